@@ -1,0 +1,369 @@
+"""Benchmark of the Titans memory write-and-read (libtitansmem) on B200.
+
+One step = one tm_run over a whole workload: every chunk of every stream goes
+through A1..A8 (stage inputs, forward of keys and queries, residual, backward,
+coefficient scan, weight-update contractions, fused state update, chunk walk).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 3]
+    python bench.py --impl reference ...     # the float64 oracle on host cores
+
+Multi-GPU (torchrun): weak scaling; every rank runs its own full copy of the
+workload (its own seed) with no collective on the data path; timing is the max
+over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gen import workloads as W  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+FLUSH_BYTES = 512 * 1024 * 1024
+SM_COUNT = 148
+
+
+def algorithmic_counts(w: W.Workload, T: int) -> dict:
+    """Work the method must do for one pass over the workload.
+    FLOPs/token = 4P (forward of keys and queries) + 2(P - P1) (backward data,
+    layers 2..L) + 4P (the W and S weight-update contractions) = 10P - 2P1.
+    State bytes per chunk = 16P (fp32 W and S read and written once)."""
+    dims = w.dims
+    P = W.param_count(dims)
+    P1 = dims[0] * dims[1]
+    tokens = w.streams * T
+    chunks = w.streams * (T // w.C)
+    tok_el = 4 if w.dtype == "f32" else 2
+    return {
+        "tokens": tokens,
+        "flops": float(10 * P - 2 * P1) * tokens,
+        "state_bytes": 16.0 * P * chunks,
+        "token_io_bytes": float(3 * w.d * tok_el + 12 + 4 * w.d) * tokens,
+    }
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "sm_max_mhz": d.get("sm_max_mhz", 1965.0), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons during timing."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def cpu_oracle_sample(w: W.Workload, budget_s: float = 15.0, streams=None, T=None) -> dict:
+    """Time the float64 oracle, as it stands, on a bounded sample of the
+    workload: all streams (up to the host's cores) over a token prefix sized to
+    take roughly `budget_s` seconds. Returns tokens/s and what was run."""
+    import oracle
+    cores = os.cpu_count() or 1
+    if streams is None:
+        streams = list(range(min(w.streams, cores)))
+    per_tok = 12.0 * w.P  # float64 flops per token, roughly
+    if T is None:
+        # calibrate on a short run, then size the sample to the budget
+        Tc = max(w.C, min(w.T, 64 // w.C * w.C or w.C))
+        sub = W.generate(w, streams=streams, T=Tc)
+        t0 = time.perf_counter()
+        oracle.run_workload(w, sub, threads=len(streams))
+        dt = max(time.perf_counter() - t0, 1e-4)
+        T = int(budget_s / dt * Tc)
+        T = max(w.C, min(w.T, T // w.C * w.C))
+    sub = W.generate(w, streams=streams, T=T)
+    t0 = time.perf_counter()
+    oracle.run_workload(w, sub, threads=len(streams))
+    dt = time.perf_counter() - t0
+    tokens = len(streams) * T
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": min(len(streams), cores),
+            "kind": "oracle", "seconds": dt, "approx_flops_per_token": per_tok,
+            "sample": f"{len(streams)} of {w.streams} streams x first {T} of {w.T} tokens",
+            "streams": streams, "T": T}
+
+
+def run_reference(args, w: W.Workload):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    steps = []
+    sample = None
+    budget = max(2.0, 60.0 / max(args.steps + args.warmup, 1))
+    for i in range(args.warmup + args.steps):
+        r = cpu_oracle_sample(w, budget_s=budget) if sample is None else \
+            cpu_oracle_sample(w, streams=sample[0], T=sample[1])
+        if sample is None:
+            sample = (r["streams"], r["T"])
+        if i >= args.warmup:
+            steps.append(r)
+    val = statistics.mean(s["value"] for s in steps)
+    line = {"impl": "reference", "metric": "memory tokens/sec (write+read)", "value": val,
+            "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * statistics.mean(s["seconds"] for s in steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "C": w.C, "dims": w.dims},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": steps[0]["cores"],
+                             "kind": "oracle", "sample": steps[0]["sample"]},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", type=int, default=3, help="workload index 0..4")
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--literal-gates", action="store_true",
+                    help="draw the gates exactly as specified (the MLP memories overflow)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = W.get_literal(args.workload) if args.literal_gates else W.get(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    from test_trained_neural_b200 import NeuralMemory
+
+    rank, world, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    seed_w = w if rank == 0 else W.Workload(**{**w.__dict__, "index": w.index + 1000 * rank})
+    inp = W.generate(seed_w)
+    pinned = {}
+    for key in ("k", "v", "q"):
+        a = np.ascontiguousarray(inp[key])
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if w.dtype == "bf16" else torch.from_numpy(a)
+        pinned[key] = t.reshape(w.B, w.H, w.T, w.d).pin_memory()
+    for key in ("theta", "eta", "alpha", "W0", "S0"):
+        pinned[key] = torch.from_numpy(np.ascontiguousarray(inp[key])).reshape(
+            w.B, w.H, *inp[key].shape[1:]).pin_memory()
+    del inp
+    d_in = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
+    mem = NeuralMemory(w.L, w.d, w.expansion, path=args.path)
+    path_used = mem.query_path(w.B, w.H, w.T, w.C, d_in["k"].dtype)
+    ws = mem.alloc_workspace(w.B, w.H, w.T, w.C, d_in["k"].dtype, dev)
+    y = torch.empty((w.B, w.H, w.T, w.d), dtype=torch.float32, device=dev)
+    We = torch.empty_like(d_in["W0"])
+    Se = torch.empty_like(d_in["S0"])
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        mem.run(d_in["k"], d_in["v"], d_in["q"], d_in["theta"], d_in["eta"], d_in["alpha"],
+                d_in["W0"], d_in["S0"], w.C, y=y, W_end=We, S_end=Se, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    mem.sync(ws, stream)
+    torch.cuda.synchronize()
+    ok = bool(torch.isfinite(y).all() and torch.isfinite(We).all())
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()  # L2 flush between steps, outside the timed events
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    t_wall = time.perf_counter() - t_wall
+    clk = clocks.stop()
+    mem.sync(ws, stream)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    ms = statistics.mean(step_ms)
+    ms_max = max_over_ranks(ms, world)
+
+    cnt = algorithmic_counts(w, w.T)
+    value = world * cnt["tokens"] / (ms_max * 1e-3)
+    peaks = measured_peaks()
+    hbm = peaks["hbm_gbs"] * 1e9
+    tens = peaks["bf16_tflops_sustained"] * 1e12
+    t_flop = cnt["flops"] / tens
+    t_state = (cnt["state_bytes"] + cnt["token_io_bytes"]) / hbm
+    chunk_roofline_s = max(t_flop, t_state)
+    sec = ms * 1e-3
+    if path_used == "tc":
+        roof = {"bound": "tensor", "achieved": cnt["flops"] / sec / 1e12,
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "peak_source": peaks["source"] + " bf16 sustained"}
+    else:
+        sm_mhz = clk.get("sm_mhz") or peaks["sm_max_mhz"]
+        alu_peak = SM_COUNT * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
+        roof = {"bound": "alu", "achieved": cnt["flops"] / sec / 1e12, "peak": alu_peak,
+                "unit": "TFLOP/s", "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 x max clock",
+                "sm_mhz_seen": sm_mhz}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = "tc_chunk_kernel" if path_used == "tc" else "simt_chunk_kernel"
+
+    e2e = None
+    if not args.no_e2e:
+        # End to end through the public API: pinned host inputs -> device,
+        # tm_run, device -> host of the reads and the final state, every step.
+        h_y = torch.empty(y.shape, dtype=torch.float32, pin_memory=True)
+        h_W = torch.empty(We.shape, dtype=torch.float32, pin_memory=True)
+        h_S = torch.empty(Se.shape, dtype=torch.float32, pin_memory=True)
+        bi = sum(v.numel() * v.element_size() for v in pinned.values())
+        bo = sum(v.numel() * v.element_size() for v in (h_y, h_W, h_S))
+        e_ms = []
+        for i in range(max(2, min(args.steps, 3))):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for k2, v2 in pinned.items():
+                d_in[k2].copy_(v2, non_blocking=True)
+            step()
+            h_y.copy_(y, non_blocking=True)
+            h_W.copy_(We, non_blocking=True)
+            h_S.copy_(Se, non_blocking=True)
+            b.record(stream)
+            torch.cuda.synchronize()
+            e_ms.append(a.elapsed_time(b))
+        e_ms_max = max_over_ranks(statistics.mean(e_ms), world)
+        e2e = {"value": world * cnt["tokens"] / (e_ms_max * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e_ms_max}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample(w)
+        cpu.pop("streams", None)
+        cpu.pop("T", None)
+    if rank == 0:
+        line = {
+            "metric": "memory tokens/sec (write+read)",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" and path_used == "tc" else
+                     ("bf16-in/f32" if w.dtype == "bf16" else "f32"),
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "C": w.C, "dims": w.dims,
+                       "theta_damping": w.theta_damping, "alpha_damping": w.alpha_damping, "path": path_used,
+                       "l2": "flushed between steps (512 MB write)", "parallelism": f"replicas{world}"},
+            "roofline": roof,
+            "chunk_roofline": {"t_flop_ms": t_flop * 1e3, "t_state_io_ms": t_state * 1e3,
+                               "bound": "state" if t_state > t_flop else "flop",
+                               "frac": chunk_roofline_s / (ms_max * 1e-3),
+                               "state_resident": "hbm/l2" if path_used != "tc" else "on-chip"},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
+            "clocks": clk, "finite": ok, "wall_s": t_wall, "step_ms": step_ms,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -32,7 +32,9 @@ Draw recipe (fixed; changing it changes every stored expectation)
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
+import os
 from typing import Sequence
 
 import numpy as np
@@ -58,6 +60,8 @@ class Workload:
     xavier_w0: bool
     spike_p: float = 0.0
     spike_sigma: float = 0.0
+    theta_damping: float = 1.0  # multiplies the theta draws
+    alpha_damping: float = 1.0  # multiplies the alpha draws (eta is never damped)
 
     @property
     def dims(self) -> list:
@@ -113,8 +117,46 @@ WORKLOADS = [
 ]
 
 
+# Gate damping of the MLP workloads. Drawn literally, theta ~ U[.001, .1] (or
+# U[.001, .05]) and alpha ~ U[0, .01] (or U[0, .005]) make a depth >= 2 memory
+# fed i.i.d. keys and values overflow within a few chunks; lowering theta alone
+# makes it collapse to zero under the forgetting, and the band in between is a
+# knife edge that gives way over a long stream (the float64 oracle shows all
+# three). Scaling the theta draws by 0.03 and the alpha draws by 0.01 keeps
+# every MLP workload finite, non-zero and insensitive to small perturbations
+# over its full length. The linear workload is stable as drawn.
+MLP_THETA_DAMPING = 0.03
+MLP_ALPHA_DAMPING = 0.01
+
+
 def get(index: int) -> Workload:
+    """Workload `index` as used for parity and benchmarking (damped gates for
+    the MLP memories)."""
+    w = WORKLOADS[index]
+    if w.L >= 2:
+        return dataclasses.replace(w, theta_damping=MLP_THETA_DAMPING,
+                                   alpha_damping=MLP_ALPHA_DAMPING)
+    return w
+
+
+def get_literal(index: int) -> Workload:
+    """Workload `index` with the gate ranges exactly as specified."""
     return WORKLOADS[index]
+
+
+def make(L: int, d: int, expansion: int, B: int, H: int, T: int, C: int, dtype: str = "bf16",
+         theta=(0.001, 0.1), eta=(0.8, 0.99), alpha=(0.0, 0.01), theta_damping=None,
+         alpha_damping=None, index: int = 100, xavier_w0: bool = True,
+         spike_p: float = 0.0, spike_sigma: float = 0.0) -> Workload:
+    """A custom workload (tests use small ones); seed = 1000 + index. The gate
+    damping defaults to that of the MLP workloads for L >= 2, none for L = 1."""
+    if theta_damping is None:
+        theta_damping = MLP_THETA_DAMPING if L >= 2 else 1.0
+    if alpha_damping is None:
+        alpha_damping = MLP_ALPHA_DAMPING if L >= 2 else 1.0
+    return Workload(index, f"custom-{index}", L, d, expansion, B, H, T, C, dtype, tuple(theta),
+                    tuple(eta), tuple(alpha), xavier_w0, spike_p, spike_sigma, theta_damping,
+                    alpha_damping)
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -162,9 +204,9 @@ def draw_stream(w: Workload, s: int, T: int | None = None, seed: int | None = No
         k = rng.standard_normal((BLOCK, d))
         v = rng.standard_normal((BLOCK, d))
         q = rng.standard_normal((BLOCK, d))
-        th = rng.uniform(w.theta[0], w.theta[1], BLOCK)
+        th = rng.uniform(w.theta[0], w.theta[1], BLOCK) * w.theta_damping
         et = rng.uniform(w.eta[0], w.eta[1], BLOCK)
-        al = rng.uniform(w.alpha[0], w.alpha[1], BLOCK)
+        al = rng.uniform(w.alpha[0], w.alpha[1], BLOCK) * w.alpha_damping
         if w.spike_p > 0.0:
             mask = rng.uniform(0.0, 1.0, BLOCK) < w.spike_p
             nsp = int(mask.sum())
@@ -211,11 +253,25 @@ def generate(w: Workload, streams: Sequence[int] | None = None, T: int | None = 
         out[g] = np.empty((n, T), dtype=np.float32)
     out["W0"] = np.empty((n, w.P), dtype=np.float32)
     out["S0"] = np.zeros((n, w.P), dtype=np.float32)
-    heads = {}
-    for i, s in enumerate(streams):
+
+    def fill(i_s):
+        i, s = i_s
         st = draw_stream(w, s, T, seed)
         for key in ("k", "v", "q", "theta", "eta", "alpha"):
             out[key][i] = st[key]
+
+    # Each stream has its own generator, so streams can be drawn concurrently
+    # (numpy releases the GIL inside its fill loops); the bytes do not depend
+    # on the thread count.
+    workers = min(n, os.cpu_count() or 1, 32)
+    if workers > 1:
+        with concurrent.futures.ThreadPoolExecutor(workers) as ex:
+            list(ex.map(fill, enumerate(streams)))
+    else:
+        for i_s in enumerate(streams):
+            fill(i_s)
+    heads = {}
+    for i, s in enumerate(streams):
         h = s % w.H
         if h not in heads:
             heads[h] = draw_w0_head(w, h, seed)

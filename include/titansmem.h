@@ -1,0 +1,155 @@
+/*
+ * libtitansmem: chunked write-and-read of the Titans neural long-term memory
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The memory M is a bias-free MLP of depth L (1..4) per stream, where a stream
+ * is one (batch entry, head) pair. Depth 1 is the linear map W. Between layers
+ * the activation is SiLU; after the last layer there is none. Widths are
+ * n_0 = d_h, n_1..n_{L-1} = expansion * d_h, n_L = d_h.
+ *   ("Titans, explained", glossary entry "M — the memory"; "titans-pytorch"
+ *    review: the "simple 1-4 layer MLP" neural memory)
+ *
+ * One call processes T tokens per stream in chunks of C tokens. For every
+ * token t of a chunk:
+ *   u_t = grad_W || M(k_t) - v_t ||^2, taken at the chunk-start weights
+ *         ("Titans, explained", step 2 "Measure surprise" and step 6 "Make it
+ *          trainable in parallel")
+ *   S_t = eta_t S_{t-1} - theta_t u_t        (step 3, momentum)
+ *   W_t = (1 - alpha_t) W_{t-1} + S_t        (step 4, forget then write)
+ *   y_t = M(q_t) through the chunk-start weights, no write   (step 5)
+ * The chunk of token t starts at t - (t mod C), tokens counted from 0
+ *   ("Attack of the Titans", section "Parallel training").
+ * The chunk-start weights are those at the end of the previous chunk (W0 for
+ * the first chunk of a call). Momentum S carries across chunks and calls.
+ *
+ * State layout ("parameter vector", P floats per stream): layer l = 1..L is a
+ * row-major [n_l x n_{l-1}] block, blocks end to end in layer order, so layer l
+ * starts at offset sum_{m<l} n_m n_{m-1}. tm_param_count() returns P.
+ *
+ * Carrying (W_end, S_end) of one call into (W0, S0) of the next, with the split
+ * on a chunk boundary, equals one longer call ("titans-pytorch" review, section
+ * "NeuralMemory as a standalone module": mem_state is state you carry forward).
+ *
+ * Threading: a tm_ctx may be used from one host thread at a time. Calls are
+ * asynchronous on the given stream; calls that overlap on the GPU must not
+ * share a workspace.
+ */
+#ifndef TITANSMEM_H
+#define TITANSMEM_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define TM_API __attribute__((visibility("default")))
+#else
+#define TM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct tm_ctx tm_ctx; /* opaque; owned by the library */
+
+typedef enum {
+  TM_OK = 0,
+  TM_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, T % C != 0 ... */
+  TM_ERR_UNSUPPORTED = 2,  /* valid but not implemented (shape, dtype, path)   */
+  TM_ERR_CUDA = 3,         /* a CUDA runtime call failed (launch, sync ...)    */
+  TM_ERR_OOM = 4,          /* host allocation failed, or workspace too small   */
+  TM_ERR_TIMEOUT = 5,      /* a bounded device-side wait expired               */
+  TM_ERR_DEVICE = 6        /* the device reported an internal consistency error */
+} tm_status;
+
+typedef enum { TM_ACT_SILU = 0 } tm_act;
+
+typedef enum {
+  TM_F32 = 0,  /* k, v, q are float32; fp32 arithmetic throughout            */
+  TM_BF16 = 1  /* k, v, q are bfloat16; tensor-core path, fp32 state        */
+} tm_dtype;
+
+typedef enum {
+  TM_PATH_AUTO = 0,  /* TM_BF16 -> tensor cores when the shape has a kernel, else SIMT */
+  TM_PATH_SIMT = 1,  /* fp32 CUDA-core kernel for any supported shape and dtype        */
+  TM_PATH_TC = 2     /* tcgen05 tensor-core kernel; TM_ERR_UNSUPPORTED if none fits    */
+} tm_path;
+
+/*
+ * Create a context for a memory of depth L (1..4), head dimension d_h and
+ * hidden expansion (ignored for L == 1). Host-only: allocates the small host
+ * object *out and nothing on the device.
+ * Supported: d_h in [1, 1024] and a multiple of 4; expansion * d_h <= 4096.
+ * Returns TM_ERR_INVALID_ARG for out == NULL or out-of-range values.
+ */
+TM_API tm_status tm_create(int L, int d_h, int expansion, tm_act act, tm_ctx **out);
+
+/* Destroy a context (NULL is accepted). Host-only. */
+TM_API tm_status tm_destroy(tm_ctx *ctx);
+
+/* P, the number of floats in one stream's parameter vector; 0 for NULL. */
+TM_API size_t tm_param_count(const tm_ctx *ctx);
+
+/* Select the kernel family used by tm_run (default TM_PATH_AUTO). Host-only. */
+TM_API tm_status tm_set_path(tm_ctx *ctx, tm_path path);
+
+/* The kernel family tm_run would use for these arguments. Host-only. */
+TM_API tm_status tm_query_path(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype,
+                        tm_path *out);
+
+/*
+ * Bytes of device workspace tm_run needs for this problem. Host-only. The
+ * workspace holds the device status word (first 256 bytes) plus per-stream
+ * activations of the CUDA-core path.
+ */
+TM_API tm_status tm_workspace_size(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype,
+                            size_t *bytes);
+
+/*
+ * Run the chunked write-and-read for B*H independent streams on `stream`
+ * (a cudaStream_t, NULL = legacy default stream). Asynchronous; allocates
+ * nothing on the device.
+ *
+ *   k, q   [B, H, T, d_h]  in_dtype, device     keys and queries
+ *   v      [B, H, T, d_h]  in_dtype, device     values
+ *   theta, eta, alpha [B, H, T] float32, device  per-token gates
+ *   W0, S0 [B, H, P] float32, device             state at the start of the call
+ *   y      [B, H, T, d_h] float32, device        reads M(q_t), output
+ *   W_end, S_end [B, H, P] float32, device       state after the last token
+ *   workspace: device buffer of at least tm_workspace_size() bytes, 256-byte
+ *              aligned; contents on entry are ignored.
+ *
+ * All pointers must be 16-byte aligned. W_end may equal W0 and S_end may equal
+ * S0 (in-place update); no other aliasing is allowed, and y must not overlap
+ * any input. Requires T % C == 0, 1 <= C <= 256, T >= C.
+ *
+ * Errors: argument problems return at once with no launch (TM_ERR_OOM when
+ * workspace_bytes is too small). A device-side error (an expired bounded wait,
+ * an internal check) is recorded in the workspace's status word, which every
+ * tm_run clears on `stream` before its kernels start; call tm_sync() after a
+ * tm_run to learn that call's device-side status.
+ */
+TM_API tm_status tm_run(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype,
+                 const void *k, const void *v, const void *q,
+                 const float *theta, const float *eta, const float *alpha,
+                 const float *W0, const float *S0,
+                 float *y, float *W_end, float *S_end,
+                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Wait for `stream`, then read and clear the device status word in
+ * `workspace`. Returns TM_OK, TM_ERR_TIMEOUT or TM_ERR_DEVICE from the
+ * kernels, or TM_ERR_CUDA if the stream itself reports an error.
+ */
+TM_API tm_status tm_sync(tm_ctx *ctx, void *workspace, void *stream);
+
+/* Static, NUL-terminated description of a status code. */
+TM_API const char *tm_status_string(tm_status status);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+TM_API int tm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TITANSMEM_H */

@@ -1,0 +1,222 @@
+// C-ABI of libtitansmem: argument checks, workspace accounting, kernel choice.
+// The operation each entry point performs is documented in include/titansmem.h.
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "tm_internal.h"
+
+struct tm_ctx {
+  int L;
+  int d;
+  int expansion;
+  int dims[tmem::kMaxL + 1];
+  size_t layer_off[tmem::kMaxL + 1];
+  size_t P;
+  tm_path path;
+};
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb) {
+  auto x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+tm_status check_shape(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype dt) {
+  if (!ctx) return TM_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || T < 1 || C < 1) return TM_ERR_INVALID_ARG;
+  if (C > tmem::kMaxC || T < C || T % C != 0) return TM_ERR_INVALID_ARG;
+  if (dt != TM_F32 && dt != TM_BF16) return TM_ERR_INVALID_ARG;
+  if ((long long)B * H > (1LL << 31) - 1) return TM_ERR_INVALID_ARG;
+  return TM_OK;
+}
+
+tmem::Problem make_problem(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype dt) {
+  tmem::Problem p{};
+  p.L = ctx->L;
+  for (int l = 0; l <= ctx->L; ++l) {
+    p.dims[l] = ctx->dims[l];
+    p.layer_off[l] = ctx->layer_off[l];
+  }
+  p.P = ctx->P;
+  p.B = B;
+  p.H = H;
+  p.T = T;
+  p.C = C;
+  p.streams = B * H;
+  p.in_dtype = dt;
+  return p;
+}
+
+tm_path choose_path(const tm_ctx *ctx, const tmem::Problem &p) {
+  if (ctx->path == TM_PATH_SIMT) return TM_PATH_SIMT;
+  if (ctx->path == TM_PATH_TC) return TM_PATH_TC;
+  if (p.in_dtype == TM_BF16 && tmem::tc_supported(p)) return TM_PATH_TC;
+  return TM_PATH_SIMT;
+}
+
+size_t scratch_bytes(tm_path path, const tmem::Problem &p) {
+  return path == TM_PATH_TC ? tmem::tc_scratch_bytes(p) : tmem::simt_scratch_bytes(p);
+}
+
+}  // namespace
+
+extern "C" {
+
+tm_status tm_create(int L, int d_h, int expansion, tm_act act, tm_ctx **out) {
+  if (!out) return TM_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (L < 1 || L > tmem::kMaxL || d_h < 1 || d_h > 1024 || d_h % 4 != 0) return TM_ERR_INVALID_ARG;
+  if (act != TM_ACT_SILU) return TM_ERR_INVALID_ARG;
+  if (L > 1 && (expansion < 1 || (long long)expansion * d_h > 4096)) return TM_ERR_INVALID_ARG;
+  tm_ctx *c = new (std::nothrow) tm_ctx();
+  if (!c) return TM_ERR_OOM;
+  c->L = L;
+  c->d = d_h;
+  c->expansion = L > 1 ? expansion : 1;
+  c->dims[0] = d_h;
+  for (int l = 1; l < L; ++l) c->dims[l] = expansion * d_h;
+  c->dims[L] = d_h;
+  size_t off = 0;
+  for (int l = 1; l <= L; ++l) {
+    c->layer_off[l - 1] = off;
+    off += (size_t)c->dims[l] * c->dims[l - 1];
+  }
+  c->layer_off[L] = off;
+  c->P = off;
+  c->path = TM_PATH_AUTO;
+  *out = c;
+  return TM_OK;
+}
+
+tm_status tm_destroy(tm_ctx *ctx) {
+  delete ctx;
+  return TM_OK;
+}
+
+size_t tm_param_count(const tm_ctx *ctx) { return ctx ? ctx->P : 0; }
+
+tm_status tm_set_path(tm_ctx *ctx, tm_path path) {
+  if (!ctx) return TM_ERR_INVALID_ARG;
+  if (path != TM_PATH_AUTO && path != TM_PATH_SIMT && path != TM_PATH_TC) return TM_ERR_INVALID_ARG;
+  ctx->path = path;
+  return TM_OK;
+}
+
+tm_status tm_query_path(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype,
+                        tm_path *out) {
+  if (!out) return TM_ERR_INVALID_ARG;
+  tm_status st = check_shape(ctx, B, H, T, C, in_dtype);
+  if (st != TM_OK) return st;
+  tmem::Problem p = make_problem(ctx, B, H, T, C, in_dtype);
+  tm_path path = choose_path(ctx, p);
+  if (path == TM_PATH_TC && !tmem::tc_supported(p)) return TM_ERR_UNSUPPORTED;
+  *out = path;
+  return TM_OK;
+}
+
+tm_status tm_workspace_size(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype,
+                            size_t *bytes) {
+  if (!bytes) return TM_ERR_INVALID_ARG;
+  tm_status st = check_shape(ctx, B, H, T, C, in_dtype);
+  if (st != TM_OK) return st;
+  tmem::Problem p = make_problem(ctx, B, H, T, C, in_dtype);
+  tm_path path = choose_path(ctx, p);
+  if (path == TM_PATH_TC && !tmem::tc_supported(p)) return TM_ERR_UNSUPPORTED;
+  *bytes = tmem::kStatusBytes + scratch_bytes(path, p);
+  return TM_OK;
+}
+
+tm_status tm_run(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype, const void *k,
+                 const void *v, const void *q, const float *theta, const float *eta,
+                 const float *alpha, const float *W0, const float *S0, float *y, float *W_end,
+                 float *S_end, void *workspace, size_t workspace_bytes, void *stream) {
+  tm_status st = check_shape(ctx, B, H, T, C, in_dtype);
+  if (st != TM_OK) return st;
+  const void *ptrs[] = {k, v, q, theta, eta, alpha, W0, S0, y, W_end, S_end, workspace};
+  for (const void *p : ptrs)
+    if (!p || !aligned16(p)) return TM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TM_ERR_INVALID_ARG;
+
+  tmem::Problem p = make_problem(ctx, B, H, T, C, in_dtype);
+  const size_t tok_el = in_dtype == TM_BF16 ? 2 : 4;
+  const size_t ntok = (size_t)p.streams * (size_t)T;
+  const size_t tok_bytes = ntok * (size_t)ctx->d * tok_el;
+  const size_t y_bytes = ntok * (size_t)ctx->d * 4;
+  const size_t gate_bytes = ntok * 4;
+  const size_t st_bytes = (size_t)p.streams * ctx->P * 4;
+  // y must not overlap any input or other output.
+  const void *ins[] = {k, v, q, theta, eta, alpha, W0, S0, W_end, S_end};
+  const size_t insz[] = {tok_bytes, tok_bytes, tok_bytes, gate_bytes, gate_bytes, gate_bytes,
+                         st_bytes, st_bytes, st_bytes, st_bytes};
+  for (int i = 0; i < 10; ++i)
+    if (ranges_overlap(y, y_bytes, ins[i], insz[i])) return TM_ERR_INVALID_ARG;
+  // W_end may equal W0 exactly (in place) but not partially overlap anything else.
+  if (W_end != W0 && ranges_overlap(W_end, st_bytes, W0, st_bytes)) return TM_ERR_INVALID_ARG;
+  if (S_end != S0 && ranges_overlap(S_end, st_bytes, S0, st_bytes)) return TM_ERR_INVALID_ARG;
+  if (ranges_overlap(W_end, st_bytes, S_end, st_bytes)) return TM_ERR_INVALID_ARG;
+  if (ranges_overlap(W_end, st_bytes, S0, st_bytes)) return TM_ERR_INVALID_ARG;
+  if (ranges_overlap(S_end, st_bytes, W0, st_bytes)) return TM_ERR_INVALID_ARG;
+
+  tm_path path = choose_path(ctx, p);
+  if (path == TM_PATH_TC && !tmem::tc_supported(p)) return TM_ERR_UNSUPPORTED;
+  const size_t need = tmem::kStatusBytes + scratch_bytes(path, p);
+  if (workspace_bytes < need) return TM_ERR_OOM;
+  if (ranges_overlap(workspace, need, y, y_bytes)) return TM_ERR_INVALID_ARG;
+
+  p.k = k;
+  p.v = v;
+  p.q = q;
+  p.theta = theta;
+  p.eta = eta;
+  p.alpha = alpha;
+  p.W0 = W0;
+  p.S0 = S0;
+  p.y = y;
+  p.W_end = W_end;
+  p.S_end = S_end;
+  p.status = reinterpret_cast<int *>(workspace);
+  p.scratch = static_cast<char *>(workspace) + tmem::kStatusBytes;
+  p.scratch_bytes = workspace_bytes - tmem::kStatusBytes;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(p.status, 0, sizeof(int), s) != cudaSuccess) return TM_ERR_CUDA;
+  cudaError_t err = path == TM_PATH_TC ? tmem::tc_launch(p, s) : tmem::simt_launch(p, s);
+  return err == cudaSuccess ? TM_OK : TM_ERR_CUDA;
+}
+
+tm_status tm_sync(tm_ctx *ctx, void *workspace, void *stream) {
+  if (!ctx || !workspace) return TM_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int code = 0;
+  if (cudaMemcpyAsync(&code, workspace, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return TM_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return TM_ERR_CUDA;
+  if (code == tmem::kDevOk) return TM_OK;
+  const int zero = 0;
+  if (cudaMemcpyAsync(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return TM_ERR_CUDA;
+  return code == tmem::kDevTimeout ? TM_ERR_TIMEOUT : TM_ERR_DEVICE;
+}
+
+const char *tm_status_string(tm_status status) {
+  switch (status) {
+    case TM_OK: return "ok";
+    case TM_ERR_INVALID_ARG: return "invalid argument";
+    case TM_ERR_UNSUPPORTED: return "unsupported shape, dtype or path";
+    case TM_ERR_CUDA: return "CUDA runtime error";
+    case TM_ERR_OOM: return "out of memory or workspace too small";
+    case TM_ERR_TIMEOUT: return "a bounded device-side wait expired";
+    case TM_ERR_DEVICE: return "device-side consistency check failed";
+  }
+  return "unknown status";
+}
+
+int tm_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,49 @@
+// Internal declarations shared by the library's translation units (host side).
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "../../include/titansmem.h"
+
+namespace tmem {
+
+constexpr int kMaxL = 4;
+constexpr int kMaxC = 256;
+constexpr size_t kStatusBytes = 256;  // device status word lives here
+
+// Device status codes written by kernels (first error wins).
+enum DevStatus : int {
+  kDevOk = 0,
+  kDevTimeout = 1,     // a bounded wait ran out
+  kDevBadConfig = 2,   // kernel received a shape it was not built for
+};
+
+struct Problem {
+  int L;
+  int dims[kMaxL + 1];
+  size_t layer_off[kMaxL + 1];
+  size_t P;
+  int B, H, T, C;
+  int streams;
+  tm_dtype in_dtype;
+  const void *k, *v, *q;
+  const float *theta, *eta, *alpha;
+  const float *W0, *S0;
+  float *y, *W_end, *S_end;
+  int *status;            // device status word
+  void *scratch;          // per-stream activations (SIMT path)
+  size_t scratch_bytes;
+};
+
+// SIMT (CUDA-core, fp32) path.
+size_t simt_scratch_bytes(const Problem &p);
+cudaError_t simt_launch(const Problem &p, cudaStream_t stream);
+
+// Tensor-core (tcgen05) path.
+bool tc_supported(const Problem &p);
+size_t tc_scratch_bytes(const Problem &p);
+cudaError_t tc_launch(const Problem &p, cudaStream_t stream);
+
+}  // namespace tmem

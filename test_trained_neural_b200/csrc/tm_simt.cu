@@ -1,0 +1,364 @@
+// CUDA-core (fp32 FFMA) persistent chunk walker for the Titans memory.
+//
+// One CTA per stream (batch entry, head). The CTA walks the chunks of its
+// stream in order; inside a chunk it runs, with block-wide barriers between
+// the steps:
+//   A5  the gate-coefficient scan (division-free reverse recurrence),
+//   A2  forward of the chunk's keys and queries through the chunk-start weights
+//       (queries give the reads y, "Titans, explained" step 5),
+//   A3  residual G_L = 2 (M(k) - v)   (step 2: loss ||M(k) - v||^2),
+//   A4  backward G_{l-1} = (W_l^T G_l) . silu'(Z_{l-1}),
+//   A6+A7 per layer one dual-accumulator contraction over the chunk's tokens,
+//       U_W = sum_i c_i g_i x_i^T and U_S = sum_i e_i g_i x_i^T, whose epilogue
+//       applies W' = B W + c_S S - U_W and S' = A S - U_S in place
+//       (steps 3 and 4, unrolled over the chunk; "Attack of the Titans",
+//        "Parallel training": gradients at the chunk start, decay products
+//        collected per token).
+// W and S live in the caller's W_end / S_end buffers (copied from W0 / S0 at
+// the start unless they alias them). Activations of the chunk live in the
+// per-stream scratch. Everything is fp32; bf16 inputs are widened on load.
+//
+// This kernel runs every supported shape and both input dtypes. It is the
+// fp32 product path and the reference the tensor-core path is checked against
+// on small shapes.
+#include <cuda_bf16.h>
+
+#include "tm_internal.h"
+
+namespace tmem {
+namespace {
+
+constexpr int NT = 256;        // threads per CTA
+constexpr int TMt = 64;        // output tile rows
+constexpr int TNt = 64;        // output tile cols
+constexpr int TKt = 16;        // reduction tile
+constexpr int PAD = 4;
+
+struct Coef {
+  float c[kMaxC];   // weight of token i's surprise in the W update
+  float e[kMaxC];   // weight of token i's surprise in the S update
+  float Bw;         // prod (1 - alpha)     : factor on W
+  float As;         // prod eta             : factor on S in the S update
+  float cS;         // eta_1 r_1            : factor on S in the W update
+};
+
+struct SmemT {
+  float As[TKt][TMt + PAD];
+  float Bs[TKt][TNt + PAD];
+  Coef coef;
+};
+
+struct Net {
+  int L;
+  int dims[kMaxL + 1];
+  long long off[kMaxL + 1];
+  long long P;
+  int maxw;
+};
+
+__device__ __forceinline__ float load_tok(const void *p, int bf16, long long i) {
+  if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
+  return reinterpret_cast<const float *>(p)[i];
+}
+
+__device__ __forceinline__ float sigm(float z) { return 1.0f / (1.0f + expf(-z)); }
+__device__ __forceinline__ float silu(float z) { return z * sigm(z); }
+__device__ __forceinline__ float silu_prime(float z) {
+  float s = sigm(z);
+  return s * (1.0f + z * (1.0f - s));
+}
+
+// out(m, n) = sum_k A(m, k) B(n, k); A(m,k) = A[m*sam + k*sak], B(n,k) = B[n*sbn + k*sbk].
+// Every output element is handed to epi(m, n, value) exactly once.
+template <class Epi>
+__device__ void gemm(SmemT &sm, int M, int N, int K, const float *A, long long sam, long long sak,
+                     const float *B, long long sbn, long long sbk, Epi epi) {
+  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+  for (int m0 = 0; m0 < M; m0 += TMt) {
+    for (int n0 = 0; n0 < N; n0 += TNt) {
+      float acc[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+      for (int k0 = 0; k0 < K; k0 += TKt) {
+        for (int e = tid; e < TMt * TKt; e += NT) {
+          int mm, kk;
+          if (sak == 1) { kk = e % TKt; mm = e / TKt; } else { mm = e % TMt; kk = e / TMt; }
+          int gm = m0 + mm, gk = k0 + kk;
+          sm.As[kk][mm] = (gm < M && gk < K) ? A[gm * sam + gk * sak] : 0.f;
+        }
+        for (int e = tid; e < TNt * TKt; e += NT) {
+          int nn, kk;
+          if (sbk == 1) { kk = e % TKt; nn = e / TKt; } else { nn = e % TNt; kk = e / TNt; }
+          int gn = n0 + nn, gk = k0 + kk;
+          sm.Bs[kk][nn] = (gn < N && gk < K) ? B[gn * sbn + gk * sbk] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < TKt; ++kk) {
+          float a[4], b[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) a[i] = sm.As[kk][ty + 16 * i];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) b[j] = sm.Bs[kk][tx + 16 * j];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          int m = m0 + ty + 16 * i, n = n0 + tx + 16 * j;
+          if (m < M && n < N) epi(m, n, acc[i][j]);
+        }
+    }
+  }
+}
+
+// The weight update of one layer: U_W(r, c) = sum_i c_i G[i][r] X[i][c],
+// U_S(r, c) = sum_i e_i G[i][r] X[i][c], then W' = Bw W + cS S - U_W and
+// S' = As S - U_S for the [rows x cols] block at Wl / Sl.
+__device__ void update_layer(SmemT &sm, int rows, int cols, int C, const float *G, const float *X,
+                             float *Wl, float *Sl) {
+  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+  const Coef &cf = sm.coef;
+  for (int m0 = 0; m0 < rows; m0 += TMt) {
+    for (int n0 = 0; n0 < cols; n0 += TNt) {
+      float aw[4][4], as[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) aw[i][j] = as[i][j] = 0.f;
+      for (int k0 = 0; k0 < C; k0 += TKt) {
+        for (int e = tid; e < TMt * TKt; e += NT) {
+          int mm = e % TMt, kk = e / TMt;  // G[i][r]: r contiguous
+          int gm = m0 + mm, gk = k0 + kk;
+          sm.As[kk][mm] = (gm < rows && gk < C) ? G[(long long)gk * rows + gm] : 0.f;
+        }
+        for (int e = tid; e < TNt * TKt; e += NT) {
+          int nn = e % TNt, kk = e / TNt;  // X[i][c]: c contiguous
+          int gn = n0 + nn, gk = k0 + kk;
+          sm.Bs[kk][nn] = (gn < cols && gk < C) ? X[(long long)gk * cols + gn] : 0.f;
+        }
+        __syncthreads();
+        for (int kk = 0; kk < TKt && k0 + kk < C; ++kk) {
+          float ci = cf.c[k0 + kk], ei = cf.e[k0 + kk];
+          float a[4], b[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) a[i] = sm.As[kk][ty + 16 * i];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) b[j] = sm.Bs[kk][tx + 16 * j];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float ab = a[i] * b[j];
+              aw[i][j] = fmaf(ci, ab, aw[i][j]);
+              as[i][j] = fmaf(ei, ab, as[i][j]);
+            }
+        }
+        __syncthreads();
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          int r = m0 + ty + 16 * i, c = n0 + tx + 16 * j;
+          if (r < rows && c < cols) {
+            long long idx = (long long)r * cols + c;
+            float w = Wl[idx], s = Sl[idx];
+            Wl[idx] = cf.Bw * w + cf.cS * s - aw[i][j];
+            Sl[idx] = cf.As * s - as[i][j];
+          }
+        }
+    }
+  }
+}
+
+// A5: per-token coefficients of one chunk from its gates (0-based i = 0..n-1):
+//   pa_i = prod_{j>i} (1 - alpha_j),  pe_i = prod_{j>i} eta_j,
+//   r_{n-1} = 1,  r_i = pa_i + eta_{i+1} r_{i+1},
+//   c_i = theta_i r_i,  e_i = theta_i pe_i,
+//   Bw = pa_0 (1 - alpha_0),  As = pe_0 eta_0,  cS = eta_0 r_0.
+// Unrolling S_t = eta_t S_{t-1} - theta_t u_t and W_t = (1-alpha_t) W_{t-1} + S_t
+// over the chunk gives W_end = Bw W + cS S - sum c_i u_i, S_end = As S - sum e_i u_i.
+// No division, so alpha = 1 and eta = 0 are exact.
+__device__ void chunk_coefficients(Coef &cf, const float *theta, const float *eta,
+                                   const float *alpha, int n) {
+  if (threadIdx.x != 0) return;
+  float pa = 1.f, pe = 1.f, r = 1.f;
+  for (int i = n - 1; i >= 0; --i) {
+    if (i < n - 1) {
+      pa *= 1.f - alpha[i + 1];
+      pe *= eta[i + 1];
+      r = pa + eta[i + 1] * r;
+    }
+    cf.c[i] = theta[i] * r;
+    cf.e[i] = theta[i] * pe;
+  }
+  cf.Bw = pa * (1.f - alpha[0]);
+  cf.As = pe * eta[0];
+  cf.cS = eta[0] * r;
+}
+
+struct KArgs {
+  Net net;
+  int T, C, bf16;
+  const void *k, *v, *q;
+  const float *theta, *eta, *alpha, *W0, *S0;
+  float *y, *W, *S;
+  float *scratch;
+  long long scratch_per_stream;  // floats
+  int *status;
+};
+
+__global__ void __launch_bounds__(NT) simt_chunk_kernel(KArgs a) {
+  __shared__ SmemT sm;
+  const Net &n = a.net;
+  const int s = blockIdx.x;
+  const int L = n.L, C = a.C, T = a.T;
+  const int d_in = n.dims[0], d_out = n.dims[L];
+  if (C > kMaxC || C < 1) {
+    if (threadIdx.x == 0) atomicCAS(a.status, 0, kDevBadConfig);
+    return;
+  }
+  float *W = a.W + (long long)s * n.P;
+  float *S = a.S + (long long)s * n.P;
+  if (a.W0 + (long long)s * n.P != W)
+    for (long long i = threadIdx.x; i < n.P; i += NT) W[i] = a.W0[(long long)s * n.P + i];
+  if (a.S0 + (long long)s * n.P != S)
+    for (long long i = threadIdx.x; i < n.P; i += NT) S[i] = a.S0[(long long)s * n.P + i];
+
+  // scratch layout (floats): X[0..L-1] (C x n_l), Z[1..L-1] (C x n_l),
+  // Qa, Qb (C x maxw), Ga, Gb (C x maxw)
+  float *base = a.scratch + (long long)s * a.scratch_per_stream;
+  float *X[kMaxL], *Z[kMaxL];
+  float *p = base;
+  for (int l = 0; l < L; ++l) { X[l] = p; p += (long long)C * n.dims[l]; }
+  for (int l = 1; l < L; ++l) { Z[l] = p; p += (long long)C * n.dims[l]; }
+  float *Qa = p; p += (long long)C * n.maxw;
+  float *Qb = p; p += (long long)C * n.maxw;
+  float *Ga = p; p += (long long)C * n.maxw;
+  float *Gb = p;
+  __syncthreads();
+
+  const long long tok_base = (long long)s * T;
+  for (int t0 = 0; t0 < T; t0 += C) {
+    const long long tb = tok_base + t0;
+    chunk_coefficients(sm.coef, a.theta + tb, a.eta + tb, a.alpha + tb, C);
+    for (int i = threadIdx.x; i < C * d_in; i += NT) {
+      X[0][i] = load_tok(a.k, a.bf16, tb * d_in + i);
+      Qa[i] = load_tok(a.q, a.bf16, tb * d_in + i);
+    }
+    __syncthreads();
+
+    // A2 + A3: forward of the keys; keep pre-activations for the backward.
+    float *Gcur = Ga, *Gnext = Gb;
+    for (int l = 1; l <= L; ++l) {
+      const float *Wl = W + n.off[l - 1];
+      const int rows = n.dims[l], cols = n.dims[l - 1];
+      if (l < L) {
+        float *Zl = Z[l], *Xl = X[l];
+        gemm(sm, C, rows, cols, X[l - 1], cols, 1, Wl, cols, 1,
+             [&](int i, int r, float z) {
+               Zl[(long long)i * rows + r] = z;
+               Xl[(long long)i * rows + r] = silu(z);
+             });
+      } else {
+        gemm(sm, C, rows, cols, X[l - 1], cols, 1, Wl, cols, 1,
+             [&](int i, int r, float z) {
+               float vv = load_tok(a.v, a.bf16, (tb + i) * d_out + r);
+               Gcur[(long long)i * rows + r] = 2.f * (z - vv);
+             });
+      }
+      __syncthreads();
+    }
+    // A2 (read half): forward of the queries through the same weights -> y.
+    float *qin = Qa, *qout = Qb;
+    for (int l = 1; l <= L; ++l) {
+      const float *Wl = W + n.off[l - 1];
+      const int rows = n.dims[l], cols = n.dims[l - 1];
+      if (l < L) {
+        gemm(sm, C, rows, cols, qin, cols, 1, Wl, cols, 1,
+             [&](int i, int r, float z) { qout[(long long)i * rows + r] = silu(z); });
+        float *tmp = qin; qin = qout; qout = tmp;
+      } else {
+        float *y = a.y + tb * d_out;
+        gemm(sm, C, rows, cols, qin, cols, 1, Wl, cols, 1,
+             [&](int i, int r, float z) { y[(long long)i * rows + r] = z; });
+      }
+      __syncthreads();
+    }
+    // A4: backward to every layer's pre-activation gradient.
+    // G[l] for layer l is kept: the update of layer l needs it.
+    float *Gl[kMaxL + 1];
+    Gl[L] = Gcur;
+    // Keep distinct buffers: layer L in Ga, then alternate through Gb and the
+    // (no longer needed) query buffers.
+    float *pool[3] = {Gb, Qa, Qb};
+    for (int l = L; l >= 2; --l) {
+      const float *Wl = W + n.off[l - 1];
+      const int rows = n.dims[l], cols = n.dims[l - 1];
+      float *Gout = pool[(L - l) % 3];
+      const float *Zp = Z[l - 1];
+      gemm(sm, C, cols, rows, Gl[l], rows, 1, Wl, 1, cols,
+           [&](int i, int c, float g) {
+             long long idx = (long long)i * cols + c;
+             Gout[idx] = g * silu_prime(Zp[idx]);
+           });
+      Gl[l - 1] = Gout;
+      __syncthreads();
+    }
+    (void)Gnext;
+    // A6 + A7: per-layer dual contraction and fused state update.
+    for (int l = 1; l <= L; ++l) {
+      update_layer(sm, n.dims[l], n.dims[l - 1], C, Gl[l], X[l - 1], W + n.off[l - 1],
+                   S + n.off[l - 1]);
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+size_t simt_scratch_bytes(const Problem &p) {
+  long long per = 0;
+  int maxw = 0;
+  for (int l = 0; l <= p.L; ++l) maxw = p.dims[l] > maxw ? p.dims[l] : maxw;
+  for (int l = 0; l < p.L; ++l) per += (long long)p.C * p.dims[l];
+  for (int l = 1; l < p.L; ++l) per += (long long)p.C * p.dims[l];
+  per += 4LL * p.C * maxw;
+  per = (per + 63) / 64 * 64;
+  return (size_t)per * sizeof(float) * (size_t)p.streams;
+}
+
+cudaError_t simt_launch(const Problem &p, cudaStream_t stream) {
+  KArgs a;
+  a.net.L = p.L;
+  a.net.maxw = 0;
+  for (int l = 0; l <= p.L; ++l) {
+    a.net.dims[l] = p.dims[l];
+    a.net.off[l] = (long long)p.layer_off[l];
+    a.net.maxw = p.dims[l] > a.net.maxw ? p.dims[l] : a.net.maxw;
+  }
+  a.net.P = (long long)p.P;
+  a.T = p.T;
+  a.C = p.C;
+  a.bf16 = p.in_dtype == TM_BF16;
+  a.k = p.k; a.v = p.v; a.q = p.q;
+  a.theta = p.theta; a.eta = p.eta; a.alpha = p.alpha;
+  a.W0 = p.W0; a.S0 = p.S0;
+  a.y = p.y; a.W = p.W_end; a.S = p.S_end;
+  a.scratch = reinterpret_cast<float *>(p.scratch);
+  a.scratch_per_stream = (long long)(simt_scratch_bytes(p) / sizeof(float) / (size_t)p.streams);
+  a.status = p.status;
+  simt_chunk_kernel<<<p.streams, NT, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace tmem

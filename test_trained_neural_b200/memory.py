@@ -1,0 +1,108 @@
+"""Python front end of libtitansmem: the neural long-term memory write-and-read.
+
+``NeuralMemory(L, d_h, expansion).run(...)`` hands torch CUDA tensors to the C
+ABI ``tm_run``; torch only supplies device memory and the stream.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _native as N
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+class NeuralMemory:
+    """A context for memories of depth L, head dim d_h, hidden = expansion * d_h."""
+
+    def __init__(self, L: int, d_h: int, expansion: int = 4, path: str = "auto"):
+        self._lib = N.load()
+        h = ctypes.c_void_p()
+        N.check(self._lib.tm_create(L, d_h, expansion, N.TM_ACT_SILU, ctypes.byref(h)), "tm_create")
+        self._h = h
+        self.L, self.d_h, self.expansion = L, d_h, expansion
+        self.P = int(self._lib.tm_param_count(h))
+        self.set_path(path)
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            self._lib.tm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def set_path(self, path: str) -> None:
+        code = {"auto": N.TM_PATH_AUTO, "simt": N.TM_PATH_SIMT, "tc": N.TM_PATH_TC}[path]
+        N.check(self._lib.tm_set_path(self._h, code), "tm_set_path")
+        self.path = path
+
+    @staticmethod
+    def _dtype_code(t: torch.Tensor) -> int:
+        if t.dtype == torch.bfloat16:
+            return N.TM_BF16
+        if t.dtype == torch.float32:
+            return N.TM_F32
+        raise TypeError(f"k/v/q must be float32 or bfloat16, got {t.dtype}")
+
+    def query_path(self, B, H, T, C, dtype=torch.bfloat16) -> str:
+        out = ctypes.c_int()
+        code = N.TM_BF16 if dtype == torch.bfloat16 else N.TM_F32
+        N.check(self._lib.tm_query_path(self._h, B, H, T, C, code, ctypes.byref(out)), "tm_query_path")
+        return {N.TM_PATH_SIMT: "simt", N.TM_PATH_TC: "tc"}[out.value]
+
+    def workspace_size(self, B, H, T, C, dtype=torch.bfloat16) -> int:
+        out = ctypes.c_size_t()
+        code = N.TM_BF16 if dtype == torch.bfloat16 else N.TM_F32
+        N.check(self._lib.tm_workspace_size(self._h, B, H, T, C, code, ctypes.byref(out)),
+                "tm_workspace_size")
+        return int(out.value)
+
+    def alloc_workspace(self, B, H, T, C, dtype=torch.bfloat16, device="cuda") -> torch.Tensor:
+        n = self.workspace_size(B, H, T, C, dtype)
+        return torch.empty(n, dtype=torch.uint8, device=device)
+
+    def run(self, k, v, q, theta, eta, alpha, W0, S0, C, y=None, W_end=None, S_end=None,
+            workspace=None, stream=None, sync=False):
+        """Write-and-read over T tokens for B*H streams.
+
+        k, v, q: [B, H, T, d_h] float32 or bfloat16 CUDA tensors; gates [B, H, T]
+        float32; W0, S0 [B, H, P] float32. Returns (y, W_end, S_end); pass
+        W_end=W0 / S_end=S0 to update in place.
+        """
+        B, H, T, d = k.shape
+        dt = self._dtype_code(k)
+        for t in (k, v, q, theta, eta, alpha, W0, S0):
+            if not t.is_cuda or not t.is_contiguous():
+                raise ValueError("all tensors must be contiguous CUDA tensors")
+        if y is None:
+            y = torch.empty((B, H, T, d), dtype=torch.float32, device=k.device)
+        if W_end is None:
+            W_end = torch.empty_like(W0)
+        if S_end is None:
+            S_end = torch.empty_like(S0)
+        if workspace is None:
+            workspace = self.alloc_workspace(B, H, T, C, k.dtype, k.device)
+        if stream is None:
+            stream = torch.cuda.current_stream(k.device)
+        code = self._lib.tm_run(self._h, B, H, T, C, dt, _ptr(k), _ptr(v), _ptr(q), _ptr(theta),
+                                _ptr(eta), _ptr(alpha), _ptr(W0), _ptr(S0), _ptr(y), _ptr(W_end),
+                                _ptr(S_end), _ptr(workspace), workspace.numel(),
+                                ctypes.c_void_p(stream.cuda_stream))
+        N.check(code, "tm_run")
+        if sync:
+            self.sync(workspace, stream)
+        return y, W_end, S_end
+
+    def sync(self, workspace, stream=None):
+        if stream is None:
+            stream = torch.cuda.current_stream(workspace.device)
+        N.check(self._lib.tm_sync(self._h, _ptr(workspace), ctypes.c_void_p(stream.cuda_stream)),
+                "tm_sync")

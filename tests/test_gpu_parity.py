@@ -1,0 +1,194 @@
+"""GPU parity: libtitansmem against the float64 oracle on the same seeded inputs.
+
+Tolerances (max normwise relative error per stream and per output tensor, each
+layer of W and S separately): 1e-4 for fp32 arithmetic, 2e-2 for the bf16
+tensor-core path.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gen import workloads as W
+from test_trained_neural_b200 import NeuralMemory
+
+from gpu_util import gpu_to_np, parity_errors, run_lib, to_dev
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-4
+TOL_BF16_TC = 2e-2
+
+
+def check(w: W.Workload, path: str, tol: float, streams=None, T=None):
+    inp = W.generate(w, streams=streams, T=T)
+    n = len(inp["streams"])
+    B, H = (w.B, w.H) if n == w.streams else (1, n)
+    Tn = inp["k"].shape[1]
+    mem = NeuralMemory(w.L, w.d, w.expansion, path=path)
+    dev = to_dev(inp, B, H, w.dtype)
+    y, We, Se = run_lib(mem, dev, w.C)
+    ref = oracle.run_workload(w, inp)
+    errs = parity_errors(w.dims, inp["W0"], gpu_to_np(y, We, Se), ref)
+    assert all(np.isfinite(v) for v in errs.values()), errs
+    assert max(errs.values()) < tol, (w.name, path, Tn, errs)
+    return errs
+
+
+def test_linear_fp32_workload():
+    """The linear fp32 workload in full (B=H=1, d=64, T=256, C=16)."""
+    check(W.get(0), "auto", TOL_F32)
+
+
+SMALL = [  # L, d, expansion, B, H, T, C
+    (1, 16, 1, 1, 3, 48, 16),
+    (1, 64, 1, 2, 1, 40, 8),
+    (2, 16, 4, 1, 2, 64, 16),
+    (2, 32, 4, 2, 2, 96, 32),
+    (2, 64, 4, 1, 2, 128, 64),
+    (2, 24, 3, 1, 1, 30, 10),      # ragged widths (72 hidden), odd chunk count
+    (3, 16, 2, 1, 2, 48, 16),
+    (4, 32, 2, 1, 2, 128, 64),
+    (4, 16, 2, 2, 1, 40, 5),
+    (2, 32, 4, 1, 2, 32, 1),       # C = 1: token-by-token descent
+    (2, 32, 4, 1, 1, 128, 128),    # one chunk covers the whole stream
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: "L%d-d%d-e%d-B%dH%d-T%d-C%d" % c)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("damped", [True, False], ids=["damped", "literal"])
+def test_simt_small_shapes(cfg, dtype, damped):
+    """Literal gates give large writes; the short streams here stay finite."""
+    L, d, e, B, H, T, C = cfg
+    extra = {} if damped else {"theta_damping": 1.0, "alpha_damping": 1.0}
+    w = W.make(L, d, e, B, H, T, C, dtype=dtype, index=200 + sum(cfg), **extra)
+    check(w, "simt", TOL_F32)
+
+
+def test_simt_literal_gates_short_horizon():
+    """The gates exactly as specified, over the horizon where the memory is
+    still finite (a few chunks), on the README-shaped workload."""
+    w = W.get_literal(1)
+    check(w, "simt", TOL_F32, T=128)
+
+
+def _dev_inputs(w, streams=None, T=None):
+    inp = W.generate(w, streams=streams, T=T)
+    n = len(inp["streams"])
+    B, H = (w.B, w.H) if n == w.streams else (1, n)
+    return inp, to_dev(inp, B, H, w.dtype)
+
+
+@pytest.mark.parametrize("path", ["simt"])
+def test_in_place_state_equals_out_of_place(path):
+    w = W.make(2, 32, 4, 1, 2, 128, 32, index=301)
+    _, dev = _dev_inputs(w)
+    mem = NeuralMemory(w.L, w.d, w.expansion, path=path)
+    y1, We1, Se1 = run_lib(mem, dev, w.C)
+    W0, S0 = dev["W0"].clone(), dev["S0"].clone()
+    y2, We2, Se2 = mem.run(dev["k"], dev["v"], dev["q"], dev["theta"], dev["eta"], dev["alpha"],
+                           W0, S0, w.C, W_end=W0, S_end=S0, sync=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2) and torch.equal(We1, W0) and torch.equal(Se1, S0)
+
+
+@pytest.mark.parametrize("path", ["simt"])
+def test_state_carry_and_determinism(path):
+    w = W.make(2, 32, 4, 2, 1, 192, 32, index=302)
+    _, dev = _dev_inputs(w)
+    mem = NeuralMemory(w.L, w.d, w.expansion, path=path)
+    y, We, Se = run_lib(mem, dev, w.C)
+    y_b, We_b, Se_b = run_lib(mem, dev, w.C)
+    assert torch.equal(y, y_b) and torch.equal(We, We_b) and torch.equal(Se, Se_b)
+    T1 = 64
+    first = {k: (v[:, :, :T1].contiguous() if k in ("k", "v", "q", "theta", "eta", "alpha") else v)
+             for k, v in dev.items()}
+    ya, Wa, Sa = run_lib(mem, first, w.C)
+    second = {k: (v[:, :, T1:].contiguous() if k in ("k", "v", "q", "theta", "eta", "alpha") else v)
+              for k, v in dev.items()}
+    second["W0"], second["S0"] = Wa, Sa
+    yb, Wb, Sb = run_lib(mem, second, w.C)
+    assert torch.equal(torch.cat([ya, yb], dim=2), y)
+    assert torch.equal(Wb, We) and torch.equal(Sb, Se)
+
+
+@pytest.mark.parametrize("path", ["simt"])
+def test_streams_independent_and_permutable(path):
+    w = W.make(2, 16, 4, 1, 4, 64, 16, index=303)
+    inp, dev = _dev_inputs(w)
+    mem = NeuralMemory(w.L, w.d, w.expansion, path=path)
+    y, We, Se = run_lib(mem, dev, w.C)
+    perm = torch.tensor([3, 1, 0, 2], device="cuda")
+    pdev = {k: v[:, perm].contiguous() for k, v in dev.items()}
+    yp, Wp, Sp = run_lib(mem, pdev, w.C)
+    assert torch.equal(yp, y[:, perm]) and torch.equal(Wp, We[:, perm]) and torch.equal(Sp, Se[:, perm])
+
+
+def test_gate_extremes_on_gpu():
+    """alpha = 1 wipes (W_end = S_end up to rounding); theta = 0 writes nothing."""
+    w = W.make(2, 32, 4, 1, 2, 64, 16, index=304)
+    inp = W.generate(w)
+    inp["alpha"][:] = 1.0
+    dev = to_dev(inp, 1, 2, w.dtype)
+    mem = NeuralMemory(w.L, w.d, w.expansion, path="simt")
+    _, We, Se = run_lib(mem, dev, w.C)
+    assert torch.allclose(We, Se, rtol=1e-6, atol=1e-7)
+    inp = W.generate(w)
+    inp["theta"][:] = 0.0
+    dev = to_dev(inp, 1, 2, w.dtype)
+    _, We, Se = run_lib(mem, dev, w.C)
+    ref = oracle.run_workload(w, inp)
+    errs = parity_errors(w.dims, inp["W0"], gpu_to_np(torch.zeros(1, 2, 64, 32, device="cuda"), We, Se),
+                         {**ref, "y": np.zeros_like(ref["y"])})
+    assert errs["W"] < TOL_F32 and errs["S"] < TOL_F32
+
+
+# Full-size workloads, in the launch configuration the benchmark times, checked
+# on outputs the oracle can afford: every output of the smaller workloads, and
+# for the long ones the reads y of sampled streams over a prefix (the
+# recurrence is causal, so a prefix run of the oracle gives the same y).
+FULL = [(1, None, None), (2, None, None), (3, [0, 9], 2048), (4, [0, 37], 1024)]
+
+
+@pytest.mark.parametrize("idx,sample_streams,prefix", FULL, ids=lambda x: str(x))
+def test_full_size_workloads(idx, sample_streams, prefix):
+    w = W.get(idx)
+    inp = W.generate(w)
+    dev = to_dev(inp, w.B, w.H, w.dtype)
+    if sample_streams is not None:
+        del inp
+    mem = NeuralMemory(w.L, w.d, w.expansion, path="auto")
+    tol = TOL_BF16_TC if mem.query_path(w.B, w.H, w.T, w.C) == "tc" else TOL_F32
+    y, We, Se = run_lib(mem, dev, w.C)
+    assert torch.isfinite(y).all() and torch.isfinite(We).all() and torch.isfinite(Se).all()
+    if sample_streams is None:
+        ref = oracle.run_workload(w, inp)
+        errs = parity_errors(w.dims, inp["W0"], gpu_to_np(y, We, Se), ref)
+        assert max(errs.values()) < tol, errs
+    else:
+        sub = W.generate(w, streams=sample_streams, T=prefix)
+        ref = oracle.run_workload(w, sub)
+        yf = y.reshape(w.streams, w.T, w.d)
+        for i, s in enumerate(sample_streams):
+            got = yf[s, :prefix].double().cpu().numpy()
+            err = np.linalg.norm(got - ref["y"][i]) / np.linalg.norm(ref["y"][i])
+            assert err < tol, (idx, s, err)
+
+
+@pytest.mark.parametrize("idx,sample_streams,T", [(3, [0, 15], 1024), (4, [0, 63], 512)])
+def test_all_streams_short_stream_state(idx, sample_streams, T):
+    """Every stream of the long workloads over a shortened stream: the state
+    (W_end, S_end) and reads of sampled streams against the oracle."""
+    w = W.get(idx)
+    inp = W.generate(w, T=T)
+    dev = to_dev(inp, w.B, w.H, w.dtype)
+    mem = NeuralMemory(w.L, w.d, w.expansion, path="auto")
+    tol = TOL_BF16_TC if mem.query_path(w.B, w.H, T, w.C) == "tc" else TOL_F32
+    y, We, Se = run_lib(mem, dev, w.C)
+    gpu = gpu_to_np(y, We, Se)
+    sub = {k: (v[sample_streams] if k != "streams" else v) for k, v in inp.items()}
+    ref = oracle.run_workload(w, sub)
+    gsub = {k: v[sample_streams] for k, v in gpu.items()}
+    errs = parity_errors(w.dims, inp["W0"][sample_streams], gsub, ref)
+    assert max(errs.values()) < tol, errs
