@@ -215,12 +215,17 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--literal-gates", action="store_true",
                     help="draw the gates exactly as specified (the MLP memories overflow)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override T (tokens per stream), e.g. for short profiling runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     w = W.get_literal(args.workload) if args.literal_gates else W.get(args.workload)
+    if args.tokens:
+        import dataclasses
+        w = dataclasses.replace(w, T=args.tokens)
     if args.impl == "reference":
         return run_reference(args, w)
 

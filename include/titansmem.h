@@ -142,6 +142,16 @@ TM_API tm_status tm_run(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dty
  */
 TM_API tm_status tm_sync(tm_ctx *ctx, void *workspace, void *stream);
 
+/*
+ * Test hook for failure handling (process-wide, host-only). inject_timeout != 0
+ * makes every CTA of the tensor-core kernel first wait on a barrier that
+ * nothing completes, so the bounded wait expires, the kernel records
+ * TM_ERR_TIMEOUT, cleans up and returns; tm_sync() then reports it.
+ * wait_limit_ns sets the time limit of each device-side wait (0 = default 2 s).
+ * Affects launches issued after the call.
+ */
+TM_API tm_status tm_set_debug(int inject_timeout, unsigned long long wait_limit_ns);
+
 /* Static, NUL-terminated description of a status code. */
 TM_API const char *tm_status_string(tm_status status);
 

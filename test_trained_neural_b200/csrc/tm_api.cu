@@ -204,6 +204,11 @@ tm_status tm_sync(tm_ctx *ctx, void *workspace, void *stream) {
   return code == tmem::kDevTimeout ? TM_ERR_TIMEOUT : TM_ERR_DEVICE;
 }
 
+tm_status tm_set_debug(int inject_timeout, unsigned long long wait_limit_ns) {
+  tmem::tc_set_debug(inject_timeout, wait_limit_ns);
+  return TM_OK;
+}
+
 const char *tm_status_string(tm_status status) {
   switch (status) {
     case TM_OK: return "ok";

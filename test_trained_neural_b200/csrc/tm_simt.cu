@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(NT) simt_chunk_kernel(KArgs a) {
     __syncthreads();
 
     // A2 + A3: forward of the keys; keep pre-activations for the backward.
-    float *Gcur = Ga, *Gnext = Gb;
+    float *Gcur = Ga;
     for (int l = 1; l <= L; ++l) {
       const float *Wl = W + n.off[l - 1];
       const int rows = n.dims[l], cols = n.dims[l - 1];
@@ -314,7 +314,6 @@ __global__ void __launch_bounds__(NT) simt_chunk_kernel(KArgs a) {
       Gl[l - 1] = Gout;
       __syncthreads();
     }
-    (void)Gnext;
     // A6 + A7: per-layer dual contraction and fused state update.
     for (int l = 1; l <= L; ++l) {
       update_layer(sm, n.dims[l], n.dims[l - 1], C, Gl[l], X[l - 1], W + n.off[l - 1],

@@ -1,11 +1,871 @@
-// tcgen05 tensor-core path (sm_100a). Shapes without a tensor-core kernel are
-// reported unsupported and run on the CUDA-core path under TM_PATH_AUTO.
+// tcgen05 tensor-core chunk walker for depth-2 memories, M(x) = W2 silu(W1 x).
+//
+// One thread-block cluster of G CTAs walks one stream (batch entry, head).
+// CTA j of the cluster owns hidden units [64 j, 64 j + 64): rows of W1 and
+// columns of W2, so hidden = 64 G. Per chunk of C = 64 tokens:
+//
+//   A1  TMA loads keys and queries of the chunk as one 128-row bf16 tile
+//       (keys rows 0-63, queries rows 64-127), 128-byte swizzle.
+//   A5  the control warp turns the chunk's gates into per-token coefficients
+//       with warp shuffles (division-free reverse scan).
+//   A2  Z1 = [K;Q] W1_j^T        M=128 N=64  K=d   (keys and queries share W)
+//       X1 = silu(Z1)            epilogue, bf16 to shared memory
+//       Z2_j = X1 W2_j^T         M=128 N=d   K=64  (this CTA's partial sum)
+//       all-reduce of Z2 over the cluster with bulk copies between the CTAs'
+//       shared memories (the copy engine, mbarrier transaction counts, no
+//       thread-level cluster fences): each CTA stages its partial as bf16 rows
+//       and pushes rows [128/G p, 128/G (p+1)) to CTA p (reduce-scatter); CTA p
+//       sums them in fp32, writes y for query rows and G2 = 2 (Z2 - V) for key
+//       rows, and pushes its G2 rows to every CTA (all-gather) (A3).
+//   A4  G1 = (G2 W2_j) . silu'(Z1_K)        M=128(64 used) N=64 K=d
+//   A6+A7 the fp32 state of this CTA's slice, [W | S], lives in TMEM for the
+//       whole stream. Before the weight-update contractions of a chunk the
+//       epilogue pre-scales it in place, W <- B W + c_S S, S <- A S (off the
+//       critical path), and the contractions accumulate onto it:
+//       [W2' | S2']   = [W2 | S2]   + G2^T [-c X1_K | -e X1_K]   M=d N=128 K=64
+//       [W1' | S1']^T = [W1 | S1]^T + K^T  [-c G1   | -e G1]     M=d N=128 K=64
+//       (c_i, e_i fold the momentum and forget gates of the chunk into the
+//        operands), so the tensor core itself emits the updated state; the
+//       epilogue only writes the bf16 copy of W' the next chunk multiplies with.
+//   A8  the loop over chunks; TMA for chunk c+1 overlaps the write-back.
+//       W_end / S_end are written once, after the last chunk.
+//
+// ("Titans, explained" steps 2-6; "Attack of the Titans", "Parallel training":
+//  gradients at the chunk-start weights written as matrix products, decay
+//  products folded per token.)
+//
+// Warp roles: warps 0-7 epilogue (warp w reads TMEM lanes 32 (w % 4) .. +31,
+// columns half w / 4), warp 8 control (TMA, MMA issue by lane 0, scan).
+// Every wait is bounded; on expiry the kernel records TM_ERR_TIMEOUT in the
+// status word, drains its copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <cstring>
+
 #include "tm_internal.h"
+#include "tm_sm100.cuh"
 
 namespace tmem {
+namespace {
 
-bool tc_supported(const Problem &) { return false; }
+using namespace sm100;
+
+constexpr int C = 64;           // chunk size of this kernel
+constexpr int HS = 64;          // hidden units per CTA
+constexpr int EPI_WARPS = 8;
+constexpr int NTHREADS = (EPI_WARPS + 1) * 32;
+constexpr int EPI_THREADS = EPI_WARPS * 32;
+constexpr int CTL_WARP = EPI_WARPS;
+constexpr uint32_t TMEM_COLS = 512;
+
+struct TcArgs {
+  int T, P, G;
+  const __nv_bfloat16 *v;
+  const float *theta, *eta, *alpha;
+  const float *W0, *S0;
+  float *y, *W, *S;
+  int *status;
+  unsigned long long wait_ns;
+  int inject_timeout;
+};
+
+struct Coefs {
+  float c[C];
+  float e[C];
+  float Bw, As, cS, pad;
+};
+
+// Shared-memory map (bytes from a 1024-aligned base). Feature dims of the
+// d-wide buffers are allocated as 128 even for d = 64 so that the padded
+// M = 128 operands stay inside their own buffer.
+template <int D>
+struct Layout {
+  static constexpr int FD = 128;
+  static constexpr uint32_t W1 = 0;                          // W1_j^T [D x 64 hid] R=D
+  static constexpr uint32_t W2 = W1 + D * 64 * 2;            // W2_j   [D x 64 hid] R=D
+  static constexpr uint32_t XKQ = W2 + D * 64 * 2;           // [128 tok x FD]  R=128
+  static constexpr uint32_t X1 = XKQ + 128 * FD * 2;         // [128 tok x 64]  R=128
+  static constexpr uint32_t X1S = X1 + 128 * 64 * 2;         // [64 tok x 128]  R=64
+  static constexpr uint32_t G2 = X1S + 64 * 128 * 2;         // [64 tok x FD]   R=64
+  static constexpr uint32_t G1S = G2 + 64 * FD * 2;          // [64 tok x 128]  R=64
+  static constexpr uint32_t SEND = G1S + 64 * 128 * 2;       // [128 x D] bf16 partial Z2
+  static constexpr uint32_t RECV = SEND + 128 * D * 2;       // G x [128/G x D] bf16
+  static constexpr uint32_t G2OWN = RECV + 128 * D * 2;      // owned rows of G2, RB atoms
+  static constexpr uint32_t COEF = G2OWN + 64 * D * 2;       // 2 x Coefs
+  static constexpr uint32_t BARS = COEF + 2 * sizeof(Coefs);
+  static constexpr uint32_t NBARS = 16;
+  static constexpr uint32_t MISC = BARS + NBARS * 8;         // tmem slot, abort flag
+  static constexpr uint32_t TOTAL = MISC + 64;
+};
+
+enum Bar {
+  B_TMA = 0, B_COEF, B_F1, B_X1, B_F2, B_SEND, B_RECV, B_G2OWN, B_G2, B_B1, B_G1, B_U2, B_U1,
+  B_UPD, B_FIN, B_NEVER, B_COUNT
+};
+
+__device__ __forceinline__ float sigm(float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ uint4 pack8(const float *v) {
+  return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                    pack_bf16(v[6], v[7]));
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, unsigned short v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void arrive_remote_release(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                   bar_cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ bool try_wait_acquire_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Copy `bytes` from this CTA's shared memory into CTA-of-cluster shared memory
+// (dst, bar are shared::cluster addresses); completion counts on the remote bar.
+__device__ __forceinline__ void bulk_push(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "r"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ uint4 ld_cluster_u4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared::cluster.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void fence_acq_rel_cluster() {
+  asm volatile("fence.acq_rel.cluster;" ::: "memory");
+}
+// One arrival per warp on a local barrier, after every lane's shared-memory
+// writes have been made visible to the tensor cores (async proxy).
+__device__ __forceinline__ void warp_arrive_local(uint64_t *bar, int lane) {
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+}
+// One arrival per warp on the barrier of every CTA of the cluster, after every
+// lane's stores into those CTAs are visible at cluster scope.
+template <int G>
+__device__ __forceinline__ void warp_arrive_cluster(uint64_t *bar, int lane) {
+  fence_acq_rel_cluster();
+  __syncwarp();
+  if (lane == 0) {
+    const uint32_t b = smem_u32(bar);
+#pragma unroll
+    for (int p = 0; p < G; ++p) arrive_remote_release(mapa(b, p));
+  }
+}
+
+// Bounded wait that also gives up as soon as another thread of the CTA has
+// flagged an abort. cluster_scope selects acquire.cluster semantics.
+__device__ bool wait_bar(uint64_t *bar, uint32_t parity, const TcArgs &a, volatile int *abort_flag,
+                         bool cluster_scope = false) {
+  const uint32_t addr = smem_u32(bar);
+  auto probe = [&]() {
+    return cluster_scope ? try_wait_acquire_cluster(addr, parity) : mbar_try_wait(bar, parity);
+  };
+  if (probe()) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i)
+      if (probe()) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > a.wait_ns) {
+      atomicCAS(a.status, 0, kDevTimeout);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+// A5 with warp shuffles. Lane l holds tokens 2l and 2l+1 of the chunk.
+//   pa_i = prod_{j>i} (1 - alpha_j), pe_i = prod_{j>i} eta_j,
+//   r_i  = pa_i + eta_{i+1} r_{i+1}, r_{C-1} = 1   (an affine map per token,
+//          composed from the right with an inclusive suffix scan),
+//   c_i = theta_i r_i, e_i = theta_i pe_i,
+//   Bw = prod (1 - alpha), As = prod eta, cS = eta_0 r_0.
+__device__ void coef_scan_warp(Coefs &cf, const float *th, const float *et, const float *al,
+                               int lane) {
+  const int i0 = 2 * lane, i1 = 2 * lane + 1;
+  const float t0 = th[i0], t1 = th[i1], e0 = et[i0], e1 = et[i1];
+  const float f0 = 1.f - al[i0], f1 = 1.f - al[i1];
+  // inclusive suffix products over lanes of the pair products
+  float pf = f0 * f1, pe = e0 * e1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    float xf = __shfl_down_sync(0xffffffffu, pf, o);
+    float xe = __shfl_down_sync(0xffffffffu, pe, o);
+    if (lane + o < 32) { pf *= xf; pe *= xe; }
+  }
+  // exclusive suffix (products strictly after this lane's pair)
+  float nf = __shfl_down_sync(0xffffffffu, pf, 1);
+  float ne = __shfl_down_sync(0xffffffffu, pe, 1);
+  if (lane == 31) { nf = 1.f; ne = 1.f; }
+  const float pa1 = nf, pa0 = f1 * nf;   // pa for tokens i1 and i0
+  const float pe1 = ne, pe0 = e1 * ne;
+  // affine maps g_i(x) = pa_i + b_i x with b_i = eta_{i+1}; the last token's
+  // map is the constant 1. Compose the pair (g_i0 o g_i1), then suffix-scan.
+  const float eta_next = __shfl_down_sync(0xffffffffu, e0, 1);  // eta of token i1 + 1
+  const float b1 = (lane == 31) ? 0.f : eta_next;
+  const float a1 = (lane == 31) ? 1.f : pa1;
+  const float a0 = pa0, b0 = e1;                // b_{i0} = eta_{i0 + 1} = eta_{i1}
+  // pair = g_i0 o g_i1: (a0 + b0 a1, b0 b1)
+  float A = a0 + b0 * a1, Bm = b0 * b1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    float xa = __shfl_down_sync(0xffffffffu, A, o);
+    float xb = __shfl_down_sync(0xffffffffu, Bm, o);
+    if (lane + o < 32) { A = A + Bm * xa; Bm = Bm * xb; }
+  }
+  // A now equals r_{i0} (the composition ends in a constant map)
+  float An = __shfl_down_sync(0xffffffffu, A, 1);
+  const float r0 = A;
+  const float r1 = (lane == 31) ? 1.f : (a1 + b1 * An);
+  cf.c[i0] = t0 * r0;
+  cf.c[i1] = t1 * r1;
+  cf.e[i0] = t0 * pe0;
+  cf.e[i1] = t1 * pe1;
+  if (lane == 0) {
+    cf.Bw = pa0 * f0;
+    cf.As = pe0 * e0;
+    cf.cS = e0 * r0;
+  }
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    tc_chunk_kernel(const TcArgs a, const __grid_constant__ CUtensorMap map_k,
+                    const __grid_constant__ CUtensorMap map_q) {
+  using Lay = Layout<D>;
+  // Reduce-scatter of Z2 by rows: CTA p owns rows [RP p, RP (p + 1)) of the
+  // 128 (keys 0-63, queries 64-127); owners of key rows produce G2 rows.
+  constexpr int RP = 128 / G;                      // rows owned per CTA
+  constexpr int RPK = RP < 64 ? RP : 64;           // key rows owned by a key owner
+  constexpr int NQO = G >= 2 ? G / 2 : 0;          // owners of query rows only
+  constexpr int NPT = RP * D / 8 / EPI_THREADS;    // 16-byte chunks reduced per thread
+  static_assert(NPT >= 1 && RP * D / 8 % EPI_THREADS == 0, "reduce split");
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char *sm =
+      reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(sm);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Lay::BARS);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + Lay::MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + Lay::MISC + 4);
+  Coefs *coefs = reinterpret_cast<Coefs *>(sm + Lay::COEF);
+
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const uint32_t j = cluster_rank();
+  const int stream = blockIdx.x / G;
+  const int T = a.T, nchunks = T / C, P = a.P;
+  const int Hd = HS * G;             // hidden width
+  float *Wg = a.W + (long long)stream * P;
+  float *Sg = a.S + (long long)stream * P;
+  const float *W0g = a.W0 + (long long)stream * P;
+  const float *S0g = a.S0 + (long long)stream * P;
+  const long long tok0 = (long long)stream * T;
+
+  if (tid == 0) {
+    mbar_init(&bars[B_TMA], 1);
+    mbar_init(&bars[B_COEF], 32);
+    mbar_init(&bars[B_F1], 1);
+    mbar_init(&bars[B_X1], EPI_WARPS);
+    mbar_init(&bars[B_F2], 1);
+    mbar_init(&bars[B_SEND], EPI_WARPS);
+    mbar_init(&bars[B_RECV], 1);
+    mbar_init(&bars[B_G2OWN], EPI_WARPS);
+    mbar_init(&bars[B_G2], 1 + NQO);
+    mbar_init(&bars[B_B1], 1);
+    mbar_init(&bars[B_G1], EPI_WARPS);
+    mbar_init(&bars[B_U2], 1);
+    mbar_init(&bars[B_U1], 1);
+    mbar_init(&bars[B_UPD], EPI_WARPS);
+    mbar_init(&bars[B_FIN], 1);
+    mbar_init(&bars[B_NEVER], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  // Zero the operand rows that padded M = 128 contractions read but never use,
+  // so that they hold finite values: the second feature block of XKQ and G2
+  // for d = 64.
+  if (D < 128) {
+    for (uint32_t off = tid * 16; off < 128 * 128 * 2; off += NTHREADS * 16)
+      st_shared_v4(sbase + Lay::XKQ + off, make_uint4(0, 0, 0, 0));
+    for (uint32_t off = tid * 16; off < 64 * 128 * 2; off += NTHREADS * 16)
+      st_shared_v4(sbase + Lay::G2 + off, make_uint4(0, 0, 0, 0));
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cluster_arrive_release();   // every CTA's barriers are initialised
+  cluster_wait_acquire();
+  const uint32_t tm = *tmem_slot;
+  const uint32_t t_z1 = tm + 0, t_z2 = tm + 64, t_g1 = tm + 192, t_s2 = tm + 256, t_s1 = tm + 384;
+
+  if (warp < EPI_WARPS) {
+    // ---------------------------------------------------------------- epilogue warps
+    const int q = warp & 3, h = warp >> 2;
+    const int row = 32 * q + lane;                     // TMEM lane of this thread
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    // TMEM-resident state: lane d, columns [W | S] of the slice; this thread
+    // holds hidden units 32 h .. 32 h + 31 of row d.
+    //   t_s2: W2[d][64 j + n] (n < 64), S2 at n + 64
+    //   t_s1: W1[64 j + n][d] (n < 64), S1 at n + 64
+    if (row < D) {
+      float w[32], sv[32];
+      const long long g2 = (long long)Hd * D + (long long)row * Hd + HS * j + 32 * h;
+#pragma unroll
+      for (int i4 = 0; i4 < 8; ++i4) {
+        const float4 a4 = *reinterpret_cast<const float4 *>(W0g + g2 + 4 * i4);
+        const float4 b4 = *reinterpret_cast<const float4 *>(S0g + g2 + 4 * i4);
+        w[4 * i4] = a4.x; w[4 * i4 + 1] = a4.y; w[4 * i4 + 2] = a4.z; w[4 * i4 + 3] = a4.w;
+        sv[4 * i4] = b4.x; sv[4 * i4 + 1] = b4.y; sv[4 * i4 + 2] = b4.z; sv[4 * i4 + 3] = b4.w;
+      }
+      tmem_st16(t_s2 + lane_base + 32 * h, *reinterpret_cast<float(*)[16]>(&w[0]));
+      tmem_st16(t_s2 + lane_base + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&w[16]));
+      tmem_st16(t_s2 + lane_base + 64 + 32 * h, *reinterpret_cast<float(*)[16]>(&sv[0]));
+      tmem_st16(t_s2 + lane_base + 64 + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&sv[16]));
+#pragma unroll
+      for (int k8 = 0; k8 < 4; ++k8)
+        st_shared_v4(sbase + Lay::W2 + rb_chunk(D, row, 4 * h + k8), pack8(&w[8 * k8]));
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const long long g1 = (long long)(HS * j + 32 * h + i) * D + row;
+        w[i] = W0g[g1];
+        sv[i] = S0g[g1];
+      }
+      tmem_st16(t_s1 + lane_base + 32 * h, *reinterpret_cast<float(*)[16]>(&w[0]));
+      tmem_st16(t_s1 + lane_base + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&w[16]));
+      tmem_st16(t_s1 + lane_base + 64 + 32 * h, *reinterpret_cast<float(*)[16]>(&sv[0]));
+      tmem_st16(t_s1 + lane_base + 64 + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&sv[16]));
+#pragma unroll
+      for (int k8 = 0; k8 < 4; ++k8)
+        st_shared_v4(sbase + Lay::W1 + rb_chunk(D, row, 4 * h + k8), pack8(&w[8 * k8]));
+      tmem_wait_st();
+    }
+    warp_arrive_local(&bars[B_UPD], lane);
+
+    for (int cch = 0; cch < nchunks; ++cch) {
+      const uint32_t par = cch & 1;
+      const long long tb = tok0 + (long long)cch * C;
+      // Load the values V this thread needs in the reduce step now, so the
+      // loads have the whole forward pass to land.
+      uint4 vv[NPT];
+#pragma unroll
+      for (int i = 0; i < NPT; ++i) {
+        const int k = tid + i * EPI_THREADS, gr = (int)j * RP + k / (D / 8), c = k % (D / 8);
+        if (gr < C) vv[i] = *reinterpret_cast<const uint4 *>(a.v + (tb + gr) * D + 8 * c);
+      }
+      if (!wait_bar(&bars[B_COEF], par, a, abort_flag)) break;
+      const Coefs &cf = coefs[par];
+      // -------- A7, first half: W <- B W + c_S S, S <- A S in TMEM. Runs while
+      // F1 executes; the accumulating contractions later add the writes.
+      if (row < D) {
+#pragma unroll
+        for (int layer = 0; layer < 2; ++layer) {
+          const uint32_t ts = (layer ? t_s1 : t_s2) + lane_base + 32 * h;
+          float w[32], sv[32];
+          tmem_ld16(ts, *reinterpret_cast<float(*)[16]>(&w[0]));
+          tmem_ld16(ts + 16, *reinterpret_cast<float(*)[16]>(&w[16]));
+          tmem_ld16(ts + 64, *reinterpret_cast<float(*)[16]>(&sv[0]));
+          tmem_ld16(ts + 80, *reinterpret_cast<float(*)[16]>(&sv[16]));
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            w[i] = cf.Bw * w[i] + cf.cS * sv[i];
+            sv[i] = cf.As * sv[i];
+          }
+          tmem_st16(ts, *reinterpret_cast<float(*)[16]>(&w[0]));
+          tmem_st16(ts + 16, *reinterpret_cast<float(*)[16]>(&w[16]));
+          tmem_st16(ts + 64, *reinterpret_cast<float(*)[16]>(&sv[0]));
+          tmem_st16(ts + 80, *reinterpret_cast<float(*)[16]>(&sv[16]));
+        }
+        tmem_wait_st();
+      }
+      // -------- E1: X1 = silu(Z1); key rows also give -c X1 and -e X1
+      if (!wait_bar(&bars[B_F1], par, a, abort_flag)) break;
+      tc_fence_after();
+      {
+        float z[32];
+        tmem_ld16(t_z1 + lane_base + 32 * h, *reinterpret_cast<float(*)[16]>(&z[0]));
+        tmem_ld16(t_z1 + lane_base + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&z[16]));
+        tmem_wait_ld();
+        float x[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] = z[i] * sigm(z[i]);
+#pragma unroll
+        for (int k8 = 0; k8 < 4; ++k8)
+          st_shared_v4(sbase + Lay::X1 + rb_chunk(128, row, 4 * h + k8), pack8(&x[8 * k8]));
+        if (row < C) {
+          const float ci = -cf.c[row], ei = -cf.e[row];
+          float s8[8];
+#pragma unroll
+          for (int k8 = 0; k8 < 4; ++k8) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) s8[i] = ci * x[8 * k8 + i];
+            st_shared_v4(sbase + Lay::X1S + rb_chunk(64, row, 4 * h + k8), pack8(s8));
+#pragma unroll
+            for (int i = 0; i < 8; ++i) s8[i] = ei * x[8 * k8 + i];
+            st_shared_v4(sbase + Lay::X1S + rb_chunk(64, row, 8 + 4 * h + k8), pack8(s8));
+          }
+        }
+      }
+      warp_arrive_local(&bars[B_X1], lane);
+      // -------- E2: stage this CTA's partial Z2 as bf16 rows (16-byte chunk
+      // index XOR row % 8), grouped by owner; the control warp bulk-copies
+      // owner p's rows into CTA p's receive buffer.
+      if (!wait_bar(&bars[B_F2], par, a, abort_flag)) break;
+      tc_fence_after();
+      {
+        constexpr int HALF = D / 2;                    // columns of Z2 per thread
+        float z[HALF];
+#pragma unroll
+        for (int c16 = 0; c16 < HALF / 16; ++c16)
+          tmem_ld16(t_z2 + lane_base + HALF * h + 16 * c16, *reinterpret_cast<float(*)[16]>(&z[16 * c16]));
+        tmem_wait_ld();
+        const uint32_t srow = sbase + Lay::SEND + (uint32_t)(row * D * 2);
+#pragma unroll
+        for (int k8 = 0; k8 < HALF / 8; ++k8) {
+          const int c = HALF / 8 * h + k8;
+          st_shared_v4(srow + (uint32_t)((c ^ (row & 7)) << 4), pack8(&z[8 * k8]));
+        }
+      }
+      warp_arrive_local(&bars[B_SEND], lane);
+      // -------- reduce my rows over the G partials (fp32 sums, fixed order):
+      // y for query rows, G2 = 2 (Z2 - V) for key rows (A3)
+      if (!wait_bar(&bars[B_RECV], par, a, abort_flag)) break;
+      {
+        float acc[NPT][8];
+#pragma unroll
+        for (int i = 0; i < NPT; ++i) {
+          const int k = tid + i * EPI_THREADS, r = k / (D / 8), c = k % (D / 8);
+          uint4 pv[G];
+#pragma unroll
+          for (int s2 = 0; s2 < G; ++s2)
+            pv[s2] = *reinterpret_cast<const uint4 *>(sm + Lay::RECV + (s2 * RP + r) * D * 2 + ((c ^ (r & 7)) << 4));
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
+#pragma unroll
+          for (int s2 = 0; s2 < G; ++s2) {
+            const __nv_bfloat16 *pb = reinterpret_cast<const __nv_bfloat16 *>(&pv[s2]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[i][e] += __bfloat162float(pb[e]);
+          }
+          const int gr = (int)j * RP + r;
+          if (gr < C) {
+            const __nv_bfloat16 *vb = reinterpret_cast<const __nv_bfloat16 *>(&vv[i]);
+            float g[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) g[e] = 2.f * (acc[i][e] - __bfloat162float(vb[e]));
+            st_shared_v4(sbase + Lay::G2OWN + rb_chunk(RPK, r, c), pack8(g));
+          }
+        }
+        warp_arrive_local(&bars[B_G2OWN], lane);
+        // reads y of my query rows
+#pragma unroll
+        for (int i = 0; i < NPT; ++i) {
+          const int k = tid + i * EPI_THREADS, r = k / (D / 8), c = k % (D / 8);
+          const int gr = (int)j * RP + r;
+          if (gr >= C) {
+            float *yp = a.y + (tb + (gr - C)) * D + 8 * c;
+            *reinterpret_cast<float4 *>(yp) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+            *reinterpret_cast<float4 *>(yp + 4) = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+          }
+        }
+      }
+      // -------- E3: G1 = (G2 W2_j) . silu'(Z1) on key rows -> [-c G1 | -e G1]
+      if (!wait_bar(&bars[B_B1], par, a, abort_flag)) break;
+      tc_fence_after();
+      if (row < C) {
+        float gp[32], z[32];
+        tmem_ld16(t_g1 + lane_base + 32 * h, *reinterpret_cast<float(*)[16]>(&gp[0]));
+        tmem_ld16(t_g1 + lane_base + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&gp[16]));
+        tmem_ld16(t_z1 + lane_base + 32 * h, *reinterpret_cast<float(*)[16]>(&z[0]));
+        tmem_ld16(t_z1 + lane_base + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&z[16]));
+        tmem_wait_ld();
+        const float ci = -cf.c[row], ei = -cf.e[row];
+        float g1[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float s = sigm(z[i]);
+          g1[i] = gp[i] * (s * (1.f + z[i] * (1.f - s)));
+        }
+        float s8[8];
+#pragma unroll
+        for (int k8 = 0; k8 < 4; ++k8) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) s8[i] = ci * g1[8 * k8 + i];
+          st_shared_v4(sbase + Lay::G1S + rb_chunk(64, row, 4 * h + k8), pack8(s8));
+#pragma unroll
+          for (int i = 0; i < 8; ++i) s8[i] = ei * g1[8 * k8 + i];
+          st_shared_v4(sbase + Lay::G1S + rb_chunk(64, row, 8 + 4 * h + k8), pack8(s8));
+        }
+      }
+      warp_arrive_local(&bars[B_G1], lane);
+      // -------- A7, second half: the bf16 copies of W2' and W1' for the next chunk
+      if (!wait_bar(&bars[B_U2], par, a, abort_flag)) break;
+      tc_fence_after();
+      if (row < D) {
+        float w[32];
+        tmem_ld16(t_s2 + lane_base + 32 * h, *reinterpret_cast<float(*)[16]>(&w[0]));
+        tmem_ld16(t_s2 + lane_base + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&w[16]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int k8 = 0; k8 < 4; ++k8)
+          st_shared_v4(sbase + Lay::W2 + rb_chunk(D, row, 4 * h + k8), pack8(&w[8 * k8]));
+      }
+      if (!wait_bar(&bars[B_U1], par, a, abort_flag)) break;
+      tc_fence_after();
+      if (row < D) {
+        float w[32];
+        tmem_ld16(t_s1 + lane_base + 32 * h, *reinterpret_cast<float(*)[16]>(&w[0]));
+        tmem_ld16(t_s1 + lane_base + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&w[16]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int k8 = 0; k8 < 4; ++k8)
+          st_shared_v4(sbase + Lay::W1 + rb_chunk(D, row, 4 * h + k8), pack8(&w[8 * k8]));
+      }
+      warp_arrive_local(&bars[B_UPD], lane);
+    }
+    // -------- W_end, S_end: write the TMEM-resident state back once
+    if (!*abort_flag && row < D) {
+      tc_fence_after();
+      float w[32], sv[32];
+      {
+        const uint32_t ts = t_s2 + lane_base + 32 * h;
+        tmem_ld16(ts, *reinterpret_cast<float(*)[16]>(&w[0]));
+        tmem_ld16(ts + 16, *reinterpret_cast<float(*)[16]>(&w[16]));
+        tmem_ld16(ts + 64, *reinterpret_cast<float(*)[16]>(&sv[0]));
+        tmem_ld16(ts + 80, *reinterpret_cast<float(*)[16]>(&sv[16]));
+        tmem_wait_ld();
+        const long long g2 = (long long)Hd * D + (long long)row * Hd + HS * j + 32 * h;
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+          *reinterpret_cast<float4 *>(Wg + g2 + 4 * i4) = make_float4(w[4 * i4], w[4 * i4 + 1], w[4 * i4 + 2], w[4 * i4 + 3]);
+          *reinterpret_cast<float4 *>(Sg + g2 + 4 * i4) = make_float4(sv[4 * i4], sv[4 * i4 + 1], sv[4 * i4 + 2], sv[4 * i4 + 3]);
+        }
+      }
+      {
+        const uint32_t ts = t_s1 + lane_base + 32 * h;
+        tmem_ld16(ts, *reinterpret_cast<float(*)[16]>(&w[0]));
+        tmem_ld16(ts + 16, *reinterpret_cast<float(*)[16]>(&w[16]));
+        tmem_ld16(ts + 64, *reinterpret_cast<float(*)[16]>(&sv[0]));
+        tmem_ld16(ts + 80, *reinterpret_cast<float(*)[16]>(&sv[16]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const long long g1 = (long long)(HS * j + 32 * h + i) * D + row;
+          Wg[g1] = w[i];
+          Sg[g1] = sv[i];
+        }
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- control warp
+    const uint32_t i_f1 = idesc_bf16(128, 64, false, true);
+    const uint32_t i_f2 = idesc_bf16(128, D, false, false);
+    const uint32_t i_b1 = idesc_bf16(128, 64, false, true);
+    const uint32_t i_dw = idesc_bf16(128, 128, true, true);
+    const uint32_t xkq = sbase + Lay::XKQ, x1 = sbase + Lay::X1, x1s = sbase + Lay::X1S;
+    const uint32_t g2 = sbase + Lay::G2, g1s = sbase + Lay::G1S;
+    const uint32_t w1 = sbase + Lay::W1, w2 = sbase + Lay::W2;
+    constexpr uint32_t TILE_BYTES = 2u * C * D * 2u;
+    auto issue_tma = [&](int cch) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bars[B_TMA], TILE_BYTES);
+        const int y0 = (int)(tok0 + (long long)cch * C);
+#pragma unroll
+        for (int fb = 0; fb < D / 64; ++fb) {
+          tma_load_2d(sm + Lay::XKQ + fb * 128 * 128, &map_k, &bars[B_TMA], 64 * fb, y0);
+          tma_load_2d(sm + Lay::XKQ + fb * 128 * 128 + 64 * 128, &map_q, &bars[B_TMA], 64 * fb, y0);
+        }
+      }
+      __syncwarp();
+    };
+    auto scan = [&](int cch) {
+      const long long tb = tok0 + (long long)cch * C;
+      coef_scan_warp(coefs[cch & 1], a.theta + tb, a.eta + tb, a.alpha + tb, lane);
+      __syncwarp();
+      mbar_arrive(&bars[B_COEF]);
+    };
+    if (lane == 0) { prefetch_tmap(&map_k); prefetch_tmap(&map_q); }
+    int tma_inflight = 0;
+    issue_tma(0);
+    tma_inflight = 1;
+    scan(0);
+    int cch = 0;
+    for (; cch < nchunks; ++cch) {
+      const uint32_t par = cch & 1;
+      if (a.inject_timeout) {
+        // Test hook: wait on a barrier nothing ever completes.
+        if (!wait_bar(&bars[B_NEVER], 0, a, abort_flag)) break;
+      }
+      if (!wait_bar(&bars[B_TMA], par, a, abort_flag)) break;
+      tma_inflight = 0;
+      if (!wait_bar(&bars[B_UPD], par, a, abort_flag)) break;
+      tc_fence_after();
+      // this chunk's incoming bytes: G partial blocks, and all 64 rows of G2
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bars[B_RECV], (uint32_t)(G * RP * D * 2));
+        mbar_arrive_expect_tx(&bars[B_G2], (uint32_t)(C * D * 2));
+      }
+      __syncwarp();
+      // A2 first half: Z1 = [K;Q] W1_j^T
+      if (lane == 0) {
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+          umma_bf16(t_z1, desc_kmajor(xkq, 128, ks), desc_mnmajor(w1, D, ks), i_f1, ks > 0);
+        umma_commit(&bars[B_F1]);
+      }
+      __syncwarp();
+      if (!wait_bar(&bars[B_X1], par, a, abort_flag)) break;
+      tc_fence_after();
+      if (lane == 0) {
+#pragma unroll
+        for (int ks = 0; ks < HS / 16; ++ks)
+          umma_bf16(t_z2, desc_kmajor(x1, 128, ks), desc_kmajor(w2, D, ks), i_f2, ks > 0);
+        umma_commit(&bars[B_F2]);
+      }
+      __syncwarp();
+      // Coefficients of the next chunk while F2 and the all-reduce run. Only
+      // after B_X1: the epilogue has then consumed this chunk's B_COEF phase,
+      // so B_COEF can never run two phases ahead of its waiters.
+      if (cch + 1 < nchunks) scan(cch + 1);
+      // reduce-scatter: owner p gets rows [RP p, RP p + RP) of every partial
+      if (!wait_bar(&bars[B_SEND], par, a, abort_flag)) break;
+      if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < G; ++i) {
+          const uint32_t p = (j + (uint32_t)i) % G;    // staggered: no hot destination
+          bulk_push(mapa(sbase + Lay::RECV + j * (uint32_t)(RP * D * 2), p),
+                    sbase + Lay::SEND + p * (uint32_t)(RP * D * 2), (uint32_t)(RP * D * 2),
+                    mapa(smem_u32(&bars[B_RECV]), p));
+        }
+      }
+      __syncwarp();
+      // all-gather of G2: key owners push their rows (whole 1 KB swizzle
+      // atoms) to every CTA; query owners only report that they are done
+      // reading their receive buffer.
+      if (!wait_bar(&bars[B_G2OWN], par, a, abort_flag)) break;
+      if (lane == 0) {
+        if ((int)j * RP < C) {
+#pragma unroll
+          for (int i = 0; i < G; ++i) {
+            const uint32_t p = (j + (uint32_t)i) % G;
+#pragma unroll
+            for (int fb = 0; fb < D / 64; ++fb)
+              bulk_push(mapa(sbase + Lay::G2 + (uint32_t)(fb * 64 * 128) + j * (uint32_t)(RP * 128), p),
+                        sbase + Lay::G2OWN + (uint32_t)(fb * RPK * 128), (uint32_t)(RPK * 128),
+                        mapa(smem_u32(&bars[B_G2]), p));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < G; ++i)
+            arrive_remote_release(mapa(smem_u32(&bars[B_G2]), (j + (uint32_t)i) % G));
+        }
+      }
+      __syncwarp();
+      // G2 complete in this CTA's shared memory
+      if (!wait_bar(&bars[B_G2], par, a, abort_flag, true)) break;
+      tc_fence_after();
+      if (lane == 0) {
+        // A4: G1 pre-activation gradient = G2 W2_j
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+          umma_bf16(t_g1, desc_kmajor(g2, 64, ks), desc_mnmajor(w2, D, ks), i_b1, ks > 0);
+        umma_commit(&bars[B_B1]);
+        // A6+A7 for W2: [W2 | S2] += G2^T [-c X1_K | -e X1_K] onto the pre-scaled state
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks)
+          umma_bf16(t_s2, desc_mnmajor(g2, 64, ks), desc_mnmajor(x1s, 64, ks), i_dw, 1);
+        umma_commit(&bars[B_U2]);
+      }
+      __syncwarp();
+      if (!wait_bar(&bars[B_G1], par, a, abort_flag)) break;
+      tc_fence_after();
+      if (lane == 0) {
+        // A6+A7 for W1: [W1 | S1]^T += K^T [-c G1 | -e G1] onto the pre-scaled state
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks)
+          umma_bf16(t_s1, desc_mnmajor(xkq, 128, ks), desc_mnmajor(g1s, 64, ks), i_dw, 1);
+        umma_commit(&bars[B_U1]);
+      }
+      __syncwarp();
+      // the key/query tile is free once U1 is done: prefetch the next chunk
+      if (!wait_bar(&bars[B_U1], par, a, abort_flag)) break;
+      if (cch + 1 < nchunks) {
+        issue_tma(cch + 1);
+        tma_inflight = 1;
+      }
+    }
+    // Drain: no copy or MMA may be in flight when the CTA leaves. These waits
+    // ignore the abort flag but stay bounded in time.
+    if (tma_inflight && !mbar_wait(&bars[B_TMA], (uint32_t)(cch & 1), a.wait_ns))
+      atomicCAS(a.status, 0, kDevTimeout);
+    if (lane == 0) umma_commit(&bars[B_FIN]);
+    __syncwarp();
+    if (!mbar_wait(&bars[B_FIN], 0, a.wait_ns)) atomicCAS(a.status, 0, kDevTimeout);
+  }
+  tc_fence_before();
+  __syncthreads();
+  // no CTA leaves while a peer may still write into its shared memory
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tm, TMEM_COLS);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D map over [rows x d] bf16 tokens, box = 64 features x 64 tokens, 128B swizzle.
+bool make_token_map(CUtensorMap *map, const void *base, long long rows, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  std::memset(map, 0, sizeof *map);
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)C};
+  cuuint32_t es[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int cluster_size(const Problem &p) { return p.dims[1] / HS; }
+
+template <int D, int G>
+cudaError_t launch_dg(const Problem &p, cudaStream_t stream, const TcArgs &a, const CUtensorMap &mk,
+                      const CUtensorMap &mq) {
+  using Lay = Layout<D>;
+  const size_t smem = Lay::TOTAL + 1024;
+  auto kern = tc_chunk_kernel<D, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(p.streams * G));
+  cfg.blockDim = dim3(NTHREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = G;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, mk, mq);
+}
+
+}  // namespace
+
+bool tc_supported(const Problem &p) {
+  if (p.in_dtype != TM_BF16 || p.L != 2 || p.C != C) return false;
+  const int d = p.dims[0], h = p.dims[1];
+  if (d != 64 && d != 128) return false;
+  if (h % HS != 0) return false;
+  const int G = h / HS;
+  if (d == 64) return G == 1 || G == 2 || G == 4;
+  return G == 1 || G == 2 || G == 4 || G == 8;
+}
+
 size_t tc_scratch_bytes(const Problem &) { return 0; }
-cudaError_t tc_launch(const Problem &, cudaStream_t) { return cudaErrorNotSupported; }
+
+static unsigned long long g_wait_ns = 2000000000ull;  // 2 s per wait
+static int g_inject_timeout = 0;
+
+void tc_set_debug(int inject_timeout, unsigned long long wait_ns) {
+  g_inject_timeout = inject_timeout;
+  g_wait_ns = wait_ns ? wait_ns : 2000000000ull;
+}
+
+cudaError_t tc_launch(const Problem &p, cudaStream_t stream) {
+  if (!tc_supported(p)) return cudaErrorNotSupported;
+  CUtensorMap mk, mq;
+  const long long rows = (long long)p.streams * p.T;
+  if (!make_token_map(&mk, p.k, rows, p.dims[0]) || !make_token_map(&mq, p.q, rows, p.dims[0]))
+    return cudaErrorInvalidValue;
+  TcArgs a;
+  a.T = p.T;
+  a.P = (int)p.P;
+  a.G = cluster_size(p);
+  a.v = reinterpret_cast<const __nv_bfloat16 *>(p.v);
+  a.theta = p.theta;
+  a.eta = p.eta;
+  a.alpha = p.alpha;
+  a.W0 = p.W0;
+  a.S0 = p.S0;
+  a.y = p.y;
+  a.W = p.W_end;
+  a.S = p.S_end;
+  a.status = p.status;
+  a.wait_ns = g_wait_ns;
+  a.inject_timeout = g_inject_timeout;
+  const int d = p.dims[0];
+  switch (a.G) {
+    case 1: return d == 64 ? launch_dg<64, 1>(p, stream, a, mk, mq) : launch_dg<128, 1>(p, stream, a, mk, mq);
+    case 2: return d == 64 ? launch_dg<64, 2>(p, stream, a, mk, mq) : launch_dg<128, 2>(p, stream, a, mk, mq);
+    case 4: return d == 64 ? launch_dg<64, 4>(p, stream, a, mk, mq) : launch_dg<128, 4>(p, stream, a, mk, mq);
+    case 8: return launch_dg<128, 8>(p, stream, a, mk, mq);
+  }
+  return cudaErrorNotSupported;
+}
 
 }  // namespace tmem

@@ -80,9 +80,9 @@ def _dev_inputs(w, streams=None, T=None):
     return inp, to_dev(inp, B, H, w.dtype)
 
 
-@pytest.mark.parametrize("path", ["simt"])
+@pytest.mark.parametrize("path", ["simt", "tc"])
 def test_in_place_state_equals_out_of_place(path):
-    w = W.make(2, 32, 4, 1, 2, 128, 32, index=301)
+    w = W.make(2, 64, 4, 1, 2, 256, 64, index=301)
     _, dev = _dev_inputs(w)
     mem = NeuralMemory(w.L, w.d, w.expansion, path=path)
     y1, We1, Se1 = run_lib(mem, dev, w.C)
@@ -93,15 +93,15 @@ def test_in_place_state_equals_out_of_place(path):
     assert torch.equal(y1, y2) and torch.equal(We1, W0) and torch.equal(Se1, S0)
 
 
-@pytest.mark.parametrize("path", ["simt"])
+@pytest.mark.parametrize("path", ["simt", "tc"])
 def test_state_carry_and_determinism(path):
-    w = W.make(2, 32, 4, 2, 1, 192, 32, index=302)
+    w = W.make(2, 64, 2, 2, 1, 384, 64, index=302)
     _, dev = _dev_inputs(w)
     mem = NeuralMemory(w.L, w.d, w.expansion, path=path)
     y, We, Se = run_lib(mem, dev, w.C)
     y_b, We_b, Se_b = run_lib(mem, dev, w.C)
     assert torch.equal(y, y_b) and torch.equal(We, We_b) and torch.equal(Se, Se_b)
-    T1 = 64
+    T1 = 128
     first = {k: (v[:, :, :T1].contiguous() if k in ("k", "v", "q", "theta", "eta", "alpha") else v)
              for k, v in dev.items()}
     ya, Wa, Sa = run_lib(mem, first, w.C)
@@ -113,9 +113,9 @@ def test_state_carry_and_determinism(path):
     assert torch.equal(Wb, We) and torch.equal(Sb, Se)
 
 
-@pytest.mark.parametrize("path", ["simt"])
+@pytest.mark.parametrize("path", ["simt", "tc"])
 def test_streams_independent_and_permutable(path):
-    w = W.make(2, 16, 4, 1, 4, 64, 16, index=303)
+    w = W.make(2, 64, 1, 1, 4, 128, 64, index=303)
     inp, dev = _dev_inputs(w)
     mem = NeuralMemory(w.L, w.d, w.expansion, path=path)
     y, We, Se = run_lib(mem, dev, w.C)
@@ -192,3 +192,68 @@ def test_all_streams_short_stream_state(idx, sample_streams, T):
     gsub = {k: v[sample_streams] for k, v in gpu.items()}
     errs = parity_errors(w.dims, inp["W0"][sample_streams], gsub, ref)
     assert max(errs.values()) < tol, errs
+
+
+# ---------------------------------------------------------------- tensor cores
+TC_SHAPES = [  # d, expansion (hidden = 64 G), B, H, T
+    (64, 1, 1, 1, 64),
+    (64, 2, 1, 2, 192),
+    (64, 4, 2, 2, 256),
+    (128, 1, 1, 1, 128),
+    (128, 2, 1, 1, 256),
+    (128, 4, 1, 3, 320),
+    (128, 4, 1, 1, 64),
+]
+
+
+@pytest.mark.parametrize("cfg", TC_SHAPES, ids=lambda c: "d%d-e%d-B%dH%d-T%d" % c)
+def test_tc_small_shapes(cfg):
+    d, e, B, H, T = cfg
+    w = W.make(2, d, e, B, H, T, 64, index=400 + sum(cfg))
+    mem = NeuralMemory(2, d, e)
+    assert mem.query_path(B, H, T, 64) == "tc"
+    check(w, "tc", TOL_BF16_TC)
+
+
+def test_tc_cluster_of_eight_d128():
+    """Hidden 512 split over a cluster of 8 CTAs (the long-stream shape)."""
+    check(W.make(2, 128, 4, 1, 2, 256, 64, index=410), "tc", TOL_BF16_TC)
+
+
+def test_tc_literal_gates_short_stream():
+    """Gates exactly as specified over a finite horizon: large writes."""
+    check(W.make(2, 64, 4, 1, 2, 128, 64, index=411, theta_damping=1.0, alpha_damping=1.0),
+          "tc", TOL_BF16_TC)
+
+
+def test_tc_matches_simt_path():
+    w = W.make(2, 128, 4, 1, 2, 512, 64, index=412)
+    inp, dev = _dev_inputs(w)
+    out = {}
+    for path in ("simt", "tc"):
+        mem = NeuralMemory(2, 128, 4, path=path)
+        out[path] = gpu_to_np(*run_lib(mem, dev, w.C))
+    errs = parity_errors(w.dims, inp["W0"], out["tc"], out["simt"])
+    assert max(errs.values()) < TOL_BF16_TC, errs
+
+
+def test_tc_timeout_is_reported_and_context_survives():
+    """A wait that nothing completes expires after 1 ms; the kernel records
+    TM_ERR_TIMEOUT, cleans up and returns; the next call works."""
+    from test_trained_neural_b200 import _native as N
+    from test_trained_neural_b200._native import TitansMemError
+    lib = N.load()
+    w = W.make(2, 64, 2, 1, 2, 128, 64, index=413)
+    inp, dev = _dev_inputs(w)
+    mem = NeuralMemory(2, 64, 2, path="tc")
+    assert lib.tm_set_debug(1, 1_000_000) == N.TM_OK
+    try:
+        with pytest.raises(TitansMemError) as ei:
+            run_lib(mem, dev, w.C)
+        assert ei.value.code == N.TM_ERR_TIMEOUT
+    finally:
+        lib.tm_set_debug(0, 0)
+    y, We, Se = run_lib(mem, dev, w.C)
+    ref = oracle.run_workload(w, inp)
+    errs = parity_errors(w.dims, inp["W0"], gpu_to_np(y, We, Se), ref)
+    assert max(errs.values()) < TOL_BF16_TC, errs
