@@ -136,6 +136,33 @@ TM_API tm_status tm_run(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dty
                  void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * tm_run without a workspace, for callers that must not allocate device
+ * memory where they run the memory (a latency-bound serving loop, where
+ * cudaMalloc/cudaFree may synchronize the device; a framework whose memory
+ * manager owns all device memory). This entry point has no counterpart in the
+ * method's description: it only changes where the scratch lives.
+ *
+ * Same arguments and semantics as tm_run, minus the workspace. It always runs
+ * the CUDA-core (fp32) kernel, whose per-stream activations go to a fixed
+ * 16 MiB array inside the library's device memory (held by every GPU that
+ * loads the library until the process exits). Problems that need more than
+ * 16 MiB of activations are refused with TM_ERR_OOM before any CUDA call.
+ * Allocates nothing and calls no allocating routine.
+ *
+ * The first call on each device looks up the array's device address; make
+ * that first call before any stream capture. All calls on a device share the
+ * array (it keeps the last call's contents; every call clears its status
+ * word): calls whose kernels overlap on the GPU race and must be serialised
+ * by the caller. Device-side errors are not reported through tm_sync (there
+ * is no caller workspace); argument errors are returned as by tm_run.
+ */
+TM_API tm_status tm_run_noalloc(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype,
+                                const void *k, const void *v, const void *q,
+                                const float *theta, const float *eta, const float *alpha,
+                                const float *W0, const float *S0,
+                                float *y, float *W_end, float *S_end, void *stream);
+
+/*
  * Wait for `stream`, then read and clear the device status word in
  * `workspace`. Returns TM_OK, TM_ERR_TIMEOUT or TM_ERR_DEVICE from the
  * kernels, or TM_ERR_CUDA if the stream itself reports an error.

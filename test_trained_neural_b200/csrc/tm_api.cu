@@ -65,6 +65,16 @@ size_t scratch_bytes(tm_path path, const tmem::Problem &p) {
 
 }  // namespace
 
+namespace tmem {
+// Validated problem description of a context, for entry points that live in
+// other translation units.
+bool problem_from_ctx(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype dt, Problem *out) {
+  if (!out || check_shape(ctx, B, H, T, C, dt) != TM_OK) return false;
+  *out = make_problem(ctx, B, H, T, C, dt);
+  return true;
+}
+}  // namespace tmem
+
 extern "C" {
 
 tm_status tm_create(int L, int d_h, int expansion, tm_act act, tm_ctx **out) {

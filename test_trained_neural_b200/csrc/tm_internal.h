@@ -37,6 +37,9 @@ struct Problem {
   size_t scratch_bytes;
 };
 
+// Shape checks of tm_run, shared with the other C entry points.
+bool problem_from_ctx(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype dt, Problem *out);
+
 // SIMT (CUDA-core, fp32) path.
 size_t simt_scratch_bytes(const Problem &p);
 cudaError_t simt_launch(const Problem &p, cudaStream_t stream);
