@@ -100,11 +100,18 @@ struct Layout {
 };
 
 enum Bar {
-  B_TMA = 0, B_COEF, B_F1, B_X1, B_F2, B_SEND, B_RECV, B_G2OWN, B_G2, B_B1, B_G1, B_U2, B_U1,
+  B_TMA = 0, B_COEF, B_F1, B_X1, B_F2, B_QFREE, B_RECV, B_G2OWN, B_G2, B_B1, B_G1, B_U2, B_U1,
   B_UPD, B_FIN, B_NEVER, B_COUNT
 };
 
-__device__ __forceinline__ float sigm(float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); }
+// sigmoid(z) = 1/2 + tanh(z/2)/2, with the hardware tanh approximation (one
+// MUFU operation; its error is far below the bf16 rounding of the results).
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float sigm(float z) { return fmaf(0.5f, tanh_approx(0.5f * z), 0.5f); }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -283,6 +290,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   constexpr int RPK = RP < 64 ? RP : 64;           // key rows owned by a key owner
   constexpr int NQO = G >= 2 ? G / 2 : 0;          // owners of query rows only
   constexpr int NPT = RP * D / 8 / EPI_THREADS;    // 16-byte chunks reduced per thread
+  constexpr int SWZ = (D / 16 < 8 ? D / 16 : 8) - 1; // chunk swizzle mask of a half row
   static_assert(NPT >= 1 && RP * D / 8 % EPI_THREADS == 0, "reduce split");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *sm =
@@ -310,10 +318,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&bars[B_F1], 1);
     mbar_init(&bars[B_X1], EPI_WARPS);
     mbar_init(&bars[B_F2], 1);
-    mbar_init(&bars[B_SEND], EPI_WARPS);
     mbar_init(&bars[B_RECV], 1);
     mbar_init(&bars[B_G2OWN], EPI_WARPS);
-    mbar_init(&bars[B_G2], 1 + NQO);
+    mbar_init(&bars[B_G2], 1);
+    mbar_init(&bars[B_QFREE], NQO > 0 ? NQO : 1);
     mbar_init(&bars[B_B1], 1);
     mbar_init(&bars[B_G1], EPI_WARPS);
     mbar_init(&bars[B_U2], 1);
@@ -439,6 +447,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int k8 = 0; k8 < 4; ++k8)
           st_shared_v4(sbase + Lay::X1 + rb_chunk(128, row, 4 * h + k8), pack8(&x[8 * k8]));
+        // X1 feeds the next MMA: publish it first
+        warp_arrive_local(&bars[B_X1], lane);
+        // the scaled copies are only needed by the W2 update, much later (they
+        // reach the tensor cores through the fence of the B_G2OWN arrival)
         if (row < C) {
           const float ci = -cf.c[row], ei = -cf.e[row];
           float s8[8];
@@ -453,12 +465,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
       }
-      warp_arrive_local(&bars[B_X1], lane);
-      // -------- E2: stage this CTA's partial Z2 as bf16 rows (16-byte chunk
-      // index XOR row % 8), grouped by owner; the control warp bulk-copies
-      // owner p's rows into CTA p's receive buffer.
+      // -------- E2: stage this CTA's partial Z2 as bf16, [half][row][d/2]
+      // (16-byte chunk index XOR row), and let each warp bulk-copy the rows it
+      // staged into their owners' receive buffers (reduce-scatter by rows:
+      // CTA p owns rows [RP p, RP p + RP)).
       if (!wait_bar(&bars[B_F2], par, a, abort_flag)) break;
       tc_fence_after();
+      // Query rows (warps of lane quarters 2, 3) reuse send and receive space
+      // that the query owners read in the previous chunk: wait for their
+      // release (normally long given). Key rows need no such wait: the key
+      // owners' G2 of the previous chunk already proved it.
+      if (NQO > 0 && q >= 2 && cch > 0 &&
+          !wait_bar(&bars[B_QFREE], (uint32_t)((cch - 1) & 1), a, abort_flag, true))
+        break;
       {
         constexpr int HALF = D / 2;                    // columns of Z2 per thread
         float z[HALF];
@@ -466,14 +485,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int c16 = 0; c16 < HALF / 16; ++c16)
           tmem_ld16(t_z2 + lane_base + HALF * h + 16 * c16, *reinterpret_cast<float(*)[16]>(&z[16 * c16]));
         tmem_wait_ld();
-        const uint32_t srow = sbase + Lay::SEND + (uint32_t)(row * D * 2);
+        const uint32_t srow = sbase + Lay::SEND + (uint32_t)(h * 128 * D + row * D);
 #pragma unroll
-        for (int k8 = 0; k8 < HALF / 8; ++k8) {
-          const int c = HALF / 8 * h + k8;
-          st_shared_v4(srow + (uint32_t)((c ^ (row & 7)) << 4), pack8(&z[8 * k8]));
+        for (int k8 = 0; k8 < HALF / 8; ++k8)
+          st_shared_v4(srow + (uint32_t)((k8 ^ (row & SWZ)) << 4), pack8(&z[8 * k8]));
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          constexpr int RPP = RP < 32 ? RP : 32;       // rows per push
+#pragma unroll
+          for (int i = 0; i < 32 / RPP; ++i) {
+            const int r0 = 32 * q + i * RPP, p = r0 / RP, rin = r0 - p * RP;
+            bulk_push(mapa(sbase + Lay::RECV + (uint32_t)(j * 2 * RP * D + h * RP * D + rin * D), (uint32_t)p),
+                      sbase + Lay::SEND + (uint32_t)(h * 128 * D + r0 * D), (uint32_t)(RPP * D),
+                      mapa(smem_u32(&bars[B_RECV]), (uint32_t)p));
+          }
         }
+        __syncwarp();
       }
-      warp_arrive_local(&bars[B_SEND], lane);
       // -------- reduce my rows over the G partials (fp32 sums, fixed order):
       // y for query rows, G2 = 2 (Z2 - V) for key rows (A3)
       if (!wait_bar(&bars[B_RECV], par, a, abort_flag)) break;
@@ -485,7 +515,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           uint4 pv[G];
 #pragma unroll
           for (int s2 = 0; s2 < G; ++s2)
-            pv[s2] = *reinterpret_cast<const uint4 *>(sm + Lay::RECV + (s2 * RP + r) * D * 2 + ((c ^ (r & 7)) << 4));
+            pv[s2] = *reinterpret_cast<const uint4 *>(sm + Lay::RECV + s2 * 2 * RP * D + (c / (D / 16)) * RP * D +
+                                                       r * D + (((c % (D / 16)) ^ (r & SWZ)) << 4));
 #pragma unroll
           for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
 #pragma unroll
@@ -674,21 +705,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // after B_X1: the epilogue has then consumed this chunk's B_COEF phase,
       // so B_COEF can never run two phases ahead of its waiters.
       if (cch + 1 < nchunks) scan(cch + 1);
-      // reduce-scatter: owner p gets rows [RP p, RP p + RP) of every partial
-      if (!wait_bar(&bars[B_SEND], par, a, abort_flag)) break;
-      if (lane == 0) {
-#pragma unroll
-        for (int i = 0; i < G; ++i) {
-          const uint32_t p = (j + (uint32_t)i) % G;    // staggered: no hot destination
-          bulk_push(mapa(sbase + Lay::RECV + j * (uint32_t)(RP * D * 2), p),
-                    sbase + Lay::SEND + p * (uint32_t)(RP * D * 2), (uint32_t)(RP * D * 2),
-                    mapa(smem_u32(&bars[B_RECV]), p));
-        }
-      }
-      __syncwarp();
       // all-gather of G2: key owners push their rows (whole 1 KB swizzle
-      // atoms) to every CTA; query owners only report that they are done
-      // reading their receive buffer.
+      // atoms) to every CTA; query owners report that they are done reading
+      // their receive buffer (B_QFREE, off the critical path).
       if (!wait_bar(&bars[B_G2OWN], par, a, abort_flag)) break;
       if (lane == 0) {
         if ((int)j * RP < C) {
@@ -702,9 +721,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         mapa(smem_u32(&bars[B_G2]), p));
           }
         } else {
+          // done reading this chunk's receive buffer: query rows of the next
+          // chunk may be pushed here
 #pragma unroll
           for (int i = 0; i < G; ++i)
-            arrive_remote_release(mapa(smem_u32(&bars[B_G2]), (j + (uint32_t)i) % G));
+            arrive_remote_release(mapa(smem_u32(&bars[B_QFREE]), (j + (uint32_t)i) % G));
         }
       }
       __syncwarp();
