@@ -285,6 +285,10 @@ def main():
     ms_max = max_over_ranks(ms, world)
 
     cnt = algorithmic_counts(w, w.T)
+    # kernels of this library per tm_run: one persistent kernel (cluster or
+    # CUDA-core path), or for the layered path an init and a coefficient kernel
+    # plus 3L - 1 GEMMs per chunk
+    launches_per_step = 2 + (3 * w.L - 1) * (w.T // w.C) if path_used == "tcl" else 1
     value = aggregate_throughput(cnt["tokens"], world, ms_max * 1e-3)
     peaks = measured_peaks()
     hbm = peaks["hbm_gbs"] * 1e9
@@ -293,7 +297,7 @@ def main():
     t_state = (cnt["state_bytes"] + cnt["token_io_bytes"]) / hbm
     chunk_roofline_s = max(t_flop, t_state)
     sec = ms * 1e-3
-    if path_used == "tc":
+    if path_used in ("tc", "tcl"):
         # The kernel runs alone at the maximum SM clock, far from the power
         # cap, so the burst figure is the denominator.
         roof = {"bound": "tensor", "achieved": cnt["flops"] / sec / 1e12,
@@ -307,7 +311,7 @@ def main():
                 "sm_mhz_seen": sm_mhz}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = None
-    roof["kernel"] = "tc_chunk_kernel" if path_used == "tc" else "simt_chunk_kernel"
+    roof["kernel"] = {"tc": "tc_chunk_kernel", "tcl": "tcl_gemm_kernel"}.get(path_used, "simt_chunk_kernel")
 
     e2e = None
     if not args.no_e2e:
@@ -347,7 +351,7 @@ def main():
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if w.dtype == "bf16" and path_used == "tc" else
+            "dtype": "bf16" if w.dtype == "bf16" and path_used in ("tc", "tcl") else
                      ("bf16-in/f32" if w.dtype == "bf16" else "f32"),
             "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "C": w.C, "dims": w.dims,
@@ -357,8 +361,8 @@ def main():
             "chunk_roofline": {"t_flop_ms": t_flop * 1e3, "t_state_io_ms": t_state * 1e3,
                                "bound": "state" if t_state > t_flop else "flop",
                                "frac": chunk_roofline_s / (ms_max * 1e-3),
-                               "state_resident": "hbm/l2" if path_used != "tc" else "on-chip"},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
+                               "state_resident": "on-chip" if path_used == "tc" else "hbm/l2"},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps * launches_per_step,
             "clocks": clk, "finite": ok, "wall_s": t_wall, "step_ms": step_ms,
         }
         print(json.dumps(line), flush=True)

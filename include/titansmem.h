@@ -69,9 +69,13 @@ typedef enum {
 } tm_dtype;
 
 typedef enum {
-  TM_PATH_AUTO = 0,  /* TM_BF16 -> tensor cores when the shape has a kernel, else SIMT */
-  TM_PATH_SIMT = 1,  /* fp32 CUDA-core kernel for any supported shape and dtype        */
-  TM_PATH_TC = 2     /* tcgen05 tensor-core kernel; TM_ERR_UNSUPPORTED if none fits    */
+  TM_PATH_AUTO = 0,        /* TM_BF16: cluster kernel, else layered kernels, else SIMT     */
+  TM_PATH_SIMT = 1,        /* fp32 CUDA-core kernel for any supported shape and dtype      */
+  TM_PATH_TC = 2,          /* tcgen05 cluster kernel, state resident on chip (L = 2,
+                              d in {64, 128}, hidden = 64 G, C = 64); else unsupported     */
+  TM_PATH_TC_LAYERED = 3   /* tcgen05 batched GEMMs, one launch per layer phase and chunk;
+                              state in W_end / S_end (widths multiples of 64, C in
+                              {64, 128}); else unsupported                                  */
 } tm_path;
 
 /*

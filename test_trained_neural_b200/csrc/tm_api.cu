@@ -53,14 +53,22 @@ tmem::Problem make_problem(const tm_ctx *ctx, int B, int H, int T, int C, tm_dty
 }
 
 tm_path choose_path(const tm_ctx *ctx, const tmem::Problem &p) {
-  if (ctx->path == TM_PATH_SIMT) return TM_PATH_SIMT;
-  if (ctx->path == TM_PATH_TC) return TM_PATH_TC;
+  if (ctx->path != TM_PATH_AUTO) return ctx->path;
   if (p.in_dtype == TM_BF16 && tmem::tc_supported(p)) return TM_PATH_TC;
+  if (p.in_dtype == TM_BF16 && tmem::tcl_supported(p)) return TM_PATH_TC_LAYERED;
   return TM_PATH_SIMT;
 }
 
+bool path_supported(tm_path path, const tmem::Problem &p) {
+  if (path == TM_PATH_TC) return tmem::tc_supported(p);
+  if (path == TM_PATH_TC_LAYERED) return tmem::tcl_supported(p);
+  return true;
+}
+
 size_t scratch_bytes(tm_path path, const tmem::Problem &p) {
-  return path == TM_PATH_TC ? tmem::tc_scratch_bytes(p) : tmem::simt_scratch_bytes(p);
+  if (path == TM_PATH_TC) return tmem::tc_scratch_bytes(p);
+  if (path == TM_PATH_TC_LAYERED) return tmem::tcl_scratch_bytes(p);
+  return tmem::simt_scratch_bytes(p);
 }
 
 }  // namespace
@@ -112,7 +120,8 @@ size_t tm_param_count(const tm_ctx *ctx) { return ctx ? ctx->P : 0; }
 
 tm_status tm_set_path(tm_ctx *ctx, tm_path path) {
   if (!ctx) return TM_ERR_INVALID_ARG;
-  if (path != TM_PATH_AUTO && path != TM_PATH_SIMT && path != TM_PATH_TC) return TM_ERR_INVALID_ARG;
+  if (path != TM_PATH_AUTO && path != TM_PATH_SIMT && path != TM_PATH_TC && path != TM_PATH_TC_LAYERED)
+    return TM_ERR_INVALID_ARG;
   ctx->path = path;
   return TM_OK;
 }
@@ -124,7 +133,7 @@ tm_status tm_query_path(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype 
   if (st != TM_OK) return st;
   tmem::Problem p = make_problem(ctx, B, H, T, C, in_dtype);
   tm_path path = choose_path(ctx, p);
-  if (path == TM_PATH_TC && !tmem::tc_supported(p)) return TM_ERR_UNSUPPORTED;
+  if (!path_supported(path, p)) return TM_ERR_UNSUPPORTED;
   *out = path;
   return TM_OK;
 }
@@ -136,7 +145,7 @@ tm_status tm_workspace_size(const tm_ctx *ctx, int B, int H, int T, int C, tm_dt
   if (st != TM_OK) return st;
   tmem::Problem p = make_problem(ctx, B, H, T, C, in_dtype);
   tm_path path = choose_path(ctx, p);
-  if (path == TM_PATH_TC && !tmem::tc_supported(p)) return TM_ERR_UNSUPPORTED;
+  if (!path_supported(path, p)) return TM_ERR_UNSUPPORTED;
   *bytes = tmem::kStatusBytes + scratch_bytes(path, p);
   return TM_OK;
 }
@@ -173,7 +182,7 @@ tm_status tm_run(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype, con
   if (ranges_overlap(S_end, st_bytes, W0, st_bytes)) return TM_ERR_INVALID_ARG;
 
   tm_path path = choose_path(ctx, p);
-  if (path == TM_PATH_TC && !tmem::tc_supported(p)) return TM_ERR_UNSUPPORTED;
+  if (!path_supported(path, p)) return TM_ERR_UNSUPPORTED;
   const size_t need = tmem::kStatusBytes + scratch_bytes(path, p);
   if (workspace_bytes < need) return TM_ERR_OOM;
   if (ranges_overlap(workspace, need, y, y_bytes)) return TM_ERR_INVALID_ARG;
@@ -195,7 +204,9 @@ tm_status tm_run(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype, con
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(p.status, 0, sizeof(int), s) != cudaSuccess) return TM_ERR_CUDA;
-  cudaError_t err = path == TM_PATH_TC ? tmem::tc_launch(p, s) : tmem::simt_launch(p, s);
+  cudaError_t err = path == TM_PATH_TC           ? tmem::tc_launch(p, s)
+                    : path == TM_PATH_TC_LAYERED ? tmem::tcl_launch(p, s)
+                                                 : tmem::simt_launch(p, s);
   return err == cudaSuccess ? TM_OK : TM_ERR_CUDA;
 }
 
@@ -216,6 +227,7 @@ tm_status tm_sync(tm_ctx *ctx, void *workspace, void *stream) {
 
 tm_status tm_set_debug(int inject_timeout, unsigned long long wait_limit_ns) {
   tmem::tc_set_debug(inject_timeout, wait_limit_ns);
+  tmem::tcl_set_wait(wait_limit_ns);
   return TM_OK;
 }
 

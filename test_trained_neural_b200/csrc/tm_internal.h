@@ -48,6 +48,12 @@ cudaError_t simt_launch(const Problem &p, cudaStream_t stream);
 bool tc_supported(const Problem &p);
 size_t tc_scratch_bytes(const Problem &p);
 cudaError_t tc_launch(const Problem &p, cudaStream_t stream);
+// Layer-by-layer tensor-core path (batched tcgen05 GEMMs per phase).
+bool tcl_supported(const Problem &p);
+size_t tcl_scratch_bytes(const Problem &p);
+cudaError_t tcl_launch(const Problem &p, cudaStream_t stream);
+void tcl_set_wait(unsigned long long wait_ns);
+
 // Test hooks of the tensor-core path: make the first wait of every CTA one
 // that nothing completes, and/or shorten the per-wait time limit (0 = 2 s).
 void tc_set_debug(int inject_timeout, unsigned long long wait_ns);

@@ -80,7 +80,7 @@ def _dev_inputs(w, streams=None, T=None):
     return inp, to_dev(inp, B, H, w.dtype)
 
 
-@pytest.mark.parametrize("path", ["simt", "tc"])
+@pytest.mark.parametrize("path", ["simt", "tc", "tcl"])
 def test_in_place_state_equals_out_of_place(path):
     w = W.make(2, 64, 4, 1, 2, 256, 64, index=301)
     _, dev = _dev_inputs(w)
@@ -93,7 +93,7 @@ def test_in_place_state_equals_out_of_place(path):
     assert torch.equal(y1, y2) and torch.equal(We1, W0) and torch.equal(Se1, S0)
 
 
-@pytest.mark.parametrize("path", ["simt", "tc"])
+@pytest.mark.parametrize("path", ["simt", "tc", "tcl"])
 def test_state_carry_and_determinism(path):
     w = W.make(2, 64, 2, 2, 1, 384, 64, index=302)
     _, dev = _dev_inputs(w)
@@ -113,7 +113,7 @@ def test_state_carry_and_determinism(path):
     assert torch.equal(Wb, We) and torch.equal(Sb, Se)
 
 
-@pytest.mark.parametrize("path", ["simt", "tc"])
+@pytest.mark.parametrize("path", ["simt", "tc", "tcl"])
 def test_streams_independent_and_permutable(path):
     w = W.make(2, 64, 1, 1, 4, 128, 64, index=303)
     inp, dev = _dev_inputs(w)
@@ -159,7 +159,7 @@ def test_full_size_workloads(idx, sample_streams, prefix):
     if sample_streams is not None:
         del inp
     mem = NeuralMemory(w.L, w.d, w.expansion, path="auto")
-    tol = TOL_BF16_TC if mem.query_path(w.B, w.H, w.T, w.C) == "tc" else TOL_F32
+    tol = TOL_BF16_TC if mem.query_path(w.B, w.H, w.T, w.C) in ("tc", "tcl") else TOL_F32
     y, We, Se = run_lib(mem, dev, w.C)
     assert torch.isfinite(y).all() and torch.isfinite(We).all() and torch.isfinite(Se).all()
     if sample_streams is None:
@@ -184,7 +184,7 @@ def test_all_streams_short_stream_state(idx, sample_streams, T):
     inp = W.generate(w, T=T)
     dev = to_dev(inp, w.B, w.H, w.dtype)
     mem = NeuralMemory(w.L, w.d, w.expansion, path="auto")
-    tol = TOL_BF16_TC if mem.query_path(w.B, w.H, T, w.C) == "tc" else TOL_F32
+    tol = TOL_BF16_TC if mem.query_path(w.B, w.H, T, w.C) in ("tc", "tcl") else TOL_F32
     y, We, Se = run_lib(mem, dev, w.C)
     gpu = gpu_to_np(y, We, Se)
     sub = {k: (v[sample_streams] if k != "streams" else v) for k, v in inp.items()}
@@ -257,3 +257,41 @@ def test_tc_timeout_is_reported_and_context_survives():
     ref = oracle.run_workload(w, inp)
     errs = parity_errors(w.dims, inp["W0"], gpu_to_np(y, We, Se), ref)
     assert max(errs.values()) < TOL_BF16_TC, errs
+
+
+# ------------------------------------------------- layered tensor-core kernels
+TCL_SHAPES = [  # L, d, expansion, B, H, T, C
+    (1, 64, 1, 1, 2, 128, 64),      # linear memory
+    (2, 64, 2, 1, 2, 256, 64),
+    (2, 128, 3, 1, 1, 128, 64),     # hidden 384: 128-wide output tiles
+    (2, 192, 2, 1, 1, 128, 64),     # d = 192: 64-wide tiles, partial M tiles
+    (3, 64, 2, 2, 1, 256, 128),     # C = 128: two row tiles of keys and queries
+    (4, 64, 2, 1, 2, 256, 128),
+    (4, 128, 2, 1, 1, 256, 128),    # the deep workload's layer shapes
+]
+
+
+@pytest.mark.parametrize("cfg", TCL_SHAPES, ids=lambda c: "L%d-d%d-e%d-B%dH%d-T%d-C%d" % c)
+def test_tcl_small_shapes(cfg):
+    L, d, e, B, H, T, C = cfg
+    w = W.make(L, d, e, B, H, T, C, index=600 + sum(cfg))
+    check(w, "tcl", TOL_BF16_TC)
+
+
+def test_tcl_literal_gates_short_stream():
+    check(W.make(2, 64, 2, 1, 2, 128, 64, index=620, theta_damping=1.0, alpha_damping=1.0),
+          "tcl", TOL_BF16_TC)
+
+
+def test_tcl_matches_cluster_kernel():
+    """The two tensor-core designs on a shape both support."""
+    w = W.make(2, 64, 4, 1, 2, 512, 64, index=621)
+    inp, dev = _dev_inputs(w)
+    out = {}
+    for path in ("tc", "tcl"):
+        mem = NeuralMemory(2, 64, 4, path=path)
+        out[path] = gpu_to_np(*run_lib(mem, dev, w.C))
+    errs = parity_errors(w.dims, inp["W0"], out["tcl"], out["tc"])
+    assert max(errs.values()) < TOL_BF16_TC, errs
+
+
