@@ -28,8 +28,8 @@ namespace {
 
 using namespace sm100;
 
-constexpr int NT = 128;          // 4 warps: warp w reads TMEM lanes 32w..32w+31
-constexpr int STAGES = 3;
+constexpr int NT = 256;          // 8 warps: warp w reads TMEM lanes 32 (w % 4) .. +31,
+                                 // columns half w / 4 of the tile
 constexpr int KB = 64;           // K block (one 128-byte swizzle atom of bf16)
 
 enum Kind { K_FWD = 0, K_FWD_LAST = 1, K_BWD = 2, K_DW = 3 };
@@ -87,7 +87,9 @@ __device__ bool wait_b(uint64_t *bar, uint32_t par, const GemmArgs &a) {
 // [256 x 64] (K-major) or [64 x 256] (MN-major). All in the row-block layout.
 constexpr uint32_t A_BYTES = 128 * KB * 2;       // 16 KB
 constexpr uint32_t B_BYTES = 256 * KB * 2;       // 32 KB
-constexpr uint32_t STAGE_BYTES = 2 * A_BYTES + B_BYTES;
+constexpr uint32_t STAGE_BYTES_DW = 2 * A_BYTES + B_BYTES;   // 64 KB, 3 stages
+constexpr uint32_t STAGE_BYTES_MM = A_BYTES + B_BYTES;       // 48 KB, 4 stages
+constexpr int STAGES_MAX = 4;
 
 // A tile loads. mt: 128-row tile index (forward/backward) or 128-column tile
 // of the transposed operand (update).
@@ -107,7 +109,7 @@ __device__ __forceinline__ void load_stage(const GemmArgs &a, const CUtensorMap 
     const int brow0 = (int)(s * a.b_rows_per_stream + a.b_row_off) + kb * KB;
     for (int f = 0; f < a.N / 64; ++f)
       tma_load_2d(st + 2 * A_BYTES + f * 64 * 128, mB, bar, a.N * nt + 64 * f, brow0);
-    return;
+    return;  // DW stage: [A_c | A_e | B]
   }
   // A: K-major [128 rows x 64] (rows = tokens); two 64-row pieces.
   for (int piece = 0; piece < 2; ++piece) {
@@ -124,11 +126,11 @@ __device__ __forceinline__ void load_stage(const GemmArgs &a, const CUtensorMap 
     // B: W_l as [K = n_l rows, N = n_{l-1} features], MN-major; 64 K rows per stage
     const int brow0 = s * a.b_rows_per_stream + kb * KB;
     for (int f = 0; f < a.N / 64; ++f)
-      tma_load_2d(st + 2 * A_BYTES + f * 64 * 128, mB, bar, a.N * nt + 64 * f, brow0);
+      tma_load_2d(st + A_BYTES + f * 64 * 128, mB, bar, a.N * nt + 64 * f, brow0);
   } else {
     // B: W_l rows = N (K-major), up to 256 rows in 64-row pieces
     for (int piece = 0; piece < a.N / 64; ++piece)
-      tma_load_2d(st + 2 * A_BYTES + piece * 64 * 128, mB, bar, kb * KB,
+      tma_load_2d(st + A_BYTES + piece * 64 * 128, mB, bar, kb * KB,
                   s * a.b_rows_per_stream + a.N * nt + 64 * piece);
   }
 }
@@ -139,16 +141,18 @@ __global__ void __launch_bounds__(NT, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *sm =
       reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t full[STAGES], empty[STAGES], done;
+  __shared__ uint64_t full[STAGES_MAX], empty[STAGES_MAX], done;
   __shared__ uint32_t tslot;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int s = blockIdx.z, mt = blockIdx.y, nt = blockIdx.x;
   const int kind = a.kind;
   const int nk = a.K / KB;
   const uint32_t ncols = kind == K_DW ? 512u : 256u;
+  const int STAGES = kind == K_DW ? 3 : 4;
+  const uint32_t STAGE_BYTES = kind == K_DW ? STAGE_BYTES_DW : STAGE_BYTES_MM;
 
   if (tid == 0) {
-    for (int i = 0; i < STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < STAGES_MAX; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     mbar_init(&done, 1);
     fence_barrier_init();
   }
@@ -158,6 +162,9 @@ __global__ void __launch_bounds__(NT, 1)
   tc_fence_after();
   const uint32_t tm = tslot;
   bool ok = true;
+  // Programmatic dependent launch: everything above overlapped the previous
+  // kernel's tail; its outputs are read only after this wait.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (tid == 0) {
     const uint32_t tx = kind == K_DW ? (uint32_t)(2 * A_BYTES + (uint32_t)a.N * KB * 2)
@@ -182,10 +189,10 @@ __global__ void __launch_bounds__(NT, 1)
           umma_bf16(tm, desc_mnmajor(base, 64, ks), bd, idesc, (kb | ks) != 0);
           umma_bf16(tm + 256, desc_mnmajor(base + A_BYTES, 64, ks), bd, idesc, (kb | ks) != 0);
         } else if (kind == K_BWD) {
-          umma_bf16(tm, desc_kmajor(base, 128, ks), desc_mnmajor(base + 2 * A_BYTES, 64, ks), idesc,
+          umma_bf16(tm, desc_kmajor(base, 128, ks), desc_mnmajor(base + A_BYTES, 64, ks), idesc,
                     (kb | ks) != 0);
         } else {
-          umma_bf16(tm, desc_kmajor(base, 128, ks), desc_kmajor(base + 2 * A_BYTES, a.N, ks), idesc,
+          umma_bf16(tm, desc_kmajor(base, 128, ks), desc_kmajor(base + A_BYTES, a.N, ks), idesc,
                     (kb | ks) != 0);
         }
       }
@@ -199,17 +206,22 @@ __global__ void __launch_bounds__(NT, 1)
     umma_commit(&done);
   }
   __syncwarp();
+  // the next kernel may start its prologue now (it waits for our completion
+  // before reading anything we write)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // ------------------------------------------------------------ epilogue
   if (!mbar_wait(&done, 0, a.wait_ns)) { atomicCAS(a.status, 0, kDevTimeout); ok = false; }
   tc_fence_after();
-  const int row = 32 * warp + lane;              // TMEM lane = output row of the tile
-  const uint32_t lb = (uint32_t)(32 * warp) << 16;
+  const int row = 32 * (warp & 3) + lane;        // TMEM lane = output row of the tile
+  const uint32_t lb = (uint32_t)(32 * (warp & 3)) << 16;
+  const int half = warp >> 2;                    // this warp's half of the tile's columns
+  const int cbeg = half * (a.N / 2), cend = cbeg + a.N / 2;
   if (ok) {
     if (kind == K_FWD || kind == K_FWD_LAST || kind == K_BWD) {
       const int r = 128 * mt + row;              // row of the per-stream matrix
       const bool key = r < a.C;
       const bool valid = (kind == K_BWD) ? key : (r < 2 * a.C);
-      for (int c0 = 0; c0 < a.N; c0 += 16) {
+      for (int c0 = cbeg; c0 < cend; c0 += 16) {
         float z[16];
         tmem_ld16(tm + lb + c0, z);
         tmem_wait_ld();
@@ -283,35 +295,51 @@ __global__ void __launch_bounds__(NT, 1)
       const float4 sc = *reinterpret_cast<const float4 *>(a.scal + 4 * ((long long)s * a.nchunks + a.chunk));
       float *Wl = a.W + (long long)s * a.P + a.layer_off;
       float *Sl = a.S + (long long)s * a.P + a.layer_off;
-      for (int c0 = 0; c0 < a.N; c0 += 16) {
-        float uw[16], us[16];
-        tmem_ld16(tm + lb + c0, uw);
-        tmem_ld16(tm + lb + 256 + c0, us);
-        tmem_wait_ld();
-        if (!valid) continue;
+      for (int c0 = cbeg; c0 < cend; c0 += 64) {
         const int col = a.N * nt + c0;
         const long long g = (long long)wr * a.n_out + col;
-        float w[16], sv[16];
+        const int ncol = cend - c0 < 64 ? cend - c0 : 64;  // 64, or 32 for a 64-wide tile
+        // all of this thread's W and S loads of the piece in flight at once
+        float4 w4[16], s4[16];
+        if (valid) {
 #pragma unroll
-        for (int i4 = 0; i4 < 4; ++i4) {
-          const float4 w4 = *reinterpret_cast<const float4 *>(Wl + g + 4 * i4);
-          const float4 s4 = *reinterpret_cast<const float4 *>(Sl + g + 4 * i4);
-          w[4 * i4] = w4.x; w[4 * i4 + 1] = w4.y; w[4 * i4 + 2] = w4.z; w[4 * i4 + 3] = w4.w;
-          sv[4 * i4] = s4.x; sv[4 * i4 + 1] = s4.y; sv[4 * i4 + 2] = s4.z; sv[4 * i4 + 3] = s4.w;
+          for (int i4 = 0; i4 < 16; ++i4) {
+            if (4 * i4 < ncol) {
+              w4[i4] = *reinterpret_cast<const float4 *>(Wl + g + 4 * i4);
+              s4[i4] = *reinterpret_cast<const float4 *>(Sl + g + 4 * i4);
+            }
+          }
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          w[i] = sc.x * w[i] + sc.z * sv[i] + uw[i];
-          sv[i] = sc.y * sv[i] + us[i];
-        }
+        for (int q16 = 0; q16 < 4; ++q16) {
+          if (16 * q16 >= ncol) break;
+          float uw[16], us[16];
+          tmem_ld16(tm + lb + c0 + 16 * q16, uw);
+          tmem_ld16(tm + lb + 256 + c0 + 16 * q16, us);
+          tmem_wait_ld();
+          if (!valid) continue;
+          float w[16], sv[16];
 #pragma unroll
-        for (int i4 = 0; i4 < 4; ++i4) {
-          *reinterpret_cast<float4 *>(Wl + g + 4 * i4) = make_float4(w[4 * i4], w[4 * i4 + 1], w[4 * i4 + 2], w[4 * i4 + 3]);
-          *reinterpret_cast<float4 *>(Sl + g + 4 * i4) = make_float4(sv[4 * i4], sv[4 * i4 + 1], sv[4 * i4 + 2], sv[4 * i4 + 3]);
+          for (int i4 = 0; i4 < 4; ++i4) {
+            const float4 a4 = w4[4 * q16 + i4], b4 = s4[4 * q16 + i4];
+            w[4 * i4] = a4.x; w[4 * i4 + 1] = a4.y; w[4 * i4 + 2] = a4.z; w[4 * i4 + 3] = a4.w;
+            sv[4 * i4] = b4.x; sv[4 * i4 + 1] = b4.y; sv[4 * i4 + 2] = b4.z; sv[4 * i4 + 3] = b4.w;
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            w[i] = sc.x * w[i] + sc.z * sv[i] + uw[i];
+            sv[i] = sc.y * sv[i] + us[i];
+          }
+          const long long gq = g + 16 * q16;
+#pragma unroll
+          for (int i4 = 0; i4 < 4; ++i4) {
+            *reinterpret_cast<float4 *>(Wl + gq + 4 * i4) = make_float4(w[4 * i4], w[4 * i4 + 1], w[4 * i4 + 2], w[4 * i4 + 3]);
+            *reinterpret_cast<float4 *>(Sl + gq + 4 * i4) = make_float4(sv[4 * i4], sv[4 * i4 + 1], sv[4 * i4 + 2], sv[4 * i4 + 3]);
+          }
+          __nv_bfloat16 *wb = a.Wbf + (long long)s * a.M * a.n_out + gq;
+          *reinterpret_cast<uint4 *>(wb) = pack8(w);
+          *reinterpret_cast<uint4 *>(wb + 8) = pack8(w + 8);
         }
-        __nv_bfloat16 *wb = a.Wbf + (long long)s * a.M * a.n_out + g;
-        *reinterpret_cast<uint4 *>(wb) = pack8(w);
-        *reinterpret_cast<uint4 *>(wb + 8) = pack8(w + 8);
       }
     }
   }
@@ -445,13 +473,21 @@ bool dims_ok(const Problem &p) {
   return true;
 }
 
-constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+constexpr size_t SMEM_BYTES = 3 * STAGE_BYTES_DW + 1024;   // = 4 * STAGE_BYTES_MM + 1024
 
 cudaError_t launch_gemm(const GemmArgs &a, const CUtensorMap &mA, const CUtensorMap &mA2,
                         const CUtensorMap &mB, int streams, int mtiles, int ntiles, cudaStream_t st) {
-  dim3 grid((unsigned)ntiles, (unsigned)mtiles, (unsigned)streams);
-  tcl_gemm_kernel<<<grid, NT, SMEM_BYTES, st>>>(a, mA, mA2, mB);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)ntiles, (unsigned)mtiles, (unsigned)streams);
+  cfg.blockDim = dim3(NT);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tcl_gemm_kernel, a, mA, mA2, mB);
 }
 
 }  // namespace
@@ -517,7 +553,14 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
       return cudaErrorInvalidValue;
     if (l < L && !map2d(&mx[l], bf(cv.x[l]), (long long)S * 2 * C, nl, 64)) return cudaErrorInvalidValue;
   }
-  auto tile_n = [](int n) { return n % 256 == 0 ? 256 : (n % 128 == 0 ? 128 : 64); };
+  // Widest tile that divides n and still gives about one CTA per SM.
+  auto tile_for = [&](int n, int mtiles) {
+    for (int t = 256; t >= 64; t /= 2) {
+      if (n % t) continue;
+      if ((long long)S * mtiles * (n / t) >= 128 || t == 64) return t;
+    }
+    return 64;
+  };
 
   GemmArgs base;
   std::memset(&base, 0, sizeof base);
@@ -541,7 +584,7 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
       const int nl = p.dims[l], np = p.dims[l - 1];
       a.kind = l < L ? K_FWD : K_FWD_LAST;
       a.chunk = ch;
-      a.N = tile_n(nl);
+      a.N = tile_for(nl, 2 * C / 128);
       a.K = np;
       a.M = 2 * C;
       a.n_out = nl;
@@ -559,7 +602,7 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
       const int nl = p.dims[l], np = p.dims[l - 1];
       a.kind = K_BWD;
       a.chunk = ch;
-      a.N = tile_n(np);
+      a.N = tile_for(np, 1);
       a.K = nl;
       a.M = C;
       a.n_out = np;
@@ -576,7 +619,7 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
       const int nl = p.dims[l], np = p.dims[l - 1];
       a.kind = K_DW;
       a.chunk = ch;
-      a.N = tile_n(np);
+      a.N = tile_for(np, (nl + 127) / 128);
       a.K = C;
       a.M = nl;
       a.n_out = np;
