@@ -200,6 +200,104 @@ def run_reference(args, w: W.Workload):
     print(json.dumps(line), flush=True)
 
 
+def sweep_chunk(args, w: W.Workload, sizes):
+    """Chunk-size trade-off: the same workload timed at several chunk sizes C
+    (gradients of a chunk are taken at its start weights, so C changes the
+    method's result as well as its speed; this times it, it does not compare
+    results). One JSON line per size: path taken, ms per pass, tokens/s."""
+    import dataclasses
+
+    import torch
+    from test_trained_neural_b200 import NeuralMemory
+
+    dev = torch.device("cuda", 0)
+    inp = W.generate(w)
+    d_in = {}
+    for key in ("k", "v", "q"):
+        a = np.ascontiguousarray(inp[key])
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if w.dtype == "bf16" else torch.from_numpy(a)
+        d_in[key] = t.reshape(w.B, w.H, w.T, w.d).to(dev)
+    for key in ("theta", "eta", "alpha", "W0", "S0"):
+        d_in[key] = torch.from_numpy(np.ascontiguousarray(inp[key])).reshape(w.B, w.H, *inp[key].shape[1:]).to(dev)
+    y = torch.empty((w.B, w.H, w.T, w.d), dtype=torch.float32, device=dev)
+    We, Se = torch.empty_like(d_in["W0"]), torch.empty_like(d_in["S0"])
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    for C in sizes:
+        wc = dataclasses.replace(w, C=C)
+        if wc.T % C:
+            continue
+        mem = NeuralMemory(w.L, w.d, w.expansion, path=args.path)
+        try:
+            path = mem.query_path(w.B, w.H, w.T, C, d_in["k"].dtype)
+        except Exception as ex:  # no kernel for this size on the forced path
+            print(json.dumps({"chunk": C, "unsupported": str(ex)}), flush=True)
+            continue
+        ws = mem.alloc_workspace(w.B, w.H, w.T, C, d_in["k"].dtype, dev)
+        stream = torch.cuda.current_stream(dev)
+
+        def step():
+            mem.run(d_in["k"], d_in["v"], d_in["q"], d_in["theta"], d_in["eta"], d_in["alpha"],
+                    d_in["W0"], d_in["S0"], C, y=y, W_end=We, S_end=Se, workspace=ws, stream=stream)
+        for _ in range(args.warmup):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            step()
+            a1.record(stream)
+            torch.cuda.synchronize()
+            ms.append(a0.elapsed_time(a1))
+        mem.sync(ws, stream)
+        t = statistics.mean(ms)
+        print(json.dumps({"metric": "memory tokens/sec (write+read)", "workload": w.name, "T": w.T,
+                          "chunk": C, "path": path, "ms_per_pass": t,
+                          "tokens_per_s": w.streams * w.T / (t * 1e-3),
+                          "workspace_bytes": ws.numel()}), flush=True)
+
+
+def bench_prologue(args, w: W.Workload):
+    """The step before the memory on the workload's k, v, q: one fused launch of
+    the depthwise causal convolution (width args.conv_width) and the L2
+    normalisation of keys and queries. HBM-bound: the algorithmic traffic is
+    each of k, v, q read once and written once."""
+    import torch
+    from test_trained_neural_b200 import prologue
+
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    xs = [torch.randn((w.B, w.H, w.T, w.d), generator=g, device=dev).to(dt) for _ in range(3)]
+    fs = [0.5 * torch.randn((w.H, w.d, args.conv_width), generator=g, device=dev) for _ in range(3)]
+    outs = tuple(torch.empty_like(x) for x in xs)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        prologue(*xs, *fs, out=outs)
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+        prologue(*xs, *fs, out=outs)
+        a1.record()
+        torch.cuda.synchronize()
+        ms.append(a0.elapsed_time(a1))
+    t = statistics.mean(ms) * 1e-3
+    bytes_ = 2.0 * 3 * xs[0].numel() * xs[0].element_size()
+    peak = measured_peaks()
+    gbs = bytes_ / t / 1e9
+    print(json.dumps({"metric": "prologue tokens/sec", "value": w.streams * w.T / t, "unit": "tokens/s",
+                      "ms": t * 1e3, "workload": w.name, "width": args.conv_width,
+                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak["hbm_gbs"],
+                                   "unit": "GB/s", "frac": gbs / peak["hbm_gbs"],
+                                   "peak_source": peak["source"] + " HBM copy"}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -212,6 +310,13 @@ def main():
                     help="draw the gates exactly as specified (the MLP memories overflow)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (tokens per stream), e.g. for short profiling runs")
+    ap.add_argument("--chunk", type=int, default=None, help="override the chunk size C")
+    ap.add_argument("--prologue", action="store_true",
+                    help="time the convolution + normalisation step before the memory instead")
+    ap.add_argument("--conv-width", type=int, default=4)
+    ap.add_argument("--sweep-chunk", default=None,
+                    help="comma-separated chunk sizes: time each (same workload, T as given) "
+                         "and print one JSON line per size instead of the benchmark line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
@@ -221,6 +326,13 @@ def main():
     if args.tokens:
         import dataclasses
         w = dataclasses.replace(w, T=args.tokens)
+    if args.chunk:
+        import dataclasses
+        w = dataclasses.replace(w, C=args.chunk)
+    if args.sweep_chunk:
+        return sweep_chunk(args, w, [int(x) for x in args.sweep_chunk.split(",")])
+    if args.prologue:
+        return bench_prologue(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
 

@@ -74,8 +74,8 @@ typedef enum {
   TM_PATH_TC = 2,          /* tcgen05 cluster kernel, state resident on chip (L = 2,
                               d in {64, 128}, hidden = 64 G, C = 64); else unsupported     */
   TM_PATH_TC_LAYERED = 3   /* tcgen05 batched GEMMs, one launch per layer phase and chunk;
-                              state in W_end / S_end (widths multiples of 64, C in
-                              {64, 128}); else unsupported                                  */
+                              state in W_end / S_end (widths multiples of 64, C a
+                              multiple of 64 up to 256); else unsupported                   */
 } tm_path;
 
 /*
@@ -172,6 +172,31 @@ TM_API tm_status tm_run_noalloc(tm_ctx *ctx, int B, int H, int T, int C, tm_dtyp
  * kernels, or TM_ERR_CUDA if the stream itself reports an error.
  */
 TM_API tm_status tm_sync(tm_ctx *ctx, void *workspace, void *stream);
+
+/*
+ * The step before the memory: a short depthwise causal convolution of the
+ * projected keys, values and queries, followed by L2 normalisation of every
+ * key and query row ("Titans, explained", step 1: "the projections are
+ * followed by a short depthwise convolution, and keys and queries are
+ * l2-normalized"). One fused launch for the three tensors; allocates nothing.
+ *
+ *   x_in  (k_in, v_in, q_in)  [B, H, T, d] in_dtype, device
+ *   filt  (filt_k, ...)       [H, d, width] float32, device: out[t, c] =
+ *                             sum_{j=0}^{width-1} filt[h, c, j] x[t - j, c]
+ *   hist  (hist_k, ...)       [B, H, width-1, d] in_dtype, device, or NULL:
+ *                             the last width-1 tokens before this call
+ *                             (NULL = zeros); row width-1+t holds token t < 0
+ *   x_out (k_out, ...)        [B, H, T, d] in_dtype, device; must not overlap
+ *                             any input. A zero key/query row stays zero.
+ * Requires 1 <= width <= 8, T >= 1, 16-byte aligned pointers, and d in
+ * {32, 64} or a multiple of 128 up to 768 (TM_ERR_UNSUPPORTED otherwise). Returns TM_ERR_INVALID_ARG for bad arguments (no launch),
+ * TM_ERR_CUDA if the launch fails.
+ */
+TM_API tm_status tm_prologue(int B, int H, int T, int d, int width, tm_dtype in_dtype,
+                             const void *k_in, const void *v_in, const void *q_in,
+                             const float *filt_k, const float *filt_v, const float *filt_q,
+                             const void *hist_k, const void *hist_v, const void *hist_q,
+                             void *k_out, void *v_out, void *q_out, void *stream);
 
 /*
  * Test hook for failure handling (process-wide, host-only). inject_timeout != 0

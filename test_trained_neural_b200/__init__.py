@@ -3,5 +3,5 @@
 The compute lives in libtitansmem.so (CUDA, C ABI in include/titansmem.h);
 this package is its thin Python binding.
 """
-from .memory import NeuralMemory  # noqa: F401
+from .memory import NeuralMemory, prologue  # noqa: F401
 from ._native import TitansMemError  # noqa: F401

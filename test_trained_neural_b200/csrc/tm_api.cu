@@ -225,6 +225,35 @@ tm_status tm_sync(tm_ctx *ctx, void *workspace, void *stream) {
   return code == tmem::kDevTimeout ? TM_ERR_TIMEOUT : TM_ERR_DEVICE;
 }
 
+tm_status tm_prologue(int B, int H, int T, int d, int width, tm_dtype in_dtype, const void *k_in,
+                      const void *v_in, const void *q_in, const float *filt_k, const float *filt_v,
+                      const float *filt_q, const void *hist_k, const void *hist_v, const void *hist_q,
+                      void *k_out, void *v_out, void *q_out, void *stream) {
+  if (B < 1 || H < 1 || T < 1 || d < 1 || d > 768 || width < 1 || width > 8) return TM_ERR_INVALID_ARG;
+  if (!tmem::prologue_supported_d(d)) return TM_ERR_UNSUPPORTED;
+  if (in_dtype != TM_F32 && in_dtype != TM_BF16) return TM_ERR_INVALID_ARG;
+  if ((long long)B * H > (1LL << 16) - 1 || T > (1 << 30)) return TM_ERR_INVALID_ARG;
+  const void *in[3] = {k_in, v_in, q_in};
+  const float *filt[3] = {filt_k, filt_v, filt_q};
+  const void *hist[3] = {hist_k, hist_v, hist_q};
+  void *out[3] = {k_out, v_out, q_out};
+  const size_t el = in_dtype == TM_BF16 ? 2 : 4;
+  const size_t tens = (size_t)B * H * T * d * el;
+  for (int i = 0; i < 3; ++i) {
+    if (!in[i] || !filt[i] || !out[i]) return TM_ERR_INVALID_ARG;
+    const void *ps[] = {in[i], filt[i], out[i], hist[i]};
+    for (const void *p : ps)
+      if (p && (reinterpret_cast<uintptr_t>(p) & 15u)) return TM_ERR_INVALID_ARG;
+    for (int j = 0; j < 3; ++j)
+      if (ranges_overlap(out[i], tens, in[j], tens)) return TM_ERR_INVALID_ARG;
+    for (int j = 0; j < i; ++j)
+      if (ranges_overlap(out[i], tens, out[j], tens)) return TM_ERR_INVALID_ARG;
+  }
+  cudaError_t e = tmem::prologue_launch(B * H, H, T, d, width, in_dtype == TM_BF16, in, filt, hist, out,
+                                        reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? TM_OK : TM_ERR_CUDA;
+}
+
 tm_status tm_set_debug(int inject_timeout, unsigned long long wait_limit_ns) {
   tmem::tc_set_debug(inject_timeout, wait_limit_ns);
   tmem::tcl_set_wait(wait_limit_ns);

@@ -54,6 +54,12 @@ size_t tcl_scratch_bytes(const Problem &p);
 cudaError_t tcl_launch(const Problem &p, cudaStream_t stream);
 void tcl_set_wait(unsigned long long wait_ns);
 
+// Depthwise causal convolution + L2 normalisation before the memory.
+bool prologue_supported_d(int d);
+cudaError_t prologue_launch(int streams, int H, int T, int d, int w, bool bf16, const void *const in[3],
+                            const float *const filt[3], const void *const hist[3], void *const out[3],
+                            cudaStream_t stream);
+
 // Test hooks of the tensor-core path: make the first wait of every CTA one
 // that nothing completes, and/or shorten the per-wait time limit (0 = 2 s).
 void tc_set_debug(int inject_timeout, unsigned long long wait_ns);

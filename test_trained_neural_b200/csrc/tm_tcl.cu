@@ -494,7 +494,7 @@ cudaError_t launch_gemm(const GemmArgs &a, const CUtensorMap &mA, const CUtensor
 
 bool tcl_supported(const Problem &p) {
   if (p.in_dtype != TM_BF16) return false;
-  if (p.C != 64 && p.C != 128) return false;
+  if (p.C % 64 != 0 || p.C > 256) return false;
   if (!dims_ok(p)) return false;
   for (int l = 0; l <= p.L; ++l)
     if (p.dims[l] > 4096) return false;
@@ -602,7 +602,7 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
       const int nl = p.dims[l], np = p.dims[l - 1];
       a.kind = K_BWD;
       a.chunk = ch;
-      a.N = tile_for(np, 1);
+      a.N = tile_for(np, (C + 127) / 128);
       a.K = nl;
       a.M = C;
       a.n_out = np;
@@ -610,7 +610,7 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
       a.b_rows_per_stream = nl;
       a.sp_in = bf(cv.sp[l - 1]);
       a.g_out = bf(cv.g[l - 1]); a.gc_out = bf(cv.gc[l - 1]); a.ge_out = bf(cv.ge[l - 1]);
-      err = launch_gemm(a, mg[l], mg[l], mwb[l], S, 1, np / a.N, stream);
+      err = launch_gemm(a, mg[l], mg[l], mwb[l], S, (C + 127) / 128, np / a.N, stream);
       if (err != cudaSuccess) return err;
     }
     // weight-update contractions with the fused state update

@@ -107,3 +107,25 @@ class NeuralMemory:
             stream = torch.cuda.current_stream(workspace.device)
         N.check(self._lib.tm_sync(self._h, _ptr(workspace), ctypes.c_void_p(stream.cuda_stream)),
                 "tm_sync")
+
+
+def prologue(k, v, q, filt_k, filt_v, filt_q, hist=None, out=None, stream=None):
+    """Depthwise causal convolution of k, v, q ([B, H, T, d], float32 or
+    bfloat16, CUDA) with per-head filters [H, d, width] (float32), then L2
+    normalisation of the key and query rows. hist: optional (hk, hv, hq)
+    [B, H, width-1, d] tails of the previous call. Returns (k', v', q')."""
+    lib = N.load()
+    B, H, T, d = k.shape
+    width = filt_k.shape[-1]
+    dt = N.TM_BF16 if k.dtype == torch.bfloat16 else N.TM_F32
+    if out is None:
+        out = (torch.empty_like(k), torch.empty_like(v), torch.empty_like(q))
+    hk, hv, hq = hist if hist is not None else (None, None, None)
+    hp = lambda t: None if t is None else _ptr(t)
+    if stream is None:
+        stream = torch.cuda.current_stream(k.device)
+    code = lib.tm_prologue(B, H, T, d, width, dt, _ptr(k), _ptr(v), _ptr(q), _ptr(filt_k),
+                           _ptr(filt_v), _ptr(filt_q), hp(hk), hp(hv), hp(hq), _ptr(out[0]),
+                           _ptr(out[1]), _ptr(out[2]), ctypes.c_void_p(stream.cuda_stream))
+    N.check(code, "tm_prologue")
+    return out

@@ -268,6 +268,8 @@ TCL_SHAPES = [  # L, d, expansion, B, H, T, C
     (3, 64, 2, 2, 1, 256, 128),     # C = 128: two row tiles of keys and queries
     (4, 64, 2, 1, 2, 256, 128),
     (4, 128, 2, 1, 1, 256, 128),    # the deep workload's layer shapes
+    (2, 64, 2, 1, 2, 384, 192),     # C = 192: a partial row tile in the backward
+    (2, 128, 2, 1, 1, 512, 256),    # C = 256: four key/query row tiles, pipelined K loop
 ]
 
 
