@@ -259,6 +259,18 @@ def sweep_chunk(args, w: W.Workload, sizes):
                           "workspace_bytes": ws.numel()}), flush=True)
 
 
+def launches_per_run(w: W.Workload, path: str) -> int:
+    """Kernels of this library per tm_run: one persistent kernel (cluster or
+    CUDA-core path); for the layered path an init and a coefficient kernel,
+    then per chunk either one fused forward + backward launch and L update
+    launches (every width at most 256) or 3L - 1 phase launches."""
+    if path not in ("tcl", "tcl-phased"):
+        return 1
+    fused = path == "tcl" and max(w.dims) <= 256
+    per_chunk = 1 + w.L if fused else 3 * w.L - 1
+    return 2 + per_chunk * (w.T // w.C)
+
+
 def bench_prologue(args, w: W.Workload):
     """The step before the memory on the workload's k, v, q: one fused launch of
     the depthwise causal convolution (width args.conv_width) and the L2
@@ -304,7 +316,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", type=int, default=3, help="workload index 0..4")
-    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc", "tcl", "tcl-phased"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--literal-gates", action="store_true",
                     help="draw the gates exactly as specified (the MLP memories overflow)")
@@ -397,10 +409,7 @@ def main():
     ms_max = max_over_ranks(ms, world)
 
     cnt = algorithmic_counts(w, w.T)
-    # kernels of this library per tm_run: one persistent kernel (cluster or
-    # CUDA-core path), or for the layered path an init and a coefficient kernel
-    # plus 3L - 1 GEMMs per chunk
-    launches_per_step = 2 + (3 * w.L - 1) * (w.T // w.C) if path_used == "tcl" else 1
+    launches_per_step = launches_per_run(w, path_used)
     value = aggregate_throughput(cnt["tokens"], world, ms_max * 1e-3)
     peaks = measured_peaks()
     hbm = peaks["hbm_gbs"] * 1e9
@@ -409,7 +418,7 @@ def main():
     t_state = (cnt["state_bytes"] + cnt["token_io_bytes"]) / hbm
     chunk_roofline_s = max(t_flop, t_state)
     sec = ms * 1e-3
-    if path_used in ("tc", "tcl"):
+    if path_used in ("tc", "tcl", "tcl-phased"):
         # The kernel runs alone at the maximum SM clock, far from the power
         # cap, so the burst figure is the denominator.
         roof = {"bound": "tensor", "achieved": cnt["flops"] / sec / 1e12,
@@ -423,7 +432,8 @@ def main():
                 "sm_mhz_seen": sm_mhz}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = None
-    roof["kernel"] = {"tc": "tc_chunk_kernel", "tcl": "tcl_gemm_kernel"}.get(path_used, "simt_chunk_kernel")
+    roof["kernel"] = {"tc": "tc_chunk_kernel", "tcl": "tcl_fb_kernel + tcl_gemm_kernel",
+                      "tcl-phased": "tcl_gemm_kernel"}.get(path_used, "simt_chunk_kernel")
 
     e2e = None
     if not args.no_e2e:
@@ -463,7 +473,7 @@ def main():
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if w.dtype == "bf16" and path_used in ("tc", "tcl") else
+            "dtype": "bf16" if w.dtype == "bf16" and path_used in ("tc", "tcl", "tcl-phased") else
                      ("bf16-in/f32" if w.dtype == "bf16" else "f32"),
             "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "C": w.C, "dims": w.dims,

@@ -73,9 +73,13 @@ typedef enum {
   TM_PATH_SIMT = 1,        /* fp32 CUDA-core kernel for any supported shape and dtype      */
   TM_PATH_TC = 2,          /* tcgen05 cluster kernel, state resident on chip (L = 2,
                               d in {64, 128}, hidden = 64 G, C = 64); else unsupported     */
-  TM_PATH_TC_LAYERED = 3   /* tcgen05 batched GEMMs, one launch per layer phase and chunk;
-                              state in W_end / S_end (widths multiples of 64, C a
-                              multiple of 64 up to 256); else unsupported                   */
+  TM_PATH_TC_LAYERED = 3,  /* tcgen05 batched GEMMs per chunk; state in W_end / S_end
+                              (widths multiples of 64, C a multiple of 64 up to 256); when
+                              every width is at most 256 the forward and backward of a
+                              chunk run as one fused launch, then one update launch per
+                              layer; else unsupported                                      */
+  TM_PATH_TC_PHASED = 4    /* as TM_PATH_TC_LAYERED, but every forward, backward and
+                              update phase its own launch (same results; for comparison)   */
 } tm_path;
 
 /*

@@ -34,6 +34,7 @@ struct Problem {
   float *y, *W_end, *S_end;
   int *status;            // device status word
   void *scratch;          // per-stream activations (SIMT path)
+  int fuse_fb;            // layered path: fused forward + backward launch where supported
   size_t scratch_bytes;
 };
 

@@ -90,6 +90,15 @@ constexpr uint32_t B_BYTES = 256 * KB * 2;       // 32 KB
 constexpr uint32_t STAGE_BYTES_DW = 2 * A_BYTES + B_BYTES;   // 64 KB, 3 stages
 constexpr uint32_t STAGE_BYTES_MM = A_BYTES + B_BYTES;       // 48 KB, 4 stages
 constexpr int STAGES_MAX = 4;
+// The update GEMM's output tiles are at most 128 columns wide, so its two
+// accumulators take 256 TMEM columns and, for C <= 128 (two K blocks, two
+// stages), its ring 96 KB: two CTAs fit on an SM and one layer's update
+// overlaps the next one's.
+constexpr int DW_MAXN = 128;
+__host__ __device__ constexpr int dw_stages(int nk) { return nk <= 2 ? 2 : 3; }
+__host__ __device__ constexpr uint32_t dw_stage_bytes(int N) { return 2 * A_BYTES + (uint32_t)N * KB * 2; }
+// the epilogue's staging buffer (U_W and U_S of a 64-column piece) reuses the ring
+constexpr uint32_t DW_STAGE_U = 2 * 128 * 64 * 4;
 
 // A tile loads. mt: 128-row tile index (forward/backward) or 128-column tile
 // of the transposed operand (update).
@@ -135,21 +144,22 @@ __device__ __forceinline__ void load_stage(const GemmArgs &a, const CUtensorMap 
   }
 }
 
-__global__ void __launch_bounds__(NT, 1)
-    tcl_gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap mA,
-                    const __grid_constant__ CUtensorMap mA2, const __grid_constant__ CUtensorMap mB) {
+// One output tile (stream s, row tile mt, column tile nt) of a phase GEMM.
+// KIND is one of the phases.
+template <int KIND>
+__device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &mA, const CUtensorMap &mA2,
+                                          const CUtensorMap &mB, const int s, const int mt, const int nt) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *sm =
       reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t full[STAGES_MAX], empty[STAGES_MAX], done;
   __shared__ uint32_t tslot;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int s = blockIdx.z, mt = blockIdx.y, nt = blockIdx.x;
-  const int kind = a.kind;
+  constexpr int kind = KIND;
   const int nk = a.K / KB;
-  const uint32_t ncols = kind == K_DW ? 512u : 256u;
-  const int STAGES = kind == K_DW ? 3 : 4;
-  const uint32_t STAGE_BYTES = kind == K_DW ? STAGE_BYTES_DW : STAGE_BYTES_MM;
+  const uint32_t ncols = 256u;                 // DW: U_W in columns [0, 128), U_S in [128, 256)
+  const int STAGES = kind == K_DW ? dw_stages(nk) : 4;
+  const uint32_t STAGE_BYTES = kind == K_DW ? dw_stage_bytes(a.N) : STAGE_BYTES_MM;
 
   if (tid == 0) {
     for (int i = 0; i < STAGES_MAX; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
@@ -162,6 +172,25 @@ __global__ void __launch_bounds__(NT, 1)
   tc_fence_after();
   const uint32_t tm = tslot;
   bool ok = true;
+  // Update: this thread's share of a 64-column piece of the fp32 state tile,
+  // in a coalesced mapping (16 threads per 256-byte row piece, rows
+  // tid/16 + 16 i). The first piece is requested while thread 0 issues the
+  // MMAs (the others skip that loop).
+  float4 wpre[8], spre[8];
+  const int dw_c4 = tid % 16, dw_r0 = tid / 16;
+  auto dw_prefetch = [&](int pc) {
+    float *Wl = a.W + (long long)s * a.P + a.layer_off;
+    float *Sl = a.S + (long long)s * a.P + a.layer_off;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int wr = 128 * mt + dw_r0 + 16 * i;
+      if (wr < a.M) {
+        const long long g = (long long)wr * a.n_out + a.N * nt + 64 * pc + 4 * dw_c4;
+        wpre[i] = *reinterpret_cast<const float4 *>(Wl + g);
+        spre[i] = *reinterpret_cast<const float4 *>(Sl + g);
+      }
+    }
+  };
   // Programmatic dependent launch: everything above overlapped the previous
   // kernel's tail; its outputs are read only after this wait.
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -187,7 +216,7 @@ __global__ void __launch_bounds__(NT, 1)
         if (kind == K_DW) {
           const uint64_t bd = desc_mnmajor(base + 2 * A_BYTES, 64, ks);
           umma_bf16(tm, desc_mnmajor(base, 64, ks), bd, idesc, (kb | ks) != 0);
-          umma_bf16(tm + 256, desc_mnmajor(base + A_BYTES, 64, ks), bd, idesc, (kb | ks) != 0);
+          umma_bf16(tm + 128, desc_mnmajor(base + A_BYTES, 64, ks), bd, idesc, (kb | ks) != 0);
         } else if (kind == K_BWD) {
           umma_bf16(tm, desc_kmajor(base, 128, ks), desc_mnmajor(base + A_BYTES, 64, ks), idesc,
                     (kb | ks) != 0);
@@ -205,6 +234,7 @@ __global__ void __launch_bounds__(NT, 1)
     }
     umma_commit(&done);
   }
+  if constexpr (kind == K_DW) dw_prefetch(0);
   __syncwarp();
   // the next kernel may start its prologue now (it waits for our completion
   // before reading anything we write)
@@ -217,7 +247,7 @@ __global__ void __launch_bounds__(NT, 1)
   const int half = warp >> 2;                    // this warp's half of the tile's columns
   const int cbeg = half * (a.N / 2), cend = cbeg + a.N / 2;
   if (ok) {
-    if (kind == K_FWD || kind == K_FWD_LAST || kind == K_BWD) {
+    if constexpr (kind == K_FWD || kind == K_FWD_LAST || kind == K_BWD) {
       const int r = 128 * mt + row;              // row of the per-stream matrix
       const bool key = r < a.C;
       const bool valid = (kind == K_BWD) ? key : (r < 2 * a.C);
@@ -288,64 +318,448 @@ __global__ void __launch_bounds__(NT, 1)
           *reinterpret_cast<uint4 *>(a.ge_out + o + 8) = pack8(ge + 8);
         }
       }
-    } else {
-      // update: row of W_l = 128 mt + row, columns N nt + [0, N)
-      const int wr = 128 * mt + row;
-      const bool valid = wr < a.M;
-      const float4 sc = *reinterpret_cast<const float4 *>(a.scal + 4 * ((long long)s * a.nchunks + a.chunk));
-      float *Wl = a.W + (long long)s * a.P + a.layer_off;
-      float *Sl = a.S + (long long)s * a.P + a.layer_off;
-      for (int c0 = cbeg; c0 < cend; c0 += 64) {
-        const int col = a.N * nt + c0;
-        const long long g = (long long)wr * a.n_out + col;
-        const int ncol = cend - c0 < 64 ? cend - c0 : 64;  // 64, or 32 for a 64-wide tile
-        // all of this thread's W and S loads of the piece in flight at once
-        float4 w4[16], s4[16];
-        if (valid) {
+    }
+  }
+  if constexpr (kind == K_DW) {
+    // Update, one 64-column piece at a time: (1) each thread moves its TMEM
+    // lane's 32 columns of U_W and U_S into shared memory (16-byte slots of a
+    // 256-byte row, slot index XOR row % 16: conflict-free both ways);
+    // (2) the tile is then updated row-contiguously, W' = B W + c_S S + U_W,
+    // S' = A S + U_S, with the prefetched state, and the next piece's state is
+    // requested before the stores.
+    float *uw = reinterpret_cast<float *>(sm);
+    float *us = uw + 128 * 64;
+    const float4 sc = *reinterpret_cast<const float4 *>(a.scal + 4 * ((long long)s * a.nchunks + a.chunk));
+    float *Wl = a.W + (long long)s * a.P + a.layer_off;
+    float *Sl = a.S + (long long)s * a.P + a.layer_off;
+    __nv_bfloat16 *Wb = a.Wbf + (long long)s * a.M * a.n_out;
+    const int npc = a.N / 64;
+    for (int pc = 0; pc < npc; ++pc) {
+      if (ok) {
+        const uint32_t c0 = (uint32_t)(64 * pc + 32 * half);
 #pragma unroll
-          for (int i4 = 0; i4 < 16; ++i4) {
-            if (4 * i4 < ncol) {
-              w4[i4] = *reinterpret_cast<const float4 *>(Wl + g + 4 * i4);
-              s4[i4] = *reinterpret_cast<const float4 *>(Sl + g + 4 * i4);
-            }
-          }
-        }
-#pragma unroll
-        for (int q16 = 0; q16 < 4; ++q16) {
-          if (16 * q16 >= ncol) break;
-          float uw[16], us[16];
-          tmem_ld16(tm + lb + c0 + 16 * q16, uw);
-          tmem_ld16(tm + lb + 256 + c0 + 16 * q16, us);
+        for (int acc = 0; acc < 2; ++acc) {      // U_W, then U_S
+          float u0[16], u1[16];
+          tmem_ld16(tm + lb + 128 * acc + c0, u0);
+          tmem_ld16(tm + lb + 128 * acc + c0 + 16, u1);
           tmem_wait_ld();
-          if (!valid) continue;
-          float w[16], sv[16];
+          float *dst = (acc ? us : uw) + row * 64;
 #pragma unroll
-          for (int i4 = 0; i4 < 4; ++i4) {
-            const float4 a4 = w4[4 * q16 + i4], b4 = s4[4 * q16 + i4];
-            w[4 * i4] = a4.x; w[4 * i4 + 1] = a4.y; w[4 * i4 + 2] = a4.z; w[4 * i4 + 3] = a4.w;
-            sv[4 * i4] = b4.x; sv[4 * i4 + 1] = b4.y; sv[4 * i4 + 2] = b4.z; sv[4 * i4 + 3] = b4.w;
+          for (int j = 0; j < 8; ++j) {
+            const int slot = (8 * half + j) ^ (row & 15);
+            const float *src = j < 4 ? u0 + 4 * j : u1 + 4 * (j - 4);
+            *reinterpret_cast<float4 *>(dst + 4 * slot) = make_float4(src[0], src[1], src[2], src[3]);
           }
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            w[i] = sc.x * w[i] + sc.z * sv[i] + uw[i];
-            sv[i] = sc.y * sv[i] + us[i];
-          }
-          const long long gq = g + 16 * q16;
-#pragma unroll
-          for (int i4 = 0; i4 < 4; ++i4) {
-            *reinterpret_cast<float4 *>(Wl + gq + 4 * i4) = make_float4(w[4 * i4], w[4 * i4 + 1], w[4 * i4 + 2], w[4 * i4 + 3]);
-            *reinterpret_cast<float4 *>(Sl + gq + 4 * i4) = make_float4(sv[4 * i4], sv[4 * i4 + 1], sv[4 * i4 + 2], sv[4 * i4 + 3]);
-          }
-          __nv_bfloat16 *wb = a.Wbf + (long long)s * a.M * a.n_out + gq;
-          *reinterpret_cast<uint4 *>(wb) = pack8(w);
-          *reinterpret_cast<uint4 *>(wb + 8) = pack8(w + 8);
         }
       }
+      __syncthreads();
+      if (ok) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = dw_r0 + 16 * i;
+          const int wr = 128 * mt + r;
+          if (wr >= a.M) continue;
+          const int slot = dw_c4 ^ (r & 15);
+          const float4 u4 = *reinterpret_cast<const float4 *>(uw + r * 64 + 4 * slot);
+          const float4 v4 = *reinterpret_cast<const float4 *>(us + r * 64 + 4 * slot);
+          const float4 w4 = wpre[i], s4 = spre[i];
+          const float4 wn = make_float4(sc.x * w4.x + sc.z * s4.x + u4.x, sc.x * w4.y + sc.z * s4.y + u4.y,
+                                        sc.x * w4.z + sc.z * s4.z + u4.z, sc.x * w4.w + sc.z * s4.w + u4.w);
+          const float4 sn = make_float4(sc.y * s4.x + v4.x, sc.y * s4.y + v4.y, sc.y * s4.z + v4.z,
+                                        sc.y * s4.w + v4.w);
+          const long long g = (long long)wr * a.n_out + a.N * nt + 64 * pc + 4 * dw_c4;
+          *reinterpret_cast<float4 *>(Wl + g) = wn;
+          *reinterpret_cast<float4 *>(Sl + g) = sn;
+          *reinterpret_cast<uint2 *>(Wb + g) = make_uint2(pack_bf16(wn.x, wn.y), pack_bf16(wn.z, wn.w));
+        }
+        if (pc + 1 < npc) dw_prefetch(pc + 1);
+      }
+      __syncthreads();
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tm, ncols);
+}
+
+// Forward and backward phases: one launch per layer, grid = (column tiles,
+// row tiles, streams).
+template <int KIND>
+__global__ void __launch_bounds__(NT, 1)
+    tcl_gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap mA,
+                    const __grid_constant__ CUtensorMap mA2, const __grid_constant__ CUtensorMap mB) {
+  gemm_tile<KIND>(a, mA, mA2, mB, blockIdx.z, blockIdx.y, blockIdx.x);
+}
+
+// The update of every layer of a chunk in one launch: the layers' output
+// tiles are numbered one after another (layer, then stream, row tile, column
+// tile). Limited to 128 registers so that two CTAs share an SM; the fixed
+// latency of a tile (operand loads, MMAs, staging) is then hidden by the
+// tiles running beside it instead of being paid once per layer.
+struct DwGroup {
+  GemmArgs l[kMaxL];
+  int first[kMaxL + 1];              // first tile of each layer; first[L] = total
+  int mtiles[kMaxL], ntiles[kMaxL];
+  int L;
+};
+struct DwMaps {
+  CUtensorMap a[kMaxL], a2[kMaxL], b[kMaxL];
+};
+
+__global__ void __launch_bounds__(NT, 2)
+    tcl_dw_kernel(const __grid_constant__ DwGroup g, const __grid_constant__ DwMaps m) {
+  const int t = blockIdx.x;
+  int l = 0;
+  while (l + 1 < g.L && t >= g.first[l + 1]) ++l;
+  const int i = t - g.first[l];
+  const int per_stream = g.mtiles[l] * g.ntiles[l];
+  const int s = i / per_stream, j = i % per_stream;
+  gemm_tile<K_DW>(g.l[l], m.a[l], m.a2[l], m.b[l], s, j / g.ntiles[l], j % g.ntiles[l]);
+}
+
+// ------------------------------------------------------------------------
+// Fused forward + backward of one chunk, for memories whose every layer is at
+// most 256 wide. One CTA per (128-row tile of the chunk's [keys; queries],
+// stream) runs the whole chain that the per-phase kernels run as 2L - 1
+// launches: the tile's rows stay in shared memory (bf16, row-block layout,
+// overwritten in place by each epilogue) and the accumulator in TMEM, while
+// the bf16 weights stream through a ring of TMA stages whose prefetch runs
+// ahead across layer boundaries (the next layer's slices land during the
+// current epilogue). Rows of a tile are independent through every layer, so
+// no other CTA is involved.
+//   forward  l = 1..L: Z_l = X_{l-1} W_l^T (K-major W slices of 64 columns)
+//   backward l = L..2: G_{l-1} = (G_l W_l) . silu'(Z_{l-1}) (MN-major W slices
+//            of 64 rows); tiles without key rows stop after the forward.
+// Outputs are those the update GEMMs read: X_l and silu'(Z_l) of key rows,
+// -c G_l and -e G_l; and y for query rows.
+constexpr int FB_STAGES = 4;
+constexpr uint32_t FB_STAGE = 256 * KB * 2;          // 32 KB: one 64-wide slice of W_l
+constexpr uint32_t FB_ABUF = 128 * 256 * 2;          // 64 KB: the tile's rows
+constexpr size_t FB_SMEM = FB_ABUF + FB_STAGES * FB_STAGE + 1024;
+constexpr int FB_MAXD = 256;
+constexpr int FB_NT = 512;           // 16 warps: warp w reads TMEM lanes 32 (w % 4) .. +31,
+                                     // columns quarter w / 4 of the phase's output
+
+struct FbArgs {
+  int L, C, T, chunk;
+  int dims[kMaxL + 1];
+  __nv_bfloat16 *x_out[kMaxL + 1];   // [streams, 2C, d_l], key rows written (l = 1..L-1)
+  __nv_bfloat16 *sp_out[kMaxL + 1];  // [streams, C, d_l] silu'(Z_l) of key rows
+  __nv_bfloat16 *gc_out[kMaxL + 1];  // [streams, C, d_l] -c G_l
+  __nv_bfloat16 *ge_out[kMaxL + 1];  // [streams, C, d_l] -e G_l
+  float *y;                          // [streams, T, d]
+  const __nv_bfloat16 *v;            // [streams, T, d]
+  const float *coef;                 // [streams, T, 2]
+  int *status;
+  unsigned long long wait_ns;
+};
+
+struct FbMaps {
+  CUtensorMap k, q;
+  CUtensorMap w[kMaxL + 1];          // w[l]: bf16 W_l of every stream, [streams * d_l, d_{l-1}]
+};
+
+struct FbPhase {
+  int bwd, l, ns, N;                 // backward?, layer, 64-wide K slices, output width
+};
+
+__device__ __forceinline__ FbPhase fb_phase(const FbArgs &a, int p) {
+  FbPhase f;
+  if (p < a.L) {
+    f.bwd = 0; f.l = p + 1; f.ns = a.dims[p] / KB; f.N = a.dims[p + 1];
+  } else {
+    f.bwd = 1; f.l = a.L - (p - a.L); f.ns = a.dims[f.l] / KB; f.N = a.dims[f.l - 1];
+  }
+  return f;
+}
+
+// Issue the TMA loads of global weight slice g (counting slices over all
+// phases of this tile) into stage g % FB_STAGES.
+__device__ __forceinline__ void fb_load_slice(const FbArgs &a, const FbMaps &m, unsigned char *ring,
+                                              uint64_t *full, int s, int g) {
+  int p = 0, kb = g;
+  FbPhase f = fb_phase(a, 0);
+  while (kb >= f.ns) { kb -= f.ns; f = fb_phase(a, ++p); }
+  const int st = g % FB_STAGES;
+  unsigned char *dst = ring + st * FB_STAGE;
+  const CUtensorMap *mw = &m.w[f.l];
+  const int dl = a.dims[f.l];
+  mbar_arrive_expect_tx(&full[st], (uint32_t)f.N * KB * 2);
+  if (!f.bwd) {
+    for (int piece = 0; piece < f.N / 64; ++piece)   // rows of W_l, K-major slice kb
+      tma_load_2d(dst + piece * 64 * 128, mw, &full[st], kb * KB, s * dl + 64 * piece);
+  } else {
+    for (int blk = 0; blk < f.N / 64; ++blk)         // 64 rows (K) of W_l, MN-major
+      tma_load_2d(dst + blk * 64 * 128, mw, &full[st], 64 * blk, s * dl + kb * KB);
+  }
+}
+
+__device__ __forceinline__ void st_shared_v4(unsigned char *p, uint4 v) {
+  *reinterpret_cast<uint4 *>(p) = v;
+}
+
+__global__ void __launch_bounds__(FB_NT, 1)
+    tcl_fb_kernel(const __grid_constant__ FbArgs a, const __grid_constant__ FbMaps m) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char *abuf =
+      reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char *ring = abuf + FB_ABUF;
+  __shared__ uint64_t full[FB_STAGES], empty[FB_STAGES], xbar, done;
+  __shared__ uint32_t tslot;
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int mt = blockIdx.x, s = blockIdx.y;
+  const int C = a.C, L = a.L;
+  const bool has_keys = 128 * mt < C;
+  const int nphase = has_keys ? 2 * L - 1 : L;
+  int total = 0;
+  for (int p = 0; p < nphase; ++p) total += fb_phase(a, p).ns;
+
+  if (tid == 0) {
+    for (int i = 0; i < FB_STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    mbar_init(&xbar, 1);
+    mbar_init(&done, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) { tmem_alloc(&tslot, 256); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = tslot;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  int issued = 0, consumed = 0;      // weight slices (thread 0's bookkeeping)
+  bool x_waited = false;
+  if (tid == 0) {
+    prefetch_tmap(&m.k);
+    prefetch_tmap(&m.q);
+    // the tile's input rows: 64-row pieces of keys or queries
+    const int d0 = a.dims[0];
+    mbar_arrive_expect_tx(&xbar, (uint32_t)(128 * d0 * 2));
+    for (int piece = 0; piece < 2; ++piece) {
+      const int r = 128 * mt + 64 * piece;
+      const CUtensorMap *src = r < C ? &m.k : &m.q;
+      const int row = s * a.T + a.chunk * C + (r < C ? r : r - C);
+      for (int f = 0; f < d0 / 64; ++f)
+        tma_load_2d(abuf + f * 128 * 128 + piece * 64 * 128, src, &xbar, 64 * f, row);
+    }
+    for (; issued < total && issued < FB_STAGES; ++issued) fb_load_slice(a, m, ring, full, s, issued);
+  }
+
+  const int row = 32 * (warp & 3) + lane;        // TMEM lane = row of the tile
+  const uint32_t lb = (uint32_t)(32 * (warp & 3)) << 16;
+  const int quarter = warp >> 2;
+  const int r = 128 * mt + row;                  // row of the stream's [keys; queries]
+  const bool key = r < C;
+  const long long tok = (long long)s * a.T + (long long)a.chunk * C + (key ? r : r - C);
+  // key rows of this tile (keys precede queries) and their (c, e)
+  const int nkey = C - 128 * mt >= 128 ? 128 : (C - 128 * mt > 0 ? C - 128 * mt : 0);
+  __shared__ float2 cef[128];
+  if (tid < nkey)
+    cef[tid] = *reinterpret_cast<const float2 *>(a.coef + 2 * ((long long)s * a.T + (long long)a.chunk * C + 128 * mt + tid));
+  __syncthreads();
+
+  for (int p = 0; p < nphase; ++p) {
+    const FbPhase f = fb_phase(a, p);
+    if (tid == 0) {
+      bool ok = true;
+      if (!x_waited) {
+        ok = mbar_wait(&xbar, 0, a.wait_ns);
+        x_waited = true;
+      }
+      const uint32_t idesc = idesc_bf16(128, f.N, false, f.bwd != 0);
+      const uint32_t abase = smem_u32(abuf);
+      for (int kb = 0; kb < f.ns && ok; ++kb) {
+        const int g = consumed;
+        const int st = g % FB_STAGES;
+        const uint32_t ph = (uint32_t)((g / FB_STAGES) & 1);
+        if (!mbar_wait(&full[st], ph, a.wait_ns)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t bb = smem_u32(ring + st * FB_STAGE);
+        for (int ks = 0; ks < KB / 16; ++ks) {
+          const uint64_t ad = desc_kmajor(abase + kb * 128 * 128, 128, ks);
+          const uint64_t bd = f.bwd ? desc_mnmajor(bb, 64, ks) : desc_kmajor(bb, f.N, ks);
+          umma_bf16(tm, ad, bd, idesc, (kb | ks) != 0);
+        }
+        umma_commit(&empty[st]);
+        ++consumed;
+        // refill the stage of the previous slice (its MMAs have had the time of
+        // this slice's issue to finish), so two slices of MMAs overlap
+        while (ok && issued < total && issued - FB_STAGES <= g - 1) {
+          const int j = issued - FB_STAGES;
+          if (!mbar_wait(&empty[j % FB_STAGES], (uint32_t)((j / FB_STAGES) & 1), a.wait_ns)) ok = false;
+          else fb_load_slice(a, m, ring, full, s, issued++);
+        }
+      }
+      if (!ok) { atomicCAS(a.status, 0, kDevTimeout); abort_flag = 1; }
+      umma_commit(&done);
+      // the last slice's stage: refilled now, so the next phase's weights land
+      // during this phase's epilogue
+      while (ok && issued < total && issued - FB_STAGES <= consumed - 1) {
+        const int j = issued - FB_STAGES;
+        if (!mbar_wait(&empty[j % FB_STAGES], (uint32_t)((j / FB_STAGES) & 1), a.wait_ns)) {
+          ok = false;
+          atomicCAS(a.status, 0, kDevTimeout);
+          abort_flag = 1;
+        } else {
+          fb_load_slice(a, m, ring, full, s, issued++);
+        }
+      }
+    }
+    __syncwarp();
+    if (p == nphase - 1) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (!mbar_wait(&done, (uint32_t)(p & 1), a.wait_ns)) {
+      atomicCAS(a.status, 0, kDevTimeout);
+      abort_flag = 1;
+    }
+    tc_fence_after();
+    if (!*(volatile int *)&abort_flag) {
+      const int N = f.N, cbeg = quarter * (N / 4), cend = cbeg + N / 4;
+      const int lnch = N == 64 ? 3 : (N == 128 ? 4 : (N == 256 ? 5 : 0));   // log2 of the
+      const int nch = N / 8;                     // 16-byte chunks of a bf16 row (0: 192 wide)
+      const bool last_fwd = !f.bwd && f.l == L;
+      // Global traffic goes through the tile in shared memory, row-contiguous:
+      // consecutive threads move consecutive 16-byte chunks of a row.
+      auto rc_of = [&](int i, int &rr, int &ch) {
+        if (lnch) { rr = i >> lnch; ch = i & (nch - 1); }
+        else { rr = i / nch; ch = i - rr * nch; }
+      };
+      auto copy_in = [&](const __nv_bfloat16 *src, long long row0) {
+        for (int i = tid; i < nkey * nch; i += FB_NT) {
+          int rr, ch;
+          rc_of(i, rr, ch);
+          st_shared_v4(abuf + rb_chunk(128, rr, ch),
+                       *reinterpret_cast<const uint4 *>(src + (row0 + rr) * N + 8 * ch));
+        }
+      };
+      auto copy_out = [&](__nv_bfloat16 *dst, long long row0) {
+        for (int i = tid; i < nkey * nch; i += FB_NT) {
+          int rr, ch;
+          rc_of(i, rr, ch);
+          *reinterpret_cast<uint4 *>(dst + (row0 + rr) * N + 8 * ch) =
+              *reinterpret_cast<const uint4 *>(abuf + rb_chunk(128, rr, ch));
+        }
+      };
+      auto copy_out_scaled = [&](int lo) {      // -c G and -e G of the key rows
+        __nv_bfloat16 *gc = a.gc_out[lo], *ge = a.ge_out[lo];
+        const long long row0 = (long long)s * C + 128 * mt;
+        for (int i = tid; i < nkey * nch; i += FB_NT) {
+          int rr, ch;
+          rc_of(i, rr, ch);
+          const uint4 u = *reinterpret_cast<const uint4 *>(abuf + rb_chunk(128, rr, ch));
+          const __nv_bfloat16 *hb = reinterpret_cast<const __nv_bfloat16 *>(&u);
+          const float2 k2 = cef[rr];
+          float vc[8], ve[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float g = __bfloat162float(hb[j]);
+            vc[j] = -k2.x * g;
+            ve[j] = -k2.y * g;
+          }
+          const long long o = (row0 + rr) * N + 8 * ch;
+          *reinterpret_cast<uint4 *>(gc + o) = pack8(vc);
+          *reinterpret_cast<uint4 *>(ge + o) = pack8(ve);
+        }
+      };
+      // this thread's 16 TMEM columns starting at c0 (lane = row)
+      auto tld16 = [&](int c0, float (&z)[16]) {
+        tmem_ld16(tm + lb + c0, z);
+        tmem_wait_ld();
+      };
+      if (!f.bwd && !last_fwd) {
+        // hidden layer: silu'(Z) of key rows out first, then X = silu(Z) for
+        // every row (the next layer's operand) and out for key rows
+        if (nkey > 0) {
+          for (int c0 = cbeg; c0 < cend; c0 += 16) {
+            float z[16];
+            tld16(c0, z);
+            if (!key) continue;
+            float sp[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float sg = sigm(z[i]);
+              sp[i] = sg * (1.f + z[i] * (1.f - sg));
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i) st_shared_v4(abuf + rb_chunk(128, row, c0 / 8 + i), pack8(sp + 8 * i));
+          }
+          __syncthreads();
+          copy_out(a.sp_out[f.l], (long long)s * C + 128 * mt);
+          __syncthreads();
+        }
+        for (int c0 = cbeg; c0 < cend; c0 += 16) {
+          float z[16];
+          tld16(c0, z);
+          float x[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) x[i] = z[i] * sigm(z[i]);
+#pragma unroll
+          for (int i = 0; i < 2; ++i) st_shared_v4(abuf + rb_chunk(128, row, c0 / 8 + i), pack8(x + 8 * i));
+        }
+        if (nkey > 0) {
+          __syncthreads();
+          copy_out(a.x_out[f.l], (long long)s * 2 * C + 128 * mt);
+        }
+      } else {
+        // gradient rows: G_L = 2 (Z_L - V) or G_{l-1} = (G_l W_l) . silu'(Z_{l-1});
+        // the other operand comes into the tile first
+        const int lo = f.bwd ? f.l - 1 : L;
+        if (nkey > 0) {
+          if (f.bwd) copy_in(a.sp_out[lo], (long long)s * C + 128 * mt);
+          else copy_in(a.v, (long long)s * a.T + (long long)a.chunk * C + 128 * mt);
+          __syncthreads();
+        }
+        for (int c0 = cbeg; c0 < cend; c0 += 16) {
+          float z[16];
+          tld16(c0, z);
+          if (!key) {
+            if (last_fwd) {                      // query row of the last layer: the read y
+              float *yo = a.y + tok * N + c0;
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<float4 *>(yo + 4 * i) =
+                    make_float4(z[4 * i], z[4 * i + 1], z[4 * i + 2], z[4 * i + 3]);
+            }
+            continue;
+          }
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            unsigned char *cp = abuf + rb_chunk(128, row, c0 / 8 + i);
+            const uint4 u = *reinterpret_cast<const uint4 *>(cp);
+            const __nv_bfloat16 *hb = reinterpret_cast<const __nv_bfloat16 *>(&u);
+            float g[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float h = __bfloat162float(hb[j]);
+              g[j] = f.bwd ? z[8 * i + j] * h : 2.f * (z[8 * i + j] - h);
+            }
+            st_shared_v4(cp, pack8(g));
+          }
+        }
+        if (nkey > 0) {
+          __syncthreads();
+          copy_out_scaled(lo);
+        }
+      }
+    }
+    // the tile (generic-proxy writes) is read by the next phase's MMAs
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (*(volatile int *)&abort_flag) break;
+  }
+  if (tid == 0) {
+    // after an abort: wait (bounded) for the copies still in flight into this CTA
+    if (!x_waited) mbar_wait(&xbar, 0, a.wait_ns);
+    for (int g = consumed; g < issued; ++g)
+      mbar_wait(&full[g % FB_STAGES], (uint32_t)((g / FB_STAGES) & 1), a.wait_ns);
+  }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tm, 256);
 }
 
 // A5 for every chunk of every stream at once: one thread per (stream, chunk)
@@ -475,6 +889,26 @@ bool dims_ok(const Problem &p) {
 
 constexpr size_t SMEM_BYTES = 3 * STAGE_BYTES_DW + 1024;   // = 4 * STAGE_BYTES_MM + 1024
 
+bool fb_ok(const Problem &p) {
+  for (int l = 0; l <= p.L; ++l)
+    if (p.dims[l] > FB_MAXD) return false;
+  return true;
+}
+
+cudaError_t launch_fb(const FbArgs &a, const FbMaps &m, int streams, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * a.C / 128), (unsigned)streams);
+  cfg.blockDim = dim3(FB_NT);
+  cfg.dynamicSmemBytes = FB_SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tcl_fb_kernel, a, m);
+}
+
 cudaError_t launch_gemm(const GemmArgs &a, const CUtensorMap &mA, const CUtensorMap &mA2,
                         const CUtensorMap &mB, int streams, int mtiles, int ntiles, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
@@ -487,7 +921,26 @@ cudaError_t launch_gemm(const GemmArgs &a, const CUtensorMap &mA, const CUtensor
   at[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, tcl_gemm_kernel, a, mA, mA2, mB);
+  switch (a.kind) {
+    case K_FWD: return cudaLaunchKernelEx(&cfg, tcl_gemm_kernel<K_FWD>, a, mA, mA2, mB);
+    case K_FWD_LAST: return cudaLaunchKernelEx(&cfg, tcl_gemm_kernel<K_FWD_LAST>, a, mA, mA2, mB);
+    case K_BWD: return cudaLaunchKernelEx(&cfg, tcl_gemm_kernel<K_BWD>, a, mA, mA2, mB);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_dw(const DwGroup &g, const DwMaps &m, size_t smem, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)g.first[g.L]);
+  cfg.blockDim = dim3(NT);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tcl_dw_kernel, g, m);
 }
 
 }  // namespace
@@ -509,8 +962,14 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
   if (!tcl_supported(p)) return cudaErrorNotSupported;
   static bool attr_done = false;
   if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(tcl_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_BYTES);
+    cudaError_t e = cudaSuccess;
+    const void *kerns[4] = {(const void *)tcl_gemm_kernel<K_FWD>, (const void *)tcl_gemm_kernel<K_FWD_LAST>,
+                            (const void *)tcl_gemm_kernel<K_BWD>, (const void *)tcl_dw_kernel};
+    for (const void *k : kerns) {
+      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+    }
+    e = cudaFuncSetAttribute(tcl_fb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FB_SMEM);
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
@@ -577,9 +1036,69 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
   base.y = p.y;
   base.v = reinterpret_cast<const __nv_bfloat16 *>(p.v);
 
-  for (int ch = 0; ch < nchunks; ++ch) {
-    // forward of keys and queries, layer by layer
+  // the update launch: per layer, tiles of 128 rows of W_l x (128 or 64) columns
+  DwGroup dg;
+  DwMaps dm;
+  std::memset(&dg, 0, sizeof dg);
+  std::memset(&dm, 0, sizeof dm);
+  dg.L = L;
+  size_t dw_smem = 0;
+  for (int l = 1; l <= L; ++l) {
+    GemmArgs &a = dg.l[l - 1];
+    a = base;
+    const int nl = p.dims[l], np = p.dims[l - 1];
+    a.kind = K_DW;
+    a.N = np % DW_MAXN == 0 ? DW_MAXN : 64;
+    a.K = C;
+    a.M = nl;
+    a.n_out = np;
+    a.a_rows_per_stream = C;
+    a.b_rows_per_stream = l == 1 ? T : 2 * C;
+    a.layer_off = (long long)p.layer_off[l - 1];
+    a.Wbf = wbf + ia.boff[l - 1];
+    dg.mtiles[l - 1] = (nl + 127) / 128;
+    dg.ntiles[l - 1] = np / a.N;
+    dg.first[l] = dg.first[l - 1] + S * dg.mtiles[l - 1] * dg.ntiles[l - 1];
+    dm.a[l - 1] = mgc[l];
+    dm.a2[l - 1] = mge[l];
+    dm.b[l - 1] = l == 1 ? mk : mx[l - 1];
+    const size_t sm = (size_t)dw_stages(C / KB) * dw_stage_bytes(a.N) + 1024;
+    if (sm > dw_smem) dw_smem = sm;
+  }
+
+  const bool fused = p.fuse_fb && fb_ok(p);
+  FbArgs fa;
+  FbMaps fm;
+  if (fused) {
+    std::memset(&fa, 0, sizeof fa);
+    std::memset(&fm, 0, sizeof fm);
+    fa.L = L;
+    fa.C = C;
+    fa.T = T;
+    for (int l = 0; l <= L; ++l) fa.dims[l] = p.dims[l];
     for (int l = 1; l <= L; ++l) {
+      if (l < L) { fa.x_out[l] = bf(cv.x[l]); fa.sp_out[l] = bf(cv.sp[l]); }
+      fa.gc_out[l] = bf(cv.gc[l]);
+      fa.ge_out[l] = bf(cv.ge[l]);
+      fm.w[l] = mwb[l];
+    }
+    fm.k = mk;
+    fm.q = mq;
+    fa.y = p.y;
+    fa.v = reinterpret_cast<const __nv_bfloat16 *>(p.v);
+    fa.coef = coef;
+    fa.status = p.status;
+    fa.wait_ns = g_tcl_wait_ns;
+  }
+
+  for (int ch = 0; ch < nchunks; ++ch) {
+    if (fused) {
+      fa.chunk = ch;
+      err = launch_fb(fa, fm, S, stream);
+      if (err != cudaSuccess) return err;
+    }
+    // forward of keys and queries, layer by layer
+    for (int l = 1; l <= L && !fused; ++l) {
       GemmArgs a = base;
       const int nl = p.dims[l], np = p.dims[l - 1];
       a.kind = l < L ? K_FWD : K_FWD_LAST;
@@ -597,7 +1116,7 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
       if (err != cudaSuccess) return err;
     }
     // backward to every hidden layer
-    for (int l = L; l >= 2; --l) {
+    for (int l = L; l >= 2 && !fused; --l) {
       GemmArgs a = base;
       const int nl = p.dims[l], np = p.dims[l - 1];
       a.kind = K_BWD;
@@ -613,24 +1132,13 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
       err = launch_gemm(a, mg[l], mg[l], mwb[l], S, (C + 127) / 128, np / a.N, stream);
       if (err != cudaSuccess) return err;
     }
-    // weight-update contractions with the fused state update
+    // weight-update contractions of every layer, with the fused state update
     for (int l = 1; l <= L; ++l) {
-      GemmArgs a = base;
-      const int nl = p.dims[l], np = p.dims[l - 1];
-      a.kind = K_DW;
-      a.chunk = ch;
-      a.N = tile_for(np, (nl + 127) / 128);
-      a.K = C;
-      a.M = nl;
-      a.n_out = np;
-      a.a_rows_per_stream = C;
-      a.b_rows_per_stream = l == 1 ? T : 2 * C;
-      a.b_row_off = l == 1 ? (long long)ch * C : 0;
-      a.layer_off = (long long)p.layer_off[l - 1];
-      a.Wbf = wbf + ia.boff[l - 1];
-      err = launch_gemm(a, mgc[l], mge[l], l == 1 ? mk : mx[l - 1], S, (nl + 127) / 128, np / a.N, stream);
-      if (err != cudaSuccess) return err;
+      dg.l[l - 1].chunk = ch;
+      dg.l[l - 1].b_row_off = l == 1 ? (long long)ch * C : 0;
     }
+    err = launch_dw(dg, dm, dw_smem, stream);
+    if (err != cudaSuccess) return err;
   }
   return cudaSuccess;
 }

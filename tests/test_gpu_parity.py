@@ -159,7 +159,7 @@ def test_full_size_workloads(idx, sample_streams, prefix):
     if sample_streams is not None:
         del inp
     mem = NeuralMemory(w.L, w.d, w.expansion, path="auto")
-    tol = TOL_BF16_TC if mem.query_path(w.B, w.H, w.T, w.C) in ("tc", "tcl") else TOL_F32
+    tol = TOL_BF16_TC if mem.query_path(w.B, w.H, w.T, w.C) in ("tc", "tcl", "tcl-phased") else TOL_F32
     y, We, Se = run_lib(mem, dev, w.C)
     assert torch.isfinite(y).all() and torch.isfinite(We).all() and torch.isfinite(Se).all()
     if sample_streams is None:
@@ -184,7 +184,7 @@ def test_all_streams_short_stream_state(idx, sample_streams, T):
     inp = W.generate(w, T=T)
     dev = to_dev(inp, w.B, w.H, w.dtype)
     mem = NeuralMemory(w.L, w.d, w.expansion, path="auto")
-    tol = TOL_BF16_TC if mem.query_path(w.B, w.H, T, w.C) in ("tc", "tcl") else TOL_F32
+    tol = TOL_BF16_TC if mem.query_path(w.B, w.H, T, w.C) in ("tc", "tcl", "tcl-phased") else TOL_F32
     y, We, Se = run_lib(mem, dev, w.C)
     gpu = gpu_to_np(y, We, Se)
     sub = {k: (v[sample_streams] if k != "streams" else v) for k, v in inp.items()}
@@ -273,11 +273,30 @@ TCL_SHAPES = [  # L, d, expansion, B, H, T, C
 ]
 
 
+@pytest.mark.parametrize("path", ["tcl", "tcl-phased"])
 @pytest.mark.parametrize("cfg", TCL_SHAPES, ids=lambda c: "L%d-d%d-e%d-B%dH%d-T%d-C%d" % c)
-def test_tcl_small_shapes(cfg):
+def test_tcl_small_shapes(cfg, path):
+    """Layered path; "tcl" runs the fused forward + backward kernel wherever
+    every width is at most 256, "tcl-phased" one launch per phase."""
     L, d, e, B, H, T, C = cfg
     w = W.make(L, d, e, B, H, T, C, index=600 + sum(cfg))
-    check(w, "tcl", TOL_BF16_TC)
+    check(w, path, TOL_BF16_TC)
+
+
+def test_tcl_fused_matches_phased():
+    """The fused forward + backward kernel against the per-phase launches on
+    the deep workload's layer shapes. Both round G to bf16 for the next MMA;
+    the fused kernel forms -c G and -e G from that bf16 G (one more rounding,
+    at most half a bf16 ulp per element) where the per-phase one scales the
+    fp32 G, hence a bound a little above bf16 resolution."""
+    w = W.make(4, 128, 2, 2, 2, 512, 128, index=630)
+    inp, dev = _dev_inputs(w)
+    out = {}
+    for path in ("tcl", "tcl-phased"):
+        mem = NeuralMemory(w.L, w.d, w.expansion, path=path)
+        out[path] = gpu_to_np(*run_lib(mem, dev, w.C))
+    errs = parity_errors(w.dims, inp["W0"], out["tcl"], out["tcl-phased"])
+    assert max(errs.values()) < 5e-3, errs
 
 
 def test_tcl_literal_gates_short_stream():
