@@ -259,18 +259,6 @@ def sweep_chunk(args, w: W.Workload, sizes):
                           "workspace_bytes": ws.numel()}), flush=True)
 
 
-def launches_per_run(w: W.Workload, path: str) -> int:
-    """Kernels of this library per tm_run: one persistent kernel (cluster or
-    CUDA-core path); for the layered path an init and a coefficient kernel,
-    then per chunk either one fused forward + backward launch and L update
-    launches (every width at most 256) or 3L - 1 phase launches."""
-    if path not in ("tcl", "tcl-phased"):
-        return 1
-    fused = path == "tcl" and max(w.dims) <= 256
-    per_chunk = 1 + w.L if fused else 3 * w.L - 1
-    return 2 + per_chunk * (w.T // w.C)
-
-
 def bench_prologue(args, w: W.Workload):
     """The step before the memory on the workload's k, v, q: one fused launch of
     the depthwise causal convolution (width args.conv_width) and the L2
@@ -409,7 +397,7 @@ def main():
     ms_max = max_over_ranks(ms, world)
 
     cnt = algorithmic_counts(w, w.T)
-    launches_per_step = launches_per_run(w, path_used)
+    launches_per_step = mem.launch_count(w.B, w.H, w.T, w.C, d_in["k"].dtype)
     value = aggregate_throughput(cnt["tokens"], world, ms_max * 1e-3)
     peaks = measured_peaks()
     hbm = peaks["hbm_gbs"] * 1e9

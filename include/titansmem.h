@@ -105,6 +105,17 @@ TM_API tm_status tm_query_path(const tm_ctx *ctx, int B, int H, int T, int C, tm
                         tm_path *out);
 
 /*
+ * Number of kernel launches one tm_run of this problem makes (no counterpart
+ * in the method's description; for profiling and accounting). Host-only;
+ * same errors as tm_query_path. The layered paths split the B*H streams into
+ * up to 8 groups run on concurrent CUDA streams (one group's forward and
+ * backward beside another group's update); the environment variable
+ * TM_TCL_GROUPS (1..8), read once per process, overrides the split.
+ */
+TM_API tm_status tm_launch_count(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype,
+                                 long long *out);
+
+/*
  * Bytes of device workspace tm_run needs for this problem. Host-only. The
  * workspace holds the device status word (first 256 bytes) plus per-stream
  * activations of the CUDA-core path.

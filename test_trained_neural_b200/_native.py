@@ -26,6 +26,7 @@ SIGNATURES = {
     "tm_param_count": (_SZ, [_P]),
     "tm_set_path": (_I, [_P, _I]),
     "tm_query_path": (_I, [_P, _I, _I, _I, _I, _I, ctypes.POINTER(_I)]),
+    "tm_launch_count": (_I, [_P, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_longlong)]),
     "tm_workspace_size": (_I, [_P, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]),
     "tm_run": (_I, [_P, _I, _I, _I, _I, _I] + [_P] * 11 + [_P, _SZ, _P]),
     "tm_run_noalloc": (_I, [_P, _I, _I, _I, _I, _I] + [_P] * 11 + [_P]),

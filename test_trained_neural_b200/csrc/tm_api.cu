@@ -15,6 +15,12 @@ struct tm_ctx {
   size_t layer_off[tmem::kMaxL + 1];
   size_t P;
   tm_path path;
+  // layered path: side CUDA streams and events, created on first use on
+  // device `dev`; one context's calls must not run concurrently
+  int dev = -1;
+  cudaStream_t side[tmem::kMaxGroups - 1] = {};
+  cudaEvent_t ev_fork = nullptr;
+  cudaEvent_t ev_join[tmem::kMaxGroups - 1] = {};
 };
 
 namespace {
@@ -112,7 +118,42 @@ tm_status tm_create(int L, int d_h, int expansion, tm_act act, tm_ctx **out) {
   return TM_OK;
 }
 
+namespace {
+
+void release_side(tm_ctx *ctx) {
+  for (int i = 0; i < tmem::kMaxGroups - 1; ++i) {
+    if (ctx->side[i]) cudaStreamDestroy(ctx->side[i]);
+    if (ctx->ev_join[i]) cudaEventDestroy(ctx->ev_join[i]);
+    ctx->side[i] = nullptr;
+    ctx->ev_join[i] = nullptr;
+  }
+  if (ctx->ev_fork) cudaEventDestroy(ctx->ev_fork);
+  ctx->ev_fork = nullptr;
+  ctx->dev = -1;
+}
+
+// Side streams and events for `groups` concurrent groups, on the current device.
+bool ensure_side(tm_ctx *ctx, int groups) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (ctx->dev != dev) release_side(ctx);
+  ctx->dev = dev;
+  if (groups > 1 && !ctx->ev_fork &&
+      cudaEventCreateWithFlags(&ctx->ev_fork, cudaEventDisableTiming) != cudaSuccess)
+    return false;
+  for (int i = 0; i < groups - 1; ++i) {
+    if (!ctx->side[i] && cudaStreamCreateWithFlags(&ctx->side[i], cudaStreamNonBlocking) != cudaSuccess)
+      return false;
+    if (!ctx->ev_join[i] && cudaEventCreateWithFlags(&ctx->ev_join[i], cudaEventDisableTiming) != cudaSuccess)
+      return false;
+  }
+  return true;
+}
+
+}  // namespace
+
 tm_status tm_destroy(tm_ctx *ctx) {
+  if (ctx) release_side(ctx);
   delete ctx;
   return TM_OK;
 }
@@ -137,6 +178,19 @@ tm_status tm_query_path(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype 
   tm_path path = choose_path(ctx, p);
   if (!path_supported(path, p)) return TM_ERR_UNSUPPORTED;
   *out = path;
+  return TM_OK;
+}
+
+tm_status tm_launch_count(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype,
+                          long long *out) {
+  if (!out) return TM_ERR_INVALID_ARG;
+  tm_status st = check_shape(ctx, B, H, T, C, in_dtype);
+  if (st != TM_OK) return st;
+  tmem::Problem p = make_problem(ctx, B, H, T, C, in_dtype);
+  tm_path path = choose_path(ctx, p);
+  if (!path_supported(path, p)) return TM_ERR_UNSUPPORTED;
+  p.fuse_fb = path == TM_PATH_TC_LAYERED;
+  *out = (path == TM_PATH_TC_LAYERED || path == TM_PATH_TC_PHASED) ? tmem::tcl_launch_count(p) : 1;
   return TM_OK;
 }
 
@@ -207,6 +261,17 @@ tm_status tm_run(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype, con
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(p.status, 0, sizeof(int), s) != cudaSuccess) return TM_ERR_CUDA;
   p.fuse_fb = path == TM_PATH_TC_LAYERED;
+  if (path == TM_PATH_TC_LAYERED || path == TM_PATH_TC_PHASED) {
+    const int groups = tmem::tcl_group_count(p);
+    if (groups > 1) {
+      if (!ensure_side(ctx, groups)) return TM_ERR_CUDA;
+      for (int i = 0; i < groups - 1; ++i) {
+        p.side_streams[i] = ctx->side[i];
+        p.ev_join[i] = ctx->ev_join[i];
+      }
+      p.ev_fork = ctx->ev_fork;
+    }
+  }
   cudaError_t err = path == TM_PATH_TC ? tmem::tc_launch(p, s)
                     : (path == TM_PATH_TC_LAYERED || path == TM_PATH_TC_PHASED) ? tmem::tcl_launch(p, s)
                                                                               : tmem::simt_launch(p, s);

@@ -11,6 +11,7 @@ namespace tmem {
 
 constexpr int kMaxL = 4;
 constexpr int kMaxC = 256;
+constexpr int kMaxGroups = 8;         // layered path: concurrent groups of streams
 constexpr size_t kStatusBytes = 256;  // device status word lives here
 
 // Device status codes written by kernels (first error wins).
@@ -35,6 +36,11 @@ struct Problem {
   int *status;            // device status word
   void *scratch;          // per-stream activations (SIMT path)
   int fuse_fb;            // layered path: fused forward + backward launch where supported
+  // layered path: CUDA streams and events (owned by the context) for groups
+  // 1.. of the streams; group 0 runs on the caller's stream
+  void *side_streams[kMaxGroups - 1];
+  void *ev_fork;
+  void *ev_join[kMaxGroups - 1];
   size_t scratch_bytes;
 };
 
@@ -49,10 +55,12 @@ cudaError_t simt_launch(const Problem &p, cudaStream_t stream);
 bool tc_supported(const Problem &p);
 size_t tc_scratch_bytes(const Problem &p);
 cudaError_t tc_launch(const Problem &p, cudaStream_t stream);
-// Layer-by-layer tensor-core path (batched tcgen05 GEMMs per phase).
+// Layer-by-layer tensor-core path 
 bool tcl_supported(const Problem &p);
 size_t tcl_scratch_bytes(const Problem &p);
 cudaError_t tcl_launch(const Problem &p, cudaStream_t stream);
+int tcl_group_count(const Problem &p);   // CUDA streams tcl_launch uses
+long long tcl_launch_count(const Problem &p);
 void tcl_set_wait(unsigned long long wait_ns);
 
 // Depthwise causal convolution + L2 normalisation before the memory.

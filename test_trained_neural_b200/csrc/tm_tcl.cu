@@ -18,7 +18,9 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <cstdlib>
 #include <cstring>
+#include <vector>
 
 #include "tm_internal.h"
 #include "tm_sm100.cuh"
@@ -437,8 +439,9 @@ constexpr uint32_t FB_STAGE = 256 * KB * 2;          // 32 KB: one 64-wide slice
 constexpr uint32_t FB_ABUF = 128 * 256 * 2;          // 64 KB: the tile's rows
 constexpr size_t FB_SMEM = FB_ABUF + FB_STAGES * FB_STAGE + 1024;
 constexpr int FB_MAXD = 256;
-constexpr int FB_NT = 512;           // 16 warps: warp w reads TMEM lanes 32 (w % 4) .. +31,
-                                     // columns quarter w / 4 of the phase's output
+constexpr int FB_EPI = 512;          // 16 epilogue warps: warp w reads TMEM lanes 32 (w % 4) ..
+                                     // +31, columns quarter w / 4 of the phase's output
+constexpr int FB_NT = FB_EPI + 32;   // and one producer warp (TMA loads, MMA issue)
 
 struct FbArgs {
   int L, C, T, chunk;
@@ -498,27 +501,31 @@ __device__ __forceinline__ void st_shared_v4(unsigned char *p, uint4 v) {
   *reinterpret_cast<uint4 *>(p) = v;
 }
 
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(FB_EPI) : "memory"); }
+
 __global__ void __launch_bounds__(FB_NT, 1)
     tcl_fb_kernel(const __grid_constant__ FbArgs a, const __grid_constant__ FbMaps m) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *abuf =
       reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char *ring = abuf + FB_ABUF;
-  __shared__ uint64_t full[FB_STAGES], empty[FB_STAGES], xbar, done;
+  __shared__ uint64_t full[FB_STAGES], empty[FB_STAGES], xbar, done, ready;
   __shared__ uint32_t tslot;
   __shared__ int abort_flag;
+  __shared__ float2 cef[128];
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int mt = blockIdx.x, s = blockIdx.y;
   const int C = a.C, L = a.L;
   const bool has_keys = 128 * mt < C;
   const int nphase = has_keys ? 2 * L - 1 : L;
-  int total = 0;
-  for (int p = 0; p < nphase; ++p) total += fb_phase(a, p).ns;
+  // key rows of this tile (keys precede queries)
+  const int nkey = C - 128 * mt >= 128 ? 128 : (C - 128 * mt > 0 ? C - 128 * mt : 0);
 
   if (tid == 0) {
     for (int i = 0; i < FB_STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     mbar_init(&xbar, 1);
     mbar_init(&done, 1);
+    mbar_init(&ready, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -529,125 +536,97 @@ __global__ void __launch_bounds__(FB_NT, 1)
   const uint32_t tm = tslot;
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  int issued = 0, consumed = 0;      // weight slices (thread 0's bookkeeping)
-  bool x_waited = false;
-  if (tid == 0) {
-    prefetch_tmap(&m.k);
-    prefetch_tmap(&m.q);
-    // the tile's input rows: 64-row pieces of keys or queries
-    const int d0 = a.dims[0];
-    mbar_arrive_expect_tx(&xbar, (uint32_t)(128 * d0 * 2));
-    for (int piece = 0; piece < 2; ++piece) {
-      const int r = 128 * mt + 64 * piece;
-      const CUtensorMap *src = r < C ? &m.k : &m.q;
-      const int row = s * a.T + a.chunk * C + (r < C ? r : r - C);
-      for (int f = 0; f < d0 / 64; ++f)
-        tma_load_2d(abuf + f * 128 * 128 + piece * 64 * 128, src, &xbar, 64 * f, row);
-    }
-    for (; issued < total && issued < FB_STAGES; ++issued) fb_load_slice(a, m, ring, full, s, issued);
-  }
-
-  const int row = 32 * (warp & 3) + lane;        // TMEM lane = row of the tile
-  const uint32_t lb = (uint32_t)(32 * (warp & 3)) << 16;
-  const int quarter = warp >> 2;
-  const int r = 128 * mt + row;                  // row of the stream's [keys; queries]
-  const bool key = r < C;
-  const long long tok = (long long)s * a.T + (long long)a.chunk * C + (key ? r : r - C);
-  // key rows of this tile (keys precede queries) and their (c, e)
-  const int nkey = C - 128 * mt >= 128 ? 128 : (C - 128 * mt > 0 ? C - 128 * mt : 0);
-  __shared__ float2 cef[128];
-  if (tid < nkey)
-    cef[tid] = *reinterpret_cast<const float2 *>(a.coef + 2 * ((long long)s * a.T + (long long)a.chunk * C + 128 * mt + tid));
-  __syncthreads();
-
-  for (int p = 0; p < nphase; ++p) {
-    const FbPhase f = fb_phase(a, p);
-    if (tid == 0) {
+  if (warp == FB_EPI / 32) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int total = 0;
+      for (int p = 0; p < nphase; ++p) total += fb_phase(a, p).ns;
+      int issued = 0, consumed = 0;
+      prefetch_tmap(&m.k);
+      prefetch_tmap(&m.q);
+      const int d0 = a.dims[0];
+      mbar_arrive_expect_tx(&xbar, (uint32_t)(128 * d0 * 2));
+      for (int piece = 0; piece < 2; ++piece) {
+        const int r = 128 * mt + 64 * piece;
+        const CUtensorMap *src = r < C ? &m.k : &m.q;
+        const int row = s * a.T + a.chunk * C + (r < C ? r : r - C);
+        for (int f = 0; f < d0 / 64; ++f)
+          tma_load_2d(abuf + f * 128 * 128 + piece * 64 * 128, src, &xbar, 64 * f, row);
+      }
+      for (; issued < total && issued < FB_STAGES; ++issued) fb_load_slice(a, m, ring, full, s, issued);
       bool ok = true;
-      if (!x_waited) {
-        ok = mbar_wait(&xbar, 0, a.wait_ns);
-        x_waited = true;
-      }
-      const uint32_t idesc = idesc_bf16(128, f.N, false, f.bwd != 0);
-      const uint32_t abase = smem_u32(abuf);
-      for (int kb = 0; kb < f.ns && ok; ++kb) {
-        const int g = consumed;
-        const int st = g % FB_STAGES;
-        const uint32_t ph = (uint32_t)((g / FB_STAGES) & 1);
-        if (!mbar_wait(&full[st], ph, a.wait_ns)) { ok = false; break; }
+      for (int p = 0; p < nphase && ok; ++p) {
+        const FbPhase f = fb_phase(a, p);
+        // the tile holds this phase's A operand: the input rows, or the
+        // previous epilogue's output
+        ok = p == 0 ? mbar_wait(&xbar, 0, a.wait_ns) : mbar_wait(&ready, (uint32_t)((p - 1) & 1), a.wait_ns);
         tc_fence_after();
-        const uint32_t bb = smem_u32(ring + st * FB_STAGE);
-        for (int ks = 0; ks < KB / 16; ++ks) {
-          const uint64_t ad = desc_kmajor(abase + kb * 128 * 128, 128, ks);
-          const uint64_t bd = f.bwd ? desc_mnmajor(bb, 64, ks) : desc_kmajor(bb, f.N, ks);
-          umma_bf16(tm, ad, bd, idesc, (kb | ks) != 0);
+        const uint32_t idesc = idesc_bf16(128, f.N, false, f.bwd != 0);
+        const uint32_t abase = smem_u32(abuf);
+        // A phase has at most FB_STAGES slices and all of them were requested
+        // before it began (the refills below run a phase ahead), so the MMAs
+        // of a phase issue back to back.
+        for (int kb = 0; kb < f.ns && ok; ++kb) {
+          const int g = consumed;
+          const int st = g % FB_STAGES;
+          if (!mbar_wait(&full[st], (uint32_t)((g / FB_STAGES) & 1), a.wait_ns)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t bb = smem_u32(ring + st * FB_STAGE);
+          for (int ks = 0; ks < KB / 16; ++ks) {
+            const uint64_t ad = desc_kmajor(abase + kb * 128 * 128, 128, ks);
+            const uint64_t bd = f.bwd ? desc_mnmajor(bb, 64, ks) : desc_kmajor(bb, f.N, ks);
+            umma_bf16(tm, ad, bd, idesc, (kb | ks) != 0);
+          }
+          umma_commit(&empty[st]);
+          ++consumed;
         }
-        umma_commit(&empty[st]);
-        ++consumed;
-        // refill the stage of the previous slice (its MMAs have had the time of
-        // this slice's issue to finish), so two slices of MMAs overlap
-        while (ok && issued < total && issued - FB_STAGES <= g - 1) {
+        if (!ok) { atomicCAS(a.status, 0, kDevTimeout); abort_flag = 1; }
+        umma_commit(&done);
+        // refill the consumed stages with the next phase's slices as the MMAs
+        // finish; they land while the epilogue runs
+        while (ok && issued < total && issued - FB_STAGES <= consumed - 1) {
           const int j = issued - FB_STAGES;
-          if (!mbar_wait(&empty[j % FB_STAGES], (uint32_t)((j / FB_STAGES) & 1), a.wait_ns)) ok = false;
-          else fb_load_slice(a, m, ring, full, s, issued++);
+          if (!mbar_wait(&empty[j % FB_STAGES], (uint32_t)((j / FB_STAGES) & 1), a.wait_ns)) {
+            ok = false;
+            atomicCAS(a.status, 0, kDevTimeout);
+            abort_flag = 1;
+          } else {
+            fb_load_slice(a, m, ring, full, s, issued++);
+          }
         }
       }
-      if (!ok) { atomicCAS(a.status, 0, kDevTimeout); abort_flag = 1; }
-      umma_commit(&done);
-      // the last slice's stage: refilled now, so the next phase's weights land
-      // during this phase's epilogue
-      while (ok && issued < total && issued - FB_STAGES <= consumed - 1) {
-        const int j = issued - FB_STAGES;
-        if (!mbar_wait(&empty[j % FB_STAGES], (uint32_t)((j / FB_STAGES) & 1), a.wait_ns)) {
-          ok = false;
-          atomicCAS(a.status, 0, kDevTimeout);
-          abort_flag = 1;
-        } else {
-          fb_load_slice(a, m, ring, full, s, issued++);
-        }
-      }
+      // after an abort: wait (bounded) for the copies still in flight into this CTA
+      for (int g = consumed; g < issued; ++g)
+        mbar_wait(&full[g % FB_STAGES], (uint32_t)((g / FB_STAGES) & 1), a.wait_ns);
     }
     __syncwarp();
-    if (p == nphase - 1) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (!mbar_wait(&done, (uint32_t)(p & 1), a.wait_ns)) {
-      atomicCAS(a.status, 0, kDevTimeout);
-      abort_flag = 1;
-    }
-    tc_fence_after();
-    if (!*(volatile int *)&abort_flag) {
-      const int N = f.N, cbeg = quarter * (N / 4), cend = cbeg + N / 4;
-      const int lnch = N == 64 ? 3 : (N == 128 ? 4 : (N == 256 ? 5 : 0));   // log2 of the
-      const int nch = N / 8;                     // 16-byte chunks of a bf16 row (0: 192 wide)
-      const bool last_fwd = !f.bwd && f.l == L;
-      // Global traffic goes through the tile in shared memory, row-contiguous:
-      // consecutive threads move consecutive 16-byte chunks of a row.
-      auto rc_of = [&](int i, int &rr, int &ch) {
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int row = 32 * (warp & 3) + lane;      // TMEM lane = row of the tile
+    const uint32_t lb = (uint32_t)(32 * (warp & 3)) << 16;
+    const int quarter = warp >> 2;
+    const int r = 128 * mt + row;                // row of the stream's [keys; queries]
+    const bool key = r < C;
+    const long long tok = (long long)s * a.T + (long long)a.chunk * C + (key ? r : r - C);
+    if (tid < nkey)
+      cef[tid] = *reinterpret_cast<const float2 *>(a.coef + 2 * ((long long)s * a.T + (long long)a.chunk * C + 128 * mt + tid));
+    epi_sync();
+    // Global traffic of the tile's outputs that the update reads (X, -c G,
+    // -e G) leaves from the tile in shared memory, row-contiguous, after the
+    // next phase's MMAs have been released (they only read the tile too).
+    int pend_kind = 0, pend_l = 0, pend_N = 0;   // 1: X_l, 2: -c G_l and -e G_l
+    auto flush = [&]() {
+      if (!pend_kind || nkey == 0) return;
+      const int N = pend_N, nch = N / 8;
+      const int lnch = N == 64 ? 3 : (N == 128 ? 4 : (N == 256 ? 5 : 0));
+      for (int i = tid; i < nkey * nch; i += FB_EPI) {
+        int rr, ch;
         if (lnch) { rr = i >> lnch; ch = i & (nch - 1); }
         else { rr = i / nch; ch = i - rr * nch; }
-      };
-      auto copy_in = [&](const __nv_bfloat16 *src, long long row0) {
-        for (int i = tid; i < nkey * nch; i += FB_NT) {
-          int rr, ch;
-          rc_of(i, rr, ch);
-          st_shared_v4(abuf + rb_chunk(128, rr, ch),
-                       *reinterpret_cast<const uint4 *>(src + (row0 + rr) * N + 8 * ch));
-        }
-      };
-      auto copy_out = [&](__nv_bfloat16 *dst, long long row0) {
-        for (int i = tid; i < nkey * nch; i += FB_NT) {
-          int rr, ch;
-          rc_of(i, rr, ch);
-          *reinterpret_cast<uint4 *>(dst + (row0 + rr) * N + 8 * ch) =
-              *reinterpret_cast<const uint4 *>(abuf + rb_chunk(128, rr, ch));
-        }
-      };
-      auto copy_out_scaled = [&](int lo) {      // -c G and -e G of the key rows
-        __nv_bfloat16 *gc = a.gc_out[lo], *ge = a.ge_out[lo];
-        const long long row0 = (long long)s * C + 128 * mt;
-        for (int i = tid; i < nkey * nch; i += FB_NT) {
-          int rr, ch;
-          rc_of(i, rr, ch);
-          const uint4 u = *reinterpret_cast<const uint4 *>(abuf + rb_chunk(128, rr, ch));
+        const uint4 u = *reinterpret_cast<const uint4 *>(abuf + rb_chunk(128, rr, ch));
+        if (pend_kind == 1) {
+          *reinterpret_cast<uint4 *>(a.x_out[pend_l] + ((long long)s * 2 * C + 128 * mt + rr) * N + 8 * ch) = u;
+        } else {
           const __nv_bfloat16 *hb = reinterpret_cast<const __nv_bfloat16 *>(&u);
           const float2 k2 = cef[rr];
           float vc[8], ve[8];
@@ -657,76 +636,73 @@ __global__ void __launch_bounds__(FB_NT, 1)
             vc[j] = -k2.x * g;
             ve[j] = -k2.y * g;
           }
-          const long long o = (row0 + rr) * N + 8 * ch;
-          *reinterpret_cast<uint4 *>(gc + o) = pack8(vc);
-          *reinterpret_cast<uint4 *>(ge + o) = pack8(ve);
+          const long long o = ((long long)s * C + 128 * mt + rr) * N + 8 * ch;
+          *reinterpret_cast<uint4 *>(a.gc_out[pend_l] + o) = pack8(vc);
+          *reinterpret_cast<uint4 *>(a.ge_out[pend_l] + o) = pack8(ve);
         }
-      };
-      // this thread's 16 TMEM columns starting at c0 (lane = row)
-      auto tld16 = [&](int c0, float (&z)[16]) {
+      }
+      pend_kind = 0;
+    };
+    for (int p = 0; p < nphase; ++p) {
+      const FbPhase f = fb_phase(a, p);
+      const int N = f.N, cbeg = quarter * (N / 4), cend = cbeg + N / 4;
+      const bool last_fwd = !f.bwd && f.l == L;
+      const bool grad = f.bwd || last_fwd;
+      // this thread's other operand of a gradient phase (V, or silu' of the
+      // layer below, which this same thread stored going forward), requested
+      // before the MMAs finish
+      uint4 aux[8];
+      if (grad && key) {
+        const __nv_bfloat16 *src = f.bwd ? a.sp_out[f.l - 1] + ((long long)s * C + r) * N
+                                         : a.v + tok * N;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (8 * i < N / 4) aux[i] = *reinterpret_cast<const uint4 *>(src + cbeg + 8 * i);
+      }
+      flush();                                   // the previous phase's outputs
+      if (tid == 0 && !mbar_wait(&done, (uint32_t)(p & 1), a.wait_ns)) {
+        atomicCAS(a.status, 0, kDevTimeout);
+        abort_flag = 1;
+      }
+      epi_sync();
+      if (*(volatile int *)&abort_flag) break;
+      tc_fence_after();
+#pragma unroll
+      for (int step = 0; step < FB_MAXD / 4 / 16; ++step) {
+        const int c0 = cbeg + 16 * step;
+        if (c0 >= cend) break;
+        float z[16];
         tmem_ld16(tm + lb + c0, z);
         tmem_wait_ld();
-      };
-      if (!f.bwd && !last_fwd) {
-        // hidden layer: silu'(Z) of key rows out first, then X = silu(Z) for
-        // every row (the next layer's operand) and out for key rows
-        if (nkey > 0) {
-          for (int c0 = cbeg; c0 < cend; c0 += 16) {
-            float z[16];
-            tld16(c0, z);
-            if (!key) continue;
-            float sp[16];
+        if (!grad) {
+          // hidden layer: X = silu(Z) for every row (the next operand), and
+          // silu'(Z) of key rows straight out
+          float x[16], sp[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float sg = sigm(z[i]);
-              sp[i] = sg * (1.f + z[i] * (1.f - sg));
-            }
-#pragma unroll
-            for (int i = 0; i < 2; ++i) st_shared_v4(abuf + rb_chunk(128, row, c0 / 8 + i), pack8(sp + 8 * i));
+          for (int i = 0; i < 16; ++i) {
+            const float sg = sigm(z[i]);
+            x[i] = z[i] * sg;
+            sp[i] = sg * (1.f + z[i] * (1.f - sg));
           }
-          __syncthreads();
-          copy_out(a.sp_out[f.l], (long long)s * C + 128 * mt);
-          __syncthreads();
-        }
-        for (int c0 = cbeg; c0 < cend; c0 += 16) {
-          float z[16];
-          tld16(c0, z);
-          float x[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) x[i] = z[i] * sigm(z[i]);
 #pragma unroll
           for (int i = 0; i < 2; ++i) st_shared_v4(abuf + rb_chunk(128, row, c0 / 8 + i), pack8(x + 8 * i));
-        }
-        if (nkey > 0) {
-          __syncthreads();
-          copy_out(a.x_out[f.l], (long long)s * 2 * C + 128 * mt);
-        }
-      } else {
-        // gradient rows: G_L = 2 (Z_L - V) or G_{l-1} = (G_l W_l) . silu'(Z_{l-1});
-        // the other operand comes into the tile first
-        const int lo = f.bwd ? f.l - 1 : L;
-        if (nkey > 0) {
-          if (f.bwd) copy_in(a.sp_out[lo], (long long)s * C + 128 * mt);
-          else copy_in(a.v, (long long)s * a.T + (long long)a.chunk * C + 128 * mt);
-          __syncthreads();
-        }
-        for (int c0 = cbeg; c0 < cend; c0 += 16) {
-          float z[16];
-          tld16(c0, z);
-          if (!key) {
-            if (last_fwd) {                      // query row of the last layer: the read y
-              float *yo = a.y + tok * N + c0;
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                *reinterpret_cast<float4 *>(yo + 4 * i) =
-                    make_float4(z[4 * i], z[4 * i + 1], z[4 * i + 2], z[4 * i + 3]);
-            }
-            continue;
+          if (key) {
+            __nv_bfloat16 *so = a.sp_out[f.l] + ((long long)s * C + r) * N + c0;
+            *reinterpret_cast<uint4 *>(so) = pack8(sp);
+            *reinterpret_cast<uint4 *>(so + 8) = pack8(sp + 8);
           }
+        } else if (!key) {
+          if (last_fwd) {                        // query row of the last layer: the read y
+            float *yo = a.y + tok * N + c0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              *reinterpret_cast<float4 *>(yo + 4 * i) = make_float4(z[4 * i], z[4 * i + 1], z[4 * i + 2], z[4 * i + 3]);
+          }
+        } else {
+          // G_L = 2 (Z_L - V) or G_{l-1} = (G_l W_l) . silu'(Z_{l-1})
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
-            unsigned char *cp = abuf + rb_chunk(128, row, c0 / 8 + i);
-            const uint4 u = *reinterpret_cast<const uint4 *>(cp);
+            const uint4 u = aux[2 * step + i];
             const __nv_bfloat16 *hb = reinterpret_cast<const __nv_bfloat16 *>(&u);
             float g[8];
 #pragma unroll
@@ -734,27 +710,21 @@ __global__ void __launch_bounds__(FB_NT, 1)
               const float h = __bfloat162float(hb[j]);
               g[j] = f.bwd ? z[8 * i + j] * h : 2.f * (z[8 * i + j] - h);
             }
-            st_shared_v4(cp, pack8(g));
+            st_shared_v4(abuf + rb_chunk(128, row, c0 / 8 + i), pack8(g));
           }
         }
-        if (nkey > 0) {
-          __syncthreads();
-          copy_out_scaled(lo);
-        }
       }
+      // the tile (generic-proxy writes) is read by the next phase's MMAs
+      fence_proxy_async_smem();
+      tc_fence_before();
+      epi_sync();
+      if (tid == 0) mbar_arrive(&ready);
+      pend_kind = grad ? 2 : (nkey > 0 ? 1 : 0);
+      pend_l = f.bwd ? f.l - 1 : f.l;
+      pend_N = N;
+      if (grad && !has_keys) pend_kind = 0;
     }
-    // the tile (generic-proxy writes) is read by the next phase's MMAs
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (*(volatile int *)&abort_flag) break;
-  }
-  if (tid == 0) {
-    // after an abort: wait (bounded) for the copies still in flight into this CTA
-    if (!x_waited) mbar_wait(&xbar, 0, a.wait_ns);
-    for (int g = consumed; g < issued; ++g)
-      mbar_wait(&full[g % FB_STAGES], (uint32_t)((g / FB_STAGES) & 1), a.wait_ns);
+    if (!*(volatile int *)&abort_flag) flush();
   }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   tc_fence_before();
@@ -954,35 +924,54 @@ bool tcl_supported(const Problem &p) {
   return true;
 }
 
-size_t tcl_scratch_bytes(const Problem &p) { return carve(p).total; }
 
 static unsigned long long g_tcl_wait_ns = 2000000000ull;
 
-cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
-  if (!tcl_supported(p)) return cudaErrorNotSupported;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaSuccess;
-    const void *kerns[4] = {(const void *)tcl_gemm_kernel<K_FWD>, (const void *)tcl_gemm_kernel<K_FWD_LAST>,
-                            (const void *)tcl_gemm_kernel<K_BWD>, (const void *)tcl_dw_kernel};
-    for (const void *k : kerns) {
-      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-      if (e != cudaSuccess) return e;
-    }
-    e = cudaFuncSetAttribute(tcl_fb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FB_SMEM);
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
-  const Carve cv = carve(p);
-  unsigned char *ws = static_cast<unsigned char *>(p.scratch);
-  float *coef = reinterpret_cast<float *>(ws + cv.coef);
-  float *scal = reinterpret_cast<float *>(ws + cv.scal);
-  __nv_bfloat16 *wbf = reinterpret_cast<__nv_bfloat16 *>(ws + cv.wbf);
-  auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16 *>(ws + off); };
-  const int L = p.L, C = p.C, T = p.T, S = p.streams, nchunks = T / C;
-  const int d = p.dims[0];
+namespace {
 
+// One group of streams: its slice of every tensor, its own workspace carve
+// and CUDA stream, and everything its launches need.
+struct TclGroup {
+  Problem p;
+  cudaStream_t st;
+  Carve cv;
+  unsigned char *ws;
+  float *coef, *scal;
+  __nv_bfloat16 *wbf;
+  int L, C, T, S, nchunks;
   InitArgs ia;
+  CUtensorMap mk, mq, mwb[kMaxL + 1], mx[kMaxL + 1], mg[kMaxL + 1], mgc[kMaxL + 1], mge[kMaxL + 1];
+  GemmArgs base;
+  DwGroup dg;
+  DwMaps dm;
+  size_t dw_smem;
+  bool fused;
+  FbArgs fa;
+  FbMaps fm;
+
+  __nv_bfloat16 *bf(size_t off) const { return reinterpret_cast<__nv_bfloat16 *>(ws + off); }
+  // Widest tile that divides n and still gives about one CTA per SM.
+  int tile_for(int n, int mtiles) const {
+    for (int t = 256; t >= 64; t /= 2) {
+      if (n % t) continue;
+      if ((long long)S * mtiles * (n / t) >= 128 || t == 64) return t;
+    }
+    return 64;
+  }
+  cudaError_t setup();
+  cudaError_t chunk(int ch);
+};
+
+cudaError_t TclGroup::setup() {
+  cv = carve(p);
+  ws = static_cast<unsigned char *>(p.scratch);
+  coef = reinterpret_cast<float *>(ws + cv.coef);
+  scal = reinterpret_cast<float *>(ws + cv.scal);
+  wbf = reinterpret_cast<__nv_bfloat16 *>(ws + cv.wbf);
+  L = p.L; C = p.C; T = p.T; S = p.streams; nchunks = T / C;
+  const int d = p.dims[0];
+  cudaStream_t stream = st;
+
   ia.W0 = p.W0; ia.S0 = p.S0; ia.W = p.W_end; ia.S = p.S_end; ia.Wbf = wbf;
   ia.P = (long long)p.P; ia.streams = S; ia.L = L;
   long long bo = 0;
@@ -1000,7 +989,6 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
   if (err != cudaSuccess) return err;
 
   // tensor maps, built once per call
-  CUtensorMap mk, mq, mwb[kMaxL + 1], mx[kMaxL + 1], mg[kMaxL + 1], mgc[kMaxL + 1], mge[kMaxL + 1];
   if (!map2d(&mk, p.k, (long long)S * T, d, 64) || !map2d(&mq, p.q, (long long)S * T, d, 64))
     return cudaErrorInvalidValue;
   for (int l = 1; l <= L; ++l) {
@@ -1012,16 +1000,7 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
       return cudaErrorInvalidValue;
     if (l < L && !map2d(&mx[l], bf(cv.x[l]), (long long)S * 2 * C, nl, 64)) return cudaErrorInvalidValue;
   }
-  // Widest tile that divides n and still gives about one CTA per SM.
-  auto tile_for = [&](int n, int mtiles) {
-    for (int t = 256; t >= 64; t /= 2) {
-      if (n % t) continue;
-      if ((long long)S * mtiles * (n / t) >= 128 || t == 64) return t;
-    }
-    return 64;
-  };
 
-  GemmArgs base;
   std::memset(&base, 0, sizeof base);
   base.C = C;
   base.T = T;
@@ -1037,12 +1016,10 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
   base.v = reinterpret_cast<const __nv_bfloat16 *>(p.v);
 
   // the update launch: per layer, tiles of 128 rows of W_l x (128 or 64) columns
-  DwGroup dg;
-  DwMaps dm;
   std::memset(&dg, 0, sizeof dg);
   std::memset(&dm, 0, sizeof dm);
   dg.L = L;
-  size_t dw_smem = 0;
+  dw_smem = 0;
   for (int l = 1; l <= L; ++l) {
     GemmArgs &a = dg.l[l - 1];
     a = base;
@@ -1066,9 +1043,7 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
     if (sm > dw_smem) dw_smem = sm;
   }
 
-  const bool fused = p.fuse_fb && fb_ok(p);
-  FbArgs fa;
-  FbMaps fm;
+  fused = p.fuse_fb && fb_ok(p);
   if (fused) {
     std::memset(&fa, 0, sizeof fa);
     std::memset(&fm, 0, sizeof fm);
@@ -1090,57 +1065,175 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
     fa.status = p.status;
     fa.wait_ns = g_tcl_wait_ns;
   }
+  return cudaSuccess;
+}
 
-  for (int ch = 0; ch < nchunks; ++ch) {
-    if (fused) {
-      fa.chunk = ch;
-      err = launch_fb(fa, fm, S, stream);
-      if (err != cudaSuccess) return err;
-    }
-    // forward of keys and queries, layer by layer
-    for (int l = 1; l <= L && !fused; ++l) {
-      GemmArgs a = base;
-      const int nl = p.dims[l], np = p.dims[l - 1];
-      a.kind = l < L ? K_FWD : K_FWD_LAST;
-      a.chunk = ch;
-      a.N = tile_for(nl, 2 * C / 128);
-      a.K = np;
-      a.M = 2 * C;
-      a.n_out = nl;
-      a.a_split_kq = l == 1;
-      a.a_rows_per_stream = 2 * C;
-      a.b_rows_per_stream = nl;
-      if (l < L) { a.x_out = bf(cv.x[l]); a.sp_out = bf(cv.sp[l]); }
-      a.g_out = bf(cv.g[L]); a.gc_out = bf(cv.gc[L]); a.ge_out = bf(cv.ge[L]);
-      err = launch_gemm(a, l == 1 ? mk : mx[l - 1], mq, mwb[l], S, 2 * C / 128, nl / a.N, stream);
-      if (err != cudaSuccess) return err;
-    }
-    // backward to every hidden layer
-    for (int l = L; l >= 2 && !fused; --l) {
-      GemmArgs a = base;
-      const int nl = p.dims[l], np = p.dims[l - 1];
-      a.kind = K_BWD;
-      a.chunk = ch;
-      a.N = tile_for(np, (C + 127) / 128);
-      a.K = nl;
-      a.M = C;
-      a.n_out = np;
-      a.a_rows_per_stream = C;
-      a.b_rows_per_stream = nl;
-      a.sp_in = bf(cv.sp[l - 1]);
-      a.g_out = bf(cv.g[l - 1]); a.gc_out = bf(cv.gc[l - 1]); a.ge_out = bf(cv.ge[l - 1]);
-      err = launch_gemm(a, mg[l], mg[l], mwb[l], S, (C + 127) / 128, np / a.N, stream);
-      if (err != cudaSuccess) return err;
-    }
-    // weight-update contractions of every layer, with the fused state update
-    for (int l = 1; l <= L; ++l) {
-      dg.l[l - 1].chunk = ch;
-      dg.l[l - 1].b_row_off = l == 1 ? (long long)ch * C : 0;
-    }
-    err = launch_dw(dg, dm, dw_smem, stream);
+cudaError_t TclGroup::chunk(int ch) {
+  cudaStream_t stream = st;
+  cudaError_t err = cudaSuccess;
+  if (fused) {
+    fa.chunk = ch;
+    err = launch_fb(fa, fm, S, stream);
     if (err != cudaSuccess) return err;
   }
-  return cudaSuccess;
+  // forward of keys and queries, layer by layer
+  for (int l = 1; l <= L && !fused; ++l) {
+    GemmArgs a = base;
+    const int nl = p.dims[l], np = p.dims[l - 1];
+    a.kind = l < L ? K_FWD : K_FWD_LAST;
+    a.chunk = ch;
+    a.N = tile_for(nl, 2 * C / 128);
+    a.K = np;
+    a.M = 2 * C;
+    a.n_out = nl;
+    a.a_split_kq = l == 1;
+    a.a_rows_per_stream = 2 * C;
+    a.b_rows_per_stream = nl;
+    if (l < L) { a.x_out = bf(cv.x[l]); a.sp_out = bf(cv.sp[l]); }
+    a.g_out = bf(cv.g[L]); a.gc_out = bf(cv.gc[L]); a.ge_out = bf(cv.ge[L]);
+    err = launch_gemm(a, l == 1 ? mk : mx[l - 1], mq, mwb[l], S, 2 * C / 128, nl / a.N, stream);
+    if (err != cudaSuccess) return err;
+  }
+  // backward to every hidden layer
+  for (int l = L; l >= 2 && !fused; --l) {
+    GemmArgs a = base;
+    const int nl = p.dims[l], np = p.dims[l - 1];
+    a.kind = K_BWD;
+    a.chunk = ch;
+    a.N = tile_for(np, (C + 127) / 128);
+    a.K = nl;
+    a.M = C;
+    a.n_out = np;
+    a.a_rows_per_stream = C;
+    a.b_rows_per_stream = nl;
+    a.sp_in = bf(cv.sp[l - 1]);
+    a.g_out = bf(cv.g[l - 1]); a.gc_out = bf(cv.gc[l - 1]); a.ge_out = bf(cv.ge[l - 1]);
+    err = launch_gemm(a, mg[l], mg[l], mwb[l], S, (C + 127) / 128, np / a.N, stream);
+    if (err != cudaSuccess) return err;
+  }
+  // weight-update contractions of every layer, with the fused state update
+  for (int l = 1; l <= L; ++l) {
+    dg.l[l - 1].chunk = ch;
+    dg.l[l - 1].b_row_off = l == 1 ? (long long)ch * C : 0;
+  }
+  err = launch_dw(dg, dm, dw_smem, stream);
+  return err;
+}
+
+// Streams split into groups issued on separate CUDA streams: one group's
+// (latency-bound) forward/backward kernel runs beside another group's
+// (bandwidth-bound) update. TM_TCL_GROUPS (1..8) overrides the choice.
+int tcl_groups(const Problem &p) {
+  static int forced = -1;
+  if (forced < 0) {
+    const char *e = std::getenv("TM_TCL_GROUPS");
+    forced = e ? std::atoi(e) : 0;
+    if (forced < 0 || forced > kMaxGroups) forced = 0;
+  }
+  // about eight streams per group (measured on the depth-4 workload, 64
+  // streams: 1 group 32.5 ms, 2: 30.8, 4: 26.4, 8: 25.4)
+  int g = forced ? forced : p.streams / 8;
+  if (g > kMaxGroups) g = kMaxGroups;
+  if (g > p.streams) g = p.streams;
+  return g < 1 ? 1 : g;
+}
+
+Problem group_slice(const Problem &p, int g, int groups) {
+  const int s0 = (int)((long long)p.streams * g / groups), s1 = (int)((long long)p.streams * (g + 1) / groups);
+  Problem q = p;
+  const size_t el = p.in_dtype == TM_BF16 ? 2 : 4;
+  const size_t td = (size_t)p.T * p.dims[0];
+  q.streams = s1 - s0;
+  q.B = 1;
+  q.H = q.streams;
+  q.k = static_cast<const char *>(p.k) + s0 * td * el;
+  q.v = static_cast<const char *>(p.v) + s0 * td * el;
+  q.q = static_cast<const char *>(p.q) + s0 * td * el;
+  q.theta = p.theta + (size_t)s0 * p.T;
+  q.eta = p.eta + (size_t)s0 * p.T;
+  q.alpha = p.alpha + (size_t)s0 * p.T;
+  q.W0 = p.W0 + (size_t)s0 * p.P;
+  q.S0 = p.S0 + (size_t)s0 * p.P;
+  q.W_end = p.W_end + (size_t)s0 * p.P;
+  q.S_end = p.S_end + (size_t)s0 * p.P;
+  q.y = p.y + (size_t)s0 * td;
+  return q;
+}
+
+size_t group_bytes(const Problem &p, int groups) {
+  size_t m = 0;
+  for (int g = 0; g < groups; ++g) {
+    const size_t b = carve(group_slice(p, g, groups)).total;
+    if (b > m) m = b;
+  }
+  return m;
+}
+
+}  // namespace
+
+size_t tcl_scratch_bytes(const Problem &p) {
+  const int G = tcl_groups(p);
+  return (size_t)G * group_bytes(p, G);
+}
+
+int tcl_group_count(const Problem &p) { return tcl_supported(p) ? tcl_groups(p) : 1; }
+
+long long tcl_launch_count(const Problem &p) {
+  // per group: init and coefficient kernels, then per chunk the fused
+  // forward + backward (or 2L - 1 phase launches) and one update launch
+  const long long per_chunk = (p.fuse_fb && fb_ok(p)) ? 2 : 2LL * p.L;
+  return (long long)tcl_group_count(p) * (2 + per_chunk * (p.T / p.C));
+}
+
+cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
+  if (!tcl_supported(p)) return cudaErrorNotSupported;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaSuccess;
+    const void *kerns[4] = {(const void *)tcl_gemm_kernel<K_FWD>, (const void *)tcl_gemm_kernel<K_FWD_LAST>,
+                            (const void *)tcl_gemm_kernel<K_BWD>, (const void *)tcl_dw_kernel};
+    for (const void *k : kerns) {
+      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+    }
+    e = cudaFuncSetAttribute(tcl_fb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FB_SMEM);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  const int G = tcl_groups(p);
+  if (G > 1 && (!p.side_streams[G - 2] || !p.ev_fork || !p.ev_join[G - 2])) return cudaErrorInvalidValue;
+  const size_t gb = group_bytes(p, G);
+  std::vector<TclGroup> groups((size_t)G);
+  cudaError_t err = cudaSuccess;
+  if (G > 1) {
+    err = cudaEventRecord(static_cast<cudaEvent_t>(p.ev_fork), stream);
+    for (int g = 1; g < G && err == cudaSuccess; ++g)
+      err = cudaStreamWaitEvent(static_cast<cudaStream_t>(p.side_streams[g - 1]),
+                                static_cast<cudaEvent_t>(p.ev_fork), 0);
+    if (err != cudaSuccess) return err;
+  }
+  for (int g = 0; g < G && err == cudaSuccess; ++g) {
+    TclGroup &t = groups[(size_t)g];
+    t.p = group_slice(p, g, G);
+    t.p.scratch = static_cast<unsigned char *>(p.scratch) + (size_t)g * gb;
+    t.p.scratch_bytes = gb;
+    t.st = g == 0 ? stream : static_cast<cudaStream_t>(p.side_streams[g - 1]);
+    err = t.setup();
+  }
+  // launches of the groups interleaved chunk by chunk
+  const int nchunks = p.T / p.C;
+  for (int ch = 0; ch < nchunks && err == cudaSuccess; ++ch)
+    for (int g = 0; g < G && err == cudaSuccess; ++g) err = groups[(size_t)g].chunk(ch);
+  if (G > 1) {
+    // join (also after an error, so that the caller's stream never runs ahead
+    // of work already queued on the side streams)
+    for (int g = 1; g < G; ++g) {
+      cudaEvent_t ev = static_cast<cudaEvent_t>(p.ev_join[g - 1]);
+      if (cudaEventRecord(ev, static_cast<cudaStream_t>(p.side_streams[g - 1])) == cudaSuccess)
+        cudaStreamWaitEvent(stream, ev, 0);
+    }
+  }
+  return err;
 }
 
 void tcl_set_wait(unsigned long long wait_ns) { g_tcl_wait_ns = wait_ns ? wait_ns : 2000000000ull; }

@@ -60,6 +60,13 @@ class NeuralMemory:
         return {N.TM_PATH_SIMT: "simt", N.TM_PATH_TC: "tc", N.TM_PATH_TC_LAYERED: "tcl",
                 N.TM_PATH_TC_PHASED: "tcl-phased"}[out.value]
 
+    def launch_count(self, B, H, T, C, dtype=torch.bfloat16) -> int:
+        """Kernel launches one run() of this problem makes."""
+        out = ctypes.c_longlong()
+        code = N.TM_BF16 if dtype == torch.bfloat16 else N.TM_F32
+        N.check(self._lib.tm_launch_count(self._h, B, H, T, C, code, ctypes.byref(out)), "tm_launch_count")
+        return int(out.value)
+
     def workspace_size(self, B, H, T, C, dtype=torch.bfloat16) -> int:
         out = ctypes.c_size_t()
         code = N.TM_BF16 if dtype == torch.bfloat16 else N.TM_F32

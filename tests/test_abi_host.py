@@ -99,6 +99,28 @@ def test_path_selection_and_query():
     lib.tm_destroy(h)
 
 
+def test_launch_count():
+    """Launches per tm_run: one persistent kernel, or for the layered paths
+    per group of streams an init and a coefficient kernel plus, per chunk,
+    the fused forward/backward (or 2L - 1 phase launches) and one update."""
+    import os
+    lib = N.load()
+    _, h = create(2, 64, 4)
+    n = ctypes.c_longlong()
+    assert lib.tm_launch_count(h, 1, 2, 256, 64, N.TM_F32, ctypes.byref(n)) == N.TM_OK
+    assert n.value == 1
+    assert lib.tm_launch_count(h, 1, 2, 256, 64, N.TM_BF16, None) == N.TM_ERR_INVALID_ARG
+    groups = int(os.environ.get("TM_TCL_GROUPS", "0"))
+    for path, per_chunk in ((N.TM_PATH_TC_LAYERED, 2), (N.TM_PATH_TC_PHASED, 2 * 2)):
+        assert lib.tm_set_path(h, path) == N.TM_OK
+        for B, H in ((1, 2), (2, 4), (3, 3)):
+            S = B * H
+            g = max(1, min(groups or min(S // 8, 8), S))
+            assert lib.tm_launch_count(h, B, H, 256, 64, N.TM_BF16, ctypes.byref(n)) == N.TM_OK
+            assert n.value == g * (2 + per_chunk * 4), (path, B, H, n.value)
+    lib.tm_destroy(h)
+
+
 def _run(lib, h, ptrs, B=1, H=1, T=64, C=16, dt=N.TM_F32, ws_bytes=1 << 30):
     args = [ctypes.c_void_p(x) for x in ptrs]
     return lib.tm_run(h, B, H, T, C, dt, *args[:11], args[11], ws_bytes, None)

@@ -270,6 +270,8 @@ TCL_SHAPES = [  # L, d, expansion, B, H, T, C
     (4, 128, 2, 1, 1, 256, 128),    # the deep workload's layer shapes
     (2, 64, 2, 1, 2, 384, 192),     # C = 192: a partial row tile in the backward
     (2, 128, 2, 1, 1, 512, 256),    # C = 256: four key/query row tiles, pipelined K loop
+    (2, 64, 2, 3, 3, 256, 64),      # 9 streams: two concurrent groups of 4 and 5
+    (4, 64, 2, 2, 4, 256, 128),     # 8 streams in two groups, depth 4
 ]
 
 
