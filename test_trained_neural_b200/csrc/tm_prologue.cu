@@ -24,7 +24,7 @@ namespace tmem {
 namespace {
 
 constexpr int RB = 8;        // output rows per row group
-constexpr int MAXW = 8;      // largest filter width
+constexpr int MAXW_ALL = 8;  // largest filter width
 constexpr int NT = 256;      // target threads per CTA
 
 struct ProArgs {
@@ -89,8 +89,9 @@ __device__ __forceinline__ void store4(void *p, long long i, const float o[4]) {
 template <typename T>
 __device__ __forceinline__ T pick(int z, T a, T b, T c) { return z == 0 ? a : (z == 1 ? b : c); }
 
-template <bool BF16>
-__global__ void __launch_bounds__(NT) prologue_kernel(const ProArgs a) {
+// MAXW: taps held in registers (4 or 8; taps beyond the filter width are zero)
+template <bool BF16, bool WIDE, int MAXW>
+__global__ void __launch_bounds__(NT, (!WIDE && MAXW == 4) ? 3 : 2) prologue_kernel(const ProArgs a) {
   using El = typename std::conditional<BF16, __nv_bfloat16, float>::type;
   __shared__ float part[NT / 32][RB];        // per-warp partial sums of squares (d > 128)
   const int s = blockIdx.y, z = blockIdx.z;
@@ -124,6 +125,36 @@ __global__ void __launch_bounds__(NT) prologue_kernel(const ProArgs a) {
       ld_pred(f[j][e], fp + e * w + (j < w ? j : 0), j < w);
     }
 
+  const bool norm = z != 1;                  // keys and queries: unit L2 norm per row
+  if constexpr (!WIDE && MAXW == 4) {
+    // a row group lies inside one warp: each output row is formed, reduced
+    // with shuffles, scaled and stored on its own (few live registers, so
+    // more CTAs and more loads in flight per SM)
+    const int width = d4;
+#pragma unroll
+    for (int r = 0; r < RB; ++r) {
+      float o[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < MAXW; ++j) {
+        float x[4];
+        raw[r + MAXW - 1 - j].to_f32(x);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[e] = fmaf(f[j][e], x[e], o[e]);
+      }
+      if (norm) {
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ss = fmaf(o[e], o[e], ss);
+        for (int off = width / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float scale = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[e] *= scale;
+      }
+      const long long t = tb + r;
+      if (t < T) store4<BF16>(out, base + t * d + c, o);
+    }
+    return;
+  } else {
   float o[RB][4];
 #pragma unroll
   for (int r = 0; r < RB; ++r)
@@ -142,7 +173,7 @@ __global__ void __launch_bounds__(NT) prologue_kernel(const ProArgs a) {
     }
   }
 
-  if (z != 1) {                              // keys and queries: unit L2 norm per row
+  if (norm) {
     float ss[RB];
 #pragma unroll
     for (int r = 0; r < RB; ++r) {
@@ -180,6 +211,7 @@ __global__ void __launch_bounds__(NT) prologue_kernel(const ProArgs a) {
     const long long t = tb + r;
     if (t < T) store4<BF16>(out, base + t * d + c, o[r]);
   }
+  }
 }
 
 int rows_groups_per_cta(int d) {
@@ -196,7 +228,7 @@ bool prologue_supported_d(int d) {
 cudaError_t prologue_launch(int streams, int H, int T, int d, int w, bool bf16, const void *const in[3],
                             const float *const filt[3], const void *const hist[3], void *const out[3],
                             cudaStream_t stream) {
-  if (!prologue_supported_d(d) || w < 1 || w > MAXW) return cudaErrorNotSupported;
+  if (!prologue_supported_d(d) || w < 1 || w > MAXW_ALL) return cudaErrorNotSupported;
   ProArgs a;
   a.T = T;
   a.d = d;
@@ -212,10 +244,16 @@ cudaError_t prologue_launch(int streams, int H, int T, int d, int w, bool bf16, 
   const int RL = rows_groups_per_cta(d);
   const int rows = RL * RB;
   dim3 grid((unsigned)((T + rows - 1) / rows), (unsigned)streams, 3);
-  if (bf16)
-    prologue_kernel<true><<<grid, RL * (d / 4), 0, stream>>>(a);
-  else
-    prologue_kernel<false><<<grid, RL * (d / 4), 0, stream>>>(a);
+  const dim3 block((unsigned)(RL * (d / 4)));
+  const bool wide = d / 4 > 32, short_filter = w <= 4;
+  auto go = [&](auto kern) { kern<<<grid, block, 0, stream>>>(a); };
+  if (bf16) {
+    if (wide) short_filter ? go(prologue_kernel<true, true, 4>) : go(prologue_kernel<true, true, 8>);
+    else short_filter ? go(prologue_kernel<true, false, 4>) : go(prologue_kernel<true, false, 8>);
+  } else {
+    if (wide) short_filter ? go(prologue_kernel<false, true, 4>) : go(prologue_kernel<false, true, 8>);
+    else short_filter ? go(prologue_kernel<false, false, 4>) : go(prologue_kernel<false, false, 8>);
+  }
   return cudaGetLastError();
 }
 

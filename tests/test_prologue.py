@@ -74,6 +74,7 @@ def _f64(a, dtype):
     (2, 2, 200, 256, 8, "f32", True),       # norm reduced across two warps
     (1, 1, 70, 768, 5, "bf16", True),       # widest row: six warps per row
     (3, 1, 9, 128, 2, "f32", True),         # sequence shorter than one tile
+    (1, 2, 100, 128, 6, "bf16", True),      # filter wider than 4 taps, rows inside one warp
 ])
 def test_prologue_matches_oracle(B, H, T, d, width, dtype, hist):
     from test_trained_neural_b200 import prologue
