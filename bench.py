@@ -259,6 +259,23 @@ def sweep_chunk(args, w: W.Workload, sizes):
                           "workspace_bytes": ws.numel()}), flush=True)
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# the cluster kernel, from one ncu --set full capture of a shortened case of
+# the long d=128 workload (16 streams x 4096 tokens: 68.39 MB read, 13.09 MB
+# written; the summary is kept under profiles/). The kernel's traffic grows
+# with the tokens it processes (inputs and reads stream through once, the
+# state stays on chip), so a full launch is that figure scaled by tokens.
+CAPTURED_TRAFFIC = {("tc", "mlp2-d128-long"): (68.387072e6 + 13.085184e6, 16 * 4096)}
+
+
+def traffic_per_launch(path: str, w: W.Workload):
+    rec = CAPTURED_TRAFFIC.get((path, w.name))
+    if rec is None:
+        return None
+    nbytes, tokens = rec
+    return nbytes * (w.streams * w.T) / tokens
+
+
 def bench_prologue(args, w: W.Workload):
     """The step before the memory on the workload's k, v, q: one fused launch of
     the depthwise causal convolution (width args.conv_width) and the L2
@@ -419,7 +436,7 @@ def main():
                 "unit": "TFLOP/s", "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 x max clock",
                 "sm_mhz_seen": sm_mhz}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = traffic_per_launch(path_used, w)
     roof["kernel"] = {"tc": "tc_chunk_kernel", "tcl": "tcl_fb_kernel + tcl_gemm_kernel",
                       "tcl-phased": "tcl_gemm_kernel"}.get(path_used, "simt_chunk_kernel")
 
