@@ -78,8 +78,13 @@ typedef enum {
                               every width is at most 256 the forward and backward of a
                               chunk run as one fused launch, then one update launch per
                               layer; else unsupported                                      */
-  TM_PATH_TC_PHASED = 4    /* as TM_PATH_TC_LAYERED, but every forward, backward and
+  TM_PATH_TC_PHASED = 4,   /* as TM_PATH_TC_LAYERED, but every forward, backward and
                               update phase its own launch (same results; for comparison)   */
+  TM_PATH_TC_GLOBAL = 5    /* as TM_PATH_TC, but the CTAs of a stream exchange through
+                              global memory instead of a cluster's shared memory (all
+                              B*H*hidden/64 CTAs must fit on the SMs at once, else
+                              unsupported). TM_PATH_TC itself uses this form, beside the
+                              clusters, for the streams whose clusters do not fit at once */
 } tm_path;
 
 /*

@@ -16,7 +16,7 @@ TM_OK, TM_ERR_INVALID_ARG, TM_ERR_UNSUPPORTED, TM_ERR_CUDA, TM_ERR_OOM, TM_ERR_T
     TM_ERR_DEVICE = range(7)
 TM_ACT_SILU = 0
 TM_F32, TM_BF16 = 0, 1
-TM_PATH_AUTO, TM_PATH_SIMT, TM_PATH_TC, TM_PATH_TC_LAYERED, TM_PATH_TC_PHASED = 0, 1, 2, 3, 4
+TM_PATH_AUTO, TM_PATH_SIMT, TM_PATH_TC, TM_PATH_TC_LAYERED, TM_PATH_TC_PHASED, TM_PATH_TC_GLOBAL = 0, 1, 2, 3, 4, 5
 
 # name -> (restype, argtypes); mirrors include/titansmem.h
 _P, _I, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t

@@ -56,6 +56,7 @@ tmem::Problem make_problem(const tm_ctx *ctx, int B, int H, int T, int C, tm_dty
   p.streams = B * H;
   p.in_dtype = dt;
   p.fuse_fb = 1;
+  p.tc_global = ctx->path == TM_PATH_TC_GLOBAL;
   return p;
 }
 
@@ -67,13 +68,13 @@ tm_path choose_path(const tm_ctx *ctx, const tmem::Problem &p) {
 }
 
 bool path_supported(tm_path path, const tmem::Problem &p) {
-  if (path == TM_PATH_TC) return tmem::tc_supported(p);
+  if (path == TM_PATH_TC || path == TM_PATH_TC_GLOBAL) return tmem::tc_supported(p);
   if (path == TM_PATH_TC_LAYERED || path == TM_PATH_TC_PHASED) return tmem::tcl_supported(p);
   return true;
 }
 
 size_t scratch_bytes(tm_path path, const tmem::Problem &p) {
-  if (path == TM_PATH_TC) return tmem::tc_scratch_bytes(p);
+  if (path == TM_PATH_TC || path == TM_PATH_TC_GLOBAL) return tmem::tc_scratch_bytes(p);
   if (path == TM_PATH_TC_LAYERED || path == TM_PATH_TC_PHASED) return tmem::tcl_scratch_bytes(p);
   return tmem::simt_scratch_bytes(p);
 }
@@ -163,7 +164,7 @@ size_t tm_param_count(const tm_ctx *ctx) { return ctx ? ctx->P : 0; }
 tm_status tm_set_path(tm_ctx *ctx, tm_path path) {
   if (!ctx) return TM_ERR_INVALID_ARG;
   if (path != TM_PATH_AUTO && path != TM_PATH_SIMT && path != TM_PATH_TC && path != TM_PATH_TC_LAYERED &&
-      path != TM_PATH_TC_PHASED)
+      path != TM_PATH_TC_PHASED && path != TM_PATH_TC_GLOBAL)
     return TM_ERR_INVALID_ARG;
   ctx->path = path;
   return TM_OK;
@@ -272,7 +273,7 @@ tm_status tm_run(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype, con
       p.ev_fork = ctx->ev_fork;
     }
   }
-  cudaError_t err = path == TM_PATH_TC ? tmem::tc_launch(p, s)
+  cudaError_t err = (path == TM_PATH_TC || path == TM_PATH_TC_GLOBAL) ? tmem::tc_launch(p, s)
                     : (path == TM_PATH_TC_LAYERED || path == TM_PATH_TC_PHASED) ? tmem::tcl_launch(p, s)
                                                                               : tmem::simt_launch(p, s);
   return err == cudaSuccess ? TM_OK : TM_ERR_CUDA;

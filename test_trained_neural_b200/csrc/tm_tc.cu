@@ -68,7 +68,19 @@ struct TcArgs {
   int *status;
   unsigned long long wait_ns;
   int inject_timeout;
+  // Exchange through global memory (streams whose cluster does not fit
+  // beside the others): per stream, receive buffers and G2 rows, double
+  // buffered by chunk parity, and monotonic arrival counters.
+  unsigned char *xrecv;          // [stream][dest][parity][G x 2 x RP x d] bf16
+  unsigned char *xg2;            // [stream][parity][64 x d] bf16, row-block layout
+  unsigned *xflag;               // [stream][G + 1] counters, 128 bytes apart
 };
+
+// Exchange buffer sizes per stream (bytes) and counter stride (in unsigned).
+constexpr int XFLAG_STRIDE = 32;
+__host__ __device__ constexpr size_t xrecv_bytes(int D, int G) { return (size_t)G * 2 * (2 * 128 * D); }
+__host__ __device__ constexpr size_t xg2_bytes(int D) { return (size_t)2 * 64 * D * 2; }
+__host__ __device__ constexpr size_t xflag_bytes(int G) { return (size_t)(G + 1) * XFLAG_STRIDE * 4; }
 
 struct Coefs {
   float c[C];
@@ -161,6 +173,32 @@ __device__ __forceinline__ void bulk_push(uint32_t dst, uint32_t src, uint32_t b
       "r"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
+// Global-memory exchange: bulk copy shared -> global, completion, proxy fence,
+// release counter, acquire poll, bulk copy global -> shared.
+__device__ __forceinline__ void bulk_store_global(void *gdst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_and_wait() {
+  asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ void red_release_add(unsigned *p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void bulk_load_global(uint32_t dst, const void *gsrc, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(gsrc), "r"(bytes), "r"(bar)
+      : "memory");
+}
 __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
   float4 v;
   asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
@@ -225,6 +263,23 @@ __device__ bool wait_bar(uint64_t *bar, uint32_t parity, const TcArgs &a, volati
   }
 }
 
+// Bounded wait until a global arrival counter reaches target (acquire).
+__device__ bool wait_flag(const unsigned *flag, unsigned target, const TcArgs &a, volatile int *abort_flag) {
+  if ((int)(ld_acquire(flag) - target) >= 0) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i)
+      if ((int)(ld_acquire(flag) - target) >= 0) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > a.wait_ns) {
+      atomicCAS(a.status, 0, kDevTimeout);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
 // A5 with warp shuffles. Lane l holds tokens 2l and 2l+1 of the chunk.
 //   pa_i = prod_{j>i} (1 - alpha_j), pe_i = prod_{j>i} eta_j,
 //   r_i  = pa_i + eta_{i+1} r_{i+1}, r_{C-1} = 1   (an affine map per token,
@@ -279,7 +334,11 @@ __device__ void coef_scan_warp(Coefs &cf, const float *th, const float *et, cons
   }
 }
 
-template <int D, int G>
+// XG = false: the G CTAs of a stream form a cluster and exchange through
+// each other's shared memory. XG = true: the same walker without a cluster,
+// the exchange going through global memory (used for streams whose cluster
+// does not fit beside the others; all G CTAs of a stream must be resident).
+template <int D, int G, bool XG>
 __global__ void __launch_bounds__(NTHREADS, 1)
     tc_chunk_kernel(const TcArgs a, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_q) {
@@ -292,6 +351,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   constexpr int NPT = RP * D / 8 / EPI_THREADS;    // 16-byte chunks reduced per thread
   constexpr int SWZ = (D / 16 < 8 ? D / 16 : 8) - 1; // chunk swizzle mask of a half row
   static_assert(NPT >= 1 && RP * D / 8 % EPI_THREADS == 0, "reduce split");
+  constexpr int NSIG = 2 * G * (RP >= 32 ? RP / 32 : 1);   // row pushes a CTA receives per chunk
+  constexpr int NKO = RP >= C ? 1 : C / RP;                 // CTAs owning key rows
+  constexpr uint32_t XDEST = 2 * 128 * D;                   // bytes of one receive buffer
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *sm =
       reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -302,8 +364,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   Coefs *coefs = reinterpret_cast<Coefs *>(sm + Lay::COEF);
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const uint32_t j = cluster_rank();
+  const uint32_t j = XG ? (uint32_t)(blockIdx.x % G) : cluster_rank();
   const int stream = blockIdx.x / G;
+  unsigned *const xfl = XG ? a.xflag + (size_t)stream * (G + 1) * XFLAG_STRIDE : nullptr;
+  unsigned char *const xrv = XG ? a.xrecv + (size_t)stream * xrecv_bytes(D, G) : nullptr;
+  unsigned char *const xg2 = XG ? a.xg2 + (size_t)stream * xg2_bytes(D) : nullptr;
   const int T = a.T, nchunks = T / C, P = a.P;
   const int Hd = HS * G;             // hidden width
   float *Wg = a.W + (long long)stream * P;
@@ -348,8 +413,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  cluster_arrive_release();   // every CTA's barriers are initialised
-  cluster_wait_acquire();
+  if constexpr (!XG) {
+    cluster_arrive_release();   // every CTA's barriers are initialised
+    cluster_wait_acquire();
+    // every CTA of this grid is resident: a kernel launched after this one
+    // with programmatic serialization (the global-exchange walker for the
+    // streams that did not fit) may take the SMs left free
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  }
   const uint32_t tm = *tmem_slot;
   const uint32_t t_z1 = tm + 0, t_z2 = tm + 64, t_g1 = tm + 192, t_s2 = tm + 256, t_s1 = tm + 384;
 
@@ -475,7 +546,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // that the query owners read in the previous chunk: wait for their
       // release (normally long given). Key rows need no such wait: the key
       // owners' G2 of the previous chunk already proved it.
-      if (NQO > 0 && q >= 2 && cch > 0 &&
+      // (The global exchange double-buffers by chunk parity instead: a peer
+      // writes chunk c+2 only after this CTA's push of chunk c+1, which
+      // follows its reads of chunk c.)
+      if (!XG && NQO > 0 && q >= 2 && cch > 0 &&
           !wait_bar(&bars[B_QFREE], (uint32_t)((cch - 1) & 1), a, abort_flag, true))
         break;
       {
@@ -497,16 +571,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int i = 0; i < 32 / RPP; ++i) {
             const int r0 = 32 * q + i * RPP, p = r0 / RP, rin = r0 - p * RP;
-            bulk_push(mapa(sbase + Lay::RECV + (uint32_t)(j * 2 * RP * D + h * RP * D + rin * D), (uint32_t)p),
-                      sbase + Lay::SEND + (uint32_t)(h * 128 * D + r0 * D), (uint32_t)(RPP * D),
-                      mapa(smem_u32(&bars[B_RECV]), (uint32_t)p));
+            const uint32_t off = (uint32_t)(j * 2 * RP * D + h * RP * D + rin * D);
+            const uint32_t src = sbase + Lay::SEND + (uint32_t)(h * 128 * D + r0 * D);
+            if constexpr (XG)
+              bulk_store_global(xrv + (size_t)(p * 2 + (int)par) * XDEST + off, src, (uint32_t)(RPP * D));
+            else
+              bulk_push(mapa(sbase + Lay::RECV + off, (uint32_t)p), src, (uint32_t)(RPP * D),
+                        mapa(smem_u32(&bars[B_RECV]), (uint32_t)p));
+          }
+          if constexpr (XG) {
+            // the rows are in global memory before the owners are told
+            bulk_commit_and_wait();
+            fence_proxy_async_global();
+#pragma unroll
+            for (int i = 0; i < 32 / RPP; ++i) red_release_add(xfl + ((32 * q + i * RPP) / RP) * XFLAG_STRIDE, 1u);
           }
         }
         __syncwarp();
       }
       // -------- reduce my rows over the G partials (fp32 sums, fixed order):
       // y for query rows, G2 = 2 (Z2 - V) for key rows (A3)
-      if (!wait_bar(&bars[B_RECV], par, a, abort_flag)) break;
+      if (XG ? !wait_flag(xfl + j * XFLAG_STRIDE, (unsigned)(NSIG * (cch + 1)), a, abort_flag)
+             : !wait_bar(&bars[B_RECV], par, a, abort_flag))
+        break;
       {
         float acc[NPT][8];
 #pragma unroll
@@ -514,9 +601,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const int k = tid + i * EPI_THREADS, r = k / (D / 8), c = k % (D / 8);
           uint4 pv[G];
 #pragma unroll
-          for (int s2 = 0; s2 < G; ++s2)
-            pv[s2] = *reinterpret_cast<const uint4 *>(sm + Lay::RECV + s2 * 2 * RP * D + (c / (D / 16)) * RP * D +
-                                                       r * D + (((c % (D / 16)) ^ (r & SWZ)) << 4));
+          for (int s2 = 0; s2 < G; ++s2) {
+            const uint32_t off = (uint32_t)(s2 * 2 * RP * D + (c / (D / 16)) * RP * D + r * D +
+                                            (((c % (D / 16)) ^ (r & SWZ)) << 4));
+            if constexpr (XG)
+              pv[s2] = __ldcg(reinterpret_cast<const uint4 *>(xrv + (size_t)(j * 2 + par) * XDEST + off));
+            else
+              pv[s2] = *reinterpret_cast<const uint4 *>(sm + Lay::RECV + off);
+          }
 #pragma unroll
           for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
 #pragma unroll
@@ -680,7 +772,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tc_fence_after();
       // this chunk's incoming bytes: G partial blocks, and all 64 rows of G2
       if (lane == 0) {
-        mbar_arrive_expect_tx(&bars[B_RECV], (uint32_t)(G * RP * D * 2));
+        if (!XG) mbar_arrive_expect_tx(&bars[B_RECV], (uint32_t)(G * RP * D * 2));
         mbar_arrive_expect_tx(&bars[B_G2], (uint32_t)(C * D * 2));
       }
       __syncwarp();
@@ -710,7 +802,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // their receive buffer (B_QFREE, off the critical path).
       if (!wait_bar(&bars[B_G2OWN], par, a, abort_flag)) break;
       if (lane == 0) {
-        if ((int)j * RP < C) {
+        if ((int)j * RP < C && XG) {
+          // G2 rows to global memory, then one arrival for every reader
+#pragma unroll
+          for (int fb = 0; fb < D / 64; ++fb)
+            bulk_store_global(xg2 + (size_t)par * (64 * D * 2) + fb * 64 * 128 + j * (uint32_t)(RP * 128),
+                              sbase + Lay::G2OWN + (uint32_t)(fb * RPK * 128), (uint32_t)(RPK * 128));
+          bulk_commit_and_wait();
+          fence_proxy_async_global();
+          red_release_add(xfl + G * XFLAG_STRIDE, 1u);
+        } else if ((int)j * RP < C) {
 #pragma unroll
           for (int i = 0; i < G; ++i) {
             const uint32_t p = (j + (uint32_t)i) % G;
@@ -720,7 +821,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         sbase + Lay::G2OWN + (uint32_t)(fb * RPK * 128), (uint32_t)(RPK * 128),
                         mapa(smem_u32(&bars[B_G2]), p));
           }
-        } else {
+        } else if (!XG) {
           // done reading this chunk's receive buffer: query rows of the next
           // chunk may be pushed here
 #pragma unroll
@@ -729,8 +830,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       __syncwarp();
+      if constexpr (XG) {
+        // every key owner's rows of this chunk are out: copy G2 in
+        int ok = 1;
+        if (lane == 0) {
+          ok = wait_flag(xfl + G * XFLAG_STRIDE, (unsigned)(NKO * (cch + 1)), a, abort_flag) ? 1 : 0;
+          if (ok) {
+            fence_proxy_async_global();
+            bulk_load_global(g2, xg2 + (size_t)par * (64 * D * 2), (uint32_t)(C * D * 2), smem_u32(&bars[B_G2]));
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      }
       // G2 complete in this CTA's shared memory
-      if (!wait_bar(&bars[B_G2], par, a, abort_flag, true)) break;
+      if (!wait_bar(&bars[B_G2], par, a, abort_flag, !XG)) break;
       tc_fence_after();
       if (lane == 0) {
         // A4: G1 pre-activation gradient = G2 W2_j
@@ -772,11 +885,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
-  // no CTA leaves while a peer may still write into its shared memory
-  cluster_arrive_release();
-  cluster_wait_acquire();
+  if constexpr (!XG) {
+    // no CTA leaves while a peer may still write into its shared memory
+    cluster_arrive_release();
+    cluster_wait_acquire();
+  }
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tm, TMEM_COLS);
+  // launched behind the cluster walker: do not complete before it, so that
+  // later work in the stream sees both done
+  if constexpr (XG) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -812,19 +930,46 @@ bool make_token_map(CUtensorMap *map, const void *base, long long rows, int d) {
 
 int cluster_size(const Problem &p) { return p.dims[1] / HS; }
 
-template <int D, int G>
-cudaError_t launch_dg(const Problem &p, cudaStream_t stream, const TcArgs &a, const CUtensorMap &mk,
-                      const CUtensorMap &mq) {
+template <int D, int G, bool XG>
+cudaError_t launch_dg(int streams, cudaStream_t stream, const TcArgs &a, const CUtensorMap &mk,
+                      const CUtensorMap &mq, bool after_primary) {
   using Lay = Layout<D>;
   const size_t smem = Lay::TOTAL + 1024;
-  auto kern = tc_chunk_kernel<D, G>;
+  auto kern = tc_chunk_kernel<D, G, XG>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(p.streams * G));
+  cfg.gridDim = dim3((unsigned)(streams * G));
   cfg.blockDim = dim3(NTHREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  if (!XG) {
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = G;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+  } else if (after_primary) {
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, kern, a, mk, mq);
+}
+
+template <int D, int G>
+int max_clusters_dg() {
+  using Lay = Layout<D>;
+  const size_t smem = Lay::TOTAL + 1024;
+  auto kern = tc_chunk_kernel<D, G, false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(G * 64));
+  cfg.blockDim = dim3(NTHREADS);
+  cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = G;
@@ -832,7 +977,65 @@ cudaError_t launch_dg(const Problem &p, cudaStream_t stream, const TcArgs &a, co
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a, mk, mq);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+// Clusters of this shape that can be resident at once (0 if unknown), and
+// the SM count; both cached per process.
+int max_clusters(int d, int G) {
+  static int cache[2][9] = {};
+  static bool done[2][9] = {};
+  const int di = d == 64 ? 0 : 1;
+  if (!done[di][G]) {
+    int n = 0;
+    switch (G) {
+      case 1: n = d == 64 ? max_clusters_dg<64, 1>() : max_clusters_dg<128, 1>(); break;
+      case 2: n = d == 64 ? max_clusters_dg<64, 2>() : max_clusters_dg<128, 2>(); break;
+      case 4: n = d == 64 ? max_clusters_dg<64, 4>() : max_clusters_dg<128, 4>(); break;
+      case 8: n = max_clusters_dg<128, 8>(); break;
+    }
+    cache[di][G] = n;
+    done[di][G] = true;
+  }
+  return cache[di][G];
+}
+
+int sm_count() {
+  static int n = -1;
+  if (n < 0) {
+    int dev = 0;
+    n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+  }
+  return n;
+}
+
+size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Streams run by the global-exchange walker: with `all`, every stream (when
+// all CTAs fit on the SMs at once); otherwise the streams beyond the
+// clusters that fit, when their CTAs fit on the SMs those clusters leave.
+int global_streams(const Problem &p, bool all) {
+  const int G = cluster_size(p), sms = sm_count();
+  if (all) return (sms > 0 && p.streams * G <= sms) ? p.streams : -1;
+  const int mx = max_clusters(p.dims[0], G);
+  if (mx <= 0 || p.streams <= mx) return 0;
+  const int rest = p.streams - mx;
+  return rest * G <= sms - mx * G ? rest : 0;
+}
+
+size_t exchange_bytes(int d, int G, int nx) {
+  if (nx <= 0) return 0;
+  return up256((size_t)nx * xflag_bytes(G)) + up256((size_t)nx * xg2_bytes(d)) +
+         up256((size_t)nx * xrecv_bytes(d, G));
 }
 
 }  // namespace
@@ -843,11 +1046,15 @@ bool tc_supported(const Problem &p) {
   if (d != 64 && d != 128) return false;
   if (h % HS != 0) return false;
   const int G = h / HS;
-  if (d == 64) return G == 1 || G == 2 || G == 4;
-  return G == 1 || G == 2 || G == 4 || G == 8;
+  const bool shape = d == 64 ? (G == 1 || G == 2 || G == 4) : (G == 1 || G == 2 || G == 4 || G == 8);
+  if (!shape) return false;
+  return !p.tc_global || global_streams(p, true) >= 0;
 }
 
-size_t tc_scratch_bytes(const Problem &) { return 0; }
+size_t tc_scratch_bytes(const Problem &p) {
+  const int nx = global_streams(p, p.tc_global != 0);
+  return exchange_bytes(p.dims[0], cluster_size(p), nx);
+}
 
 static unsigned long long g_wait_ns = 2000000000ull;  // 2 s per wait
 static int g_inject_timeout = 0;
@@ -857,34 +1064,67 @@ void tc_set_debug(int inject_timeout, unsigned long long wait_ns) {
   g_wait_ns = wait_ns ? wait_ns : 2000000000ull;
 }
 
+namespace {
+
+template <int D, int G>
+cudaError_t launch_both(const Problem &p, cudaStream_t stream, int nc, int nx, unsigned char *xbuf) {
+  const size_t td = (size_t)p.T * D;
+  TcArgs base;
+  std::memset(&base, 0, sizeof base);
+  base.T = p.T;
+  base.P = (int)p.P;
+  base.G = G;
+  base.status = p.status;
+  base.wait_ns = g_wait_ns;
+  base.inject_timeout = g_inject_timeout;
+  // streams [s0, s0 + n) of the problem
+  auto run = [&](int s0, int n, bool xg, bool after) -> cudaError_t {
+    CUtensorMap mk, mq;
+    const __nv_bfloat16 *k = static_cast<const __nv_bfloat16 *>(p.k) + (size_t)s0 * td;
+    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(p.q) + (size_t)s0 * td;
+    if (!make_token_map(&mk, k, (long long)n * p.T, D) || !make_token_map(&mq, q, (long long)n * p.T, D))
+      return cudaErrorInvalidValue;
+    TcArgs a = base;
+    a.v = static_cast<const __nv_bfloat16 *>(p.v) + (size_t)s0 * td;
+    a.theta = p.theta + (size_t)s0 * p.T;
+    a.eta = p.eta + (size_t)s0 * p.T;
+    a.alpha = p.alpha + (size_t)s0 * p.T;
+    a.W0 = p.W0 + (size_t)s0 * p.P;
+    a.S0 = p.S0 + (size_t)s0 * p.P;
+    a.y = p.y + (size_t)s0 * td;
+    a.W = p.W_end + (size_t)s0 * p.P;
+    a.S = p.S_end + (size_t)s0 * p.P;
+    if (!xg) return launch_dg<D, G, false>(n, stream, a, mk, mq, false);
+    a.xflag = reinterpret_cast<unsigned *>(xbuf);
+    a.xg2 = xbuf + up256((size_t)n * xflag_bytes(G));
+    a.xrecv = a.xg2 + up256((size_t)n * xg2_bytes(D));
+    return launch_dg<D, G, true>(n, stream, a, mk, mq, after);
+  };
+  cudaError_t e = cudaSuccess;
+  if (nx > 0) {
+    e = cudaMemsetAsync(xbuf, 0, (size_t)nx * xflag_bytes(G), stream);
+    if (e != cudaSuccess) return e;
+  }
+  if (nc > 0) e = run(0, nc, false, false);
+  if (e == cudaSuccess && nx > 0) e = run(nc, nx, true, nc > 0);
+  return e;
+}
+
+}  // namespace
+
 cudaError_t tc_launch(const Problem &p, cudaStream_t stream) {
   if (!tc_supported(p)) return cudaErrorNotSupported;
-  CUtensorMap mk, mq;
-  const long long rows = (long long)p.streams * p.T;
-  if (!make_token_map(&mk, p.k, rows, p.dims[0]) || !make_token_map(&mq, p.q, rows, p.dims[0]))
-    return cudaErrorInvalidValue;
-  TcArgs a;
-  a.T = p.T;
-  a.P = (int)p.P;
-  a.G = cluster_size(p);
-  a.v = reinterpret_cast<const __nv_bfloat16 *>(p.v);
-  a.theta = p.theta;
-  a.eta = p.eta;
-  a.alpha = p.alpha;
-  a.W0 = p.W0;
-  a.S0 = p.S0;
-  a.y = p.y;
-  a.W = p.W_end;
-  a.S = p.S_end;
-  a.status = p.status;
-  a.wait_ns = g_wait_ns;
-  a.inject_timeout = g_inject_timeout;
-  const int d = p.dims[0];
-  switch (a.G) {
-    case 1: return d == 64 ? launch_dg<64, 1>(p, stream, a, mk, mq) : launch_dg<128, 1>(p, stream, a, mk, mq);
-    case 2: return d == 64 ? launch_dg<64, 2>(p, stream, a, mk, mq) : launch_dg<128, 2>(p, stream, a, mk, mq);
-    case 4: return d == 64 ? launch_dg<64, 4>(p, stream, a, mk, mq) : launch_dg<128, 4>(p, stream, a, mk, mq);
-    case 8: return launch_dg<128, 8>(p, stream, a, mk, mq);
+  const int G = cluster_size(p), d = p.dims[0];
+  const int nx = global_streams(p, p.tc_global != 0);
+  if (nx < 0) return cudaErrorNotSupported;
+  const int nc = p.streams - nx;
+  unsigned char *xbuf = static_cast<unsigned char *>(p.scratch);
+  if (nx > 0 && (!xbuf || p.scratch_bytes < exchange_bytes(d, G, nx))) return cudaErrorInvalidValue;
+  switch (G) {
+    case 1: return d == 64 ? launch_both<64, 1>(p, stream, nc, nx, xbuf) : launch_both<128, 1>(p, stream, nc, nx, xbuf);
+    case 2: return d == 64 ? launch_both<64, 2>(p, stream, nc, nx, xbuf) : launch_both<128, 2>(p, stream, nc, nx, xbuf);
+    case 4: return d == 64 ? launch_both<64, 4>(p, stream, nc, nx, xbuf) : launch_both<128, 4>(p, stream, nc, nx, xbuf);
+    case 8: return launch_both<128, 8>(p, stream, nc, nx, xbuf);
   }
   return cudaErrorNotSupported;
 }

@@ -41,7 +41,8 @@ class NeuralMemory:
 
     def set_path(self, path: str) -> None:
         code = {"auto": N.TM_PATH_AUTO, "simt": N.TM_PATH_SIMT, "tc": N.TM_PATH_TC,
-                "tcl": N.TM_PATH_TC_LAYERED, "tcl-phased": N.TM_PATH_TC_PHASED}[path]
+                "tcl": N.TM_PATH_TC_LAYERED, "tcl-phased": N.TM_PATH_TC_PHASED,
+                "tc-global": N.TM_PATH_TC_GLOBAL}[path]
         N.check(self._lib.tm_set_path(self._h, code), "tm_set_path")
         self.path = path
 
@@ -58,7 +59,7 @@ class NeuralMemory:
         code = N.TM_BF16 if dtype == torch.bfloat16 else N.TM_F32
         N.check(self._lib.tm_query_path(self._h, B, H, T, C, code, ctypes.byref(out)), "tm_query_path")
         return {N.TM_PATH_SIMT: "simt", N.TM_PATH_TC: "tc", N.TM_PATH_TC_LAYERED: "tcl",
-                N.TM_PATH_TC_PHASED: "tcl-phased"}[out.value]
+                N.TM_PATH_TC_PHASED: "tcl-phased", N.TM_PATH_TC_GLOBAL: "tc-global"}[out.value]
 
     def launch_count(self, B, H, T, C, dtype=torch.bfloat16) -> int:
         """Kernel launches one run() of this problem makes."""

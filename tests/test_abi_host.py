@@ -90,6 +90,7 @@ def test_path_selection_and_query():
     assert lib.tm_query_path(h, 1, 1, 256, 16, N.TM_F32, ctypes.byref(p)) == N.TM_OK
     assert p.value == N.TM_PATH_SIMT
     assert lib.tm_set_path(h, 9) == N.TM_ERR_INVALID_ARG
+    assert lib.tm_set_path(h, N.TM_PATH_TC_GLOBAL) == N.TM_OK
     assert lib.tm_set_path(h, N.TM_PATH_TC_PHASED) == N.TM_OK
     assert lib.tm_query_path(h, 1, 1, 256, 64, N.TM_BF16, ctypes.byref(p)) == N.TM_OK
     assert p.value == N.TM_PATH_TC_PHASED

@@ -215,6 +215,41 @@ def test_tc_small_shapes(cfg):
     check(w, "tc", TOL_BF16_TC)
 
 
+@pytest.mark.parametrize("cfg", TC_SHAPES + [(128, 4, 1, 2, 256)], ids=lambda c: "d%d-e%d-B%dH%d-T%d" % c)
+def test_tc_global_exchange_small_shapes(cfg):
+    """The chunk walker with its CTAs exchanging through global memory (no
+    cluster): against the oracle, and bit for bit against the cluster form
+    (same bf16 partials, same fp32 summation order)."""
+    d, e, B, H, T = cfg
+    w = W.make(2, d, e, B, H, T, 64, index=420 + sum(cfg))
+    check(w, "tc-global", TOL_BF16_TC)
+    inp, dev = _dev_inputs(w)
+    outs = {}
+    for path in ("tc", "tc-global"):
+        mem = NeuralMemory(2, d, e, path=path)
+        outs[path] = gpu_to_np(*run_lib(mem, dev, w.C))
+    for key in ("y", "W_end", "S_end"):
+        np.testing.assert_array_equal(outs["tc"][key], outs["tc-global"][key], err_msg=key)
+
+
+def test_tc_streams_beyond_resident_clusters():
+    """16 streams of the long d=128 shape: 15 clusters of 8 fit at once, the
+    16th stream runs beside them on the global-exchange walker. Every
+    stream against the oracle, and the whole result bit for bit against the
+    all-global form."""
+    w = W.make(2, 128, 4, 1, 16, 256, 64, index=430)
+    mem = NeuralMemory(2, 128, 4)
+    assert mem.query_path(1, 16, 256, 64) == "tc"
+    check(w, "tc", TOL_BF16_TC)
+    inp, dev = _dev_inputs(w)
+    outs = {}
+    for path in ("tc", "tc-global"):
+        m = NeuralMemory(2, 128, 4, path=path)
+        outs[path] = gpu_to_np(*run_lib(m, dev, w.C))
+    for key in ("y", "W_end", "S_end"):
+        np.testing.assert_array_equal(outs["tc"][key], outs["tc-global"][key], err_msg=key)
+
+
 def test_tc_cluster_of_eight_d128():
     """Hidden 512 split over a cluster of 8 CTAs (the long-stream shape)."""
     check(W.make(2, 128, 4, 1, 2, 256, 64, index=410), "tc", TOL_BF16_TC)
