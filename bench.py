@@ -259,13 +259,14 @@ def sweep_chunk(args, w: W.Workload, sizes):
                           "workspace_bytes": ws.numel()}), flush=True)
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
-# the cluster kernel, from one ncu --set full capture of a shortened case of
-# the long d=128 workload (16 streams x 4096 tokens: 68.39 MB read, 13.09 MB
-# written; the summary is kept under profiles/). The kernel's traffic grows
-# with the tokens it processes (inputs and reads stream through once, the
-# state stays on chip), so a full launch is that figure scaled by tokens.
-CAPTURED_TRAFFIC = {("tc", "mlp2-d128-long"): (68.387072e6 + 13.085184e6, 16 * 4096)}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one run of the
+# chunk walker (the cluster kernel for 15 streams and the global-exchange
+# kernel for the 16th), from one ncu --set full capture of a shortened case
+# of the long d=128 workload (16 streams x 4096 tokens: 64.16 + 9.94 MB and
+# 4.32 + 0 MB; the summary is kept under profiles/). The traffic grows with
+# the tokens processed (inputs and reads stream through once, the state stays
+# on chip), so a full run is that figure scaled by tokens.
+CAPTURED_TRAFFIC = {("tc", "mlp2-d128-long"): (64.163584e6 + 9.935360e6 + 4.315904e6, 16 * 4096)}
 
 
 def traffic_per_launch(path: str, w: W.Workload):
@@ -437,7 +438,8 @@ def main():
                 "sm_mhz_seen": sm_mhz}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = traffic_per_launch(path_used, w)
-    roof["kernel"] = {"tc": "tc_chunk_kernel", "tcl": "tcl_fb_kernel + tcl_gemm_kernel",
+    roof["kernel"] = {"tc": "tc_chunk_kernel (cluster and global-exchange forms)",
+                      "tcl": "tcl_fb_kernel + tcl_dw_kernel",
                       "tcl-phased": "tcl_gemm_kernel"}.get(path_used, "simt_chunk_kernel")
 
     e2e = None

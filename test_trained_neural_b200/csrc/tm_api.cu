@@ -191,7 +191,9 @@ tm_status tm_launch_count(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtyp
   tm_path path = choose_path(ctx, p);
   if (!path_supported(path, p)) return TM_ERR_UNSUPPORTED;
   p.fuse_fb = path == TM_PATH_TC_LAYERED;
-  *out = (path == TM_PATH_TC_LAYERED || path == TM_PATH_TC_PHASED) ? tmem::tcl_launch_count(p) : 1;
+  *out = (path == TM_PATH_TC_LAYERED || path == TM_PATH_TC_PHASED) ? tmem::tcl_launch_count(p)
+         : (path == TM_PATH_TC || path == TM_PATH_TC_GLOBAL)       ? tmem::tc_launch_count(p)
+                                                                   : 1;
   return TM_OK;
 }
 

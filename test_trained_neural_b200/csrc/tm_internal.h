@@ -55,6 +55,7 @@ cudaError_t simt_launch(const Problem &p, cudaStream_t stream);
 // Tensor-core (tcgen05) path.
 bool tc_supported(const Problem &p);
 size_t tc_scratch_bytes(const Problem &p);
+int tc_launch_count(const Problem &p);
 cudaError_t tc_launch(const Problem &p, cudaStream_t stream);
 // Layer-by-layer tensor-core path 
 bool tcl_supported(const Problem &p);

@@ -1051,6 +1051,12 @@ bool tc_supported(const Problem &p) {
   return !p.tc_global || global_streams(p, true) >= 0;
 }
 
+int tc_launch_count(const Problem &p) {
+  const int nx = global_streams(p, p.tc_global != 0);
+  if (nx < 0) return 0;
+  return (p.streams - nx > 0 ? 1 : 0) + (nx > 0 ? 1 : 0);
+}
+
 size_t tc_scratch_bytes(const Problem &p) {
   const int nx = global_streams(p, p.tc_global != 0);
   return exchange_bytes(p.dims[0], cluster_size(p), nx);
