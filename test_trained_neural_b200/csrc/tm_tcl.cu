@@ -520,6 +520,10 @@ __global__ void __launch_bounds__(FB_NT, 1)
   const int nphase = has_keys ? 2 * L - 1 : L;
   // key rows of this tile (keys precede queries)
   const int nkey = C - 128 * mt >= 128 ? 128 : (C - 128 * mt > 0 ? C - 128 * mt : 0);
+  // silu'(Z_l) of key rows for the backward: the last two hidden layers keep
+  // it in TMEM (bf16 pairs in columns 256-383 and 384-511, beside the
+  // accumulator in 0-255); earlier layers go through global memory
+  auto sp_slot = [&](int l) -> int { return L - 1 - l < 2 ? 256 + 128 * ((L - 1 - l) & 1) : -1; };
 
   if (tid == 0) {
     for (int i = 0; i < FB_STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
@@ -529,7 +533,7 @@ __global__ void __launch_bounds__(FB_NT, 1)
     abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0) { tmem_alloc(&tslot, 256); tmem_relinquish(); }
+  if (warp == 0) { tmem_alloc(&tslot, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -652,7 +656,8 @@ __global__ void __launch_bounds__(FB_NT, 1)
       // layer below, which this same thread stored going forward), requested
       // before the MMAs finish
       uint4 aux[8];
-      if (grad && key) {
+      const int spt = f.bwd ? sp_slot(f.l - 1) : -1;      // silu' of the layer below in TMEM?
+      if (grad && key && spt < 0) {
         const __nv_bfloat16 *src = f.bwd ? a.sp_out[f.l - 1] + ((long long)s * C + r) * N
                                          : a.v + tok * N;
 #pragma unroll
@@ -687,9 +692,17 @@ __global__ void __launch_bounds__(FB_NT, 1)
 #pragma unroll
           for (int i = 0; i < 2; ++i) st_shared_v4(abuf + rb_chunk(128, row, c0 / 8 + i), pack8(x + 8 * i));
           if (key) {
-            __nv_bfloat16 *so = a.sp_out[f.l] + ((long long)s * C + r) * N + c0;
-            *reinterpret_cast<uint4 *>(so) = pack8(sp);
-            *reinterpret_cast<uint4 *>(so + 8) = pack8(sp + 8);
+            const int slot = sp_slot(f.l);
+            if (slot >= 0) {
+              uint32_t pk[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) pk[i] = pack_bf16(sp[2 * i], sp[2 * i + 1]);
+              tmem_st8(tm + lb + (uint32_t)(slot + c0 / 2), pk);
+            } else {
+              __nv_bfloat16 *so = a.sp_out[f.l] + ((long long)s * C + r) * N + c0;
+              *reinterpret_cast<uint4 *>(so) = pack8(sp);
+              *reinterpret_cast<uint4 *>(so + 8) = pack8(sp + 8);
+            }
           }
         } else if (!key) {
           if (last_fwd) {                        // query row of the last layer: the read y
@@ -700,6 +713,13 @@ __global__ void __launch_bounds__(FB_NT, 1)
           }
         } else {
           // G_L = 2 (Z_L - V) or G_{l-1} = (G_l W_l) . silu'(Z_{l-1})
+          if (spt >= 0) {
+            uint32_t pk[8];
+            tmem_ld8(tm + lb + (uint32_t)(spt + c0 / 2), pk);
+            tmem_wait_ld();
+            aux[2 * step] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            aux[2 * step + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             const uint4 u = aux[2 * step + i];
@@ -714,6 +734,7 @@ __global__ void __launch_bounds__(FB_NT, 1)
           }
         }
       }
+      if (!grad) tmem_wait_st();                 // silu' stored into TMEM above
       // the tile (generic-proxy writes) is read by the next phase's MMAs
       fence_proxy_async_smem();
       tc_fence_before();
@@ -729,7 +750,7 @@ __global__ void __launch_bounds__(FB_NT, 1)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tm, 256);
+  if (warp == 0) tmem_dealloc(tm, 512);
 }
 
 // A5 for every chunk of every stream at once: one thread per (stream, chunk)
