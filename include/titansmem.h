@@ -53,7 +53,7 @@ typedef struct tm_ctx tm_ctx; /* opaque; owned by the library */
 
 typedef enum {
   TM_OK = 0,
-  TM_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, T % C != 0 ... */
+  TM_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size ...                 */
   TM_ERR_UNSUPPORTED = 2,  /* valid but not implemented (shape, dtype, path)   */
   TM_ERR_CUDA = 3,         /* a CUDA runtime call failed (launch, sync ...)    */
   TM_ERR_OOM = 4,          /* host allocation failed, or workspace too small   */
@@ -144,7 +144,10 @@ TM_API tm_status tm_workspace_size(const tm_ctx *ctx, int B, int H, int T, int C
  *
  * All pointers must be 16-byte aligned. W_end may equal W0 and S_end may equal
  * S0 (in-place update); no other aliasing is allowed, and y must not overlap
- * any input. Requires T % C == 0, 1 <= C <= 256, T >= C.
+ * any input. Requires 1 <= C <= 256 and T >= 1. Chunks start at multiples
+ * of C; when C does not divide T the last chunk is shorter (T % C tokens). On
+ * the tensor-core paths the whole chunks run first and that last chunk runs
+ * after them on the CUDA-core kernel, from the state they left.
  *
  * Errors: argument problems return at once with no launch (TM_ERR_OOM when
  * workspace_bytes is too small). A device-side error (an expired bounded wait,

@@ -35,7 +35,7 @@ bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb) {
 tm_status check_shape(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype dt) {
   if (!ctx) return TM_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || T < 1 || C < 1) return TM_ERR_INVALID_ARG;
-  if (C > tmem::kMaxC || T < C || T % C != 0) return TM_ERR_INVALID_ARG;
+  if (C > tmem::kMaxC) return TM_ERR_INVALID_ARG;
   if (dt != TM_F32 && dt != TM_BF16) return TM_ERR_INVALID_ARG;
   if ((long long)B * H > (1LL << 31) - 1) return TM_ERR_INVALID_ARG;
   return TM_OK;
@@ -57,6 +57,10 @@ tmem::Problem make_problem(const tm_ctx *ctx, int B, int H, int T, int C, tm_dty
   p.in_dtype = dt;
   p.fuse_fb = 1;
   p.tc_global = ctx->path == TM_PATH_TC_GLOBAL;
+  // the tensor-core paths run the whole chunks; a shorter last chunk
+  // (T % C tokens) runs after them on the CUDA-core kernel
+  p.T_run = T - T % C;
+  p.t_begin = 0;
   return p;
 }
 
@@ -73,10 +77,20 @@ bool path_supported(tm_path path, const tmem::Problem &p) {
   return true;
 }
 
+bool tensor_path(tm_path path) {
+  return path == TM_PATH_TC || path == TM_PATH_TC_GLOBAL || path == TM_PATH_TC_LAYERED ||
+         path == TM_PATH_TC_PHASED;
+}
+
+// Workspace after the status word. A tensor-core path with a shorter last
+// chunk runs it afterwards on the CUDA-core kernel, in the same space.
 size_t scratch_bytes(tm_path path, const tmem::Problem &p) {
-  if (path == TM_PATH_TC || path == TM_PATH_TC_GLOBAL) return tmem::tc_scratch_bytes(p);
-  if (path == TM_PATH_TC_LAYERED || path == TM_PATH_TC_PHASED) return tmem::tcl_scratch_bytes(p);
-  return tmem::simt_scratch_bytes(p);
+  size_t b = tmem::simt_scratch_bytes(p);
+  if (!tensor_path(path)) return b;
+  const size_t m = (path == TM_PATH_TC || path == TM_PATH_TC_GLOBAL) ? tmem::tc_scratch_bytes(p)
+                                                                    : tmem::tcl_scratch_bytes(p);
+  if (p.T_run == p.T) return m;
+  return m > b ? m : b;
 }
 
 }  // namespace
@@ -191,9 +205,14 @@ tm_status tm_launch_count(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtyp
   tm_path path = choose_path(ctx, p);
   if (!path_supported(path, p)) return TM_ERR_UNSUPPORTED;
   p.fuse_fb = path == TM_PATH_TC_LAYERED;
-  *out = (path == TM_PATH_TC_LAYERED || path == TM_PATH_TC_PHASED) ? tmem::tcl_launch_count(p)
-         : (path == TM_PATH_TC || path == TM_PATH_TC_GLOBAL)       ? tmem::tc_launch_count(p)
-                                                                   : 1;
+  long long n = 1;
+  if (tensor_path(path)) {
+    n = p.T_run == 0 ? 0
+        : (path == TM_PATH_TC_LAYERED || path == TM_PATH_TC_PHASED) ? tmem::tcl_launch_count(p)
+                                                                    : tmem::tc_launch_count(p);
+    if (p.T_run < p.T) n += 1;                 // the shorter last chunk
+  }
+  *out = n;
   return TM_OK;
 }
 
@@ -275,9 +294,24 @@ tm_status tm_run(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype, con
       p.ev_fork = ctx->ev_fork;
     }
   }
-  cudaError_t err = (path == TM_PATH_TC || path == TM_PATH_TC_GLOBAL) ? tmem::tc_launch(p, s)
-                    : (path == TM_PATH_TC_LAYERED || path == TM_PATH_TC_PHASED) ? tmem::tcl_launch(p, s)
-                                                                              : tmem::simt_launch(p, s);
+  cudaError_t err = cudaSuccess;
+  if (!tensor_path(path)) {
+    p.T_run = p.T;                             // the CUDA-core kernel runs the short chunk itself
+    err = tmem::simt_launch(p, s);
+  } else {
+    if (p.T_run > 0)
+      err = (path == TM_PATH_TC || path == TM_PATH_TC_GLOBAL) ? tmem::tc_launch(p, s) : tmem::tcl_launch(p, s);
+    if (err == cudaSuccess && p.T_run < p.T) {
+      // the shorter last chunk, from the state the whole chunks left
+      tmem::Problem q = p;
+      q.t_begin = p.T_run;
+      if (p.T_run > 0) {
+        q.W0 = p.W_end;
+        q.S0 = p.S_end;
+      }
+      err = tmem::simt_launch(q, s);
+    }
+  }
   return err == cudaSuccess ? TM_OK : TM_ERR_CUDA;
 }
 

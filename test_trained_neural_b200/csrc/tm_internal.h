@@ -27,6 +27,8 @@ struct Problem {
   size_t layer_off[kMaxL + 1];
   size_t P;
   int B, H, T, C;
+  int T_run;              // tokens per stream the launch processes (from t_begin); T is the stride
+  int t_begin;            // CUDA-core path: first token of each stream
   int streams;
   tm_dtype in_dtype;
   const void *k, *v, *q;

@@ -209,6 +209,7 @@ __device__ void chunk_coefficients(Coef &cf, const float *theta, const float *et
 struct KArgs {
   Net net;
   int T, C, bf16;
+  int t_begin;                   // first token of each stream to process
   const void *k, *v, *q;
   const float *theta, *eta, *alpha, *W0, *S0;
   float *y, *W, *S;
@@ -248,10 +249,12 @@ __global__ void __launch_bounds__(NT) simt_chunk_kernel(KArgs a) {
   __syncthreads();
 
   const long long tok_base = (long long)s * T;
-  for (int t0 = 0; t0 < T; t0 += C) {
+  // chunks start at t_begin + multiples of C; the last one may be shorter
+  for (int t0 = a.t_begin; t0 < T; t0 += C) {
     const long long tb = tok_base + t0;
-    chunk_coefficients(sm.coef, a.theta + tb, a.eta + tb, a.alpha + tb, C);
-    for (int i = threadIdx.x; i < C * d_in; i += NT) {
+    const int Cc = T - t0 < C ? T - t0 : C;       // tokens in this chunk
+    chunk_coefficients(sm.coef, a.theta + tb, a.eta + tb, a.alpha + tb, Cc);
+    for (int i = threadIdx.x; i < Cc * d_in; i += NT) {
       X[0][i] = load_tok(a.k, a.bf16, tb * d_in + i);
       Qa[i] = load_tok(a.q, a.bf16, tb * d_in + i);
     }
@@ -264,13 +267,13 @@ __global__ void __launch_bounds__(NT) simt_chunk_kernel(KArgs a) {
       const int rows = n.dims[l], cols = n.dims[l - 1];
       if (l < L) {
         float *Zl = Z[l], *Xl = X[l];
-        gemm(sm, C, rows, cols, X[l - 1], cols, 1, Wl, cols, 1,
+        gemm(sm, Cc, rows, cols, X[l - 1], cols, 1, Wl, cols, 1,
              [&](int i, int r, float z) {
                Zl[(long long)i * rows + r] = z;
                Xl[(long long)i * rows + r] = silu(z);
              });
       } else {
-        gemm(sm, C, rows, cols, X[l - 1], cols, 1, Wl, cols, 1,
+        gemm(sm, Cc, rows, cols, X[l - 1], cols, 1, Wl, cols, 1,
              [&](int i, int r, float z) {
                float vv = load_tok(a.v, a.bf16, (tb + i) * d_out + r);
                Gcur[(long long)i * rows + r] = 2.f * (z - vv);
@@ -284,12 +287,12 @@ __global__ void __launch_bounds__(NT) simt_chunk_kernel(KArgs a) {
       const float *Wl = W + n.off[l - 1];
       const int rows = n.dims[l], cols = n.dims[l - 1];
       if (l < L) {
-        gemm(sm, C, rows, cols, qin, cols, 1, Wl, cols, 1,
+        gemm(sm, Cc, rows, cols, qin, cols, 1, Wl, cols, 1,
              [&](int i, int r, float z) { qout[(long long)i * rows + r] = silu(z); });
         float *tmp = qin; qin = qout; qout = tmp;
       } else {
         float *y = a.y + tb * d_out;
-        gemm(sm, C, rows, cols, qin, cols, 1, Wl, cols, 1,
+        gemm(sm, Cc, rows, cols, qin, cols, 1, Wl, cols, 1,
              [&](int i, int r, float z) { y[(long long)i * rows + r] = z; });
       }
       __syncthreads();
@@ -306,7 +309,7 @@ __global__ void __launch_bounds__(NT) simt_chunk_kernel(KArgs a) {
       const int rows = n.dims[l], cols = n.dims[l - 1];
       float *Gout = pool[(L - l) % 3];
       const float *Zp = Z[l - 1];
-      gemm(sm, C, cols, rows, Gl[l], rows, 1, Wl, 1, cols,
+      gemm(sm, Cc, cols, rows, Gl[l], rows, 1, Wl, 1, cols,
            [&](int i, int c, float g) {
              long long idx = (long long)i * cols + c;
              Gout[idx] = g * silu_prime(Zp[idx]);
@@ -316,7 +319,7 @@ __global__ void __launch_bounds__(NT) simt_chunk_kernel(KArgs a) {
     }
     // A6 + A7: per-layer dual contraction and fused state update.
     for (int l = 1; l <= L; ++l) {
-      update_layer(sm, n.dims[l], n.dims[l - 1], C, Gl[l], X[l - 1], W + n.off[l - 1],
+      update_layer(sm, n.dims[l], n.dims[l - 1], Cc, Gl[l], X[l - 1], W + n.off[l - 1],
                    S + n.off[l - 1]);
     }
     __syncthreads();
@@ -348,6 +351,7 @@ cudaError_t simt_launch(const Problem &p, cudaStream_t stream) {
   a.net.P = (long long)p.P;
   a.T = p.T;
   a.C = p.C;
+  a.t_begin = p.t_begin;
   a.bf16 = p.in_dtype == TM_BF16;
   a.k = p.k; a.v = p.v; a.q = p.q;
   a.theta = p.theta; a.eta = p.eta; a.alpha = p.alpha;

@@ -61,6 +61,7 @@ constexpr uint32_t TMEM_COLS = 512;
 
 struct TcArgs {
   int T, P, G;
+  int nchunks;                   // chunks per stream to process (T is the token stride)
   const __nv_bfloat16 *v;
   const float *theta, *eta, *alpha;
   const float *W0, *S0;
@@ -369,7 +370,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   unsigned *const xfl = XG ? a.xflag + (size_t)stream * (G + 1) * XFLAG_STRIDE : nullptr;
   unsigned char *const xrv = XG ? a.xrecv + (size_t)stream * xrecv_bytes(D, G) : nullptr;
   unsigned char *const xg2 = XG ? a.xg2 + (size_t)stream * xg2_bytes(D) : nullptr;
-  const int T = a.T, nchunks = T / C, P = a.P;
+  const int T = a.T, nchunks = a.nchunks, P = a.P;
   const int Hd = HS * G;             // hidden width
   float *Wg = a.W + (long long)stream * P;
   float *Sg = a.S + (long long)stream * P;
@@ -1078,6 +1079,7 @@ cudaError_t launch_both(const Problem &p, cudaStream_t stream, int nc, int nx, u
   TcArgs base;
   std::memset(&base, 0, sizeof base);
   base.T = p.T;
+  base.nchunks = p.T_run / C;
   base.P = (int)p.P;
   base.G = G;
   base.status = p.status;

@@ -759,8 +759,7 @@ __global__ void __launch_bounds__(FB_NT, 1)
 //   r_{C-1} = 1, r_i = pa_i + eta_{i+1} r_{i+1};  c_i = theta_i r_i, e_i = theta_i pe_i;
 //   B = prod(1 - alpha), A = prod eta, c_S = eta_0 r_0.
 __global__ void tcl_coef_kernel(const float *theta, const float *eta, const float *alpha, int streams,
-                                int T, int C, float *coef, float *scal) {
-  const int nchunks = T / C;
+                                int T, int C, int nchunks, float *coef, float *scal) {
   const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (id >= (long long)streams * nchunks) return;
   const long long s = id / nchunks, ch = id % nchunks;
@@ -989,7 +988,7 @@ cudaError_t TclGroup::setup() {
   coef = reinterpret_cast<float *>(ws + cv.coef);
   scal = reinterpret_cast<float *>(ws + cv.scal);
   wbf = reinterpret_cast<__nv_bfloat16 *>(ws + cv.wbf);
-  L = p.L; C = p.C; T = p.T; S = p.streams; nchunks = T / C;
+  L = p.L; C = p.C; T = p.T; S = p.streams; nchunks = p.T_run / C;
   const int d = p.dims[0];
   cudaStream_t stream = st;
 
@@ -1005,7 +1004,7 @@ cudaError_t TclGroup::setup() {
   tcl_init_kernel<<<592, 256, 0, stream>>>(ia);
   const long long nct = (long long)S * nchunks;
   tcl_coef_kernel<<<(unsigned)((nct + 127) / 128), 128, 0, stream>>>(p.theta, p.eta, p.alpha, S, T, C,
-                                                                     coef, scal);
+                                                                     nchunks, coef, scal);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
 
@@ -1203,7 +1202,7 @@ long long tcl_launch_count(const Problem &p) {
   // per group: init and coefficient kernels, then per chunk the fused
   // forward + backward (or 2L - 1 phase launches) and one update launch
   const long long per_chunk = (p.fuse_fb && fb_ok(p)) ? 2 : 2LL * p.L;
-  return (long long)tcl_group_count(p) * (2 + per_chunk * (p.T / p.C));
+  return (long long)tcl_group_count(p) * (2 + per_chunk * (p.T_run / p.C));
 }
 
 cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
@@ -1242,7 +1241,7 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
     err = t.setup();
   }
   // launches of the groups interleaved chunk by chunk
-  const int nchunks = p.T / p.C;
+  const int nchunks = p.T_run / p.C;
   for (int ch = 0; ch < nchunks && err == cudaSuccess; ++ch)
     for (int g = 0; g < G && err == cudaSuccess; ++g) err = groups[(size_t)g].chunk(ch);
   if (G > 1) {

@@ -75,9 +75,11 @@ def test_workspace_and_shape_validation():
     out = ctypes.c_size_t()
     assert lib.tm_workspace_size(h, 4, 8, 8192, 64, N.TM_BF16, ctypes.byref(out)) == N.TM_OK
     assert out.value >= 256 and out.value % 4 == 0
-    for B, H, T, C in [(0, 1, 64, 64), (1, 0, 64, 64), (1, 1, 100, 64), (1, 1, 32, 64),
-                       (1, 1, 512, 512), (1, 1, 64, 0)]:
+    for B, H, T, C in [(0, 1, 64, 64), (1, 0, 64, 64), (1, 1, 0, 64), (1, 1, 512, 512), (1, 1, 64, 0)]:
         assert lib.tm_workspace_size(h, B, H, T, C, N.TM_BF16, ctypes.byref(out)) == N.TM_ERR_INVALID_ARG
+    # a shorter last chunk (C does not divide T, or T < C) is accepted
+    for T in (100, 32):
+        assert lib.tm_workspace_size(h, 1, 1, T, 64, N.TM_BF16, ctypes.byref(out)) == N.TM_OK
     assert lib.tm_workspace_size(h, 1, 1, 64, 64, 9, ctypes.byref(out)) == N.TM_ERR_INVALID_ARG
     assert lib.tm_workspace_size(None, 1, 1, 64, 64, N.TM_BF16, ctypes.byref(out)) == N.TM_ERR_INVALID_ARG
     lib.tm_destroy(h)
@@ -141,7 +143,7 @@ def test_run_rejects_bad_arguments_before_any_launch():
     bad_ws_align = list(base)
     bad_ws_align[11] += 16
     assert _run(lib, h, bad_ws_align) == N.TM_ERR_INVALID_ARG
-    assert _run(lib, h, base, T=60, C=16) == N.TM_ERR_INVALID_ARG
+    assert _run(lib, h, base, T=0, C=16) == N.TM_ERR_INVALID_ARG
     assert _run(lib, h, base, C=0) == N.TM_ERR_INVALID_ARG
     # y overlapping k
     ov = list(base)

@@ -336,6 +336,28 @@ def test_tcl_fused_matches_phased():
     assert max(errs.values()) < 5e-3, errs
 
 
+RAGGED = [  # L, d, expansion, B, H, T, C, dtype, path
+    (1, 64, 1, 1, 1, 100, 16, "f32", "simt"),     # linear memory, 6 whole chunks + 4 tokens
+    (2, 32, 4, 2, 1, 75, 32, "bf16", "simt"),
+    (2, 64, 4, 1, 2, 209, 64, "bf16", "tc"),       # 3 whole chunks on the cluster kernel + 17
+    (2, 64, 4, 1, 2, 40, 64, "bf16", "tc"),        # T < C: only the short chunk
+    (4, 64, 2, 1, 2, 296, 128, "bf16", "tcl"),     # 2 whole chunks, fused layered kernels + 40
+    (2, 128, 3, 1, 1, 150, 64, "bf16", "tcl"),     # per-phase layered kernels + 22
+]
+
+
+@pytest.mark.parametrize("cfg", RAGGED, ids=lambda c: "L%d-d%d-e%d-B%dH%d-T%d-C%d-%s-%s" % c)
+def test_shorter_last_chunk(cfg):
+    """C does not divide T: chunks start at multiples of C and the last one is
+    shorter (the oracle's partial last chunk). The tensor-core paths run the
+    whole chunks, then the short one on the CUDA-core kernel."""
+    L, d, e, B, H, T, C, dt, path = cfg
+    w = W.make(L, d, e, B, H, T, C, dtype=dt, index=640 + T)
+    mem = NeuralMemory(L, d, e)
+    assert mem.query_path(B, H, T, C, torch.bfloat16 if dt == "bf16" else torch.float32) == path
+    check(w, path, TOL_F32 if dt == "f32" else TOL_BF16_TC)
+
+
 def test_tcl_literal_gates_short_stream():
     check(W.make(2, 64, 2, 1, 2, 128, 64, index=620, theta_damping=1.0, alpha_damping=1.0),
           "tcl", TOL_BF16_TC)
