@@ -277,6 +277,74 @@ def traffic_per_launch(path: str, w: W.Workload):
     return nbytes * (w.streams * w.T) / tokens
 
 
+def bench_decode(args, w: W.Workload):
+    """One-token decode steps on the workload's memory shape and streams: each
+    step reads one token per stream, writes y, and updates W and S in place.
+    HBM-bound: the algorithmic traffic is every parameter of W and S read and
+    written once (16P bytes per stream) plus the token's inputs and y."""
+    import torch
+    from test_trained_neural_b200 import NeuralMemory
+
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    B, H, d = w.B, w.H, w.d
+    mem = NeuralMemory(w.L, w.d, w.expansion)
+    k, v, q = (torch.randn((B, H, d), generator=g, device=dev).to(dt) for _ in range(3))
+    k = k / k.float().norm(dim=-1, keepdim=True).to(dt)
+    q = q / q.float().norm(dim=-1, keepdim=True).to(dt)
+    theta = torch.full((B, H), 1e-3, device=dev)
+    eta = torch.full((B, H), 0.9, device=dev)
+    alpha = torch.full((B, H), 1e-3, device=dev)
+    # Cold state every step without a flush (zeroing a large buffer would leave
+    # L2 full of dirty lines whose write-back lands inside a step this short):
+    # rotate through enough independent states that together exceed L2 three
+    # times; tiny states (which L2 holds anyway) fall back to the flush.
+    state_bytes = 2 * B * H * w.P * 4
+    nbuf = -(-3 * L2_BYTES // state_bytes)
+    use_flush = nbuf > 64
+    nbuf = 1 if use_flush else max(nbuf, 2)
+    states = []
+    for _ in range(nbuf):
+        Wst = 0.05 * torch.randn((B, H, w.P), generator=g, device=dev)
+        states.append((Wst, torch.zeros_like(Wst)))
+    y = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev) if use_flush else None
+    for i in range(max(args.warmup, nbuf)):
+        Wst, Sst = states[i % nbuf]
+        mem.decode_step(k, v, q, theta, eta, alpha, Wst, Sst, y)
+    torch.cuda.synchronize()
+    # steps are issued back to back (as a serving loop does), BURST per
+    # measurement, so the host's launch time overlaps the device's work
+    BURST = 1 if use_flush else 32
+    ms = []
+    for i in range(args.steps):
+        if use_flush:
+            flush.zero_()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+        for b in range(BURST):
+            Wst, Sst = states[(i * BURST + b) % nbuf]
+            mem.decode_step(k, v, q, theta, eta, alpha, Wst, Sst, y)
+        a1.record()
+        torch.cuda.synchronize()
+        ms.append(a0.elapsed_time(a1) / BURST)
+    t = statistics.mean(ms) * 1e-3
+    streams = B * H
+    el = 2 if dt == torch.bfloat16 else 4
+    bytes_ = streams * (16.0 * w.P + 3 * d * el + 12 + 4 * d)
+    peak = measured_peaks()
+    gbs = bytes_ / t / 1e9
+    print(json.dumps({"metric": "decode tokens/sec", "value": streams / t, "unit": "tokens/s", "us": t * 1e6,
+                      "workload": w.name, "streams": streams, "finite": bool(torch.isfinite(Wst).all()),
+                      "l2": "flushed between steps" if use_flush else "%d rotating states (%.0f MB)" % (
+                          nbuf, nbuf * state_bytes / 1e6),
+                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak["hbm_gbs"], "unit": "GB/s",
+                                   "frac": gbs / peak["hbm_gbs"], "peak_source": peak["source"] + " HBM copy"}}),
+          flush=True)
+
+
 def bench_prologue(args, w: W.Workload):
     """The step before the memory on the workload's k, v, q: one fused launch of
     the depthwise causal convolution (width args.conv_width) and the L2
@@ -332,6 +400,8 @@ def main():
     ap.add_argument("--prologue", action="store_true",
                     help="time the convolution + normalisation step before the memory instead")
     ap.add_argument("--conv-width", type=int, default=4)
+    ap.add_argument("--decode", action="store_true",
+                    help="time one-token decode steps on the workload's memory and streams instead")
     ap.add_argument("--sweep-chunk", default=None,
                     help="comma-separated chunk sizes: time each (same workload, T as given) "
                          "and print one JSON line per size instead of the benchmark line")
@@ -351,6 +421,8 @@ def main():
         return sweep_chunk(args, w, [int(x) for x in args.sweep_chunk.split(",")])
     if args.prologue:
         return bench_prologue(args, w)
+    if args.decode:
+        return bench_decode(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
 

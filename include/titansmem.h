@@ -197,6 +197,32 @@ TM_API tm_status tm_run_noalloc(tm_ctx *ctx, int B, int H, int T, int C, tm_dtyp
 TM_API tm_status tm_sync(tm_ctx *ctx, void *workspace, void *stream);
 
 /*
+ * One decode step: a single token per stream, the chunk size C = 1 form of
+ * the write-and-read ("Titans, explained" steps 2-6: surprise of the token at
+ * the current weights, momentum and forgetting, then the update). With the
+ * state (W, S) before the token: y = M_W(q) (the read sees none of this
+ * token's write), then S <- eta S - theta u and W <- (1 - alpha) W + S with
+ * u = grad_W ||M_W(k) - v||^2, in place. Same results as tm_run with T = C = 1
+ * and W_end = W0, S_end = S0 (fp32 arithmetic throughout), as one launch that
+ * reads and writes every parameter of W and S once.
+ *
+ *   k, v, q   [B, H, d_h] in_dtype, device      the token of each stream
+ *   theta, eta, alpha [B, H] float32, device
+ *   W, S      [B, H, P] float32, device         state, updated in place
+ *   y         [B, H, d_h] float32, device       output
+ *
+ * Supported: depth 1 (any d_h multiple of 4 up to 4096), or depth 2 with
+ * d_h in {64, 128} and hidden = 64 G, G in {1, 2, 4, 8} (one thread-block
+ * cluster of G CTAs per stream); TM_ERR_UNSUPPORTED otherwise (use tm_run
+ * with T = C = 1). Pointers 16-byte aligned; y must not overlap any input or
+ * the state, W not S. Errors: TM_ERR_INVALID_ARG (no launch), TM_ERR_CUDA.
+ * Asynchronous on `stream`; allocates nothing.
+ */
+TM_API tm_status tm_decode_step(tm_ctx *ctx, int B, int H, tm_dtype in_dtype, const void *k, const void *v,
+                                const void *q, const float *theta, const float *eta, const float *alpha,
+                                float *W, float *S, float *y, void *stream);
+
+/*
  * The step before the memory: a short depthwise causal convolution of the
  * projected keys, values and queries, followed by L2 normalisation of every
  * key and query row ("Titans, explained", step 1: "the projections are

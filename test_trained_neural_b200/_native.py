@@ -33,6 +33,7 @@ SIGNATURES = {
     "tm_sync": (_I, [_P, _P, _P]),
     "tm_set_debug": (_I, [_I, ctypes.c_ulonglong]),
     "tm_prologue": (_I, [_I, _I, _I, _I, _I, _I] + [_P] * 12 + [_P]),
+    "tm_decode_step": (_I, [_P, _I, _I, _I] + [_P] * 9 + [_P]),
     "tm_status_string": (ctypes.c_char_p, [_I]),
     "tm_version": (_I, []),
 }

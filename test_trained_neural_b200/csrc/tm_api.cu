@@ -330,6 +330,32 @@ tm_status tm_sync(tm_ctx *ctx, void *workspace, void *stream) {
   return code == tmem::kDevTimeout ? TM_ERR_TIMEOUT : TM_ERR_DEVICE;
 }
 
+tm_status tm_decode_step(tm_ctx *ctx, int B, int H, tm_dtype in_dtype, const void *k, const void *v,
+                         const void *q, const float *theta, const float *eta, const float *alpha, float *W,
+                         float *S, float *y, void *stream) {
+  tm_status st = check_shape(ctx, B, H, 1, 1, in_dtype);
+  if (st != TM_OK) return st;
+  const void *ptrs[] = {k, v, q, theta, eta, alpha, W, S, y};
+  for (const void *p : ptrs)
+    if (!p || !aligned16(p)) return TM_ERR_INVALID_ARG;
+  const tmem::Problem p = make_problem(ctx, B, H, 1, 1, in_dtype);
+  const size_t el = in_dtype == TM_BF16 ? 2 : 4;
+  const size_t tok = (size_t)p.streams * p.dims[0] * el, gate = (size_t)p.streams * 4;
+  const size_t state = (size_t)p.streams * p.P * 4, yb = (size_t)p.streams * p.dims[0] * 4;
+  const void *ins[] = {k, v, q, theta, eta, alpha, W, S};
+  const size_t insz[] = {tok, tok, tok, gate, gate, gate, state, state};
+  for (int i = 0; i < 8; ++i)
+    if (ranges_overlap(y, yb, ins[i], insz[i])) return TM_ERR_INVALID_ARG;
+  for (int i = 0; i < 6; ++i)
+    if (ranges_overlap(W, state, ins[i], insz[i]) || ranges_overlap(S, state, ins[i], insz[i]))
+      return TM_ERR_INVALID_ARG;
+  if (ranges_overlap(W, state, S, state)) return TM_ERR_INVALID_ARG;
+  if (!tmem::decode_supported(p)) return TM_ERR_UNSUPPORTED;
+  const cudaError_t e = tmem::decode_launch(p, k, v, q, theta, eta, alpha, W, S, y,
+                                            reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? TM_OK : TM_ERR_CUDA;
+}
+
 tm_status tm_prologue(int B, int H, int T, int d, int width, tm_dtype in_dtype, const void *k_in,
                       const void *v_in, const void *q_in, const float *filt_k, const float *filt_v,
                       const float *filt_q, const void *hist_k, const void *hist_v, const void *hist_q,

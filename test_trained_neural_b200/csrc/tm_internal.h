@@ -67,6 +67,11 @@ int tcl_group_count(const Problem &p);   // CUDA streams tcl_launch uses
 long long tcl_launch_count(const Problem &p);
 void tcl_set_wait(unsigned long long wait_ns);
 
+// One-token decode step (C = 1), state updated in place.
+bool decode_supported(const Problem &p);
+cudaError_t decode_launch(const Problem &p, const void *k, const void *v, const void *q, const float *theta,
+                          const float *eta, const float *alpha, float *W, float *S, float *y, cudaStream_t st);
+
 // Depthwise causal convolution + L2 normalisation before the memory.
 bool prologue_supported_d(int d);
 cudaError_t prologue_launch(int streams, int H, int T, int d, int w, bool bf16, const void *const in[3],

@@ -111,6 +111,20 @@ class NeuralMemory:
             self.sync(workspace, stream)
         return y, W_end, S_end
 
+    def decode_step(self, k, v, q, theta, eta, alpha, W, S, y=None, stream=None):
+        """One token per stream (k, v, q [B, H, d_h]; gates [B, H]): returns
+        y = M_W(q) and updates W, S ([B, H, P] float32) in place."""
+        B, H, d = k.shape
+        if y is None:
+            y = torch.empty((B, H, d), dtype=torch.float32, device=k.device)
+        if stream is None:
+            stream = torch.cuda.current_stream(k.device)
+        code = self._lib.tm_decode_step(self._h, B, H, self._dtype_code(k), _ptr(k), _ptr(v), _ptr(q),
+                                        _ptr(theta), _ptr(eta), _ptr(alpha), _ptr(W), _ptr(S), _ptr(y),
+                                        ctypes.c_void_p(stream.cuda_stream))
+        N.check(code, "tm_decode_step")
+        return y
+
     def sync(self, workspace, stream=None):
         if stream is None:
             stream = torch.cuda.current_stream(workspace.device)
