@@ -345,6 +345,61 @@ def bench_decode(args, w: W.Workload):
           flush=True)
 
 
+def bench_backward(args, w: W.Workload):
+    """Gradients of the memory layer (depth 1) on the workload's shape: one
+    tm_backward per step (forward recomputed inside with chunk-start
+    checkpoints, then the reverse pass). CUDA-core fp32: the roofline is the
+    FP32 issue rate; about 22P FLOPs per token (forward 6P, reverse 16P)."""
+    import torch
+    from test_trained_neural_b200 import NeuralMemory
+
+    if w.L != 1:
+        raise SystemExit("--backward: depth-1 memories only")
+    dev = torch.device("cuda", 0)
+    inp = W.generate(w)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    d_in = {}
+    for key in ("k", "v", "q"):
+        a = np.ascontiguousarray(inp[key])
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if dt == torch.bfloat16 else torch.from_numpy(a)
+        d_in[key] = t.reshape(w.B, w.H, w.T, w.d).to(dev)
+    for key in ("theta", "eta", "alpha", "W0", "S0"):
+        a = np.ascontiguousarray(inp[key], dtype=np.float32)
+        d_in[key] = torch.from_numpy(a).reshape(w.B, w.H, *a.shape[1:]).to(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed)
+    dy = torch.randn((w.B, w.H, w.T, w.d), generator=g, device=dev)
+    dW = torch.randn(d_in["W0"].shape, generator=g, device=dev)
+    dS = torch.randn(d_in["S0"].shape, generator=g, device=dev)
+    mem = NeuralMemory(w.L, w.d, w.expansion)
+    run = lambda: mem.backward(d_in["k"], d_in["v"], d_in["q"], d_in["theta"], d_in["eta"], d_in["alpha"],
+                               d_in["W0"], d_in["S0"], dy, dW, dS, w.C)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        out = run()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+        out = run()
+        a1.record()
+        torch.cuda.synchronize()
+        ms.append(a0.elapsed_time(a1))
+    t = statistics.mean(ms) * 1e-3
+    tokens = w.streams * w.T
+    flops = 22.0 * w.P * tokens
+    peaks = measured_peaks()
+    alu_peak = SM_COUNT * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
+    tf = flops / t / 1e12
+    print(json.dumps({"metric": "backward tokens/sec", "value": tokens / t, "unit": "tokens/s", "ms": t * 1e3,
+                      "workload": w.name, "finite": bool(all(torch.isfinite(v).all() for v in out.values())),
+                      "roofline": {"bound": "alu", "achieved": tf, "peak": alu_peak, "unit": "TFLOP/s",
+                                   "frac": tf / alu_peak,
+                                   "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 x max clock"}}), flush=True)
+
+
 def bench_prologue(args, w: W.Workload):
     """The step before the memory on the workload's k, v, q: one fused launch of
     the depthwise causal convolution (width args.conv_width) and the L2
@@ -400,6 +455,8 @@ def main():
     ap.add_argument("--prologue", action="store_true",
                     help="time the convolution + normalisation step before the memory instead")
     ap.add_argument("--conv-width", type=int, default=4)
+    ap.add_argument("--backward", action="store_true",
+                    help="time the memory layer's gradients (depth-1 workloads) instead")
     ap.add_argument("--decode", action="store_true",
                     help="time one-token decode steps on the workload's memory and streams instead")
     ap.add_argument("--sweep-chunk", default=None,
@@ -423,6 +480,8 @@ def main():
         return bench_prologue(args, w)
     if args.decode:
         return bench_decode(args, w)
+    if args.backward:
+        return bench_backward(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
 

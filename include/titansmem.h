@@ -197,6 +197,37 @@ TM_API tm_status tm_run_noalloc(tm_ctx *ctx, int B, int H, int T, int C, tm_dtyp
 TM_API tm_status tm_sync(tm_ctx *ctx, void *workspace, void *stream);
 
 /*
+ * Gradients of the memory layer for an outer model that trains through it
+ * ("Titans, explained" and "Attack of the Titans" train the memory's inputs,
+ * k, v, q and the data-dependent gates, through the write-and-read; no
+ * kernel form is given). For the run tm_run(k, v, q, gates, W0, S0) -> (y,
+ * W_end, S_end) and upstream gradients dy, dW_end, dS_end, returns the
+ * gradients of J = sum_t <dy_t, y_t> + <dW_end, W_end> + <dS_end, S_end>:
+ *
+ *   dy                [B, H, T, d_h] float32     gradient of the reads y
+ *   dW_end, dS_end    [B, H, P] float32          gradient of the final state
+ *   dk, dv, dq        [B, H, T, d_h] float32     outputs
+ *   dtheta, deta, dalpha [B, H, T] float32       outputs
+ *   dW0, dS0          [B, H, P] float32          outputs
+ *   other arguments as for tm_run (chunk size C, a shorter last chunk allowed)
+ *
+ * Supported: depth 1 (the linear memory; deeper memories need second
+ * derivatives through the MLP, since the surprise is itself a gradient, and
+ * are not built), fp32 arithmetic; TM_ERR_UNSUPPORTED otherwise. The forward is recomputed inside
+ * (chunk-start states kept in the workspace: tm_backward_workspace_size()).
+ * Pointers 16-byte aligned; outputs must not overlap inputs or each other.
+ * Errors as for tm_run. Asynchronous on `stream`; allocates nothing.
+ */
+TM_API tm_status tm_backward_workspace_size(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype,
+                                            size_t *bytes);
+TM_API tm_status tm_backward(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype, const void *k,
+                             const void *v, const void *q, const float *theta, const float *eta,
+                             const float *alpha, const float *W0, const float *S0, const float *dy,
+                             const float *dW_end, const float *dS_end, float *dk, float *dv, float *dq,
+                             float *dtheta, float *deta, float *dalpha, float *dW0, float *dS0, void *workspace,
+                             size_t workspace_bytes, void *stream);
+
+/*
  * One decode step: a single token per stream, the chunk size C = 1 form of
  * the write-and-read ("Titans, explained" steps 2-6: surprise of the token at
  * the current weights, momentum and forgetting, then the update). With the

@@ -34,6 +34,8 @@ SIGNATURES = {
     "tm_set_debug": (_I, [_I, ctypes.c_ulonglong]),
     "tm_prologue": (_I, [_I, _I, _I, _I, _I, _I] + [_P] * 12 + [_P]),
     "tm_decode_step": (_I, [_P, _I, _I, _I] + [_P] * 9 + [_P]),
+    "tm_backward_workspace_size": (_I, [_P, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)]),
+    "tm_backward": (_I, [_P, _I, _I, _I, _I, _I] + [_P] * 20 + [ctypes.c_size_t, _P]),
     "tm_status_string": (ctypes.c_char_p, [_I]),
     "tm_version": (_I, []),
 }

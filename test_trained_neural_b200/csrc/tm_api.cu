@@ -330,6 +330,60 @@ tm_status tm_sync(tm_ctx *ctx, void *workspace, void *stream) {
   return code == tmem::kDevTimeout ? TM_ERR_TIMEOUT : TM_ERR_DEVICE;
 }
 
+tm_status tm_backward_workspace_size(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype,
+                                     size_t *bytes) {
+  if (!bytes) return TM_ERR_INVALID_ARG;
+  tm_status st = check_shape(ctx, B, H, T, C, in_dtype);
+  if (st != TM_OK) return st;
+  const tmem::Problem p = make_problem(ctx, B, H, T, C, in_dtype);
+  if (!tmem::backward_supported(p)) return TM_ERR_UNSUPPORTED;
+  *bytes = tmem::kStatusBytes + tmem::backward_scratch_bytes(p);
+  return TM_OK;
+}
+
+tm_status tm_backward(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype, const void *k, const void *v,
+                      const void *q, const float *theta, const float *eta, const float *alpha, const float *W0,
+                      const float *S0, const float *dy, const float *dW_end, const float *dS_end, float *dk,
+                      float *dv, float *dq, float *dtheta, float *deta, float *dalpha, float *dW0, float *dS0,
+                      void *workspace, size_t workspace_bytes, void *stream) {
+  tm_status st = check_shape(ctx, B, H, T, C, in_dtype);
+  if (st != TM_OK) return st;
+  const void *ptrs[] = {k, v, q, theta, eta, alpha, W0, S0, dy, dW_end, dS_end, dk, dv, dq, dtheta, deta,
+                        dalpha, dW0, dS0, workspace};
+  for (const void *p : ptrs)
+    if (!p || !aligned16(p)) return TM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TM_ERR_INVALID_ARG;
+  tmem::Problem p = make_problem(ctx, B, H, T, C, in_dtype);
+  if (!tmem::backward_supported(p)) return TM_ERR_UNSUPPORTED;
+  const size_t need = tmem::kStatusBytes + tmem::backward_scratch_bytes(p);
+  if (workspace_bytes < need) return TM_ERR_OOM;
+  const size_t S = (size_t)p.streams, el = in_dtype == TM_BF16 ? 2 : 4, d = (size_t)p.dims[0];
+  const size_t tokb = S * p.T * d * el, tokf = S * p.T * d * 4, gate = S * p.T * 4, state = S * p.P * 4;
+  const void *ins[] = {k, v, q, theta, eta, alpha, W0, S0, dy, dW_end, dS_end, workspace};
+  const size_t insz[] = {tokb, tokb, tokb, gate, gate, gate, state, state, tokf, state, state, need};
+  const void *outs[] = {dk, dv, dq, dtheta, deta, dalpha, dW0, dS0};
+  const size_t outsz[] = {tokf, tokf, tokf, gate, gate, gate, state, state};
+  for (int i = 0; i < 8; ++i) {
+    for (int j = 0; j < 12; ++j)
+      if (ranges_overlap(outs[i], outsz[i], ins[j], insz[j])) return TM_ERR_INVALID_ARG;
+    for (int j = 0; j < i; ++j)
+      if (ranges_overlap(outs[i], outsz[i], outs[j], outsz[j])) return TM_ERR_INVALID_ARG;
+  }
+  p.k = k;
+  p.v = v;
+  p.q = q;
+  p.theta = theta;
+  p.eta = eta;
+  p.alpha = alpha;
+  p.W0 = W0;
+  p.S0 = S0;
+  p.scratch = static_cast<char *>(workspace) + tmem::kStatusBytes;
+  p.scratch_bytes = workspace_bytes - tmem::kStatusBytes;
+  const cudaError_t e = tmem::backward_launch(p, dy, dW_end, dS_end, dk, dv, dq, dtheta, deta, dalpha, dW0, dS0,
+                                              reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? TM_OK : TM_ERR_CUDA;
+}
+
 tm_status tm_decode_step(tm_ctx *ctx, int B, int H, tm_dtype in_dtype, const void *k, const void *v,
                          const void *q, const float *theta, const float *eta, const float *alpha, float *W,
                          float *S, float *y, void *stream) {

@@ -67,6 +67,13 @@ int tcl_group_count(const Problem &p);   // CUDA streams tcl_launch uses
 long long tcl_launch_count(const Problem &p);
 void tcl_set_wait(unsigned long long wait_ns);
 
+// Gradients of the memory layer (depth 1) with respect to its inputs.
+bool backward_supported(const Problem &p);
+size_t backward_scratch_bytes(const Problem &p);
+cudaError_t backward_launch(const Problem &p, const float *dy, const float *dW_end, const float *dS_end,
+                            float *dk, float *dv, float *dq, float *dtheta, float *deta, float *dalpha,
+                            float *dW0, float *dS0, cudaStream_t stream);
+
 // One-token decode step (C = 1), state updated in place.
 bool decode_supported(const Problem &p);
 cudaError_t decode_launch(const Problem &p, const void *k, const void *v, const void *q, const float *theta,

@@ -63,6 +63,11 @@ __device__ __forceinline__ float load_tok(const void *p, int bf16, long long i) 
 
 __device__ __forceinline__ float sigm(float z) { return 1.0f / (1.0f + expf(-z)); }
 __device__ __forceinline__ float silu(float z) { return z * sigm(z); }
+__device__ __forceinline__ float warp_sum_simt(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
 __device__ __forceinline__ float silu_prime(float z) {
   float s = sigm(z);
   return s * (1.0f + z * (1.0f - s));
@@ -326,6 +331,214 @@ __global__ void __launch_bounds__(NT) simt_chunk_kernel(KArgs a) {
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Gradients of the linear memory (depth 1, W and S [d x d]) for an outer
+// model training through it: given dy (of the reads), dW_end and dS_end, the
+// gradients of J = sum <dy_t, y_t> + <dW_end, W_end> + <dS_end, S_end> with
+// respect to k, v, q, the gates, W0 and S0. A forward pass stores the
+// chunk-start state; the reverse pass carries (gW, gS) back through the
+// chunks. Per chunk, with r_i = W k_i - v_i, u_i = 2 r_i k_i^T and
+// m_i = -(c_i gW + e_i gS) k_i:
+//   dq_i = W^T dy_i,  dv_i = -2 m_i,  dk_i = 2 W^T m_i - 2 c_i gW^T r_i - 2 e_i gS^T r_i
+//   dc_i = -2 r_i^T gW k_i,  de_i = -2 r_i^T gS k_i
+//   dB = <gW, W>, dcS = <gW, S>, dA = <gS, S>
+//   gW <- B gW + 2 sum m_i k_i^T + sum dy_i q_i^T,   gS <- cS gW + A gS
+// and (dc, de, dB, dA, dcS) go back through the coefficient scan to the gates.
+struct BArgs {
+  int d, T, C, bf16;
+  const void *k, *v, *q;
+  const float *theta, *eta, *alpha, *W0, *S0, *dy, *dW_end, *dS_end;
+  float *dk, *dv, *dq, *dtheta, *deta, *dalpha, *dW0, *dS0;
+  float *scratch;
+  long long scratch_per_stream;
+};
+
+__device__ float block_sum(float x, float *red) {
+  x = warp_sum_simt(x);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  __syncthreads();
+  if (lane == 0) red[warp] = x;
+  __syncthreads();
+  float t = 0.f;
+  if (threadIdx.x < NT / 32) t = red[threadIdx.x];
+  if (warp == 0) t = warp_sum_simt(t);
+  if (threadIdx.x == 0) red[0] = t;
+  __syncthreads();
+  const float r = red[0];
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(NT) simt_backward_kernel(BArgs a) {
+  __shared__ SmemT sm;
+  __shared__ float red[NT / 32];
+  const int s = blockIdx.x, d = a.d, T = a.T, C = a.C, dd = d * d;
+  const int nch = (T + C - 1) / C;
+  float *p = a.scratch + (long long)s * a.scratch_per_stream;
+  float *ckW = p; p += (long long)nch * dd;
+  float *ckS = p; p += (long long)nch * dd;
+  float *Wc = p; p += dd;
+  float *Sc = p; p += dd;
+  float *gW = p; p += dd;
+  float *gS = p; p += dd;
+  float *gWn = p; p += dd;
+  float *K = p; p += (long long)C * d;
+  float *V = p; p += (long long)C * d;
+  float *Q = p; p += (long long)C * d;
+  float *DY = p; p += (long long)C * d;
+  float *R = p; p += (long long)C * d;
+  float *Am = p; p += (long long)C * d;
+  float *Bm = p; p += (long long)C * d;
+  float *Mm = p; p += (long long)C * d;
+  float *Pm = p; p += (long long)C * d;
+  float *Qm = p; p += (long long)C * d;
+  float *dc = p; p += C;
+  float *de = p; p += C;
+  float *pa = p; p += C;
+  float *pe = p; p += C;
+  float *rho = p; p += C;
+  float *dpa = p; p += C;
+  float *dpe = p; p += C;
+  float *drho = p; p += C;
+  const long long sw = (long long)s * dd, tok0 = (long long)s * T;
+
+  auto load_chunk = [&](int t0, int Cc, bool grads) {
+    for (int i = threadIdx.x; i < Cc * d; i += NT) {
+      const long long g = (tok0 + t0) * d + i;
+      K[i] = load_tok(a.k, a.bf16, g);
+      V[i] = load_tok(a.v, a.bf16, g);
+      if (grads) {
+        Q[i] = load_tok(a.q, a.bf16, g);
+        DY[i] = a.dy[g];
+      }
+    }
+    __syncthreads();
+  };
+  // ---- forward: chunk-start states
+  for (int i = threadIdx.x; i < dd; i += NT) {
+    Wc[i] = a.W0[sw + i];
+    Sc[i] = a.S0[sw + i];
+  }
+  __syncthreads();
+  for (int c = 0; c < nch; ++c) {
+    const int t0 = c * C, Cc = T - t0 < C ? T - t0 : C;
+    for (int i = threadIdx.x; i < dd; i += NT) {
+      ckW[(long long)c * dd + i] = Wc[i];
+      ckS[(long long)c * dd + i] = Sc[i];
+    }
+    chunk_coefficients(sm.coef, a.theta + tok0 + t0, a.eta + tok0 + t0, a.alpha + tok0 + t0, Cc);
+    load_chunk(t0, Cc, false);
+    // G = 2 (K W^T - V): the surprise factor of every token
+    gemm(sm, Cc, d, d, K, d, 1, Wc, d, 1, [&](int i, int r, float z) { R[i * d + r] = 2.f * (z - V[i * d + r]); });
+    __syncthreads();
+    update_layer(sm, d, d, Cc, R, K, Wc, Sc);
+    __syncthreads();
+  }
+  // ---- reverse
+  for (int i = threadIdx.x; i < dd; i += NT) {
+    gW[i] = a.dW_end[sw + i];
+    gS[i] = a.dS_end[sw + i];
+  }
+  __syncthreads();
+  for (int c = nch - 1; c >= 0; --c) {
+    const int t0 = c * C, Cc = T - t0 < C ? T - t0 : C;
+    const float *th = a.theta + tok0 + t0, *et = a.eta + tok0 + t0, *al = a.alpha + tok0 + t0;
+    const float *W = ckW + (long long)c * dd, *S = ckS + (long long)c * dd;
+    chunk_coefficients(sm.coef, th, et, al, Cc);
+    load_chunk(t0, Cc, true);
+    // residuals r_i and the products with gW, gS
+    gemm(sm, Cc, d, d, K, d, 1, W, d, 1, [&](int i, int r, float z) { R[i * d + r] = z - V[i * d + r]; });
+    gemm(sm, Cc, d, d, K, d, 1, gW, d, 1, [&](int i, int r, float z) { Am[i * d + r] = z; });
+    gemm(sm, Cc, d, d, K, d, 1, gS, d, 1, [&](int i, int r, float z) { Bm[i * d + r] = z; });
+    __syncthreads();
+    gemm(sm, Cc, d, d, R, d, 1, gW, 1, d, [&](int i, int j, float z) { Pm[i * d + j] = z; });
+    gemm(sm, Cc, d, d, R, d, 1, gS, 1, d, [&](int i, int j, float z) { Qm[i * d + j] = z; });
+    for (int e = threadIdx.x; e < Cc * d; e += NT) {
+      const int i = e / d;
+      Mm[e] = -(sm.coef.c[i] * Am[e] + sm.coef.e[i] * Bm[e]);
+    }
+    __syncthreads();
+    // coefficient gradients (warp per token) and the chunk scalars
+    for (int i = threadIdx.x / 32; i < Cc; i += NT / 32) {
+      float x = 0.f, y = 0.f;
+      for (int r = threadIdx.x % 32; r < d; r += 32) {
+        x = fmaf(R[i * d + r], Am[i * d + r], x);
+        y = fmaf(R[i * d + r], Bm[i * d + r], y);
+      }
+      x = warp_sum_simt(x);
+      y = warp_sum_simt(y);
+      if (threadIdx.x % 32 == 0) {
+        dc[i] = -2.f * x;
+        de[i] = -2.f * y;
+      }
+    }
+    float pw = 0.f, pws = 0.f, pss = 0.f;
+    for (int e = threadIdx.x; e < dd; e += NT) {
+      pw = fmaf(gW[e], W[e], pw);
+      pws = fmaf(gW[e], S[e], pws);
+      pss = fmaf(gS[e], S[e], pss);
+    }
+    const float dB = block_sum(pw, red), dcS = block_sum(pws, red), dA = block_sum(pss, red);
+    // token gradients
+    const long long gt = (tok0 + t0) * d;
+    gemm(sm, Cc, d, d, Mm, d, 1, W, 1, d, [&](int i, int j, float z) {
+      const int e = i * d + j;
+      a.dk[gt + e] = 2.f * z - 2.f * sm.coef.c[i] * Pm[e] - 2.f * sm.coef.e[i] * Qm[e];
+    });
+    gemm(sm, Cc, d, d, DY, d, 1, W, 1, d, [&](int i, int j, float z) { a.dq[gt + i * d + j] = z; });
+    for (int e = threadIdx.x; e < Cc * d; e += NT) a.dv[gt + e] = -2.f * Mm[e];
+    // gates: back through the coefficient scan (one thread, in order)
+    if (threadIdx.x == 0) {
+      pa[Cc - 1] = 1.f; pe[Cc - 1] = 1.f; rho[Cc - 1] = 1.f;
+      for (int i = Cc - 2; i >= 0; --i) {
+        pa[i] = pa[i + 1] * (1.f - al[i + 1]);
+        pe[i] = pe[i + 1] * et[i + 1];
+        rho[i] = pa[i] + et[i + 1] * rho[i + 1];
+      }
+      float *dth = a.dtheta + tok0 + t0, *det = a.deta + tok0 + t0, *dal = a.dalpha + tok0 + t0;
+      for (int i = 0; i < Cc; ++i) {
+        dth[i] = dc[i] * rho[i] + de[i] * pe[i];
+        drho[i] = dc[i] * th[i];
+        dpe[i] = de[i] * th[i];
+        dpa[i] = 0.f;
+        det[i] = 0.f;
+        dal[i] = 0.f;
+      }
+      dpa[0] += dB * (1.f - al[0]);
+      dal[0] += -dB * pa[0];
+      dpe[0] += dA * et[0];
+      det[0] += dA * pe[0];
+      det[0] += dcS * rho[0];
+      drho[0] += dcS * et[0];
+      for (int i = 0; i + 1 < Cc; ++i) {
+        dpa[i] += drho[i];
+        det[i + 1] += drho[i] * rho[i + 1];
+        drho[i + 1] += drho[i] * et[i + 1];
+        dpe[i + 1] += dpe[i] * et[i + 1];
+        det[i + 1] += dpe[i] * pe[i + 1];
+        dpa[i + 1] += dpa[i] * (1.f - al[i + 1]);
+        dal[i + 1] += -dpa[i] * pa[i + 1];
+      }
+    }
+    // the state gradients at the chunk start
+    const float Bw = sm.coef.Bw, As = sm.coef.As, cS = sm.coef.cS;
+    gemm(sm, d, d, Cc, Mm, 1, d, K, 1, d, [&](int r, int j, float z) { gWn[r * d + j] = Bw * gW[r * d + j] + 2.f * z; });
+    __syncthreads();
+    gemm(sm, d, d, Cc, DY, 1, d, Q, 1, d, [&](int r, int j, float z) { gWn[r * d + j] += z; });
+    __syncthreads();
+    for (int e = threadIdx.x; e < dd; e += NT) {
+      gS[e] = cS * gW[e] + As * gS[e];
+      gW[e] = gWn[e];
+    }
+    __syncthreads();
+  }
+  for (int e = threadIdx.x; e < dd; e += NT) {
+    a.dW0[sw + e] = gW[e];
+    a.dS0[sw + e] = gS[e];
+  }
+}
+
 }  // namespace
 
 size_t simt_scratch_bytes(const Problem &p) {
@@ -361,6 +574,36 @@ cudaError_t simt_launch(const Problem &p, cudaStream_t stream) {
   a.scratch_per_stream = (long long)(simt_scratch_bytes(p) / sizeof(float) / (size_t)p.streams);
   a.status = p.status;
   simt_chunk_kernel<<<p.streams, NT, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+bool backward_supported(const Problem &p) { return p.L == 1 && p.C <= kMaxC; }
+
+size_t backward_scratch_bytes(const Problem &p) {
+  const long long d = p.dims[0], C = p.C, nch = (p.T + p.C - 1) / p.C;
+  const long long per = 2 * nch * d * d + 5 * d * d + 10 * C * d + 8 * C;
+  return (size_t)(per * p.streams) * sizeof(float);
+}
+
+cudaError_t backward_launch(const Problem &p, const float *dy, const float *dW_end, const float *dS_end,
+                            float *dk, float *dv, float *dq, float *dtheta, float *deta, float *dalpha,
+                            float *dW0, float *dS0, cudaStream_t stream) {
+  if (!backward_supported(p)) return cudaErrorNotSupported;
+  BArgs a;
+  const long long d = p.dims[0], C = p.C, nch = (p.T + p.C - 1) / p.C;
+  a.d = (int)d;
+  a.T = p.T;
+  a.C = p.C;
+  a.bf16 = p.in_dtype == TM_BF16 ? 1 : 0;
+  a.k = p.k; a.v = p.v; a.q = p.q;
+  a.theta = p.theta; a.eta = p.eta; a.alpha = p.alpha;
+  a.W0 = p.W0; a.S0 = p.S0;
+  a.dy = dy; a.dW_end = dW_end; a.dS_end = dS_end;
+  a.dk = dk; a.dv = dv; a.dq = dq; a.dtheta = dtheta; a.deta = deta; a.dalpha = dalpha;
+  a.dW0 = dW0; a.dS0 = dS0;
+  a.scratch = static_cast<float *>(p.scratch);
+  a.scratch_per_stream = 2 * nch * d * d + 5 * d * d + 10 * C * d + 8 * C;
+  simt_backward_kernel<<<p.streams, NT, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

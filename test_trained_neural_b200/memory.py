@@ -125,6 +125,31 @@ class NeuralMemory:
         N.check(code, "tm_decode_step")
         return y
 
+    def backward(self, k, v, q, theta, eta, alpha, W0, S0, dy, dW_end, dS_end, C, stream=None):
+        """Gradients of sum <dy, y> + <dW_end, W_end> + <dS_end, S_end> for the
+        run with these inputs (depth 1). Returns a dict of float32 tensors dk,
+        dv, dq, dtheta, deta, dalpha, dW0, dS0."""
+        B, H, T, d = k.shape
+        dt = self._dtype_code(k)
+        n = ctypes.c_size_t()
+        N.check(self._lib.tm_backward_workspace_size(self._h, B, H, T, C, dt, ctypes.byref(n)),
+                "tm_backward_workspace_size")
+        ws = torch.empty(int(n.value), dtype=torch.uint8, device=k.device)
+        f32 = dict(dtype=torch.float32, device=k.device)
+        out = {"dk": torch.empty((B, H, T, d), **f32), "dv": torch.empty((B, H, T, d), **f32),
+               "dq": torch.empty((B, H, T, d), **f32), "dtheta": torch.empty((B, H, T), **f32),
+               "deta": torch.empty((B, H, T), **f32), "dalpha": torch.empty((B, H, T), **f32),
+               "dW0": torch.empty_like(W0), "dS0": torch.empty_like(S0)}
+        if stream is None:
+            stream = torch.cuda.current_stream(k.device)
+        code = self._lib.tm_backward(
+            self._h, B, H, T, C, dt, _ptr(k), _ptr(v), _ptr(q), _ptr(theta), _ptr(eta), _ptr(alpha), _ptr(W0),
+            _ptr(S0), _ptr(dy), _ptr(dW_end), _ptr(dS_end), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dq"]),
+            _ptr(out["dtheta"]), _ptr(out["deta"]), _ptr(out["dalpha"]), _ptr(out["dW0"]), _ptr(out["dS0"]),
+            _ptr(ws), ws.numel(), ctypes.c_void_p(stream.cuda_stream))
+        N.check(code, "tm_backward")
+        return out
+
     def sync(self, workspace, stream=None):
         if stream is None:
             stream = torch.cuda.current_stream(workspace.device)

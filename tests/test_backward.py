@@ -1,0 +1,71 @@
+"""Gradients of the memory layer (tm_backward, depth 1) against the float64
+gradient oracle (autograd through the restated recurrence, itself pinned
+against finite differences of the C oracle)."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from gen import workloads as W
+from oracle import backward as BW
+from test_trained_neural_b200 import NeuralMemory
+from test_trained_neural_b200 import _native as N
+
+from gpu_util import rel, to_dev
+
+TOL = 1e-4   # fp32 arithmetic against float64
+
+BACKWARD = [  # d, B, H, T, C, dtype
+    (64, 1, 1, 256, 16, "f32"),    # the linear workload's shape
+    (32, 2, 1, 40, 8, "bf16"),
+    (16, 1, 3, 50, 16, "f32"),     # a shorter last chunk (50 = 3 x 16 + 2)
+    (128, 1, 1, 64, 32, "bf16"),
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg", BACKWARD, ids=lambda c: "d%d-B%dH%d-T%d-C%d-%s" % c)
+def test_backward_matches_gradient_oracle(cfg):
+    d, B, H, T, C, dt = cfg
+    w = W.make(1, d, 1, B, H, T, C, dtype=dt, index=700 + d + T)
+    inp = W.generate(w)
+    dev = to_dev(inp, B, H, dt)
+    rng = np.random.default_rng(w.seed + 1)
+    n = B * H
+    dy = rng.standard_normal((n, T, d)).astype(np.float32)
+    dWe = rng.standard_normal((n, w.P)).astype(np.float32)
+    dSe = rng.standard_normal((n, w.P)).astype(np.float32)
+    mem = NeuralMemory(1, d, 1)
+    t = lambda a, shape: torch.from_numpy(np.ascontiguousarray(a)).reshape(shape).cuda()
+    out = mem.backward(dev["k"], dev["v"], dev["q"], dev["theta"], dev["eta"], dev["alpha"], dev["W0"], dev["S0"],
+                       t(dy, (B, H, T, d)), t(dWe, (B, H, w.P)), t(dSe, (B, H, w.P)), C)
+    torch.cuda.synchronize()
+    kf, vf, qf = (W.tokens_as_f64(inp[x], dt) for x in ("k", "v", "q"))
+    worst = {}
+    for s in range(n):
+        f32 = lambda x: np.asarray(inp[x][s], dtype=np.float32).astype(np.float64)   # as the GPU sees them
+        ref = BW.backward(w.dims, C, kf[s], vf[s], qf[s], f32("theta"), f32("eta"), f32("alpha"),
+                          f32("W0"), f32("S0"), dy[s], dWe[s], dSe[s])
+        for name, g in ref.items():
+            got = out[name].reshape(n, *g.shape).double().cpu().numpy()[s]
+            worst[name] = max(worst.get(name, 0.0), rel(got, g))
+    assert all(np.isfinite(v) for v in worst.values()), worst
+    assert max(worst.values()) < TOL, worst
+
+
+def test_backward_refuses_before_any_launch():
+    lib = N.load()
+    h = ctypes.c_void_p()
+    assert lib.tm_create(2, 64, 4, N.TM_ACT_SILU, ctypes.byref(h)) == N.TM_OK
+    n = ctypes.c_size_t()
+    assert lib.tm_backward_workspace_size(h, 1, 1, 64, 16, N.TM_F32, ctypes.byref(n)) == N.TM_ERR_UNSUPPORTED
+    lib.tm_destroy(h)
+    assert lib.tm_create(1, 64, 1, N.TM_ACT_SILU, ctypes.byref(h)) == N.TM_OK
+    assert lib.tm_backward_workspace_size(h, 1, 1, 64, 16, N.TM_F32, ctypes.byref(n)) == N.TM_OK
+    assert n.value > 256
+    p = [ctypes.c_void_p((i + 1) << 32) for i in range(20)]
+    assert lib.tm_backward(h, 1, 1, 64, 16, N.TM_F32, *p, ctypes.c_size_t(0), None) == N.TM_ERR_OOM
+    assert lib.tm_backward(h, 1, 1, 64, 16, N.TM_F32, *([None] + p[1:]), ctypes.c_size_t(1 << 30), None) == \
+        N.TM_ERR_INVALID_ARG
+    lib.tm_destroy(h)
