@@ -56,7 +56,6 @@ constexpr int HS = 64;          // hidden units per CTA
 constexpr int EPI_WARPS = 8;
 constexpr int NTHREADS = (EPI_WARPS + 1) * 32;
 constexpr int EPI_THREADS = EPI_WARPS * 32;
-constexpr int CTL_WARP = EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 
 struct TcArgs {
@@ -139,16 +138,6 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
                "r"(v.z), "r"(v.w)
                : "memory");
 }
-__device__ __forceinline__ void st_shared_u16(uint32_t addr, unsigned short v) {
-  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
-}
-__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr));
-  return v;
-}
 __device__ __forceinline__ void arrive_remote_release(uint32_t bar_cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
                    bar_cluster_addr)
@@ -200,26 +189,6 @@ __device__ __forceinline__ void bulk_load_global(uint32_t dst, const void *gsrc,
       "l"(gsrc), "r"(bytes), "r"(bar)
       : "memory");
 }
-__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
-}
-__device__ __forceinline__ uint4 ld_cluster_u4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared::cluster.v4.b32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void fence_acq_rel_cluster() {
-  asm volatile("fence.acq_rel.cluster;" ::: "memory");
-}
 // One arrival per warp on a local barrier, after every lane's shared-memory
 // writes have been made visible to the tensor cores (async proxy).
 __device__ __forceinline__ void warp_arrive_local(uint64_t *bar, int lane) {
@@ -228,19 +197,6 @@ __device__ __forceinline__ void warp_arrive_local(uint64_t *bar, int lane) {
   __syncwarp();
   if (lane == 0) mbar_arrive(bar);
 }
-// One arrival per warp on the barrier of every CTA of the cluster, after every
-// lane's stores into those CTAs are visible at cluster scope.
-template <int G>
-__device__ __forceinline__ void warp_arrive_cluster(uint64_t *bar, int lane) {
-  fence_acq_rel_cluster();
-  __syncwarp();
-  if (lane == 0) {
-    const uint32_t b = smem_u32(bar);
-#pragma unroll
-    for (int p = 0; p < G; ++p) arrive_remote_release(mapa(b, p));
-  }
-}
-
 // Bounded wait that also gives up as soon as another thread of the CTA has
 // flagged an abort. cluster_scope selects acquire.cluster semantics.
 __device__ bool wait_bar(uint64_t *bar, uint32_t parity, const TcArgs &a, volatile int *abort_flag,

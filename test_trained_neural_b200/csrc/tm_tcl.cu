@@ -99,8 +99,8 @@ constexpr int STAGES_MAX = 4;
 constexpr int DW_MAXN = 128;
 __host__ __device__ constexpr int dw_stages(int nk) { return nk <= 2 ? 2 : 3; }
 __host__ __device__ constexpr uint32_t dw_stage_bytes(int N) { return 2 * A_BYTES + (uint32_t)N * KB * 2; }
-// the epilogue's staging buffer (U_W and U_S of a 64-column piece) reuses the ring
-constexpr uint32_t DW_STAGE_U = 2 * 128 * 64 * 4;
+// (the epilogue's staging buffer for U_W and U_S of a 64-column piece, 64 KB,
+// reuses the ring, which is at least 80 KB)
 
 // A tile loads. mt: 128-row tile index (forward/backward) or 128-column tile
 // of the transposed operand (update).
