@@ -370,6 +370,47 @@ __device__ float block_sum(float x, float *red) {
   return r;
 }
 
+// Reverse-mode through the coefficient scan of one chunk (Cc tokens), one
+// thread: from the gradients of c_i, e_i, B, A, c_S to theta, eta, alpha.
+//   pa_i = prod_{j>i}(1 - alpha_j), pe_i = prod_{j>i} eta_j,
+//   rho_{C-1} = 1, rho_i = pa_i + eta_{i+1} rho_{i+1};
+//   c_i = theta_i rho_i, e_i = theta_i pe_i, B = pa_0 (1 - alpha_0),
+//   A = pe_0 eta_0, c_S = eta_0 rho_0.
+// pa .. drho: scratch of Cc floats each.
+__device__ void gate_reverse(int Cc, const float *th, const float *et, const float *al, const float *dc,
+                             const float *de, float dB, float dA, float dcS, float *dth, float *det, float *dal,
+                             float *pa, float *pe, float *rho, float *dpa, float *dpe, float *drho) {
+  pa[Cc - 1] = 1.f; pe[Cc - 1] = 1.f; rho[Cc - 1] = 1.f;
+  for (int i = Cc - 2; i >= 0; --i) {
+    pa[i] = pa[i + 1] * (1.f - al[i + 1]);
+    pe[i] = pe[i + 1] * et[i + 1];
+    rho[i] = pa[i] + et[i + 1] * rho[i + 1];
+  }
+  for (int i = 0; i < Cc; ++i) {
+    dth[i] = dc[i] * rho[i] + de[i] * pe[i];
+    drho[i] = dc[i] * th[i];
+    dpe[i] = de[i] * th[i];
+    dpa[i] = 0.f;
+    det[i] = 0.f;
+    dal[i] = 0.f;
+  }
+  dpa[0] += dB * (1.f - al[0]);
+  dal[0] += -dB * pa[0];
+  dpe[0] += dA * et[0];
+  det[0] += dA * pe[0];
+  det[0] += dcS * rho[0];
+  drho[0] += dcS * et[0];
+  for (int i = 0; i + 1 < Cc; ++i) {
+    dpa[i] += drho[i];
+    det[i + 1] += drho[i] * rho[i + 1];
+    drho[i + 1] += drho[i] * et[i + 1];
+    dpe[i + 1] += dpe[i] * et[i + 1];
+    det[i + 1] += dpe[i] * pe[i + 1];
+    dpa[i + 1] += dpa[i] * (1.f - al[i + 1]);
+    dal[i + 1] += -dpa[i] * pa[i + 1];
+  }
+}
+
 __global__ void __launch_bounds__(NT) simt_backward_kernel(BArgs a) {
   __shared__ SmemT sm;
   __shared__ float red[NT / 32];
@@ -489,38 +530,9 @@ __global__ void __launch_bounds__(NT) simt_backward_kernel(BArgs a) {
     gemm(sm, Cc, d, d, DY, d, 1, W, 1, d, [&](int i, int j, float z) { a.dq[gt + i * d + j] = z; });
     for (int e = threadIdx.x; e < Cc * d; e += NT) a.dv[gt + e] = -2.f * Mm[e];
     // gates: back through the coefficient scan (one thread, in order)
-    if (threadIdx.x == 0) {
-      pa[Cc - 1] = 1.f; pe[Cc - 1] = 1.f; rho[Cc - 1] = 1.f;
-      for (int i = Cc - 2; i >= 0; --i) {
-        pa[i] = pa[i + 1] * (1.f - al[i + 1]);
-        pe[i] = pe[i + 1] * et[i + 1];
-        rho[i] = pa[i] + et[i + 1] * rho[i + 1];
-      }
-      float *dth = a.dtheta + tok0 + t0, *det = a.deta + tok0 + t0, *dal = a.dalpha + tok0 + t0;
-      for (int i = 0; i < Cc; ++i) {
-        dth[i] = dc[i] * rho[i] + de[i] * pe[i];
-        drho[i] = dc[i] * th[i];
-        dpe[i] = de[i] * th[i];
-        dpa[i] = 0.f;
-        det[i] = 0.f;
-        dal[i] = 0.f;
-      }
-      dpa[0] += dB * (1.f - al[0]);
-      dal[0] += -dB * pa[0];
-      dpe[0] += dA * et[0];
-      det[0] += dA * pe[0];
-      det[0] += dcS * rho[0];
-      drho[0] += dcS * et[0];
-      for (int i = 0; i + 1 < Cc; ++i) {
-        dpa[i] += drho[i];
-        det[i + 1] += drho[i] * rho[i + 1];
-        drho[i + 1] += drho[i] * et[i + 1];
-        dpe[i + 1] += dpe[i] * et[i + 1];
-        det[i + 1] += dpe[i] * pe[i + 1];
-        dpa[i + 1] += dpa[i] * (1.f - al[i + 1]);
-        dal[i + 1] += -dpa[i] * pa[i + 1];
-      }
-    }
+    if (threadIdx.x == 0)
+      gate_reverse(Cc, th, et, al, dc, de, dB, dA, dcS, a.dtheta + tok0 + t0, a.deta + tok0 + t0,
+                   a.dalpha + tok0 + t0, pa, pe, rho, dpa, dpe, drho);
     // the state gradients at the chunk start
     const float Bw = sm.coef.Bw, As = sm.coef.As, cS = sm.coef.cS;
     gemm(sm, d, d, Cc, Mm, 1, d, K, 1, d, [&](int r, int j, float z) { gWn[r * d + j] = Bw * gW[r * d + j] + 2.f * z; });
@@ -534,6 +546,239 @@ __global__ void __launch_bounds__(NT) simt_backward_kernel(BArgs a) {
     __syncthreads();
   }
   for (int e = threadIdx.x; e < dd; e += NT) {
+    a.dW0[sw + e] = gW[e];
+    a.dS0[sw + e] = gS[e];
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// The same gradients for the depth-2 memory M(x) = W2 silu(W1 x) (W1 [n x d],
+// W2 [o x n]). Per token the surprise enters J through
+//   J_i = g1^T a + g2^T b,  a = M1 k, b = M2 x1,  M_l = -(c_i gW_l + e_i gS_l),
+// with z1 = W1 k, x1 = silu(z1), g2 = 2 (W2 x1 - v), h = W2^T g2,
+// g1 = h . silu'(z1); reverse mode through these vector steps gives, for the
+// chunk's tokens as matrices (rows = tokens):
+//   dG1 = a;  dH = a . silu'(z1);  dSP = a . h;  dG2 = b + dH W2^T
+//   dW2 += G2^T dH + 2 dG2^T X1;  dv = -2 dG2
+//   dX1 = 2 dG2 W2 - c (G2 gW2) - e (G2 gS2)
+//   dZ1 = dX1 . silu'(z1) + dSP . silu''(z1)
+//   dW1 += dZ1^T K;  dk = dZ1 W1 - c (G1 gW1) - e (G1 gS1)
+// and the reads y = W2 silu(W1 q) add their ordinary backward (dq, dW1, dW2).
+// The coefficient, scalar, state and gate steps are those of depth 1.
+__device__ __forceinline__ float silu_second(float z) {
+  const float s = sigm(z);
+  return s * (1.f - s) * (2.f + z * (1.f - 2.f * s));
+}
+
+struct BArgs2 {
+  int d, n, o, T, C, bf16;
+  long long P;
+  const void *k, *v, *q;
+  const float *theta, *eta, *alpha, *W0, *S0, *dy, *dW_end, *dS_end;
+  float *dk, *dv, *dq, *dtheta, *deta, *dalpha, *dW0, *dS0;
+  float *scratch;
+  long long scratch_per_stream;
+};
+
+__host__ __device__ inline long long backward2_floats(int d, int n, int o, int T, int C) {
+  const long long P = (long long)n * d + (long long)o * n, nch = (T + C - 1) / C;
+  const long long m = n > d ? (n > o ? n : o) : (d > o ? d : o);
+  return 2 * nch * P + 5 * P + 20LL * C * m + 8LL * C;
+}
+
+__global__ void __launch_bounds__(NT) simt_backward2_kernel(BArgs2 a) {
+  __shared__ SmemT sm;
+  __shared__ float red[NT / 32];
+  const int s = blockIdx.x, d = a.d, n = a.n, o = a.o, T = a.T, C = a.C;
+  const long long P = a.P, nd = (long long)n * d;
+  const int nch = (T + C - 1) / C;
+  const int m = n > d ? (n > o ? n : o) : (d > o ? d : o);
+  float *p = a.scratch + (long long)s * a.scratch_per_stream;
+  float *ckW = p; p += (long long)nch * P;
+  float *ckS = p; p += (long long)nch * P;
+  float *Wc = p; p += P;
+  float *Sc = p; p += P;
+  float *gW = p; p += P;
+  float *gS = p; p += P;
+  float *gWn = p; p += P;
+  auto take = [&]() { float *r = p; p += (long long)C * m; return r; };
+  float *K = take(), *V = take(), *Q = take(), *DY = take();
+  float *Z1 = take(), *X1 = take(), *G2 = take(), *H = take(), *G1 = take();
+  float *ZQ = take(), *XQ = take(), *KW1 = take(), *KS1 = take(), *XW2 = take(), *XS2 = take();
+  float *T1 = take(), *T2 = take(), *TO = take();
+  take(); take();
+  float *dc = p; p += C;
+  float *de = p; p += C;
+  float *pa = p; p += C;
+  float *pe = p; p += C;
+  float *rho = p; p += C;
+  float *dpa = p; p += C;
+  float *dpe = p; p += C;
+  float *drho = p; p += C;
+  const long long sw = (long long)s * P, tok0 = (long long)s * T;
+
+  auto load_chunk = [&](int t0, int Cc, bool grads) {
+    for (int i = threadIdx.x; i < Cc * d; i += NT) {
+      const long long g = (tok0 + t0) * d + i;
+      K[i] = load_tok(a.k, a.bf16, g);
+      if (grads) Q[i] = load_tok(a.q, a.bf16, g);
+    }
+    for (int i = threadIdx.x; i < Cc * o; i += NT) {
+      const long long g = (tok0 + t0) * o + i;
+      V[i] = load_tok(a.v, a.bf16, g);
+      if (grads) DY[i] = a.dy[g];
+    }
+    __syncthreads();
+  };
+  // forward of the keys at (W1, W2): Z1, X1, G2, H = G2 W2, G1
+  auto keys_forward = [&](int Cc, const float *W1, const float *W2) {
+    gemm(sm, Cc, n, d, K, d, 1, W1, d, 1, [&](int i, int j, float z) {
+      Z1[i * n + j] = z;
+      X1[i * n + j] = silu(z);
+    });
+    __syncthreads();
+    gemm(sm, Cc, o, n, X1, n, 1, W2, n, 1, [&](int i, int r, float z) { G2[i * o + r] = 2.f * (z - V[i * o + r]); });
+    __syncthreads();
+    gemm(sm, Cc, n, o, G2, o, 1, W2, 1, n, [&](int i, int j, float z) {
+      H[i * n + j] = z;
+      G1[i * n + j] = z * silu_prime(Z1[i * n + j]);
+    });
+    __syncthreads();
+  };
+  // ---- forward: chunk-start states
+  for (long long i = threadIdx.x; i < P; i += NT) {
+    Wc[i] = a.W0[sw + i];
+    Sc[i] = a.S0[sw + i];
+  }
+  __syncthreads();
+  for (int c = 0; c < nch; ++c) {
+    const int t0 = c * C, Cc = T - t0 < C ? T - t0 : C;
+    for (long long i = threadIdx.x; i < P; i += NT) {
+      ckW[(long long)c * P + i] = Wc[i];
+      ckS[(long long)c * P + i] = Sc[i];
+    }
+    chunk_coefficients(sm.coef, a.theta + tok0 + t0, a.eta + tok0 + t0, a.alpha + tok0 + t0, Cc);
+    load_chunk(t0, Cc, false);
+    keys_forward(Cc, Wc, Wc + nd);
+    update_layer(sm, o, n, Cc, G2, X1, Wc + nd, Sc + nd);
+    update_layer(sm, n, d, Cc, G1, K, Wc, Sc);
+    __syncthreads();
+  }
+  // ---- reverse
+  for (long long i = threadIdx.x; i < P; i += NT) {
+    gW[i] = a.dW_end[sw + i];
+    gS[i] = a.dS_end[sw + i];
+  }
+  __syncthreads();
+  for (int c = nch - 1; c >= 0; --c) {
+    const int t0 = c * C, Cc = T - t0 < C ? T - t0 : C;
+    const float *th = a.theta + tok0 + t0, *et = a.eta + tok0 + t0, *al = a.alpha + tok0 + t0;
+    const float *W1 = ckW + (long long)c * P, *W2 = W1 + nd;
+    const float *S = ckS + (long long)c * P;
+    const float *gW1 = gW, *gW2 = gW + nd, *gS1 = gS, *gS2 = gS + nd;
+    chunk_coefficients(sm.coef, th, et, al, Cc);
+    load_chunk(t0, Cc, true);
+    keys_forward(Cc, W1, W2);
+    gemm(sm, Cc, n, d, Q, d, 1, W1, d, 1, [&](int i, int j, float z) {
+      ZQ[i * n + j] = z;
+      XQ[i * n + j] = silu(z);
+    });
+    gemm(sm, Cc, n, d, K, d, 1, gW1, d, 1, [&](int i, int j, float z) { KW1[i * n + j] = z; });
+    gemm(sm, Cc, n, d, K, d, 1, gS1, d, 1, [&](int i, int j, float z) { KS1[i * n + j] = z; });
+    gemm(sm, Cc, o, n, X1, n, 1, gW2, n, 1, [&](int i, int r, float z) { XW2[i * o + r] = z; });
+    gemm(sm, Cc, o, n, X1, n, 1, gS2, n, 1, [&](int i, int r, float z) { XS2[i * o + r] = z; });
+    __syncthreads();
+    // coefficient gradients: dc_i = -<gW, u_i>, de_i = -<gS, u_i>
+    for (int i = threadIdx.x / 32; i < Cc; i += NT / 32) {
+      float x = 0.f, y = 0.f;
+      for (int j = threadIdx.x % 32; j < n; j += 32) {
+        x = fmaf(G1[i * n + j], KW1[i * n + j], x);
+        y = fmaf(G1[i * n + j], KS1[i * n + j], y);
+      }
+      for (int r = threadIdx.x % 32; r < o; r += 32) {
+        x = fmaf(G2[i * o + r], XW2[i * o + r], x);
+        y = fmaf(G2[i * o + r], XS2[i * o + r], y);
+      }
+      x = warp_sum_simt(x);
+      y = warp_sum_simt(y);
+      if (threadIdx.x % 32 == 0) {
+        dc[i] = -x;
+        de[i] = -y;
+      }
+    }
+    __syncthreads();
+    // a = M1 k (into KW1), b = M2 x1 (into XW2); dH (T1), dSP (T2)
+    for (int e = threadIdx.x; e < Cc * n; e += NT) {
+      const int i = e / n;
+      const float av = -(sm.coef.c[i] * KW1[e] + sm.coef.e[i] * KS1[e]);
+      KW1[e] = av;
+      T1[e] = av * silu_prime(Z1[e]);
+      T2[e] = av * H[e];
+    }
+    for (int e = threadIdx.x; e < Cc * o; e += NT) {
+      const int i = e / o;
+      XW2[e] = -(sm.coef.c[i] * XW2[e] + sm.coef.e[i] * XS2[e]);
+    }
+    __syncthreads();
+    // dG2 = b + dH W2^T (TO)
+    gemm(sm, Cc, o, n, T1, n, 1, W2, n, 1, [&](int i, int r, float z) { TO[i * o + r] = z + XW2[i * o + r]; });
+    __syncthreads();
+    // state gradient of W2: B gW2 + G2^T dH + 2 dG2^T X1 + DY^T XQ
+    const float Bw = sm.coef.Bw, As = sm.coef.As, cS = sm.coef.cS;
+    float *gWn1 = gWn, *gWn2 = gWn + nd;
+    gemm(sm, o, n, Cc, G2, 1, o, T1, 1, n, [&](int r, int j, float z) { gWn2[r * n + j] = Bw * gW2[r * n + j] + z; });
+    __syncthreads();
+    gemm(sm, o, n, Cc, TO, 1, o, X1, 1, n, [&](int r, int j, float z) { gWn2[r * n + j] += 2.f * z; });
+    __syncthreads();
+    gemm(sm, o, n, Cc, DY, 1, o, XQ, 1, n, [&](int r, int j, float z) { gWn2[r * n + j] += z; });
+    __syncthreads();
+    const long long gt_in = (tok0 + t0) * d, gt_out = (tok0 + t0) * o;
+    for (int e = threadIdx.x; e < Cc * o; e += NT) a.dv[gt_out + e] = -2.f * TO[e];
+    // dX1 = 2 dG2 W2 - c (G2 gW2) - e (G2 gS2)  (into T1, dH no longer needed)
+    gemm(sm, Cc, n, o, TO, o, 1, W2, 1, n, [&](int i, int j, float z) { T1[i * n + j] = 2.f * z; });
+    __syncthreads();
+    gemm(sm, Cc, n, o, G2, o, 1, gW2, 1, n, [&](int i, int j, float z) { T1[i * n + j] -= sm.coef.c[i] * z; });
+    __syncthreads();
+    gemm(sm, Cc, n, o, G2, o, 1, gS2, 1, n, [&](int i, int j, float z) { T1[i * n + j] -= sm.coef.e[i] * z; });
+    __syncthreads();
+    // dZ1 = dX1 . silu'(z1) + dSP . silu''(z1)  (T1)
+    for (int e = threadIdx.x; e < Cc * n; e += NT) T1[e] = T1[e] * silu_prime(Z1[e]) + T2[e] * silu_second(Z1[e]);
+    __syncthreads();
+    // reads: dZQ = (DY W2) . silu'(zq)  (T2)
+    gemm(sm, Cc, n, o, DY, o, 1, W2, 1, n, [&](int i, int j, float z) { T2[i * n + j] = z * silu_prime(ZQ[i * n + j]); });
+    __syncthreads();
+    // state gradient of W1: B gW1 + dZ1^T K + dZQ^T Q
+    gemm(sm, n, d, Cc, T1, 1, n, K, 1, d, [&](int j, int mm, float z) { gWn1[j * d + mm] = Bw * gW1[j * d + mm] + z; });
+    __syncthreads();
+    gemm(sm, n, d, Cc, T2, 1, n, Q, 1, d, [&](int j, int mm, float z) { gWn1[j * d + mm] += z; });
+    __syncthreads();
+    // dk = dZ1 W1 - c (G1 gW1) - e (G1 gS1);  dq = dZQ W1
+    gemm(sm, Cc, d, n, T1, n, 1, W1, 1, d, [&](int i, int mm, float z) { a.dk[gt_in + i * d + mm] = z; });
+    __syncthreads();
+    gemm(sm, Cc, d, n, G1, n, 1, gW1, 1, d, [&](int i, int mm, float z) { a.dk[gt_in + i * d + mm] -= sm.coef.c[i] * z; });
+    __syncthreads();
+    gemm(sm, Cc, d, n, G1, n, 1, gS1, 1, d, [&](int i, int mm, float z) { a.dk[gt_in + i * d + mm] -= sm.coef.e[i] * z; });
+    __syncthreads();
+    gemm(sm, Cc, d, n, T2, n, 1, W1, 1, d, [&](int i, int mm, float z) { a.dq[gt_in + i * d + mm] = z; });
+    // chunk scalars
+    float pw = 0.f, pws = 0.f, pss = 0.f;
+    for (long long e = threadIdx.x; e < P; e += NT) {
+      pw = fmaf(gW[e], W1[e], pw);
+      pws = fmaf(gW[e], S[e], pws);
+      pss = fmaf(gS[e], S[e], pss);
+    }
+    const float dB = block_sum(pw, red), dcS = block_sum(pws, red), dA = block_sum(pss, red);
+    if (threadIdx.x == 0)
+      gate_reverse(Cc, th, et, al, dc, de, dB, dA, dcS, a.dtheta + tok0 + t0, a.deta + tok0 + t0,
+                   a.dalpha + tok0 + t0, pa, pe, rho, dpa, dpe, drho);
+    for (long long e = threadIdx.x; e < P; e += NT) {
+      gS[e] = cS * gW[e] + As * gS[e];
+      gW[e] = gWn[e];
+    }
+    __syncthreads();
+  }
+  for (long long e = threadIdx.x; e < P; e += NT) {
     a.dW0[sw + e] = gW[e];
     a.dS0[sw + e] = gS[e];
   }
@@ -577,11 +822,12 @@ cudaError_t simt_launch(const Problem &p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-bool backward_supported(const Problem &p) { return p.L == 1 && p.C <= kMaxC; }
+bool backward_supported(const Problem &p) { return (p.L == 1 || p.L == 2) && p.C <= kMaxC; }
 
 size_t backward_scratch_bytes(const Problem &p) {
   const long long d = p.dims[0], C = p.C, nch = (p.T + p.C - 1) / p.C;
-  const long long per = 2 * nch * d * d + 5 * d * d + 10 * C * d + 8 * C;
+  const long long per = p.L == 1 ? 2 * nch * d * d + 5 * d * d + 10 * C * d + 8 * C
+                                 : backward2_floats(p.dims[0], p.dims[1], p.dims[2], p.T, p.C);
   return (size_t)(per * p.streams) * sizeof(float);
 }
 
@@ -589,6 +835,26 @@ cudaError_t backward_launch(const Problem &p, const float *dy, const float *dW_e
                             float *dk, float *dv, float *dq, float *dtheta, float *deta, float *dalpha,
                             float *dW0, float *dS0, cudaStream_t stream) {
   if (!backward_supported(p)) return cudaErrorNotSupported;
+  if (p.L == 2) {
+    BArgs2 b;
+    b.d = p.dims[0];
+    b.n = p.dims[1];
+    b.o = p.dims[2];
+    b.T = p.T;
+    b.C = p.C;
+    b.bf16 = p.in_dtype == TM_BF16 ? 1 : 0;
+    b.P = (long long)p.P;
+    b.k = p.k; b.v = p.v; b.q = p.q;
+    b.theta = p.theta; b.eta = p.eta; b.alpha = p.alpha;
+    b.W0 = p.W0; b.S0 = p.S0;
+    b.dy = dy; b.dW_end = dW_end; b.dS_end = dS_end;
+    b.dk = dk; b.dv = dv; b.dq = dq; b.dtheta = dtheta; b.deta = deta; b.dalpha = dalpha;
+    b.dW0 = dW0; b.dS0 = dS0;
+    b.scratch = static_cast<float *>(p.scratch);
+    b.scratch_per_stream = backward2_floats(b.d, b.n, b.o, p.T, p.C);
+    simt_backward2_kernel<<<p.streams, NT, 0, stream>>>(b);
+    return cudaGetLastError();
+  }
   BArgs a;
   const long long d = p.dims[0], C = p.C, nch = (p.T + p.C - 1) / p.C;
   a.d = (int)d;

@@ -1,4 +1,4 @@
-"""Gradients of the memory layer (tm_backward, depth 1) against the float64
+"""Gradients of the memory layer (tm_backward, depths 1 and 2) against the float64
 gradient oracle (autograd through the restated recurrence, itself pinned
 against finite differences of the C oracle)."""
 import ctypes
@@ -16,19 +16,22 @@ from gpu_util import rel, to_dev
 
 TOL = 1e-4   # fp32 arithmetic against float64
 
-BACKWARD = [  # d, B, H, T, C, dtype
-    (64, 1, 1, 256, 16, "f32"),    # the linear workload's shape
-    (32, 2, 1, 40, 8, "bf16"),
-    (16, 1, 3, 50, 16, "f32"),     # a shorter last chunk (50 = 3 x 16 + 2)
-    (128, 1, 1, 64, 32, "bf16"),
+BACKWARD = [  # L, d, expansion, B, H, T, C, dtype
+    (1, 64, 1, 1, 1, 256, 16, "f32"),    # the linear workload's shape
+    (1, 32, 1, 2, 1, 40, 8, "bf16"),
+    (1, 16, 1, 1, 3, 50, 16, "f32"),     # a shorter last chunk (50 = 3 x 16 + 2)
+    (1, 128, 1, 1, 1, 64, 32, "bf16"),
+    (2, 16, 4, 1, 2, 48, 16, "f32"),     # depth 2, hidden 64
+    (2, 32, 2, 2, 1, 50, 16, "bf16"),    # depth 2, a shorter last chunk
+    (2, 64, 4, 1, 1, 64, 64, "bf16"),    # depth 2, the d = 64 workload's memory
 ]
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("cfg", BACKWARD, ids=lambda c: "d%d-B%dH%d-T%d-C%d-%s" % c)
+@pytest.mark.parametrize("cfg", BACKWARD, ids=lambda c: "L%d-d%d-e%d-B%dH%d-T%d-C%d-%s" % c)
 def test_backward_matches_gradient_oracle(cfg):
-    d, B, H, T, C, dt = cfg
-    w = W.make(1, d, 1, B, H, T, C, dtype=dt, index=700 + d + T)
+    L, d, e, B, H, T, C, dt = cfg
+    w = W.make(L, d, e, B, H, T, C, dtype=dt, index=700 + d + T)
     inp = W.generate(w)
     dev = to_dev(inp, B, H, dt)
     rng = np.random.default_rng(w.seed + 1)
@@ -36,7 +39,7 @@ def test_backward_matches_gradient_oracle(cfg):
     dy = rng.standard_normal((n, T, d)).astype(np.float32)
     dWe = rng.standard_normal((n, w.P)).astype(np.float32)
     dSe = rng.standard_normal((n, w.P)).astype(np.float32)
-    mem = NeuralMemory(1, d, 1)
+    mem = NeuralMemory(L, d, e)
     t = lambda a, shape: torch.from_numpy(np.ascontiguousarray(a)).reshape(shape).cuda()
     out = mem.backward(dev["k"], dev["v"], dev["q"], dev["theta"], dev["eta"], dev["alpha"], dev["W0"], dev["S0"],
                        t(dy, (B, H, T, d)), t(dWe, (B, H, w.P)), t(dSe, (B, H, w.P)), C)
@@ -57,7 +60,7 @@ def test_backward_matches_gradient_oracle(cfg):
 def test_backward_refuses_before_any_launch():
     lib = N.load()
     h = ctypes.c_void_p()
-    assert lib.tm_create(2, 64, 4, N.TM_ACT_SILU, ctypes.byref(h)) == N.TM_OK
+    assert lib.tm_create(4, 64, 2, N.TM_ACT_SILU, ctypes.byref(h)) == N.TM_OK
     n = ctypes.c_size_t()
     assert lib.tm_backward_workspace_size(h, 1, 1, 64, 16, N.TM_F32, ctypes.byref(n)) == N.TM_ERR_UNSUPPORTED
     lib.tm_destroy(h)
