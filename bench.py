@@ -346,15 +346,15 @@ def bench_decode(args, w: W.Workload):
 
 
 def bench_backward(args, w: W.Workload):
-    """Gradients of the memory layer (depth 1) on the workload's shape: one
-    tm_backward per step (forward recomputed inside with chunk-start
-    checkpoints, then the reverse pass). CUDA-core fp32: the roofline is the
-    FP32 issue rate; about 22P FLOPs per token (forward 6P, reverse 16P)."""
+    """Gradients of the memory layer on the workload's shape: one tm_backward
+    per step (forward recomputed inside with chunk-start checkpoints, then the
+    reverse pass). CUDA-core fp32: the roofline is the FP32 issue rate. FLOPs
+    per token, counted from the kernels' matrix products (P1 = the first
+    layer's weights): 22P at depth 1, 32P - 6P1 at depth 2, 34P - 8P1 deeper
+    (forward 8P - 2P1, reverse 26P - 6P1)."""
     import torch
     from test_trained_neural_b200 import NeuralMemory
 
-    if w.L != 1:
-        raise SystemExit("--backward: depth-1 memories only")
     dev = torch.device("cuda", 0)
     inp = W.generate(w)
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
@@ -389,7 +389,8 @@ def bench_backward(args, w: W.Workload):
         ms.append(a0.elapsed_time(a1))
     t = statistics.mean(ms) * 1e-3
     tokens = w.streams * w.T
-    flops = 22.0 * w.P * tokens
+    P1 = w.dims[0] * w.dims[1]
+    flops = (22.0 * w.P if w.L == 1 else 32.0 * w.P - 6.0 * P1 if w.L == 2 else 34.0 * w.P - 8.0 * P1) * tokens
     peaks = measured_peaks()
     alu_peak = SM_COUNT * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
     tf = flops / t / 1e12

@@ -211,9 +211,9 @@ TM_API tm_status tm_sync(tm_ctx *ctx, void *workspace, void *stream);
  *   dW0, dS0          [B, H, P] float32          outputs
  *   other arguments as for tm_run (chunk size C, a shorter last chunk allowed)
  *
- * Supported: depths 1 and 2 (the surprise is itself a gradient, so the
- * backward takes second derivatives through the MLP; depth 3 and 4 are not
- * built), fp32 arithmetic; TM_ERR_UNSUPPORTED otherwise. The forward is recomputed inside
+ * Supported: every depth 1 to 4 (the surprise is itself a gradient, so the
+ * backward takes second derivatives through the MLP), fp32 arithmetic, any
+ * C the forward accepts; TM_ERR_UNSUPPORTED otherwise. The forward is recomputed inside
  * (chunk-start states kept in the workspace: tm_backward_workspace_size()).
  * Pointers 16-byte aligned; outputs must not overlap inputs or each other.
  * Errors as for tm_run. Asynchronous on `stream`; allocates nothing.

@@ -784,6 +784,257 @@ __global__ void __launch_bounds__(NT) simt_backward2_kernel(BArgs2 a) {
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// The same gradients for any depth L (used for depths 3 and 4). With
+// x_0 = k, z_l = W_l x_{l-1}, x_l = silu(z_l) (x_L = z_L), g_L = 2 (x_L - v),
+// h_{l-1} = W_l^T g_l, g_{l-1} = h_{l-1} . silu'(z_{l-1}), the surprise enters
+// J through sum_l g_l^T a_l with a_l = M_l x_{l-1}. Reverse mode:
+//   dg_l = a_l, dx_{l-1} = M_l^T g_l                      (for every l)
+//   l = 2..L:  dh = dg_{l-1} . silu'(z_{l-1});  dsp_{l-1} = dg_{l-1} . h_{l-1}
+//              dW_l += g_l dh^T;  dg_l += dh W_l^T
+//   dx_L += 2 dg_L;  dv = -2 dg_L
+//   l = L..1:  dz = dx_l . silu'(z_l) + dsp_l . silu''(z_l)   (dz = dx_L at L)
+//              dW_l += dz x_{l-1}^T;  dx_{l-1} += dz W_l;      dk = dx_0
+// and the reads add their ordinary backward.
+constexpr int BWL_ARRAYS = 2 + 9 * (kMaxL + 1) + 3;   // V, DY; 9 per level; P1, P2, dH
+
+struct BArgsL {
+  int L, T, C, bf16, maxw;
+  int dims[kMaxL + 1];
+  long long off[kMaxL + 1];
+  long long P;
+  const void *k, *v, *q;
+  const float *theta, *eta, *alpha, *W0, *S0, *dy, *dW_end, *dS_end;
+  float *dk, *dv, *dq, *dtheta, *deta, *dalpha, *dW0, *dS0;
+  float *scratch;
+  long long scratch_per_stream;
+};
+
+__host__ __device__ inline long long backwardL_floats(long long P, int maxw, int T, int C) {
+  const long long nch = (T + C - 1) / C;
+  return 2 * nch * P + 5 * P + (long long)BWL_ARRAYS * C * maxw + 8LL * C;
+}
+
+__global__ void __launch_bounds__(NT) simt_backwardL_kernel(BArgsL a) {
+  __shared__ SmemT sm;
+  __shared__ float red[NT / 32];
+  const int s = blockIdx.x, L = a.L, T = a.T, C = a.C, mw = a.maxw;
+  const int *nn = a.dims;
+  const long long P = a.P;
+  const int nch = (T + C - 1) / C;
+  float *p = a.scratch + (long long)s * a.scratch_per_stream;
+  float *ckW = p; p += (long long)nch * P;
+  float *ckS = p; p += (long long)nch * P;
+  float *Wc = p; p += P;
+  float *Sc = p; p += P;
+  float *gW = p; p += P;
+  float *gS = p; p += P;
+  float *gWn = p; p += P;
+  auto take = [&]() { float *r = p; p += (long long)C * mw; return r; };
+  float *V = take(), *DY = take();
+  float *Xk[kMaxL + 1], *Zk[kMaxL + 1], *Gk[kMaxL + 1], *Hk[kMaxL + 1];
+  float *Xq[kMaxL + 1], *Zq[kMaxL + 1], *dG[kMaxL + 1], *dSP[kMaxL + 1], *dX[kMaxL + 1], *dXq[kMaxL + 1];
+  for (int l = 0; l <= kMaxL; ++l) {
+    Xk[l] = take(); Zk[l] = take(); Gk[l] = take(); Hk[l] = take();
+    Xq[l] = take(); Zq[l] = take(); dG[l] = take(); dSP[l] = take(); dX[l] = take();
+  }
+  for (int l = 0; l <= kMaxL; ++l) dXq[l] = dX[l];   // the reads reuse dX after the keys are done
+  float *P1 = take(), *P2 = take(), *dH = take();
+  float *dc = p; p += C;
+  float *de = p; p += C;
+  float *pa = p; p += C;
+  float *pe = p; p += C;
+  float *rho = p; p += C;
+  float *dpa = p; p += C;
+  float *dpe = p; p += C;
+  float *drho = p; p += C;
+  const long long sw = (long long)s * P, tok0 = (long long)s * T;
+  const int d0 = nn[0], dL = nn[L];
+
+  auto load_chunk = [&](int t0, int Cc, bool grads) {
+    for (int i = threadIdx.x; i < Cc * d0; i += NT) {
+      const long long g = (tok0 + t0) * d0 + i;
+      Xk[0][i] = load_tok(a.k, a.bf16, g);
+      if (grads) Xq[0][i] = load_tok(a.q, a.bf16, g);
+    }
+    for (int i = threadIdx.x; i < Cc * dL; i += NT) {
+      const long long g = (tok0 + t0) * dL + i;
+      V[i] = load_tok(a.v, a.bf16, g);
+      if (grads) DY[i] = a.dy[g];
+    }
+    __syncthreads();
+  };
+  // forward of rows X[0] through W: Z[l], X[l] (X[L] = Z[L])
+  auto forward = [&](int Cc, const float *W, float **X, float **Z) {
+    for (int l = 1; l <= L; ++l) {
+      const int r = nn[l], cl = nn[l - 1];
+      float *Zl = Z[l], *Xl = X[l];
+      const bool last = l == L;
+      gemm(sm, Cc, r, cl, X[l - 1], cl, 1, W + a.off[l - 1], cl, 1, [&](int i, int j, float z) {
+        Zl[i * r + j] = z;
+        Xl[i * r + j] = last ? z : silu(z);
+      });
+      __syncthreads();
+    }
+  };
+  // the keys' backward: G[L] = 2 (X[L] - V), H[l-1] = G[l] W_l, G[l-1] = H[l-1] . silu'(Z[l-1])
+  auto keys_backward = [&](int Cc, const float *W) {
+    for (int e = threadIdx.x; e < Cc * dL; e += NT) Gk[L][e] = 2.f * (Xk[L][e] - V[e]);
+    __syncthreads();
+    for (int l = L; l >= 2; --l) {
+      const int r = nn[l], cl = nn[l - 1];
+      float *Hl = Hk[l - 1], *Gl = Gk[l - 1], *Zl = Zk[l - 1];
+      gemm(sm, Cc, cl, r, Gk[l], r, 1, W + a.off[l - 1], 1, cl, [&](int i, int j, float z) {
+        Hl[i * cl + j] = z;
+        Gl[i * cl + j] = z * silu_prime(Zl[i * cl + j]);
+      });
+      __syncthreads();
+    }
+  };
+  // ---- forward: chunk-start states
+  for (long long i = threadIdx.x; i < P; i += NT) {
+    Wc[i] = a.W0[sw + i];
+    Sc[i] = a.S0[sw + i];
+  }
+  __syncthreads();
+  for (int c = 0; c < nch; ++c) {
+    const int t0 = c * C, Cc = T - t0 < C ? T - t0 : C;
+    for (long long i = threadIdx.x; i < P; i += NT) {
+      ckW[(long long)c * P + i] = Wc[i];
+      ckS[(long long)c * P + i] = Sc[i];
+    }
+    chunk_coefficients(sm.coef, a.theta + tok0 + t0, a.eta + tok0 + t0, a.alpha + tok0 + t0, Cc);
+    load_chunk(t0, Cc, false);
+    forward(Cc, Wc, Xk, Zk);
+    keys_backward(Cc, Wc);
+    for (int l = 1; l <= L; ++l) update_layer(sm, nn[l], nn[l - 1], Cc, Gk[l], Xk[l - 1], Wc + a.off[l - 1], Sc + a.off[l - 1]);
+    __syncthreads();
+  }
+  // ---- reverse
+  for (long long i = threadIdx.x; i < P; i += NT) {
+    gW[i] = a.dW_end[sw + i];
+    gS[i] = a.dS_end[sw + i];
+  }
+  __syncthreads();
+  for (int c = nch - 1; c >= 0; --c) {
+    const int t0 = c * C, Cc = T - t0 < C ? T - t0 : C;
+    const float *th = a.theta + tok0 + t0, *et = a.eta + tok0 + t0, *al = a.alpha + tok0 + t0;
+    const float *W = ckW + (long long)c * P, *S = ckS + (long long)c * P;
+    chunk_coefficients(sm.coef, th, et, al, Cc);
+    load_chunk(t0, Cc, true);
+    forward(Cc, W, Xk, Zk);
+    keys_backward(Cc, W);
+    forward(Cc, W, Xq, Zq);
+    const float Bw = sm.coef.Bw, As = sm.coef.As, cS = sm.coef.cS;
+    for (long long e = threadIdx.x; e < P; e += NT) gWn[e] = Bw * gW[e];
+    for (int i = threadIdx.x; i < Cc; i += NT) { dc[i] = 0.f; de[i] = 0.f; }
+    __syncthreads();
+    // per layer: a_l = M_l x_{l-1} (dG[l]), dc, de, and dx_{l-1} = M_l^T g_l (dX[l-1])
+    for (int l = 1; l <= L; ++l) {
+      const int r = nn[l], cl = nn[l - 1];
+      const float *gWl = gW + a.off[l - 1], *gSl = gS + a.off[l - 1];
+      gemm(sm, Cc, r, cl, Xk[l - 1], cl, 1, gWl, cl, 1, [&](int i, int j, float z) { P1[i * r + j] = z; });
+      gemm(sm, Cc, r, cl, Xk[l - 1], cl, 1, gSl, cl, 1, [&](int i, int j, float z) { P2[i * r + j] = z; });
+      __syncthreads();
+      for (int i = threadIdx.x / 32; i < Cc; i += NT / 32) {
+        float x = 0.f, y = 0.f;
+        for (int j = threadIdx.x % 32; j < r; j += 32) {
+          x = fmaf(Gk[l][i * r + j], P1[i * r + j], x);
+          y = fmaf(Gk[l][i * r + j], P2[i * r + j], y);
+        }
+        x = warp_sum_simt(x);
+        y = warp_sum_simt(y);
+        if (threadIdx.x % 32 == 0) { dc[i] -= x; de[i] -= y; }
+      }
+      for (int e = threadIdx.x; e < Cc * r; e += NT) {
+        const int i = e / r;
+        dG[l][e] = -(sm.coef.c[i] * P1[e] + sm.coef.e[i] * P2[e]);
+      }
+      __syncthreads();
+      float *dXl = dX[l - 1];
+      gemm(sm, Cc, cl, r, Gk[l], r, 1, gWl, 1, cl, [&](int i, int j, float z) { dXl[i * cl + j] = -sm.coef.c[i] * z; });
+      __syncthreads();
+      gemm(sm, Cc, cl, r, Gk[l], r, 1, gSl, 1, cl, [&](int i, int j, float z) { dXl[i * cl + j] -= sm.coef.e[i] * z; });
+      __syncthreads();
+    }
+    // back through the keys' backward recursion
+    for (int l = 2; l <= L; ++l) {
+      const int r = nn[l], cl = nn[l - 1];
+      for (int e = threadIdx.x; e < Cc * cl; e += NT) {
+        dH[e] = dG[l - 1][e] * silu_prime(Zk[l - 1][e]);
+        dSP[l - 1][e] = dG[l - 1][e] * Hk[l - 1][e];
+      }
+      __syncthreads();
+      float *gWnl = gWn + a.off[l - 1], *dGl = dG[l];
+      gemm(sm, r, cl, Cc, Gk[l], 1, r, dH, 1, cl, [&](int rr, int j, float z) { gWnl[rr * cl + j] += z; });
+      __syncthreads();
+      gemm(sm, Cc, r, cl, dH, cl, 1, W + a.off[l - 1], cl, 1, [&](int i, int rr, float z) { dGl[i * r + rr] += z; });
+      __syncthreads();
+    }
+    const long long gout = (tok0 + t0) * dL, gin = (tok0 + t0) * d0;
+    for (int e = threadIdx.x; e < Cc * dL; e += NT) {
+      dX[L][e] = 2.f * dG[L][e];
+      a.dv[gout + e] = -2.f * dG[L][e];
+    }
+    __syncthreads();
+    // back through the keys' forward
+    for (int l = L; l >= 1; --l) {
+      const int r = nn[l], cl = nn[l - 1];
+      float *dZ = dH;
+      if (l == L) {
+        for (int e = threadIdx.x; e < Cc * r; e += NT) dZ[e] = dX[L][e];
+      } else {
+        for (int e = threadIdx.x; e < Cc * r; e += NT)
+          dZ[e] = dX[l][e] * silu_prime(Zk[l][e]) + dSP[l][e] * silu_second(Zk[l][e]);
+      }
+      __syncthreads();
+      float *gWnl = gWn + a.off[l - 1], *dXl = dX[l - 1];
+      gemm(sm, r, cl, Cc, dZ, 1, r, Xk[l - 1], 1, cl, [&](int rr, int j, float z) { gWnl[rr * cl + j] += z; });
+      __syncthreads();
+      gemm(sm, Cc, cl, r, dZ, r, 1, W + a.off[l - 1], 1, cl, [&](int i, int j, float z) { dXl[i * cl + j] += z; });
+      __syncthreads();
+    }
+    for (int e = threadIdx.x; e < Cc * d0; e += NT) a.dk[gin + e] = dX[0][e];
+    __syncthreads();
+    // the reads: ordinary backward of y = M(q)
+    for (int e = threadIdx.x; e < Cc * dL; e += NT) dXq[L][e] = DY[e];
+    __syncthreads();
+    for (int l = L; l >= 1; --l) {
+      const int r = nn[l], cl = nn[l - 1];
+      float *dZ = dH;
+      for (int e = threadIdx.x; e < Cc * r; e += NT) dZ[e] = l == L ? dXq[L][e] : dXq[l][e] * silu_prime(Zq[l][e]);
+      __syncthreads();
+      float *gWnl = gWn + a.off[l - 1], *dXl = dXq[l - 1];
+      gemm(sm, r, cl, Cc, dZ, 1, r, Xq[l - 1], 1, cl, [&](int rr, int j, float z) { gWnl[rr * cl + j] += z; });
+      __syncthreads();
+      gemm(sm, Cc, cl, r, dZ, r, 1, W + a.off[l - 1], 1, cl, [&](int i, int j, float z) { dXl[i * cl + j] = z; });
+      __syncthreads();
+    }
+    for (int e = threadIdx.x; e < Cc * d0; e += NT) a.dq[gin + e] = dXq[0][e];
+    // chunk scalars, gates, state gradients
+    float pw = 0.f, pws = 0.f, pss = 0.f;
+    for (long long e = threadIdx.x; e < P; e += NT) {
+      pw = fmaf(gW[e], W[e], pw);
+      pws = fmaf(gW[e], S[e], pws);
+      pss = fmaf(gS[e], S[e], pss);
+    }
+    const float dB = block_sum(pw, red), dcS = block_sum(pws, red), dA = block_sum(pss, red);
+    if (threadIdx.x == 0)
+      gate_reverse(Cc, th, et, al, dc, de, dB, dA, dcS, a.dtheta + tok0 + t0, a.deta + tok0 + t0,
+                   a.dalpha + tok0 + t0, pa, pe, rho, dpa, dpe, drho);
+    for (long long e = threadIdx.x; e < P; e += NT) {
+      gS[e] = cS * gW[e] + As * gS[e];
+      gW[e] = gWn[e];
+    }
+    __syncthreads();
+  }
+  for (long long e = threadIdx.x; e < P; e += NT) {
+    a.dW0[sw + e] = gW[e];
+    a.dS0[sw + e] = gS[e];
+  }
+}
+
 }  // namespace
 
 size_t simt_scratch_bytes(const Problem &p) {
@@ -822,12 +1073,15 @@ cudaError_t simt_launch(const Problem &p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-bool backward_supported(const Problem &p) { return (p.L == 1 || p.L == 2) && p.C <= kMaxC; }
+bool backward_supported(const Problem &p) { return p.L >= 1 && p.L <= kMaxL && p.C <= kMaxC; }
 
 size_t backward_scratch_bytes(const Problem &p) {
   const long long d = p.dims[0], C = p.C, nch = (p.T + p.C - 1) / p.C;
-  const long long per = p.L == 1 ? 2 * nch * d * d + 5 * d * d + 10 * C * d + 8 * C
-                                 : backward2_floats(p.dims[0], p.dims[1], p.dims[2], p.T, p.C);
+  int maxw = 0;
+  for (int l = 0; l <= p.L; ++l) maxw = p.dims[l] > maxw ? p.dims[l] : maxw;
+  const long long per = p.L == 1   ? 2 * nch * d * d + 5 * d * d + 10 * C * d + 8 * C
+                        : p.L == 2 ? backward2_floats(p.dims[0], p.dims[1], p.dims[2], p.T, p.C)
+                                   : backwardL_floats((long long)p.P, maxw, p.T, p.C);
   return (size_t)(per * p.streams) * sizeof(float);
 }
 
@@ -835,6 +1089,30 @@ cudaError_t backward_launch(const Problem &p, const float *dy, const float *dW_e
                             float *dk, float *dv, float *dq, float *dtheta, float *deta, float *dalpha,
                             float *dW0, float *dS0, cudaStream_t stream) {
   if (!backward_supported(p)) return cudaErrorNotSupported;
+  if (p.L >= 3) {
+    BArgsL b;
+    b.L = p.L;
+    b.T = p.T;
+    b.C = p.C;
+    b.bf16 = p.in_dtype == TM_BF16 ? 1 : 0;
+    b.maxw = 0;
+    for (int l = 0; l <= kMaxL; ++l) {
+      b.dims[l] = l <= p.L ? p.dims[l] : 0;
+      b.off[l] = l <= p.L ? (long long)p.layer_off[l] : 0;
+      if (l <= p.L && p.dims[l] > b.maxw) b.maxw = p.dims[l];
+    }
+    b.P = (long long)p.P;
+    b.k = p.k; b.v = p.v; b.q = p.q;
+    b.theta = p.theta; b.eta = p.eta; b.alpha = p.alpha;
+    b.W0 = p.W0; b.S0 = p.S0;
+    b.dy = dy; b.dW_end = dW_end; b.dS_end = dS_end;
+    b.dk = dk; b.dv = dv; b.dq = dq; b.dtheta = dtheta; b.deta = deta; b.dalpha = dalpha;
+    b.dW0 = dW0; b.dS0 = dS0;
+    b.scratch = static_cast<float *>(p.scratch);
+    b.scratch_per_stream = backwardL_floats(b.P, b.maxw, p.T, p.C);
+    simt_backwardL_kernel<<<p.streams, NT, 0, stream>>>(b);
+    return cudaGetLastError();
+  }
   if (p.L == 2) {
     BArgs2 b;
     b.d = p.dims[0];

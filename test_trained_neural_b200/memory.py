@@ -127,7 +127,7 @@ class NeuralMemory:
 
     def backward(self, k, v, q, theta, eta, alpha, W0, S0, dy, dW_end, dS_end, C, stream=None):
         """Gradients of sum <dy, y> + <dW_end, W_end> + <dS_end, S_end> for the
-        run with these inputs (depth 1). Returns a dict of float32 tensors dk,
+        run with these inputs (any depth). Returns a dict of float32 tensors dk,
         dv, dq, dtheta, deta, dalpha, dW0, dS0."""
         B, H, T, d = k.shape
         dt = self._dtype_code(k)

@@ -1,4 +1,4 @@
-"""Gradients of the memory layer (tm_backward, depths 1 and 2) against the float64
+"""Gradients of the memory layer (tm_backward, depths 1 to 4) against the float64
 gradient oracle (autograd through the restated recurrence, itself pinned
 against finite differences of the C oracle)."""
 import ctypes
@@ -24,6 +24,9 @@ BACKWARD = [  # L, d, expansion, B, H, T, C, dtype
     (2, 16, 4, 1, 2, 48, 16, "f32"),     # depth 2, hidden 64
     (2, 32, 2, 2, 1, 50, 16, "bf16"),    # depth 2, a shorter last chunk
     (2, 64, 4, 1, 1, 64, 64, "bf16"),    # depth 2, the d = 64 workload's memory
+    (3, 16, 2, 1, 2, 40, 16, "f32"),     # depth 3, a shorter last chunk (40 = 2 x 16 + 8)
+    (4, 16, 2, 2, 1, 48, 16, "f32"),     # depth 4
+    (4, 128, 2, 1, 1, 40, 32, "bf16"),   # the deep workload's memory 128-256-256-256-128
 ]
 
 
@@ -60,9 +63,10 @@ def test_backward_matches_gradient_oracle(cfg):
 def test_backward_refuses_before_any_launch():
     lib = N.load()
     h = ctypes.c_void_p()
-    assert lib.tm_create(4, 64, 2, N.TM_ACT_SILU, ctypes.byref(h)) == N.TM_OK
     n = ctypes.c_size_t()
-    assert lib.tm_backward_workspace_size(h, 1, 1, 64, 16, N.TM_F32, ctypes.byref(n)) == N.TM_ERR_UNSUPPORTED
+    assert lib.tm_create(4, 64, 2, N.TM_ACT_SILU, ctypes.byref(h)) == N.TM_OK
+    assert lib.tm_backward_workspace_size(h, 1, 1, 64, 16, N.TM_F32, ctypes.byref(n)) == N.TM_OK
+    assert lib.tm_backward_workspace_size(h, 1, 1, 64, 512, N.TM_F32, ctypes.byref(n)) != N.TM_OK
     lib.tm_destroy(h)
     assert lib.tm_create(1, 64, 1, N.TM_ACT_SILU, ctypes.byref(h)) == N.TM_OK
     assert lib.tm_backward_workspace_size(h, 1, 1, 64, 16, N.TM_F32, ctypes.byref(n)) == N.TM_OK

@@ -13,6 +13,7 @@ CASES = [  # dims, T, C
     ([3, 3], 5, 2),          # linear memory, partial last chunk
     ([2, 3, 2], 4, 2),       # depth 2
     ([2, 2, 2, 2], 3, 3),    # depth 3, one chunk
+    ([2, 3, 2, 3, 2], 5, 2),  # depth 4, two full chunks and a shorter last one
 ]
 
 
