@@ -21,6 +21,19 @@ struct tm_ctx {
   cudaStream_t side[tmem::kMaxGroups - 1] = {};
   cudaEvent_t ev_fork = nullptr;
   cudaEvent_t ev_join[tmem::kMaxGroups - 1] = {};
+  // layered path: its per-chunk launches as one CUDA graph, captured when a
+  // call repeats the previous call exactly (shapes, pointers, settings) and
+  // replayed while calls keep repeating it; the launch sequence is long
+  // (two launches per chunk and group) and the host's enqueue rate would
+  // otherwise pace the GPU
+  struct Key {
+    int v[12];
+    const void *ptr[12];
+  };
+  Key seen{}, graph_key{};
+  bool has_seen = false;
+  cudaStream_t cap = nullptr;
+  cudaGraphExec_t exec = nullptr;
 };
 
 namespace {
@@ -135,7 +148,16 @@ tm_status tm_create(int L, int d_h, int expansion, tm_act act, tm_ctx **out) {
 
 namespace {
 
+void drop_graph(tm_ctx *ctx) {
+  if (ctx->exec) cudaGraphExecDestroy(ctx->exec);
+  ctx->exec = nullptr;
+}
+
 void release_side(tm_ctx *ctx) {
+  drop_graph(ctx);
+  ctx->has_seen = false;
+  if (ctx->cap) cudaStreamDestroy(ctx->cap);
+  ctx->cap = nullptr;
   for (int i = 0; i < tmem::kMaxGroups - 1; ++i) {
     if (ctx->side[i]) cudaStreamDestroy(ctx->side[i]);
     if (ctx->ev_join[i]) cudaEventDestroy(ctx->ev_join[i]);
@@ -163,6 +185,58 @@ bool ensure_side(tm_ctx *ctx, int groups) {
       return false;
   }
   return true;
+}
+
+tm_ctx::Key run_key(const tm_ctx *ctx, tm_path path, const tmem::Problem &p) {
+  tm_ctx::Key k;
+  std::memset(&k, 0, sizeof k);
+  const unsigned long long w = tmem::tcl_wait_ns();
+  const int v[] = {(int)path, p.B, p.H, p.T, p.C, (int)p.in_dtype, tmem::tcl_group_count(p), ctx->dev,
+                   (int)(w & 0x7fffffff), (int)(w >> 31), p.T_run, 0};
+  std::memcpy(k.v, v, sizeof v);
+  const void *ptr[] = {p.k, p.v, p.q, p.theta, p.eta, p.alpha, p.W0, p.S0, p.y, p.W_end, p.S_end, p.scratch};
+  std::memcpy(k.ptr, ptr, sizeof ptr);
+  return k;
+}
+
+bool same_key(const tm_ctx::Key &a, const tm_ctx::Key &b) { return std::memcmp(&a, &b, sizeof a) == 0; }
+
+// Captures the layered launch sequence of `p` into ctx->exec. On any failure
+// the capture is discarded and the caller launches directly.
+bool capture_layered(tm_ctx *ctx, const tmem::Problem &p, const tm_ctx::Key &key) {
+  drop_graph(ctx);
+  if (!ctx->cap && cudaStreamCreateWithFlags(&ctx->cap, cudaStreamNonBlocking) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (cudaStreamBeginCapture(ctx->cap, cudaStreamCaptureModeRelaxed) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  const cudaError_t e = tmem::tcl_launch(p, ctx->cap);
+  cudaGraph_t g = nullptr;
+  const cudaError_t e2 = cudaStreamEndCapture(ctx->cap, &g);
+  bool ok = e == cudaSuccess && e2 == cudaSuccess && g != nullptr;
+  if (ok) ok = cudaGraphInstantiate(&ctx->exec, g, 0) == cudaSuccess;
+  if (g) cudaGraphDestroy(g);
+  if (!ok) {
+    ctx->exec = nullptr;
+    cudaGetLastError();
+    return false;
+  }
+  ctx->graph_key = key;
+  return true;
+}
+
+// The layered path: graph replay when the call repeats, else direct launches.
+cudaError_t run_layered(tm_ctx *ctx, tm_path path, const tmem::Problem &p, cudaStream_t s) {
+  const tm_ctx::Key key = run_key(ctx, path, p);
+  if (ctx->exec && same_key(key, ctx->graph_key)) return cudaGraphLaunch(ctx->exec, s);
+  if (ctx->has_seen && same_key(key, ctx->seen) && capture_layered(ctx, p, key))
+    return cudaGraphLaunch(ctx->exec, s);
+  ctx->seen = key;
+  ctx->has_seen = true;
+  return tmem::tcl_launch(p, s);
 }
 
 }  // namespace
@@ -285,8 +359,8 @@ tm_status tm_run(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype, con
   p.fuse_fb = path == TM_PATH_TC_LAYERED;
   if (path == TM_PATH_TC_LAYERED || path == TM_PATH_TC_PHASED) {
     const int groups = tmem::tcl_group_count(p);
+    if (!ensure_side(ctx, groups)) return TM_ERR_CUDA;
     if (groups > 1) {
-      if (!ensure_side(ctx, groups)) return TM_ERR_CUDA;
       for (int i = 0; i < groups - 1; ++i) {
         p.side_streams[i] = ctx->side[i];
         p.ev_join[i] = ctx->ev_join[i];
@@ -300,7 +374,7 @@ tm_status tm_run(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype, con
     err = tmem::simt_launch(p, s);
   } else {
     if (p.T_run > 0)
-      err = (path == TM_PATH_TC || path == TM_PATH_TC_GLOBAL) ? tmem::tc_launch(p, s) : tmem::tcl_launch(p, s);
+      err = (path == TM_PATH_TC || path == TM_PATH_TC_GLOBAL) ? tmem::tc_launch(p, s) : run_layered(ctx, path, p, s);
     if (err == cudaSuccess && p.T_run < p.T) {
       // the shorter last chunk, from the state the whole chunks left
       tmem::Problem q = p;

@@ -66,6 +66,7 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream);
 int tcl_group_count(const Problem &p);   // CUDA streams tcl_launch uses
 long long tcl_launch_count(const Problem &p);
 void tcl_set_wait(unsigned long long wait_ns);
+unsigned long long tcl_wait_ns();
 
 // Gradients of the memory layer (depth 1) with respect to its inputs.
 bool backward_supported(const Problem &p);

@@ -34,7 +34,7 @@ constexpr int NT = 256;          // 8 warps: warp w reads TMEM lanes 32 (w % 4) 
                                  // columns half w / 4 of the tile
 constexpr int KB = 64;           // K block (one 128-byte swizzle atom of bf16)
 
-enum Kind { K_FWD = 0, K_FWD_LAST = 1, K_BWD = 2, K_DW = 3 };
+enum Kind { K_FWD = 0, K_FWD_LAST = 1, K_BWD = 2 };
 
 struct GemmArgs {
   int kind;
@@ -84,44 +84,19 @@ __device__ bool wait_b(uint64_t *bar, uint32_t par, const GemmArgs &a) {
   return false;
 }
 
-// Shared-memory stage: A tile [128 rows x 64 k] (K-major) or, for the update
-// GEMM, two MN-major A tiles [64 tokens x 128] (c and e); B tile up to
+// Shared-memory stage: A tile [128 rows x 64 k] (K-major); B tile up to
 // [256 x 64] (K-major) or [64 x 256] (MN-major). All in the row-block layout.
 constexpr uint32_t A_BYTES = 128 * KB * 2;       // 16 KB
 constexpr uint32_t B_BYTES = 256 * KB * 2;       // 32 KB
-constexpr uint32_t STAGE_BYTES_DW = 2 * A_BYTES + B_BYTES;   // 64 KB, 3 stages
 constexpr uint32_t STAGE_BYTES_MM = A_BYTES + B_BYTES;       // 48 KB, 4 stages
 constexpr int STAGES_MAX = 4;
-// The update GEMM's output tiles are at most 128 columns wide, so its two
-// accumulators take 256 TMEM columns and, for C <= 128 (two K blocks, two
-// stages), its ring 96 KB: two CTAs fit on an SM and one layer's update
-// overlaps the next one's.
-constexpr int DW_MAXN = 128;
-__host__ __device__ constexpr int dw_stages(int nk) { return nk <= 2 ? 2 : 3; }
-__host__ __device__ constexpr uint32_t dw_stage_bytes(int N) { return 2 * A_BYTES + (uint32_t)N * KB * 2; }
-// (the epilogue's staging buffer for U_W and U_S of a 64-column piece, 64 KB,
-// reuses the ring, which is at least 80 KB)
 
-// A tile loads. mt: 128-row tile index (forward/backward) or 128-column tile
-// of the transposed operand (update).
+// A tile loads. mt: 128-row tile index.
 __device__ __forceinline__ void load_stage(const GemmArgs &a, const CUtensorMap *mA,
                                            const CUtensorMap *mA2, const CUtensorMap *mB,
                                            unsigned char *st, uint64_t *bar, int s, int mt,
                                            int nt, int kb) {
   const int kind = a.kind;
-  if (kind == K_DW) {
-    // A^T operands: -c G and -e G, rows = tokens (K), features = rows of W (M)
-    // B: X_{l-1}, rows = tokens (K), features = N. All MN-major.
-    const int row0 = s * a.a_rows_per_stream + kb * KB;
-    for (int f = 0; f < 2; ++f) {
-      tma_load_2d(st + f * 64 * 128, mA, bar, 128 * mt + 64 * f, row0);
-      tma_load_2d(st + A_BYTES + f * 64 * 128, mA2, bar, 128 * mt + 64 * f, row0);
-    }
-    const int brow0 = (int)(s * a.b_rows_per_stream + a.b_row_off) + kb * KB;
-    for (int f = 0; f < a.N / 64; ++f)
-      tma_load_2d(st + 2 * A_BYTES + f * 64 * 128, mB, bar, a.N * nt + 64 * f, brow0);
-    return;  // DW stage: [A_c | A_e | B]
-  }
   // A: K-major [128 rows x 64] (rows = tokens); two 64-row pieces.
   for (int piece = 0; piece < 2; ++piece) {
     const int r = 128 * mt + 64 * piece;         // row of the per-stream matrix
@@ -159,9 +134,9 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   constexpr int kind = KIND;
   const int nk = a.K / KB;
-  const uint32_t ncols = 256u;                 // DW: U_W in columns [0, 128), U_S in [128, 256)
-  const int STAGES = kind == K_DW ? dw_stages(nk) : 4;
-  const uint32_t STAGE_BYTES = kind == K_DW ? dw_stage_bytes(a.N) : STAGE_BYTES_MM;
+  const uint32_t ncols = 256u;
+  constexpr int STAGES = 4;
+  constexpr uint32_t STAGE_BYTES = STAGE_BYTES_MM;
 
   if (tid == 0) {
     for (int i = 0; i < STAGES_MAX; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
@@ -174,35 +149,14 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
   tc_fence_after();
   const uint32_t tm = tslot;
   bool ok = true;
-  // Update: this thread's share of a 64-column piece of the fp32 state tile,
-  // in a coalesced mapping (16 threads per 256-byte row piece, rows
-  // tid/16 + 16 i). The first piece is requested while thread 0 issues the
-  // MMAs (the others skip that loop).
-  float4 wpre[8], spre[8];
-  const int dw_c4 = tid % 16, dw_r0 = tid / 16;
-  auto dw_prefetch = [&](int pc) {
-    float *Wl = a.W + (long long)s * a.P + a.layer_off;
-    float *Sl = a.S + (long long)s * a.P + a.layer_off;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int wr = 128 * mt + dw_r0 + 16 * i;
-      if (wr < a.M) {
-        const long long g = (long long)wr * a.n_out + a.N * nt + 64 * pc + 4 * dw_c4;
-        wpre[i] = *reinterpret_cast<const float4 *>(Wl + g);
-        spre[i] = *reinterpret_cast<const float4 *>(Sl + g);
-      }
-    }
-  };
   // Programmatic dependent launch: everything above overlapped the previous
   // kernel's tail; its outputs are read only after this wait.
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (tid == 0) {
-    const uint32_t tx = kind == K_DW ? (uint32_t)(2 * A_BYTES + (uint32_t)a.N * KB * 2)
-                                     : (uint32_t)(A_BYTES + (uint32_t)a.N * KB * 2);
+    const uint32_t tx = (uint32_t)(A_BYTES + (uint32_t)a.N * KB * 2);
     uint32_t idesc;
-    if (kind == K_DW) idesc = idesc_bf16(128, a.N, true, true);
-    else if (kind == K_BWD) idesc = idesc_bf16(128, a.N, false, true);
+    if (kind == K_BWD) idesc = idesc_bf16(128, a.N, false, true);
     else idesc = idesc_bf16(128, a.N, false, false);
     for (int kb = 0; kb < nk && kb < STAGES; ++kb) {
       mbar_arrive_expect_tx(&full[kb], tx);
@@ -215,11 +169,7 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
       tc_fence_after();
       const uint32_t base = smem_u32(sm + st * STAGE_BYTES);
       for (int ks = 0; ks < KB / 16; ++ks) {
-        if (kind == K_DW) {
-          const uint64_t bd = desc_mnmajor(base + 2 * A_BYTES, 64, ks);
-          umma_bf16(tm, desc_mnmajor(base, 64, ks), bd, idesc, (kb | ks) != 0);
-          umma_bf16(tm + 128, desc_mnmajor(base + A_BYTES, 64, ks), bd, idesc, (kb | ks) != 0);
-        } else if (kind == K_BWD) {
+        if (kind == K_BWD) {
           umma_bf16(tm, desc_kmajor(base, 128, ks), desc_mnmajor(base + A_BYTES, 64, ks), idesc,
                     (kb | ks) != 0);
         } else {
@@ -236,7 +186,6 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
     }
     umma_commit(&done);
   }
-  if constexpr (kind == K_DW) dw_prefetch(0);
   __syncwarp();
   // the next kernel may start its prologue now (it waits for our completion
   // before reading anything we write)
@@ -322,63 +271,6 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
       }
     }
   }
-  if constexpr (kind == K_DW) {
-    // Update, one 64-column piece at a time: (1) each thread moves its TMEM
-    // lane's 32 columns of U_W and U_S into shared memory (16-byte slots of a
-    // 256-byte row, slot index XOR row % 16: conflict-free both ways);
-    // (2) the tile is then updated row-contiguously, W' = B W + c_S S + U_W,
-    // S' = A S + U_S, with the prefetched state, and the next piece's state is
-    // requested before the stores.
-    float *uw = reinterpret_cast<float *>(sm);
-    float *us = uw + 128 * 64;
-    const float4 sc = *reinterpret_cast<const float4 *>(a.scal + 4 * ((long long)s * a.nchunks + a.chunk));
-    float *Wl = a.W + (long long)s * a.P + a.layer_off;
-    float *Sl = a.S + (long long)s * a.P + a.layer_off;
-    __nv_bfloat16 *Wb = a.Wbf + (long long)s * a.M * a.n_out;
-    const int npc = a.N / 64;
-    for (int pc = 0; pc < npc; ++pc) {
-      if (ok) {
-        const uint32_t c0 = (uint32_t)(64 * pc + 32 * half);
-#pragma unroll
-        for (int acc = 0; acc < 2; ++acc) {      // U_W, then U_S
-          float u0[16], u1[16];
-          tmem_ld16(tm + lb + 128 * acc + c0, u0);
-          tmem_ld16(tm + lb + 128 * acc + c0 + 16, u1);
-          tmem_wait_ld();
-          float *dst = (acc ? us : uw) + row * 64;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int slot = (8 * half + j) ^ (row & 15);
-            const float *src = j < 4 ? u0 + 4 * j : u1 + 4 * (j - 4);
-            *reinterpret_cast<float4 *>(dst + 4 * slot) = make_float4(src[0], src[1], src[2], src[3]);
-          }
-        }
-      }
-      __syncthreads();
-      if (ok) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int r = dw_r0 + 16 * i;
-          const int wr = 128 * mt + r;
-          if (wr >= a.M) continue;
-          const int slot = dw_c4 ^ (r & 15);
-          const float4 u4 = *reinterpret_cast<const float4 *>(uw + r * 64 + 4 * slot);
-          const float4 v4 = *reinterpret_cast<const float4 *>(us + r * 64 + 4 * slot);
-          const float4 w4 = wpre[i], s4 = spre[i];
-          const float4 wn = make_float4(sc.x * w4.x + sc.z * s4.x + u4.x, sc.x * w4.y + sc.z * s4.y + u4.y,
-                                        sc.x * w4.z + sc.z * s4.z + u4.z, sc.x * w4.w + sc.z * s4.w + u4.w);
-          const float4 sn = make_float4(sc.y * s4.x + v4.x, sc.y * s4.y + v4.y, sc.y * s4.z + v4.z,
-                                        sc.y * s4.w + v4.w);
-          const long long g = (long long)wr * a.n_out + a.N * nt + 64 * pc + 4 * dw_c4;
-          *reinterpret_cast<float4 *>(Wl + g) = wn;
-          *reinterpret_cast<float4 *>(Sl + g) = sn;
-          *reinterpret_cast<uint2 *>(Wb + g) = make_uint2(pack_bf16(wn.x, wn.y), pack_bf16(wn.z, wn.w));
-        }
-        if (pc + 1 < npc) dw_prefetch(pc + 1);
-      }
-      __syncthreads();
-    }
-  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tm, ncols);
@@ -393,30 +285,193 @@ __global__ void __launch_bounds__(NT, 1)
   gemm_tile<KIND>(a, mA, mA2, mB, blockIdx.z, blockIdx.y, blockIdx.x);
 }
 
-// The update of every layer of a chunk in one launch: the layers' output
-// tiles are numbered one after another (layer, then stream, row tile, column
-// tile). Limited to 128 registers so that two CTAs share an SM; the fixed
-// latency of a tile (operand loads, MMAs, staging) is then hidden by the
-// tiles running beside it instead of being paid once per layer.
-struct DwGroup {
-  GemmArgs l[kMaxL];
-  int first[kMaxL + 1];              // first tile of each layer; first[L] = total
-  int mtiles[kMaxL], ntiles[kMaxL];
-  int L;
+// ------------------------------------------------------------------------
+// The state update of every layer of a chunk, in one launch. One CTA per
+// tile of 128 rows x N columns of one layer's W_l (tiles numbered layer, then
+// stream, row tile, column tile) forms the weight-update contractions
+//   U_W = sum_i (-c_i g_i) x_i^T,  U_S = sum_i (-e_i g_i) x_i^T
+// on tcgen05 (A = the MN-major -c G and -e G of the tile's rows, B = the
+// layer's inputs X; accumulators in TMEM columns 0.. and 128..), then
+//   W' = B W + c_S S + U_W,  S' = A S + U_S
+// and the bf16 copy of W' that the next chunk's forward reads.
+// The fp32 state tile travels by TMA both ways. Its loads (32-column boxes,
+// 128-byte swizzle) are issued when the CTA starts, beside the contraction's
+// operands: the previous chunk's update of these rows completed before the
+// kernels between it and this launch could start, so they need not wait for
+// the preceding kernel. After the MMAs, the thread that owns a row's TMEM
+// lane updates that row in shared memory (16-byte chunk j of row r sits at
+// j ^ (r % 8): conflict-free across the 8 rows a quarter-warp touches), and
+// the tile goes back to global memory by TMA stores. Every state byte is read
+// once and written once and a tile's loads are all in flight together.
+constexpr int UP_NT = 256;
+constexpr uint32_t UP_BOX = 128 * 128;         // one box slot: 128 rows x 128 bytes
+struct UpLayer {
+  int M, N, mtiles, ntiles, first;             // rows of W_l, tile width, tiles per stream, first tile
+  int b_rows_per_stream;                       // rows of the X source per stream
+  long long b_row_off;                         // first X row of the chunk (layer 1 reads the keys)
 };
-struct DwMaps {
-  CUtensorMap a[kMaxL], a2[kMaxL], b[kMaxL];
+struct UpArgs {
+  UpLayer l[kMaxL];
+  int L, C, chunk, nchunks;
+  const float *scal;                           // [streams, nchunks, 4] (B, A, c_S, -)
+  int *status;
+  unsigned long long wait_ns;
 };
+struct UpMaps {
+  CUtensorMap a[kMaxL], a2[kMaxL], b[kMaxL];   // -c G_l, -e G_l [S*C, d_l]; X_{l-1} (bf16, 64 x 64 boxes)
+  CUtensorMap w[kMaxL], s[kMaxL];              // fp32 W_l, S_l as {cols, rows, stream}, 32-column boxes
+  CUtensorMap wb[kMaxL];                       // bf16 W_l as {cols, rows, stream}, 64-column boxes
+};
+__host__ __device__ constexpr uint32_t up_stage_bytes(int N) { return 2 * A_BYTES + (uint32_t)N * KB * 2; }
+__host__ __device__ constexpr int up_stages(int nk) { return nk <= 2 ? 2 : 3; }
+// dynamic shared memory: the operand ring, then the W and S tiles
+__host__ __device__ constexpr size_t up_smem(int N, int nk) {
+  return (size_t)up_stages(nk) * up_stage_bytes(N) + 2 * (size_t)(N / 32) * UP_BOX + 1024;
+}
+// tile width: 128 columns when the ring and both state tiles fit (C <= 128)
+__host__ __device__ constexpr int up_width(int cols, int C) { return cols % 128 == 0 && C <= 128 ? 128 : 64; }
 
-__global__ void __launch_bounds__(NT, 2)
-    tcl_dw_kernel(const __grid_constant__ DwGroup g, const __grid_constant__ DwMaps m) {
+__device__ __forceinline__ bool up_wait(uint64_t *bar, uint32_t par, const UpArgs &a) {
+  if (mbar_wait(bar, par, a.wait_ns)) return true;
+  atomicCAS(a.status, 0, kDevTimeout);
+  return false;
+}
+
+__global__ void __launch_bounds__(UP_NT, 1)
+    tcl_update_kernel(const __grid_constant__ UpArgs a, const __grid_constant__ UpMaps m) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char *sm =
+      reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t full[3], empty[3], done, stb;
+  __shared__ uint32_t tslot;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int t = blockIdx.x;
   int l = 0;
-  while (l + 1 < g.L && t >= g.first[l + 1]) ++l;
-  const int i = t - g.first[l];
-  const int per_stream = g.mtiles[l] * g.ntiles[l];
-  const int s = i / per_stream, j = i % per_stream;
-  gemm_tile<K_DW>(g.l[l], m.a[l], m.a2[l], m.b[l], s, j / g.ntiles[l], j % g.ntiles[l]);
+  while (l + 1 < a.L && t >= a.l[l + 1].first) ++l;
+  const UpLayer &ly = a.l[l];
+  const int per = ly.mtiles * ly.ntiles, i = t - ly.first;
+  const int s = i / per, mt = (i % per) / ly.ntiles, nt = i % ly.ntiles;
+  const int N = ly.N, nk = a.C / KB, STAGES = up_stages(nk);
+  const uint32_t SB = up_stage_bytes(N);
+  unsigned char *wt = sm + STAGES * SB;        // W tile: N / 32 boxes
+  unsigned char *st = wt + (N / 32) * UP_BOX;  // S tile
+  unsigned char *wbt = sm;                     // bf16 W' tile (N / 64 boxes), in the ring once the MMAs are done
+  const int R = ly.M < 128 ? ly.M : 128;       // rows of a box
+  const int rows = ly.M - 128 * mt < 128 ? ly.M - 128 * mt : 128;   // rows of this tile
+
+  if (tid == 0) {
+    for (int k = 0; k < 3; ++k) { mbar_init(&full[k], 1); mbar_init(&empty[k], 1); }
+    mbar_init(&done, 1);
+    mbar_init(&stb, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) { tmem_alloc(&tslot, 256); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = tslot;
+  bool ok = true;
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&stb, 2u * (uint32_t)(N / 32) * (uint32_t)R * 128u);
+    for (int b = 0; b < N / 32; ++b) {
+      tma_load_3d(wt + b * UP_BOX, &m.w[l], &stb, N * nt + 32 * b, 128 * mt, s);
+      tma_load_3d(st + b * UP_BOX, &m.s[l], &stb, N * nt + 32 * b, 128 * mt, s);
+    }
+  }
+  // the operands are the preceding kernel's outputs
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (tid == 0) {
+    const uint32_t idesc = idesc_bf16(128, N, true, true);
+    auto load = [&](int stg, int kb) {
+      unsigned char *d = sm + stg * SB;
+      const int row0 = s * a.C + kb * KB;
+      for (int f = 0; f < 2; ++f) {
+        tma_load_2d(d + f * 64 * 128, &m.a[l], &full[stg], 128 * mt + 64 * f, row0);
+        tma_load_2d(d + A_BYTES + f * 64 * 128, &m.a2[l], &full[stg], 128 * mt + 64 * f, row0);
+      }
+      const int brow0 = (int)(s * ly.b_rows_per_stream + ly.b_row_off) + kb * KB;
+      for (int f = 0; f < N / 64; ++f)
+        tma_load_2d(d + 2 * A_BYTES + f * 64 * 128, &m.b[l], &full[stg], N * nt + 64 * f, brow0);
+    };
+    for (int kb = 0; kb < nk && kb < STAGES; ++kb) {
+      mbar_arrive_expect_tx(&full[kb], SB);
+      load(kb, kb);
+    }
+    for (int kb = 0; kb < nk && ok; ++kb) {
+      const int stg = kb % STAGES;
+      const uint32_t ph = (uint32_t)((kb / STAGES) & 1);
+      if (!up_wait(&full[stg], ph, a)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t base = smem_u32(sm + stg * SB);
+      for (int ks = 0; ks < KB / 16; ++ks) {
+        const uint64_t bd = desc_mnmajor(base + 2 * A_BYTES, 64, ks);
+        umma_bf16(tm, desc_mnmajor(base, 64, ks), bd, idesc, (kb | ks) != 0);
+        umma_bf16(tm + 128, desc_mnmajor(base + A_BYTES, 64, ks), bd, idesc, (kb | ks) != 0);
+      }
+      umma_commit(&empty[stg]);
+      if (kb + STAGES < nk) {
+        if (!up_wait(&empty[stg], ph, a)) { ok = false; break; }
+        mbar_arrive_expect_tx(&full[stg], SB);
+        load(stg, kb + STAGES);
+      }
+    }
+    umma_commit(&done);
+  }
+  __syncwarp();
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (!up_wait(&done, 0, a)) ok = false;
+  if (!up_wait(&stb, 0, a)) ok = false;
+  tc_fence_after();
+  ok = __syncthreads_and(ok) != 0;
+  if (ok) {
+    const float4 sc = *reinterpret_cast<const float4 *>(a.scal + 4 * ((long long)s * a.nchunks + a.chunk));
+    const int q = warp & 3, h = warp >> 2;     // TMEM lanes 32q.. (rows); column half h
+    const int r = 32 * q + lane;
+    const uint32_t lb = (uint32_t)(32 * q) << 16;
+    for (int gi = 0; gi < N / 64; ++gi) {
+      const int cg = (N / 2) * h + 32 * gi;    // first of this thread's 32 columns
+      float u0[16], u1[16], v0[16], v1[16];
+      tmem_ld16(tm + lb + (uint32_t)cg, u0);
+      tmem_ld16(tm + lb + (uint32_t)cg + 16, u1);
+      tmem_ld16(tm + lb + 128 + (uint32_t)cg, v0);
+      tmem_ld16(tm + lb + 128 + (uint32_t)cg + 16, v1);
+      tmem_wait_ld();
+      if (r >= rows) continue;
+      unsigned char *wr = wt + (cg / 32) * UP_BOX + r * 128;
+      unsigned char *sr = st + (cg / 32) * UP_BOX + r * 128;
+      unsigned char *br = wbt + (cg / 64) * UP_BOX + r * 128;
+      const int c16 = (cg % 64) / 8;           // 16-byte chunk of the bf16 row that column cg starts
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t o = (uint32_t)((j ^ (r & 7)) << 4);
+        const float *uw = j < 4 ? u0 + 4 * j : u1 + 4 * (j - 4);
+        const float *us = j < 4 ? v0 + 4 * j : v1 + 4 * (j - 4);
+        const float4 w = *reinterpret_cast<const float4 *>(wr + o);
+        const float4 x = *reinterpret_cast<const float4 *>(sr + o);
+        const float4 wn = make_float4(sc.x * w.x + sc.z * x.x + uw[0], sc.x * w.y + sc.z * x.y + uw[1],
+                                      sc.x * w.z + sc.z * x.z + uw[2], sc.x * w.w + sc.z * x.w + uw[3]);
+        const float4 sn = make_float4(sc.y * x.x + us[0], sc.y * x.y + us[1], sc.y * x.z + us[2],
+                                      sc.y * x.w + us[3]);
+        *reinterpret_cast<float4 *>(wr + o) = wn;
+        *reinterpret_cast<float4 *>(sr + o) = sn;
+        const uint32_t ob = (uint32_t)((((c16 + (j >> 1)) ^ (r & 7)) << 4) + (j & 1) * 8);
+        *reinterpret_cast<uint2 *>(br + ob) = make_uint2(pack_bf16(wn.x, wn.y), pack_bf16(wn.z, wn.w));
+      }
+    }
+  }
+  fence_proxy_async_smem();                    // the updated tiles are read by the TMA stores
+  __syncthreads();
+  if (tid == 0 && ok) {
+    for (int b = 0; b < N / 32; ++b) {
+      tma_store_3d(&m.w[l], wt + b * UP_BOX, N * nt + 32 * b, 128 * mt, s);
+      tma_store_3d(&m.s[l], st + b * UP_BOX, N * nt + 32 * b, 128 * mt, s);
+    }
+    for (int b = 0; b < N / 64; ++b) tma_store_3d(&m.wb[l], wbt + b * UP_BOX, N * nt + 64 * b, 128 * mt, s);
+    tma_store_commit_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tm, 256);
 }
 
 // ------------------------------------------------------------------------
@@ -842,6 +897,23 @@ bool map2d(CUtensorMap *m, const void *base, long long rows, int cols, int box_r
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over `streams` matrices [rows x cols] of el-byte elements, matrix
+// s at base + s * stream_stride elements; box = box_cols x box_rows x 1 with
+// the 128-byte swizzle (box_cols * el = 128).
+bool map3d(CUtensorMap *m, CUtensorMapDataType dt, int el, const void *base, int cols, int rows, int streams,
+           long long stream_stride, int box_cols, int box_rows) {
+  EncodeTiledFn fn = encode_fn_l();
+  if (!fn || box_cols * el != 128) return false;
+  std::memset(m, 0, sizeof *m);
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)streams};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * el, (cuuint64_t)stream_stride * el};
+  cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Workspace carve-up (bytes, 256-aligned pieces), per problem.
 struct Carve {
   size_t coef, scal, wbf, x[kMaxL + 1], sp[kMaxL + 1], g[kMaxL + 1], gc[kMaxL + 1], ge[kMaxL + 1];
@@ -877,7 +949,7 @@ bool dims_ok(const Problem &p) {
   return true;
 }
 
-constexpr size_t SMEM_BYTES = 3 * STAGE_BYTES_DW + 1024;   // = 4 * STAGE_BYTES_MM + 1024
+constexpr size_t SMEM_BYTES = 4 * STAGE_BYTES_MM + 1024;
 
 bool fb_ok(const Problem &p) {
   for (int l = 0; l <= p.L; ++l)
@@ -919,10 +991,10 @@ cudaError_t launch_gemm(const GemmArgs &a, const CUtensorMap &mA, const CUtensor
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_dw(const DwGroup &g, const DwMaps &m, size_t smem, cudaStream_t st) {
+cudaError_t launch_up(const UpArgs &a, const UpMaps &m, int tiles, size_t smem, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)g.first[g.L]);
-  cfg.blockDim = dim3(NT);
+  cfg.gridDim = dim3((unsigned)tiles);
+  cfg.blockDim = dim3(UP_NT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute at[1];
@@ -930,7 +1002,7 @@ cudaError_t launch_dw(const DwGroup &g, const DwMaps &m, size_t smem, cudaStream
   at[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, tcl_dw_kernel, g, m);
+  return cudaLaunchKernelEx(&cfg, tcl_update_kernel, a, m);
 }
 
 }  // namespace
@@ -962,9 +1034,10 @@ struct TclGroup {
   InitArgs ia;
   CUtensorMap mk, mq, mwb[kMaxL + 1], mx[kMaxL + 1], mg[kMaxL + 1], mgc[kMaxL + 1], mge[kMaxL + 1];
   GemmArgs base;
-  DwGroup dg;
-  DwMaps dm;
-  size_t dw_smem;
+  UpArgs ua;
+  UpMaps um;
+  int up_tiles;
+  size_t up_smem_bytes;
   bool fused;
   FbArgs fa;
   FbMaps fm;
@@ -1036,31 +1109,39 @@ cudaError_t TclGroup::setup() {
   base.v = reinterpret_cast<const __nv_bfloat16 *>(p.v);
 
   // the update launch: per layer, tiles of 128 rows of W_l x (128 or 64) columns
-  std::memset(&dg, 0, sizeof dg);
-  std::memset(&dm, 0, sizeof dm);
-  dg.L = L;
-  dw_smem = 0;
+  std::memset(&ua, 0, sizeof ua);
+  std::memset(&um, 0, sizeof um);
+  ua.L = L;
+  ua.C = C;
+  ua.nchunks = nchunks;
+  ua.scal = scal;
+  ua.status = p.status;
+  ua.wait_ns = g_tcl_wait_ns;
+  up_tiles = 0;
+  up_smem_bytes = 0;
   for (int l = 1; l <= L; ++l) {
-    GemmArgs &a = dg.l[l - 1];
-    a = base;
+    UpLayer &u = ua.l[l - 1];
     const int nl = p.dims[l], np = p.dims[l - 1];
-    a.kind = K_DW;
-    a.N = np % DW_MAXN == 0 ? DW_MAXN : 64;
-    a.K = C;
-    a.M = nl;
-    a.n_out = np;
-    a.a_rows_per_stream = C;
-    a.b_rows_per_stream = l == 1 ? T : 2 * C;
-    a.layer_off = (long long)p.layer_off[l - 1];
-    a.Wbf = wbf + ia.boff[l - 1];
-    dg.mtiles[l - 1] = (nl + 127) / 128;
-    dg.ntiles[l - 1] = np / a.N;
-    dg.first[l] = dg.first[l - 1] + S * dg.mtiles[l - 1] * dg.ntiles[l - 1];
-    dm.a[l - 1] = mgc[l];
-    dm.a2[l - 1] = mge[l];
-    dm.b[l - 1] = l == 1 ? mk : mx[l - 1];
-    const size_t sm = (size_t)dw_stages(C / KB) * dw_stage_bytes(a.N) + 1024;
-    if (sm > dw_smem) dw_smem = sm;
+    u.M = nl;
+    u.N = up_width(np, C);
+    u.mtiles = (nl + 127) / 128;
+    u.ntiles = np / u.N;
+    u.first = up_tiles;
+    u.b_rows_per_stream = l == 1 ? T : 2 * C;
+    up_tiles += S * u.mtiles * u.ntiles;
+    um.a[l - 1] = mgc[l];
+    um.a2[l - 1] = mge[l];
+    um.b[l - 1] = l == 1 ? mk : mx[l - 1];
+    const int br = nl < 128 ? nl : 128;
+    if (!map3d(&um.w[l - 1], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.W_end + p.layer_off[l - 1], np, nl, S,
+               (long long)p.P, 32, br) ||
+        !map3d(&um.s[l - 1], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.S_end + p.layer_off[l - 1], np, nl, S,
+               (long long)p.P, 32, br) ||
+        !map3d(&um.wb[l - 1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wbf + ia.boff[l - 1], np, nl, S,
+               (long long)nl * np, 64, br))
+      return cudaErrorInvalidValue;
+    const size_t sm = up_smem(u.N, C / KB);
+    if (sm > up_smem_bytes) up_smem_bytes = sm;
   }
 
   fused = p.fuse_fb && fb_ok(p);
@@ -1132,12 +1213,9 @@ cudaError_t TclGroup::chunk(int ch) {
     if (err != cudaSuccess) return err;
   }
   // weight-update contractions of every layer, with the fused state update
-  for (int l = 1; l <= L; ++l) {
-    dg.l[l - 1].chunk = ch;
-    dg.l[l - 1].b_row_off = l == 1 ? (long long)ch * C : 0;
-  }
-  err = launch_dw(dg, dm, dw_smem, stream);
-  return err;
+  ua.chunk = ch;
+  ua.l[0].b_row_off = (long long)ch * C;
+  return launch_up(ua, um, up_tiles, up_smem_bytes, stream);
 }
 
 // Streams split into groups issued on separate CUDA streams: one group's
@@ -1210,13 +1288,16 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e = cudaSuccess;
-    const void *kerns[4] = {(const void *)tcl_gemm_kernel<K_FWD>, (const void *)tcl_gemm_kernel<K_FWD_LAST>,
-                            (const void *)tcl_gemm_kernel<K_BWD>, (const void *)tcl_dw_kernel};
+    const void *kerns[3] = {(const void *)tcl_gemm_kernel<K_FWD>, (const void *)tcl_gemm_kernel<K_FWD_LAST>,
+                            (const void *)tcl_gemm_kernel<K_BWD>};
     for (const void *k : kerns) {
       e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
       if (e != cudaSuccess) return e;
     }
     e = cudaFuncSetAttribute(tcl_fb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FB_SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tcl_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)up_smem(128, 2));
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
@@ -1257,5 +1338,6 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
 }
 
 void tcl_set_wait(unsigned long long wait_ns) { g_tcl_wait_ns = wait_ns ? wait_ns : 2000000000ull; }
+unsigned long long tcl_wait_ns() { return g_tcl_wait_ns; }
 
 }  // namespace tmem

@@ -336,6 +336,37 @@ def test_tcl_fused_matches_phased():
     assert max(errs.values()) < 5e-3, errs
 
 
+def test_tcl_graph_replay_matches_direct_launches():
+    """The layered path captures its launch sequence into a CUDA graph when a
+    call repeats the previous one exactly, and replays it from then on: the
+    replays give the direct launches' results bit for bit, and read the
+    inputs' current contents (new data behind the same pointers)."""
+    w = W.make(4, 64, 2, 4, 4, 384, 128, index=640)     # 16 streams: two concurrent groups
+    _, dev = _dev_inputs(w)
+    mem = NeuralMemory(w.L, w.d, w.expansion, path="tcl")
+    y = torch.empty((w.B, w.H, w.T, w.d), dtype=torch.float32, device="cuda")
+    We, Se = torch.empty_like(dev["W0"]), torch.empty_like(dev["S0"])
+    ws = mem.alloc_workspace(w.B, w.H, w.T, w.C, dev["k"].dtype)
+    call = lambda: mem.run(dev["k"], dev["v"], dev["q"], dev["theta"], dev["eta"], dev["alpha"], dev["W0"],
+                           dev["S0"], w.C, y=y, W_end=We, S_end=Se, workspace=ws, sync=True)
+    outs = []
+    for _ in range(3):                                   # direct, capture + replay, replay
+        y.fill_(float("nan"))
+        call()
+        torch.cuda.synchronize()
+        outs.append((y.clone(), We.clone(), Se.clone()))
+    for o in outs[1:]:
+        assert all(torch.equal(a, b) for a, b in zip(o, outs[0]))
+    dev["k"].copy_(torch.flip(dev["k"], dims=[2]))
+    dev["alpha"].mul_(0.5)
+    call()
+    torch.cuda.synchronize()
+    fresh = NeuralMemory(w.L, w.d, w.expansion, path="tcl")
+    ref = run_lib(fresh, dev, w.C)
+    assert all(torch.equal(a, b) for a, b in zip((y, We, Se), ref))
+    assert not torch.equal(y, outs[0][0])
+
+
 RAGGED = [  # L, d, expansion, B, H, T, C, dtype, path
     (1, 64, 1, 1, 1, 100, 16, "f32", "simt"),     # linear memory, 6 whole chunks + 4 tokens
     (2, 32, 4, 2, 1, 75, 32, "bf16", "simt"),
