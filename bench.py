@@ -571,7 +571,7 @@ def main():
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = traffic_per_launch(path_used, w)
     roof["kernel"] = {"tc": "tc_chunk_kernel (cluster and global-exchange forms)",
-                      "tcl": "tcl_fb_kernel + tcl_dw_kernel",
+                      "tcl": "tcl_fb_kernel + tcl_update_kernel",
                       "tcl-phased": "tcl_gemm_kernel"}.get(path_used, "simt_chunk_kernel")
 
     e2e = None

@@ -467,7 +467,7 @@ __global__ void __launch_bounds__(UP_NT, 1)
       tma_store_3d(&m.s[l], st + b * UP_BOX, N * nt + 32 * b, 128 * mt, s);
     }
     for (int b = 0; b < N / 64; ++b) tma_store_3d(&m.wb[l], wbt + b * UP_BOX, N * nt + 64 * b, 128 * mt, s);
-    tma_store_commit_wait();
+    tma_store_commit_wait_read();
   }
   tc_fence_before();
   __syncthreads();
