@@ -68,7 +68,7 @@ long long tcl_launch_count(const Problem &p);
 void tcl_set_wait(unsigned long long wait_ns);
 unsigned long long tcl_wait_ns();
 
-// Gradients of the memory layer (depth 1) with respect to its inputs.
+// Gradients of the memory layer (depths 1 to 4) with respect to its inputs.
 bool backward_supported(const Problem &p);
 size_t backward_scratch_bytes(const Problem &p);
 cudaError_t backward_launch(const Problem &p, const float *dy, const float *dW_end, const float *dS_end,
