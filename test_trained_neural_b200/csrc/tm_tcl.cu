@@ -11,10 +11,12 @@
 //              W' = B W + c_S S + U_W, S' = A S + U_S (fp32 state in the
 //              caller's W_end / S_end) and the bf16 copy of W' for the next chunk
 // ("Titans, explained" steps 2-6; "Attack of the Titans", "Parallel
-//  training"). Launch order on one stream orders the phases; every kernel is
-// one output tile per CTA: TMA loads (128-byte swizzle) into a ring of
-// shared-memory stages, tcgen05 MMAs into TMEM, a 4-warp epilogue. Each
-// stream's tiles are independent (batched over streams).
+//  training"). Launch order on one stream orders the phases. For widths up to
+// 256 one fused kernel runs a tile's whole forward and backward; wider layers
+// run one launch per phase (one output tile per CTA: TMA loads with the
+// 128-byte swizzle into a ring of shared-memory stages, tcgen05 MMAs into
+// TMEM, an epilogue from TMEM); one launch updates every layer. Each stream's
+// tiles are independent (batched over streams).
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -44,7 +46,6 @@ struct GemmArgs {
   int a_rows_per_stream;         // rows of the A source per stream
   int b_rows_per_stream;
   int a_split_kq;                // layer-1 forward: rows < C from k, else from q
-  long long b_row_off;           // added to B's row coordinate (update of layer 1: keys)
   // epilogue operands
   __nv_bfloat16 *x_out;          // [streams, 2C, n] activations (forward)
   __nv_bfloat16 *sp_out;         // [streams, C, n] silu'(Z) of key rows (forward)
@@ -53,11 +54,6 @@ struct GemmArgs {
   float *y;                      // [streams, T, d] reads (last forward)
   const __nv_bfloat16 *v;        // [streams, T, d] values (last forward)
   const float *coef;             // [streams, T, 2] (c, e) per token
-  const float *scal;             // [streams, nchunks, 4] (B, A, cS, -)
-  float *W, *S;                  // fp32 state of this layer: [streams] x P stride
-  __nv_bfloat16 *Wbf;            // bf16 copy of this layer: [streams, M, N]
-  long long P, layer_off;
-  int nchunks;
   int *status;
   unsigned long long wait_ns;
 };
@@ -1098,11 +1094,6 @@ cudaError_t TclGroup::setup() {
   base.C = C;
   base.T = T;
   base.coef = coef;
-  base.scal = scal;
-  base.W = p.W_end;
-  base.S = p.S_end;
-  base.P = (long long)p.P;
-  base.nchunks = nchunks;
   base.status = p.status;
   base.wait_ns = g_tcl_wait_ns;
   base.y = p.y;
