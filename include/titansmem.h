@@ -135,9 +135,10 @@ TM_API tm_status tm_workspace_size(const tm_ctx *ctx, int B, int H, int T, int C
  * a call that repeats this context's previous call exactly (shapes, every
  * pointer, path, wait limit) captures its launch sequence into a CUDA graph
  * kept by the context (its resources are the CUDA runtime's), and identical
- * calls after it replay that graph on `stream`; any other call launches
- * directly. The graph reads whatever the pointers hold when it runs. Calls on
- * one context must not run concurrently.
+ * calls after it replay that graph on `stream`; any other call, and any call
+ * made while `stream` is being captured by the caller, launches directly. The
+ * graph reads whatever the pointers hold when it runs. Calls on one context
+ * must not run concurrently.
  *
  *   k, q   [B, H, T, d_h]  in_dtype, device     keys and queries
  *   v      [B, H, T, d_h]  in_dtype, device     values

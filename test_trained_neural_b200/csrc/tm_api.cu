@@ -229,7 +229,14 @@ bool capture_layered(tm_ctx *ctx, const tmem::Problem &p, const tm_ctx::Key &key
 }
 
 // The layered path: graph replay when the call repeats, else direct launches.
+// While the caller captures `s` into a graph of its own, the launches go
+// straight into that capture.
 cudaError_t run_layered(tm_ctx *ctx, tm_path path, const tmem::Problem &p, cudaStream_t s) {
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
+    cudaGetLastError();
+    return tmem::tcl_launch(p, s);
+  }
   const tm_ctx::Key key = run_key(ctx, path, p);
   if (ctx->exec && same_key(key, ctx->graph_key)) return cudaGraphLaunch(ctx->exec, s);
   if (ctx->has_seen && same_key(key, ctx->seen) && capture_layered(ctx, p, key))
