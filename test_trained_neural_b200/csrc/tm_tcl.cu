@@ -376,6 +376,7 @@ __global__ void __launch_bounds__(UP_NT, 1)
   }
   // the operands are the preceding kernel's outputs
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  int issued = 0, consumed = 0;                // operand stages requested / seen complete (thread 0)
   if (tid == 0) {
     const uint32_t idesc = idesc_bf16(128, N, true, true);
     auto load = [&](int stg, int kb) {
@@ -392,11 +393,13 @@ __global__ void __launch_bounds__(UP_NT, 1)
     for (int kb = 0; kb < nk && kb < STAGES; ++kb) {
       mbar_arrive_expect_tx(&full[kb], SB);
       load(kb, kb);
+      ++issued;
     }
     for (int kb = 0; kb < nk && ok; ++kb) {
       const int stg = kb % STAGES;
       const uint32_t ph = (uint32_t)((kb / STAGES) & 1);
       if (!up_wait(&full[stg], ph, a)) { ok = false; break; }
+      ++consumed;
       tc_fence_after();
       const uint32_t base = smem_u32(sm + stg * SB);
       for (int ks = 0; ks < KB / 16; ++ks) {
@@ -409,6 +412,7 @@ __global__ void __launch_bounds__(UP_NT, 1)
         if (!up_wait(&empty[stg], ph, a)) { ok = false; break; }
         mbar_arrive_expect_tx(&full[stg], SB);
         load(stg, kb + STAGES);
+        ++issued;
       }
     }
     umma_commit(&done);
@@ -464,6 +468,13 @@ __global__ void __launch_bounds__(UP_NT, 1)
     }
     for (int b = 0; b < N / 64; ++b) tma_store_3d(&m.wb[l], wbt + b * UP_BOX, N * nt + 64 * b, 128 * mt, s);
     tma_store_commit_wait_read();
+  }
+  if (!ok && tid == 0) {
+    // after an expired wait: copies and MMAs this CTA started may still be
+    // using its shared memory; give them (again bounded) time to finish
+    for (int k = consumed; k < issued; ++k) mbar_wait(&full[k % STAGES], (uint32_t)((k / STAGES) & 1), a.wait_ns);
+    mbar_wait(&stb, 0, a.wait_ns);
+    mbar_wait(&done, 0, a.wait_ns);
   }
   tc_fence_before();
   __syncthreads();
