@@ -11,16 +11,21 @@ SRC = os.path.join(HERE, "titans_oracle.c")
 LIB = os.path.join(HERE, "libtitans_oracle.so")
 
 
-def build(force: bool = False) -> str:
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
-        return LIB
+def compile_source(src: str, out: str) -> str:
+    """gcc `src` into the shared library `out` with the oracle's flags."""
     # -ffp-contract=off: no fused multiply-add, so every float64 operation is
     # rounded exactly as written.
     cmd = ["gcc", "-O2", "-std=c99", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
-           "-Wall", "-Wextra", "-o", LIB + ".tmp", SRC, "-lpthread", "-lm"]
+           "-Wall", "-Wextra", "-o", out + ".tmp", src, "-lpthread", "-lm"]
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(out + ".tmp", out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
+        return LIB
+    return compile_source(SRC, LIB)
 
 
 if __name__ == "__main__":

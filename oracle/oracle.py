@@ -5,6 +5,7 @@ arithmetic lives in titans_oracle.c; this file only marshals arrays.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -16,20 +17,37 @@ DT_F64, DT_F32, DT_BF16 = 0, 1, 2
 _lib = None
 
 
+def _open(path):
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    lib.titans_oracle_run.argtypes = [I, P, I, I, I, I, P, P, P, I, P, P, P, I, P, P,
+                                      P, P, P, P, P, P, I]
+    lib.titans_oracle_run.restype = I
+    lib.titans_oracle_surprise.argtypes = [I, P, P, P, P, P]
+    lib.titans_oracle_surprise.restype = I
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        path = _build.build()
-        lib = ctypes.CDLL(path)
-        P = ctypes.c_void_p
-        I = ctypes.c_int
-        lib.titans_oracle_run.argtypes = [I, P, I, I, I, I, P, P, P, I, P, P, P, I, P, P,
-                                          P, P, P, P, P, P, I]
-        lib.titans_oracle_run.restype = I
-        lib.titans_oracle_surprise.argtypes = [I, P, P, P, P, P]
-        lib.titans_oracle_surprise.restype = I
-        _lib = lib
+        _lib = _open(_build.build())
     return _lib
+
+
+@contextlib.contextmanager
+def use_library(path):
+    """Within the block, run() and surprise() call the oracle compiled at
+    `path` (the tests use this to show that the pins reject an oracle with a
+    planted mistake)."""
+    global _lib
+    prev = _load()
+    _lib = _open(path)
+    try:
+        yield
+    finally:
+        _lib = prev
 
 
 def _dtype_code(a: np.ndarray) -> int:
