@@ -1,11 +1,14 @@
-"""The oracle's pins reject an oracle with a plausible mistake in it.
+"""The oracles' pins reject an oracle with a plausible mistake in it.
 
 Each case plants one mistake in a copy of oracle/titans_oracle.c (a wrong
 sign, a dropped factor, a transposed operand, an off-by-one chunk start, the
 wrong weights for a read or a surprise, a wrong derivative), compiles it with
 the oracle's own flags and runs a battery of the pins against it: at least one
 pin must fail. The unmodified source, compiled the same way, must pass them
-all, so the failures come from the planted mistakes."""
+all, so the failures come from the planted mistakes. The second part does the
+same for the prologue's oracle (oracle/prologue.py): taps, causality, history
+order, the norm and which of k, v, q are normalised."""
+import importlib.util
 import os
 
 import pytest
@@ -15,6 +18,7 @@ from oracle import build as obuild
 
 import test_golden as golden
 import test_oracle_pins as pins
+import test_prologue as prologue_pins
 
 SRC = os.path.join(os.path.dirname(obuild.__file__), "titans_oracle.c")
 
@@ -83,3 +87,58 @@ def test_unmodified_oracle_passes_the_battery(tmp_path):
 def test_planted_mistake_fails_a_pin(tmp_path, name):
     old, new = MUTANTS[name]
     assert failures_with(build_variant(tmp_path, old, new)), name
+
+
+# ---------------------------------------------------------------- prologue oracle
+
+PRO_SRC = os.path.join(os.path.dirname(obuild.__file__), "prologue.py")
+
+PRO_MUTANTS = {
+    "taps reversed": ("out[t] += filt[:, j] * full[w - 1 + t - j]", "out[t] += filt[:, w - 1 - j] * full[w - 1 + t - j]"),
+    "looks ahead": ("out[t] += filt[:, j] * full[w - 1 + t - j]", "out[t] += filt[:, j] * full[min(w - 1 + t + j, T + w - 2)]"),
+    "history after the tokens": ("full = np.concatenate([hist, x], axis=0)", "full = np.concatenate([x, hist], axis=0)"),
+    "norm without the square root": ("n = np.sqrt((x * x).sum(axis=-1, keepdims=True))", "n = (x * x).sum(axis=-1, keepdims=True)"),
+    "norm over tokens": ("n = np.sqrt((x * x).sum(axis=-1, keepdims=True))", "n = np.sqrt((x * x).sum(axis=0, keepdims=True))"),
+    "values normalised": ("vv = conv_causal(v, filt_v, hist_v)", "vv = l2_normalise_rows(conv_causal(v, filt_v, hist_v))"),
+    "keys not normalised": ("kk = l2_normalise_rows(conv_causal(k, filt_k, hist_k))", "kk = conv_causal(k, filt_k, hist_k)"),
+}
+
+
+def prologue_battery():
+    return [
+        ("numpy convolve", prologue_pins.test_conv_matches_numpy_convolve),
+        ("delta and shift", prologue_pins.test_delta_and_shift_filters),
+        ("history", prologue_pins.test_history_equals_one_long_sequence),
+        ("normalisation", prologue_pins.test_normalisation),
+        ("keys and queries only", prologue_pins.test_prologue_normalises_keys_and_queries_only),
+    ]
+
+
+def prologue_failures(tmp_path, old=None, new=None, monkeypatch=None):
+    src = open(PRO_SRC).read()
+    if old is not None:
+        assert src.count(old) == 1, old
+        src = src.replace(old, new)
+    path = tmp_path / "prologue_variant.py"
+    path.write_text(src)
+    spec = importlib.util.spec_from_file_location("prologue_variant", str(path))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    monkeypatch.setattr(prologue_pins, "P", mod)
+    failed = []
+    for name, pin in prologue_battery():
+        try:
+            pin()
+        except (AssertionError, IndexError, ValueError):
+            failed.append(name)
+    return failed
+
+
+def test_unmodified_prologue_oracle_passes_the_battery(tmp_path, monkeypatch):
+    assert prologue_failures(tmp_path, monkeypatch=monkeypatch) == []
+
+
+@pytest.mark.parametrize("name", sorted(PRO_MUTANTS))
+def test_planted_prologue_mistake_fails_a_pin(tmp_path, monkeypatch, name):
+    old, new = PRO_MUTANTS[name]
+    assert prologue_failures(tmp_path, old, new, monkeypatch=monkeypatch), name

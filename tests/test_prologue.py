@@ -47,6 +47,19 @@ def test_normalisation():
     np.testing.assert_allclose(np.linalg.norm(np.delete(n, 2, axis=0), axis=1), 1.0, rtol=1e-14)
 
 
+def test_prologue_normalises_keys_and_queries_only():
+    """With identity filters (tap 0 = 1) the step reduces to row normalisation
+    of k and q (checked with numpy's norm) and leaves v exactly as it was."""
+    rng = np.random.default_rng(6)
+    k, v, q = (rng.standard_normal((7, 5)) for _ in range(3))
+    f = np.zeros((5, 3))
+    f[:, 0] = 1.0
+    kk, vv, qq = P.prologue(k, v, q, f, f, f)
+    np.testing.assert_allclose(kk, k / np.linalg.norm(k, axis=1, keepdims=True), rtol=1e-14)
+    np.testing.assert_allclose(qq, q / np.linalg.norm(q, axis=1, keepdims=True), rtol=1e-14)
+    np.testing.assert_array_equal(vv, v)
+
+
 def _rand(shape, rng, dtype):
     x = rng.standard_normal(shape).astype(np.float32)
     if dtype == "bf16":
