@@ -7,7 +7,9 @@ the oracle's own flags and runs a battery of the pins against it: at least one
 pin must fail. The unmodified source, compiled the same way, must pass them
 all, so the failures come from the planted mistakes. The second part does the
 same for the prologue's oracle (oracle/prologue.py): taps, causality, history
-order, the norm and which of k, v, q are normalised."""
+order, the norm and which of k, v, q are normalised; the third for the
+gradient oracle (oracle/backward.py), whose pins compare it with the C oracle
+and with finite differences of the C oracle."""
 import importlib.util
 import os
 
@@ -16,6 +18,7 @@ import pytest
 import oracle
 from oracle import build as obuild
 
+import test_backward_oracle as backward_pins
 import test_golden as golden
 import test_oracle_pins as pins
 import test_prologue as prologue_pins
@@ -142,3 +145,57 @@ def test_unmodified_prologue_oracle_passes_the_battery(tmp_path, monkeypatch):
 def test_planted_prologue_mistake_fails_a_pin(tmp_path, monkeypatch, name):
     old, new = PRO_MUTANTS[name]
     assert prologue_failures(tmp_path, old, new, monkeypatch=monkeypatch), name
+
+
+# ---------------------------------------------------------------- gradient oracle
+
+BW_SRC = os.path.join(os.path.dirname(obuild.__file__), "backward.py")
+
+BW_MUTANTS = {
+    "silu' sign": ("return s * (1 + z * (1 - s))", "return s * (1 - z * (1 - s))"),
+    "surprise without the factor 2": ("g = 2 * (xs[-1] - v)", "g = xs[-1] - v"),
+    "outer product transposed": ("us[l] = torch.outer(g, xs[l])", "us[l] = torch.outer(g, xs[l]).T.reshape(g.shape[0], -1)"),
+    "momentum without eta": ("S = [eta[t] * s - theta[t] * ul for s, ul in zip(S, u)]",
+                             "S = [s - theta[t] * ul for s, ul in zip(S, u)]"),
+    "reads at the current weights": ("ys.append(_forward(Wf, q[t])[1][-1])", "ys.append(_forward(W, q[t])[1][-1])"),
+    "dS_end dropped from J": ("(Se * torch.as_tensor(dS_end, dtype=torch.float64)).sum()", "0.0 * Se.sum()"),
+}
+
+
+def backward_battery():
+    c2, c4 = backward_pins.CASES[1], backward_pins.CASES[3]
+    return [
+        ("forward = C oracle (depth 2)", lambda: backward_pins.test_forward_restatement_equals_c_oracle(c2)),
+        ("forward = C oracle (depth 4)", lambda: backward_pins.test_forward_restatement_equals_c_oracle(c4)),
+        ("finite differences (depth 2)", lambda: backward_pins.test_gradients_equal_finite_differences_of_c_oracle(c2)),
+    ]
+
+
+def backward_failures(tmp_path, monkeypatch, old=None, new=None):
+    src = open(BW_SRC).read()
+    if old is not None:
+        assert src.count(old) == 1, old
+        src = src.replace(old, new)
+    path = tmp_path / "backward_variant.py"
+    path.write_text(src)
+    spec = importlib.util.spec_from_file_location("backward_variant", str(path))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    monkeypatch.setattr(backward_pins, "BW", mod)
+    failed = []
+    for name, pin in backward_battery():
+        try:
+            pin()
+        except (AssertionError, RuntimeError, ValueError):
+            failed.append(name)
+    return failed
+
+
+def test_unmodified_gradient_oracle_passes_the_battery(tmp_path, monkeypatch):
+    assert backward_failures(tmp_path, monkeypatch) == []
+
+
+@pytest.mark.parametrize("name", sorted(BW_MUTANTS))
+def test_planted_gradient_oracle_mistake_fails_a_pin(tmp_path, monkeypatch, name):
+    old, new = BW_MUTANTS[name]
+    assert backward_failures(tmp_path, monkeypatch, old, new), name
