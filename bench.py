@@ -517,9 +517,10 @@ def main():
         mem.run(d_in["k"], d_in["v"], d_in["q"], d_in["theta"], d_in["eta"], d_in["alpha"],
                 d_in["W0"], d_in["S0"], w.C, y=y, W_end=We, S_end=Se, workspace=ws, stream=stream)
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
+    with torch.cuda.nvtx.range("tm_run warm-up"):
+        for _ in range(args.warmup):
+            flush.zero_()
+            step()
     mem.sync(ws, stream)
     torch.cuda.synchronize()
     ok = bool(torch.isfinite(y).all() and torch.isfinite(We).all())
@@ -532,11 +533,12 @@ def main():
     barrier(world)
     torch.cuda.synchronize()
     t_wall = time.perf_counter()
-    for i in range(args.steps):
-        flush.zero_()  # L2 flush between steps, outside the timed events
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
+    with torch.cuda.nvtx.range("tm_run timed"):
+        for i in range(args.steps):
+            flush.zero_()  # L2 flush between steps, outside the timed events
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
     torch.cuda.synchronize()
     barrier(world)
     t_wall = time.perf_counter() - t_wall
@@ -584,19 +586,20 @@ def main():
         bi = sum(v.numel() * v.element_size() for v in pinned.values())
         bo = sum(v.numel() * v.element_size() for v in (h_y, h_W, h_S))
         e_ms = []
-        for i in range(max(2, min(args.steps, 3))):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for k2, v2 in pinned.items():
-                d_in[k2].copy_(v2, non_blocking=True)
-            step()
-            h_y.copy_(y, non_blocking=True)
-            h_W.copy_(We, non_blocking=True)
-            h_S.copy_(Se, non_blocking=True)
-            b.record(stream)
-            torch.cuda.synchronize()
-            e_ms.append(a.elapsed_time(b))
+        with torch.cuda.nvtx.range("tm_run end to end"):
+            for i in range(max(2, min(args.steps, 3))):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for k2, v2 in pinned.items():
+                    d_in[k2].copy_(v2, non_blocking=True)
+                step()
+                h_y.copy_(y, non_blocking=True)
+                h_W.copy_(We, non_blocking=True)
+                h_S.copy_(Se, non_blocking=True)
+                b.record(stream)
+                torch.cuda.synchronize()
+                e_ms.append(a.elapsed_time(b))
         e_ms_max = max_over_ranks(statistics.mean(e_ms), world)
         e2e = {"value": aggregate_throughput(cnt["tokens"], world, e_ms_max * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e_ms_max}
