@@ -465,6 +465,8 @@ def main():
                          "and print one JSON line per size instead of the benchmark line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--segment-tokens", type=int, default=0,
+                    help="tm_run_host segment length for the end-to-end leg (0 = library default)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -578,31 +580,44 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        # End to end through the public API: pinned host inputs -> device,
-        # tm_run, device -> host of the reads and the final state, every step.
+        # End to end through the public host-buffer API (tm_run_host): pinned
+        # host inputs in, the reads and the final state out, every step; the
+        # library copies segments of T in and out on side streams, overlapped
+        # with the kernels.
         h_y = torch.empty(y.shape, dtype=torch.float32, pin_memory=True)
         h_W = torch.empty(We.shape, dtype=torch.float32, pin_memory=True)
         h_S = torch.empty(Se.shape, dtype=torch.float32, pin_memory=True)
         bi = sum(v.numel() * v.element_size() for v in pinned.values())
         bo = sum(v.numel() * v.element_size() for v in (h_y, h_W, h_S))
+        seg = args.segment_tokens
+        del ws
+        hws = torch.empty(mem.host_workspace_size(w.B, w.H, w.T, w.C, d_in["k"].dtype, seg),
+                          dtype=torch.uint8, device=dev)
+
+        def e2e_step():
+            mem.run_host(pinned["k"], pinned["v"], pinned["q"], pinned["theta"], pinned["eta"],
+                         pinned["alpha"], pinned["W0"], pinned["S0"], w.C, y=h_y, W_end=h_W, S_end=h_S,
+                         workspace=hws, segment_tokens=seg, stream=stream, sync=False)
+
+        e2e_step()                       # warm-up (first use creates the copy streams)
+        torch.cuda.synchronize()
         e_ms = []
         with torch.cuda.nvtx.range("tm_run end to end"):
             for i in range(max(2, min(args.steps, 3))):
                 flush.zero_()
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(stream)
-                for k2, v2 in pinned.items():
-                    d_in[k2].copy_(v2, non_blocking=True)
-                step()
-                h_y.copy_(y, non_blocking=True)
-                h_W.copy_(We, non_blocking=True)
-                h_S.copy_(Se, non_blocking=True)
+                e2e_step()
                 b.record(stream)
                 torch.cuda.synchronize()
                 e_ms.append(a.elapsed_time(b))
+        mem.sync(hws, stream)
+        same = bool(torch.equal(h_y, y.cpu()) and torch.equal(h_W, We.cpu()) and torch.equal(h_S, Se.cpu()))
         e_ms_max = max_over_ranks(statistics.mean(e_ms), world)
         e2e = {"value": aggregate_throughput(cnt["tokens"], world, e_ms_max * 1e-3), "unit": "tokens/s",
-               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e_ms_max}
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e_ms_max,
+               "api": "tm_run_host", "segment_tokens": seg or "default (about T/8)",
+               "equal_to_device_run": same}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -619,7 +634,10 @@ def main():
                      ("bf16-in/f32" if w.dtype == "bf16" else "f32"),
             "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "C": w.C, "dims": w.dims,
-                       "theta_damping": w.theta_damping, "alpha_damping": w.alpha_damping, "path": path_used,
+                       "theta_damping": w.theta_damping, "alpha_damping": w.alpha_damping,
+                       "gates": ("literal" if (w.theta_damping == 1.0 and w.alpha_damping == 1.0) else
+                                 f"damped: theta draws x{w.theta_damping}, alpha draws x{w.alpha_damping}"),
+                       "path": path_used,
                        "l2": "flushed between steps (512 MB write)", "parallelism": f"replicas{world}"},
             "roofline": roof,
             "chunk_roofline": {"t_flop_ms": t_flop * 1e3, "t_state_io_ms": t_state * 1e3,

@@ -183,8 +183,10 @@ TM_API tm_status tm_run(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dty
  * 16 MiB of activations are refused with TM_ERR_OOM before any CUDA call.
  * Allocates nothing and calls no allocating routine.
  *
- * The first call on each device looks up the array's device address; make
- * that first call before any stream capture. All calls on a device share the
+ * The first call on each device looks up the array's device address (again
+ * after the device's context has been reset, e.g. by cudaDeviceReset, which
+ * may move the array); make that first call before any stream capture. All
+ * calls on a device share the
  * array (it keeps the last call's contents; every call clears its status
  * word): calls whose kernels overlap on the GPU race and must be serialised
  * by the caller. Device-side errors are not reported through tm_sync (there
@@ -195,6 +197,45 @@ TM_API tm_status tm_run_noalloc(tm_ctx *ctx, int B, int H, int T, int C, tm_dtyp
                                 const float *theta, const float *eta, const float *alpha,
                                 const float *W0, const float *S0,
                                 float *y, float *W_end, float *S_end, void *stream);
+
+/*
+ * The write-and-read with every input and output in HOST memory: the same
+ * operation and results as tm_run (bit for bit: the state is carried on the
+ * device between segments, and carrying the state equals one longer call,
+ * "titans-pytorch" review, "NeuralMemory as a standalone module"), with the
+ * host <-> device copies inside the call and overlapped with the kernels.
+ *
+ * T is walked in segments of `segment_tokens` tokens per stream (0 = about
+ * T / 8, rounded up to whole chunks; otherwise a multiple of C, or >= T);
+ * the last segment takes the rest. While the kernels run segment i, the
+ * inputs of segment i + 1 are copied in on one side stream and the reads y
+ * of segment i - 1 copied out on another (one cudaMemcpy2DAsync per tensor
+ * and segment). W0/S0 go in before the first segment, W_end/S_end come out
+ * after the last.
+ *
+ *   k, v, q, theta, eta, alpha, W0, S0   host memory, layouts as for tm_run
+ *   y, W_end, S_end                       host memory, outputs
+ *   workspace: device buffer of at least tm_host_workspace_size() bytes,
+ *              256-byte aligned (tm_run's workspace for one segment, the
+ *              carried state and two sets of segment buffers).
+ *
+ * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister) for
+ * the copies to overlap the kernels; pageable memory gives the same results
+ * without the overlap. Aliasing rules as for tm_run (W_end may equal W0, S_end
+ * S0). Asynchronous: the outputs are complete once `stream` has reached the
+ * point of the call (cudaStreamSynchronize or an event); the inputs must stay
+ * unchanged until then. Errors as for tm_run; tm_sync(ctx, workspace, stream)
+ * reports device-side errors of all segments. The context's calls must not run
+ * concurrently.
+ */
+TM_API tm_status tm_host_workspace_size(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype,
+                                        int segment_tokens, size_t *bytes);
+TM_API tm_status tm_run_host(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype,
+                             const void *k, const void *v, const void *q,
+                             const float *theta, const float *eta, const float *alpha,
+                             const float *W0, const float *S0,
+                             float *y, float *W_end, float *S_end,
+                             int segment_tokens, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Wait for `stream`, then read and clear the device status word in
@@ -287,11 +328,12 @@ TM_API tm_status tm_prologue(int B, int H, int T, int d, int width, tm_dtype in_
 
 /*
  * Test hook for failure handling (process-wide, host-only). inject_timeout != 0
- * makes every CTA of the tensor-core kernel first wait on a barrier that
- * nothing completes, so the bounded wait expires, the kernel records
- * TM_ERR_TIMEOUT, cleans up and returns; tm_sync() then reports it.
- * wait_limit_ns sets the time limit of each device-side wait (0 = default 2 s).
- * Affects launches issued after the call.
+ * makes every CTA of the tensor-core kernels (the cluster walker and the
+ * layered forward/backward, per-phase and update kernels) first wait on a
+ * barrier that nothing completes, so the bounded wait expires, the kernel
+ * records TM_ERR_TIMEOUT, issues nothing further, cleans up and returns;
+ * tm_sync() then reports it. wait_limit_ns sets the time limit of each
+ * device-side wait (0 = default 2 s). Affects launches issued after the call.
  */
 TM_API tm_status tm_set_debug(int inject_timeout, unsigned long long wait_limit_ns);
 

@@ -30,6 +30,8 @@ SIGNATURES = {
     "tm_workspace_size": (_I, [_P, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]),
     "tm_run": (_I, [_P, _I, _I, _I, _I, _I] + [_P] * 11 + [_P, _SZ, _P]),
     "tm_run_noalloc": (_I, [_P, _I, _I, _I, _I, _I] + [_P] * 11 + [_P]),
+    "tm_host_workspace_size": (_I, [_P, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]),
+    "tm_run_host": (_I, [_P, _I, _I, _I, _I, _I] + [_P] * 11 + [_I, _P, _SZ, _P]),
     "tm_sync": (_I, [_P, _P, _P]),
     "tm_set_debug": (_I, [_I, ctypes.c_ulonglong]),
     "tm_prologue": (_I, [_I, _I, _I, _I, _I, _I] + [_P] * 12 + [_P]),

@@ -34,6 +34,13 @@ struct tm_ctx {
   bool has_seen = false;
   cudaStream_t cap = nullptr;
   cudaGraphExec_t exec = nullptr;
+  // tm_run_host: copy streams (host -> device, device -> host) and the
+  // events that order them against the kernels, created on first use on
+  // device `hdev`
+  int hdev = -1;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t h_start = nullptr, h_done = nullptr, h_state = nullptr;
+  cudaEvent_t in_ready[2] = {}, in_free[2] = {}, y_ready[2] = {}, y_free[2] = {};
 };
 
 namespace {
@@ -116,6 +123,36 @@ bool problem_from_ctx(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype dt
   *out = make_problem(ctx, B, H, T, C, dt);
   return true;
 }
+
+bool run_aliasing_ok(const Problem &p, const void *k, const void *v, const void *q, const float *theta,
+                     const float *eta, const float *alpha, const float *W0, const float *S0, const float *y,
+                     const float *W_end, const float *S_end) {
+  const size_t tok_el = p.in_dtype == TM_BF16 ? 2 : 4;
+  const size_t ntok = (size_t)p.streams * (size_t)p.T;
+  const size_t d = (size_t)p.dims[0];
+  const size_t tok_bytes = ntok * d * tok_el;
+  const size_t y_bytes = ntok * d * 4;
+  const size_t gate_bytes = ntok * 4;
+  const size_t st_bytes = (size_t)p.streams * p.P * 4;
+  // y must not overlap any input or other output.
+  const void *ins[] = {k, v, q, theta, eta, alpha, W0, S0, W_end, S_end};
+  const size_t insz[] = {tok_bytes, tok_bytes, tok_bytes, gate_bytes, gate_bytes, gate_bytes,
+                         st_bytes, st_bytes, st_bytes, st_bytes};
+  for (int i = 0; i < 10; ++i)
+    if (ranges_overlap(y, y_bytes, ins[i], insz[i])) return false;
+  // W_end may equal W0 exactly (in place) but not partially overlap anything else.
+  if (W_end != W0 && ranges_overlap(W_end, st_bytes, W0, st_bytes)) return false;
+  if (S_end != S0 && ranges_overlap(S_end, st_bytes, S0, st_bytes)) return false;
+  if (ranges_overlap(W_end, st_bytes, S_end, st_bytes)) return false;
+  if (ranges_overlap(W_end, st_bytes, S0, st_bytes)) return false;
+  if (ranges_overlap(S_end, st_bytes, W0, st_bytes)) return false;
+  // the state outputs must not overlap the token inputs or the gates
+  const void *tin[] = {k, v, q, theta, eta, alpha};
+  for (int i = 0; i < 6; ++i)
+    if (ranges_overlap(W_end, st_bytes, tin[i], insz[i]) || ranges_overlap(S_end, st_bytes, tin[i], insz[i]))
+      return false;
+  return true;
+}
 }  // namespace tmem
 
 extern "C" {
@@ -151,6 +188,38 @@ namespace {
 void drop_graph(tm_ctx *ctx) {
   if (ctx->exec) cudaGraphExecDestroy(ctx->exec);
   ctx->exec = nullptr;
+}
+
+void release_host(tm_ctx *ctx) {
+  cudaStream_t st[] = {ctx->h2d, ctx->d2h};
+  for (cudaStream_t x : st)
+    if (x) cudaStreamDestroy(x);
+  ctx->h2d = ctx->d2h = nullptr;
+  cudaEvent_t *evs[] = {&ctx->h_start, &ctx->h_done, &ctx->h_state, &ctx->in_ready[0], &ctx->in_ready[1],
+                        &ctx->in_free[0], &ctx->in_free[1], &ctx->y_ready[0], &ctx->y_ready[1],
+                        &ctx->y_free[0], &ctx->y_free[1]};
+  for (cudaEvent_t *e : evs) {
+    if (*e) cudaEventDestroy(*e);
+    *e = nullptr;
+  }
+  ctx->hdev = -1;
+}
+
+// Copy streams and events of tm_run_host on the current device.
+bool ensure_host(tm_ctx *ctx) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (ctx->hdev != dev) release_host(ctx);
+  ctx->hdev = dev;
+  cudaStream_t *st[] = {&ctx->h2d, &ctx->d2h};
+  for (cudaStream_t *x : st)
+    if (!*x && cudaStreamCreateWithFlags(x, cudaStreamNonBlocking) != cudaSuccess) return false;
+  cudaEvent_t *evs[] = {&ctx->h_start, &ctx->h_done, &ctx->h_state, &ctx->in_ready[0], &ctx->in_ready[1],
+                        &ctx->in_free[0], &ctx->in_free[1], &ctx->y_ready[0], &ctx->y_ready[1],
+                        &ctx->y_free[0], &ctx->y_free[1]};
+  for (cudaEvent_t *e : evs)
+    if (!*e && cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
+  return true;
 }
 
 void release_side(tm_ctx *ctx) {
@@ -192,7 +261,7 @@ tm_ctx::Key run_key(const tm_ctx *ctx, tm_path path, const tmem::Problem &p) {
   std::memset(&k, 0, sizeof k);
   const unsigned long long w = tmem::tcl_wait_ns();
   const int v[] = {(int)path, p.B, p.H, p.T, p.C, (int)p.in_dtype, tmem::tcl_group_count(p), ctx->dev,
-                   (int)(w & 0x7fffffff), (int)(w >> 31), p.T_run, 0};
+                   (int)(w & 0x7fffffff), (int)(w >> 31), p.T_run, tmem::tcl_inject()};
   std::memcpy(k.v, v, sizeof v);
   const void *ptr[] = {p.k, p.v, p.q, p.theta, p.eta, p.alpha, p.W0, p.S0, p.y, p.W_end, p.S_end, p.scratch};
   std::memcpy(k.ptr, ptr, sizeof ptr);
@@ -249,7 +318,10 @@ cudaError_t run_layered(tm_ctx *ctx, tm_path path, const tmem::Problem &p, cudaS
 }  // namespace
 
 tm_status tm_destroy(tm_ctx *ctx) {
-  if (ctx) release_side(ctx);
+  if (ctx) {
+    release_side(ctx);
+    release_host(ctx);
+  }
   delete ctx;
   return TM_OK;
 }
@@ -309,10 +381,16 @@ tm_status tm_workspace_size(const tm_ctx *ctx, int B, int H, int T, int C, tm_dt
   return TM_OK;
 }
 
-tm_status tm_run(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype, const void *k,
-                 const void *v, const void *q, const float *theta, const float *eta,
-                 const float *alpha, const float *W0, const float *S0, float *y, float *W_end,
-                 float *S_end, void *workspace, size_t workspace_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// tm_run's work; clear_status = false keeps the device status word as it is
+// (tm_run_host clears it once for all of its segments).
+tm_status run_device(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype, const void *k,
+                     const void *v, const void *q, const float *theta, const float *eta,
+                     const float *alpha, const float *W0, const float *S0, float *y, float *W_end,
+                     float *S_end, void *workspace, size_t workspace_bytes, void *stream, bool clear_status) {
   tm_status st = check_shape(ctx, B, H, T, C, in_dtype);
   if (st != TM_OK) return st;
   const void *ptrs[] = {k, v, q, theta, eta, alpha, W0, S0, y, W_end, S_end, workspace};
@@ -321,24 +399,9 @@ tm_status tm_run(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype, con
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TM_ERR_INVALID_ARG;
 
   tmem::Problem p = make_problem(ctx, B, H, T, C, in_dtype);
-  const size_t tok_el = in_dtype == TM_BF16 ? 2 : 4;
-  const size_t ntok = (size_t)p.streams * (size_t)T;
-  const size_t tok_bytes = ntok * (size_t)ctx->d * tok_el;
-  const size_t y_bytes = ntok * (size_t)ctx->d * 4;
-  const size_t gate_bytes = ntok * 4;
-  const size_t st_bytes = (size_t)p.streams * ctx->P * 4;
-  // y must not overlap any input or other output.
-  const void *ins[] = {k, v, q, theta, eta, alpha, W0, S0, W_end, S_end};
-  const size_t insz[] = {tok_bytes, tok_bytes, tok_bytes, gate_bytes, gate_bytes, gate_bytes,
-                         st_bytes, st_bytes, st_bytes, st_bytes};
-  for (int i = 0; i < 10; ++i)
-    if (ranges_overlap(y, y_bytes, ins[i], insz[i])) return TM_ERR_INVALID_ARG;
-  // W_end may equal W0 exactly (in place) but not partially overlap anything else.
-  if (W_end != W0 && ranges_overlap(W_end, st_bytes, W0, st_bytes)) return TM_ERR_INVALID_ARG;
-  if (S_end != S0 && ranges_overlap(S_end, st_bytes, S0, st_bytes)) return TM_ERR_INVALID_ARG;
-  if (ranges_overlap(W_end, st_bytes, S_end, st_bytes)) return TM_ERR_INVALID_ARG;
-  if (ranges_overlap(W_end, st_bytes, S0, st_bytes)) return TM_ERR_INVALID_ARG;
-  if (ranges_overlap(S_end, st_bytes, W0, st_bytes)) return TM_ERR_INVALID_ARG;
+  const size_t y_bytes = (size_t)p.streams * (size_t)T * (size_t)ctx->d * 4;
+  if (!tmem::run_aliasing_ok(p, k, v, q, theta, eta, alpha, W0, S0, y, W_end, S_end))
+    return TM_ERR_INVALID_ARG;
 
   tm_path path = choose_path(ctx, p);
   if (!path_supported(path, p)) return TM_ERR_UNSUPPORTED;
@@ -362,7 +425,7 @@ tm_status tm_run(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype, con
   p.scratch_bytes = workspace_bytes - tmem::kStatusBytes;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(p.status, 0, sizeof(int), s) != cudaSuccess) return TM_ERR_CUDA;
+  if (clear_status && cudaMemsetAsync(p.status, 0, sizeof(int), s) != cudaSuccess) return TM_ERR_CUDA;
   p.fuse_fb = path == TM_PATH_TC_LAYERED;
   if (path == TM_PATH_TC_LAYERED || path == TM_PATH_TC_PHASED) {
     const int groups = tmem::tcl_group_count(p);
@@ -394,6 +457,185 @@ tm_status tm_run(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype, con
     }
   }
   return err == cudaSuccess ? TM_OK : TM_ERR_CUDA;
+}
+
+size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Segment length of tm_run_host: the caller's, or about an eighth of T
+// rounded up to whole chunks.
+int host_segment(int T, int C, int segment_tokens) {
+  if (segment_tokens > 0) return segment_tokens < T ? segment_tokens : T;
+  const int n = (T + 7) / 8;
+  const int seg = (n + C - 1) / C * C;
+  return seg < T ? seg : T;
+}
+
+// Device workspace of tm_run_host: tm_run's workspace for one segment first
+// (so that its status word sits at the start), then the carried state and
+// two sets of segment buffers.
+struct HostCarve {
+  size_t run, run_bytes, W, S, buf[2], k, v, q, th, et, al, y, total;
+};
+
+tm_status host_carve(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype dt, int seg, HostCarve *c) {
+  const int last = T - (T - 1) / seg * seg;    // tokens of the last segment
+  size_t ws = 0;
+  const int lens[2] = {seg, last};
+  for (int t : lens) {
+    size_t b = 0;
+    const tm_status st = tm_workspace_size(ctx, B, H, t, C, dt, &b);
+    if (st != TM_OK) return st;
+    if (b > ws) ws = b;
+  }
+  const size_t S = (size_t)B * H, d = (size_t)ctx->d, el = dt == TM_BF16 ? 2 : 4, ts = (size_t)seg;
+  std::memset(c, 0, sizeof *c);
+  size_t off = 0;
+  c->run = off;
+  c->run_bytes = up256(ws);
+  off += c->run_bytes;
+  c->W = off;
+  off += up256(S * ctx->P * 4);
+  c->S = off;
+  off += up256(S * ctx->P * 4);
+  // offsets inside one set of segment buffers
+  size_t o = 0;
+  c->k = o; o += up256(S * ts * d * el);
+  c->v = o; o += up256(S * ts * d * el);
+  c->q = o; o += up256(S * ts * d * el);
+  c->th = o; o += up256(S * ts * 4);
+  c->et = o; o += up256(S * ts * 4);
+  c->al = o; o += up256(S * ts * 4);
+  c->y = o; o += up256(S * ts * d * 4);
+  c->buf[0] = off;
+  c->buf[1] = off + o;
+  c->total = off + 2 * o;
+  return TM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+tm_status tm_run(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype, const void *k,
+                 const void *v, const void *q, const float *theta, const float *eta,
+                 const float *alpha, const float *W0, const float *S0, float *y, float *W_end,
+                 float *S_end, void *workspace, size_t workspace_bytes, void *stream) {
+  return run_device(ctx, B, H, T, C, in_dtype, k, v, q, theta, eta, alpha, W0, S0, y, W_end, S_end, workspace,
+                    workspace_bytes, stream, true);
+}
+
+tm_status tm_host_workspace_size(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype,
+                                 int segment_tokens, size_t *bytes) {
+  if (!bytes || segment_tokens < 0) return TM_ERR_INVALID_ARG;
+  tm_status st = check_shape(ctx, B, H, T, C, in_dtype);
+  if (st != TM_OK) return st;
+  const int seg = host_segment(T, C, segment_tokens);
+  if (seg < T && seg % C != 0) return TM_ERR_INVALID_ARG;
+  HostCarve c;
+  st = host_carve(ctx, B, H, T, C, in_dtype, seg, &c);
+  if (st != TM_OK) return st;
+  *bytes = c.total;
+  return TM_OK;
+}
+
+tm_status tm_run_host(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype, const void *k,
+                      const void *v, const void *q, const float *theta, const float *eta,
+                      const float *alpha, const float *W0, const float *S0, float *y, float *W_end,
+                      float *S_end, int segment_tokens, void *workspace, size_t workspace_bytes,
+                      void *stream) {
+  tm_status st = check_shape(ctx, B, H, T, C, in_dtype);
+  if (st != TM_OK) return st;
+  if (segment_tokens < 0) return TM_ERR_INVALID_ARG;
+  const void *ptrs[] = {k, v, q, theta, eta, alpha, W0, S0, y, W_end, S_end, workspace};
+  for (const void *x : ptrs)
+    if (!x) return TM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TM_ERR_INVALID_ARG;
+  const tmem::Problem p = make_problem(ctx, B, H, T, C, in_dtype);
+  if (!tmem::run_aliasing_ok(p, k, v, q, theta, eta, alpha, W0, S0, y, W_end, S_end)) return TM_ERR_INVALID_ARG;
+  const int seg = host_segment(T, C, segment_tokens);
+  if (seg < T && seg % C != 0) return TM_ERR_INVALID_ARG;
+  HostCarve c;
+  st = host_carve(ctx, B, H, T, C, in_dtype, seg, &c);
+  if (st != TM_OK) return st;
+  if (workspace_bytes < c.total) return TM_ERR_OOM;
+  {
+    // every segment's path must be one tm_run supports
+    tm_path path;
+    const int last = T - (T - 1) / seg * seg;
+    if (tm_query_path(ctx, B, H, seg, C, in_dtype, &path) != TM_OK ||
+        tm_query_path(ctx, B, H, last, C, in_dtype, &path) != TM_OK)
+      return TM_ERR_UNSUPPORTED;
+  }
+  if (!ensure_host(ctx)) return TM_ERR_CUDA;
+
+  unsigned char *ws = static_cast<unsigned char *>(workspace);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t S = (size_t)p.streams, d = (size_t)ctx->d, el = in_dtype == TM_BF16 ? 2 : 4;
+  const size_t st_bytes = S * ctx->P * 4;
+  float *dW = reinterpret_cast<float *>(ws + c.W), *dS = reinterpret_cast<float *>(ws + c.S);
+  const int nseg = (T + seg - 1) / seg;
+  auto seg_len = [&](int i) { return i + 1 < nseg ? seg : T - i * seg; };
+  // One strided copy per tensor and segment: the segment's rows of every
+  // stream, [S rows] x [n tokens x width] bytes.
+  auto copy_in = [&](int i) -> cudaError_t {
+    unsigned char *b = ws + c.buf[i & 1];
+    const size_t t0 = (size_t)i * seg, n = (size_t)seg_len(i);
+    const void *src[6] = {k, v, q, theta, eta, alpha};
+    const size_t off[6] = {c.k, c.v, c.q, c.th, c.et, c.al};
+    const size_t w[6] = {d * el, d * el, d * el, 4, 4, 4};
+    for (int j = 0; j < 6; ++j) {
+      const cudaError_t e = cudaMemcpy2DAsync(b + off[j], n * w[j], static_cast<const unsigned char *>(src[j]) + t0 * w[j],
+                                              (size_t)T * w[j], n * w[j], S, cudaMemcpyHostToDevice, ctx->h2d);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  };
+  cudaError_t e = cudaEventRecord(ctx->h_start, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(ctx->h2d, ctx->h_start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(ctx->d2h, ctx->h_start, 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dW, W0, st_bytes, cudaMemcpyHostToDevice, ctx->h2d);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dS, S0, st_bytes, cudaMemcpyHostToDevice, ctx->h2d);
+  if (e == cudaSuccess) e = copy_in(0);
+  if (e == cudaSuccess) e = cudaEventRecord(ctx->in_ready[0], ctx->h2d);
+  st = e == cudaSuccess ? TM_OK : TM_ERR_CUDA;
+  for (int i = 0; i < nseg && st == TM_OK; ++i) {
+    const int b = i & 1, n = seg_len(i);
+    unsigned char *bb = ws + c.buf[b];
+    if (i + 1 < nseg) {
+      // the next segment's inputs land while this one runs (its buffer was
+      // last read by segment i - 1)
+      e = cudaStreamWaitEvent(ctx->h2d, ctx->in_free[(i + 1) & 1], 0);
+      if (e == cudaSuccess) e = copy_in(i + 1);
+      if (e == cudaSuccess) e = cudaEventRecord(ctx->in_ready[(i + 1) & 1], ctx->h2d);
+    }
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ctx->in_ready[b], 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ctx->y_free[b], 0);   // y buffer read out (segment i - 2)
+    if (e != cudaSuccess) { st = TM_ERR_CUDA; break; }
+    float *yb = reinterpret_cast<float *>(bb + c.y);
+    st = run_device(ctx, B, H, n, C, in_dtype, bb + c.k, bb + c.v, bb + c.q, reinterpret_cast<float *>(bb + c.th),
+                    reinterpret_cast<float *>(bb + c.et), reinterpret_cast<float *>(bb + c.al), dW, dS, yb, dW, dS,
+                    ws + c.run, c.run_bytes, s, i == 0);
+    if (st != TM_OK) break;
+    e = cudaEventRecord(ctx->in_free[b], s);
+    if (e == cudaSuccess) e = cudaEventRecord(ctx->y_ready[b], s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ctx->d2h, ctx->y_ready[b], 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(y + (size_t)i * seg * d, (size_t)T * d * 4, yb, (size_t)n * d * 4, (size_t)n * d * 4, S,
+                            cudaMemcpyDeviceToHost, ctx->d2h);
+    if (e == cudaSuccess) e = cudaEventRecord(ctx->y_free[b], ctx->d2h);
+    if (e != cudaSuccess) st = TM_ERR_CUDA;
+  }
+  if (st == TM_OK) {
+    e = cudaEventRecord(ctx->h_state, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ctx->d2h, ctx->h_state, 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(W_end, dW, st_bytes, cudaMemcpyDeviceToHost, ctx->d2h);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(S_end, dS, st_bytes, cudaMemcpyDeviceToHost, ctx->d2h);
+    if (e != cudaSuccess) st = TM_ERR_CUDA;
+  }
+  // join both copy streams into the caller's stream, also after an error
+  if (cudaEventRecord(ctx->h_done, ctx->d2h) == cudaSuccess) cudaStreamWaitEvent(s, ctx->h_done, 0);
+  if (cudaEventRecord(ctx->h_state, ctx->h2d) == cudaSuccess) cudaStreamWaitEvent(s, ctx->h_state, 0);
+  return st;
 }
 
 tm_status tm_sync(tm_ctx *ctx, void *workspace, void *stream) {
@@ -522,7 +764,7 @@ tm_status tm_prologue(int B, int H, int T, int d, int width, tm_dtype in_dtype, 
 
 tm_status tm_set_debug(int inject_timeout, unsigned long long wait_limit_ns) {
   tmem::tc_set_debug(inject_timeout, wait_limit_ns);
-  tmem::tcl_set_wait(wait_limit_ns);
+  tmem::tcl_set_debug(inject_timeout, wait_limit_ns);
   return TM_OK;
 }
 

@@ -49,6 +49,12 @@ struct Problem {
 
 // Shape checks of tm_run, shared with the other C entry points.
 bool problem_from_ctx(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype dt, Problem *out);
+// Aliasing rules of tm_run's buffers for problem p (shapes filled in): y
+// overlaps no input or other output; W_end / S_end equal W0 / S0 exactly or
+// overlap nothing else. False if a rule is broken.
+bool run_aliasing_ok(const Problem &p, const void *k, const void *v, const void *q, const float *theta,
+                     const float *eta, const float *alpha, const float *W0, const float *S0, const float *y,
+                     const float *W_end, const float *S_end);
 
 // SIMT (CUDA-core, fp32) path.
 size_t simt_scratch_bytes(const Problem &p);
@@ -65,8 +71,10 @@ size_t tcl_scratch_bytes(const Problem &p);
 cudaError_t tcl_launch(const Problem &p, cudaStream_t stream);
 int tcl_group_count(const Problem &p);   // CUDA streams tcl_launch uses
 long long tcl_launch_count(const Problem &p);
-void tcl_set_wait(unsigned long long wait_ns);
+// Test hooks of the layered kernels, as tc_set_debug below.
+void tcl_set_debug(int inject_timeout, unsigned long long wait_ns);
 unsigned long long tcl_wait_ns();
+int tcl_inject();
 
 // Gradients of the memory layer (depths 1 to 4) with respect to its inputs.
 bool backward_supported(const Problem &p);

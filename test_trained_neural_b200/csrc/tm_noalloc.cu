@@ -19,6 +19,8 @@
 // caller.
 #include <mutex>
 
+#include <cuda.h>
+
 #include "tm_internal.h"
 
 namespace {
@@ -28,22 +30,62 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[tmem::kStatusBytes + kScratchMax];
 
-// Device address of g_noalloc_scratch per device. In host code the symbol
-// itself is only a host-side stand-in; the address comes from
-// cudaGetSymbolAddress with that device current.
-void *g_scratch_dev[kMaxDevices] = {};
+// Device address of g_noalloc_scratch per device, and the id of the CUDA
+// context it was looked up in. In host code the symbol itself is only a
+// host-side stand-in; the address comes from cudaGetSymbolAddress with that
+// device current. A context created after a reset of the device (for
+// example cudaDeviceReset) loads the module afresh and the array may move,
+// so the address is looked up again whenever the current context's id
+// differs from the one recorded.
+struct ScratchAddr {
+  void *ptr = nullptr;
+  unsigned long long ctx_id = 0;
+};
+ScratchAddr g_scratch_dev[kMaxDevices];
 std::mutex g_scratch_mu;
+
+// Id of the CUDA context current on this thread; 0 if none is current yet.
+// The two driver functions are resolved through the runtime, so that the
+// library loads on machines without the driver library.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (!get_current || !get_id) {
+    void *a = nullptr, *b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) != cudaSuccess ||
+        qa != cudaDriverEntryPointSuccess ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) != cudaSuccess ||
+        qb != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+    get_id = reinterpret_cast<CtxGetIdFn>(b);
+  }
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 tm_status scratch_address(void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TM_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_dev[dev]) {
+  ScratchAddr &e = g_scratch_dev[dev];
+  const unsigned long long id = current_ctx_id();
+  if (!e.ptr || id == 0 || id != e.ctx_id) {
+    // set-up for this device (and context): cudaGetSymbolAddress also makes
+    // the device's primary context current when no context is yet
     void *ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return TM_ERR_CUDA;
-    g_scratch_dev[dev] = ptr;
+    e.ptr = ptr;
+    e.ctx_id = current_ctx_id();
   }
-  *out = g_scratch_dev[dev];
+  *out = e.ptr;
   return TM_OK;
 }
 
@@ -66,6 +108,8 @@ tm_status tm_run_noalloc(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dt
   // any CUDA call.
   const size_t need = tmem::simt_scratch_bytes(p);
   if (need > kScratchMax) return TM_ERR_OOM;
+  // the same aliasing rules as tm_run
+  if (!tmem::run_aliasing_ok(p, k, v, q, theta, eta, alpha, W0, S0, y, W_end, S_end)) return TM_ERR_INVALID_ARG;
   void *base = nullptr;
   tm_status st = scratch_address(&base);
   if (st != TM_OK) return st;

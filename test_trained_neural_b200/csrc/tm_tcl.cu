@@ -56,6 +56,7 @@ struct GemmArgs {
   const float *coef;             // [streams, T, 2] (c, e) per token
   int *status;
   unsigned long long wait_ns;
+  int inject;                    // test hook: every CTA's first wait is one that nothing completes
 };
 
 __device__ __forceinline__ float tanh_approx(float x) {
@@ -77,6 +78,16 @@ __device__ __forceinline__ uint4 pack8(const float *v) {
 __device__ bool wait_b(uint64_t *bar, uint32_t par, const GemmArgs &a) {
   if (mbar_wait(bar, par, a.wait_ns)) return true;
   atomicCAS(a.status, 0, kDevTimeout);
+  return false;
+}
+
+// Test hook of failure handling: a wait on a barrier that nothing ever
+// completes. It runs out after the wait limit and is recorded like any other
+// expired wait; the caller then issues nothing and leaves through its abort
+// path. Returns false (the wait did not succeed).
+__device__ bool injected_wait(uint64_t *never, int *status, unsigned long long wait_ns) {
+  if (mbar_wait(never, 0, wait_ns)) return true;
+  atomicCAS(status, 0, kDevTimeout);
   return false;
 }
 
@@ -125,7 +136,7 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *sm =
       reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t full[STAGES_MAX], empty[STAGES_MAX], done;
+  __shared__ uint64_t full[STAGES_MAX], empty[STAGES_MAX], done, never;
   __shared__ uint32_t tslot;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   constexpr int kind = KIND;
@@ -137,6 +148,7 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
   if (tid == 0) {
     for (int i = 0; i < STAGES_MAX; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     mbar_init(&done, 1);
+    mbar_init(&never, 1);
     fence_barrier_init();
   }
   if (warp == 0) { tmem_alloc(&tslot, ncols); tmem_relinquish(); }
@@ -150,11 +162,12 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (tid == 0) {
+    if (a.inject) ok = injected_wait(&never, a.status, a.wait_ns);
     const uint32_t tx = (uint32_t)(A_BYTES + (uint32_t)a.N * KB * 2);
     uint32_t idesc;
     if (kind == K_BWD) idesc = idesc_bf16(128, a.N, false, true);
     else idesc = idesc_bf16(128, a.N, false, false);
-    for (int kb = 0; kb < nk && kb < STAGES; ++kb) {
+    for (int kb = 0; kb < nk && kb < STAGES && ok; ++kb) {
       mbar_arrive_expect_tx(&full[kb], tx);
       load_stage(a, &mA, &mA2, &mB, sm + kb * STAGE_BYTES, &full[kb], s, mt, nt, kb);
     }
@@ -189,6 +202,7 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
   // ------------------------------------------------------------ epilogue
   if (!mbar_wait(&done, 0, a.wait_ns)) { atomicCAS(a.status, 0, kDevTimeout); ok = false; }
   tc_fence_after();
+  ok = __syncthreads_and(ok) != 0;               // an expired wait anywhere skips the epilogue
   const int row = 32 * (warp & 3) + lane;        // TMEM lane = output row of the tile
   const uint32_t lb = (uint32_t)(32 * (warp & 3)) << 16;
   const int half = warp >> 2;                    // this warp's half of the tile's columns
@@ -312,6 +326,7 @@ struct UpArgs {
   const float *scal;                           // [streams, nchunks, 4] (B, A, c_S, -)
   int *status;
   unsigned long long wait_ns;
+  int inject;                                  // test hook, as in GemmArgs
 };
 struct UpMaps {
   CUtensorMap a[kMaxL], a2[kMaxL], b[kMaxL];   // -c G_l, -e G_l [S*C, d_l]; X_{l-1} (bf16, 64 x 64 boxes)
@@ -338,7 +353,7 @@ __global__ void __launch_bounds__(UP_NT, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *sm =
       reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t full[3], empty[3], done, stb;
+  __shared__ uint64_t full[3], empty[3], done, stb, never;
   __shared__ uint32_t tslot;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int t = blockIdx.x;
@@ -359,6 +374,7 @@ __global__ void __launch_bounds__(UP_NT, 1)
     for (int k = 0; k < 3; ++k) { mbar_init(&full[k], 1); mbar_init(&empty[k], 1); }
     mbar_init(&done, 1);
     mbar_init(&stb, 1);
+    mbar_init(&never, 1);
     fence_barrier_init();
   }
   if (warp == 0) { tmem_alloc(&tslot, 256); tmem_relinquish(); }
@@ -368,10 +384,15 @@ __global__ void __launch_bounds__(UP_NT, 1)
   const uint32_t tm = tslot;
   bool ok = true;
   if (tid == 0) {
-    mbar_arrive_expect_tx(&stb, 2u * (uint32_t)(N / 32) * (uint32_t)R * 128u);
-    for (int b = 0; b < N / 32; ++b) {
-      tma_load_3d(wt + b * UP_BOX, &m.w[l], &stb, N * nt + 32 * b, 128 * mt, s);
-      tma_load_3d(st + b * UP_BOX, &m.s[l], &stb, N * nt + 32 * b, 128 * mt, s);
+    if (a.inject) ok = injected_wait(&never, a.status, a.wait_ns);
+    if (ok) {
+      mbar_arrive_expect_tx(&stb, 2u * (uint32_t)(N / 32) * (uint32_t)R * 128u);
+      for (int b = 0; b < N / 32; ++b) {
+        tma_load_3d(wt + b * UP_BOX, &m.w[l], &stb, N * nt + 32 * b, 128 * mt, s);
+        tma_load_3d(st + b * UP_BOX, &m.s[l], &stb, N * nt + 32 * b, 128 * mt, s);
+      }
+    } else {
+      mbar_arrive(&stb);                       // nothing issued: release the state-tile waiters
     }
   }
   // the operands are the preceding kernel's outputs
@@ -390,7 +411,7 @@ __global__ void __launch_bounds__(UP_NT, 1)
       for (int f = 0; f < N / 64; ++f)
         tma_load_2d(d + 2 * A_BYTES + f * 64 * 128, &m.b[l], &full[stg], N * nt + 64 * f, brow0);
     };
-    for (int kb = 0; kb < nk && kb < STAGES; ++kb) {
+    for (int kb = 0; kb < nk && kb < STAGES && ok; ++kb) {
       mbar_arrive_expect_tx(&full[kb], SB);
       load(kb, kb);
       ++issued;
@@ -482,6 +503,269 @@ __global__ void __launch_bounds__(UP_NT, 1)
 }
 
 // ------------------------------------------------------------------------
+// The state update of every layer of a chunk, pipelined (chunks of at most 128
+// tokens). One CTA per unit = (layer l, stream, block of 128 rows of W_l, a
+// range of up to `tpu` 64-column tiles). The contraction's A operands, -c G
+// and -e G of the block's rows over the whole chunk (K = C), are loaded once;
+// the column tiles then stream through two shared-memory stages (X columns
+// and the fp32 W and S tiles) and two TMEM accumulator pairs (U_W | U_S), so
+// that tile j + 1's loads and MMAs overlap tile j's update and stores:
+//   warp 0      TMA loads (state tiles first: they do not depend on the
+//               previous kernel; the operands after griddepcontrol.wait)
+//   warp 1      TMEM allocation; MMA issue (M = 128 rows, N = 64, K = C)
+//   warp 2      TMA stores of W', S' and the bf16 W' of a tile, then frees
+//               the stage once the stores have read it
+//   warps 4-11  epilogue: the thread owning TMEM lane r (row r) and one half
+//               of the tile's columns computes W' = B W + c_S S + U_W,
+//               S' = A S + U_S in place and the bf16 W' into the X slot
+// Every wait is bounded and also gives up once another role has flagged an
+// abort; after an abort the producer waits (bounded) for its copies in
+// flight and the MMA warp for its MMAs before TMEM is freed.
+constexpr int UP2_NT = 384;
+constexpr int UP2_EPI0 = 4;                    // first epilogue warp
+struct Up2Layer {
+  int M, mtiles, ntiles, nranges, first;       // rows of W_l, 128-row blocks, 64-column tiles, ranges, first unit
+  int b_rows_per_stream;                       // rows of the X source per stream
+  long long b_row_off;                         // first X row of the chunk (layer 1 reads the keys)
+};
+struct Up2Args {
+  Up2Layer l[kMaxL];
+  int L, C, chunk, nchunks, tpu;
+  const float *scal;                           // [streams, nchunks, 4] (B, A, c_S, -)
+  int *status;
+  unsigned long long wait_ns;
+  int inject;                                  // test hook, as in GemmArgs
+};
+// shared memory: A operands, then two stages of {X (or bf16 W'), W, S}
+__host__ __device__ constexpr uint32_t up2_a_bytes(int C) { return 2u * (uint32_t)C * 128u; }
+__host__ __device__ constexpr uint32_t up2_x_bytes(int C) { return (uint32_t)(C > 128 ? C : 128) * 128u; }
+__host__ __device__ constexpr uint32_t up2_stage_bytes(int C) { return up2_x_bytes(C) + 4u * UP_BOX; }
+__host__ __device__ constexpr size_t up2_smem(int C) {
+  return 2 * (size_t)up2_a_bytes(C) + 2 * (size_t)up2_stage_bytes(C) + 1024;
+}
+
+// Bounded wait that also returns (false) once *abort is set; on expiry it
+// records TM_ERR_TIMEOUT and sets *abort.
+__device__ bool up2_wait(uint64_t *bar, uint32_t par, const Up2Args &a, volatile int *abort) {
+  if (mbar_try_wait(bar, par)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i)
+      if (mbar_try_wait(bar, par)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > a.wait_ns) {
+      atomicCAS(a.status, 0, kDevTimeout);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(UP2_NT, 1)
+    tcl_update2_kernel(const __grid_constant__ Up2Args a, const __grid_constant__ UpMaps m) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char *sm =
+      reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t a_full, ws_full[2], x_full[2], mma_done[2], acc_free[2], epi_done[2], stage_free[2], fin,
+      never;
+  __shared__ uint32_t tslot;
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  // this CTA's unit
+  const int u = blockIdx.x;
+  int l = 0;
+  while (l + 1 < a.L && u >= a.l[l + 1].first) ++l;
+  const Up2Layer &ly = a.l[l];
+  const int per = ly.mtiles * ly.nranges, i = u - ly.first;
+  const int s = i / per, mt = (i % per) / ly.nranges, rg = i % ly.nranges;
+  const int j0 = rg * a.tpu, j1 = (j0 + a.tpu < ly.ntiles) ? j0 + a.tpu : ly.ntiles;
+  const int nt = j1 - j0;                      // column tiles of this unit
+  const int C = a.C;
+  const int R = ly.M < 128 ? ly.M : 128;       // rows of a state box
+  const int rows = ly.M - 128 * mt < 128 ? ly.M - 128 * mt : 128;
+  const uint32_t AB = up2_a_bytes(C), XB = up2_x_bytes(C), SB = up2_stage_bytes(C);
+  unsigned char *a_cg = sm, *a_eg = sm + AB;
+  auto x_slot = [&](int b) { return sm + 2 * AB + b * SB; };
+  auto w_slot = [&](int b) { return sm + 2 * AB + b * SB + XB; };
+  auto s_slot = [&](int b) { return sm + 2 * AB + b * SB + XB + 2 * UP_BOX; };
+  const uint32_t ws_bytes = 4u * (uint32_t)R * 128u;
+  const uint32_t x_bytes = (uint32_t)C * 128u;
+
+  if (tid == 0) {
+    mbar_init(&a_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ws_full[b], 1);
+      mbar_init(&x_full[b], 1);
+      mbar_init(&mma_done[b], 1);
+      mbar_init(&acc_free[b], 8);
+      mbar_init(&epi_done[b], 8);
+      mbar_init(&stage_free[b], 1);
+    }
+    mbar_init(&fin, 1);
+    mbar_init(&never, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) { tmem_alloc(&tslot, 256); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = tslot;
+  volatile int *abort = &abort_flag;
+
+  // state tiles of the first two column tiles: issued before the wait for
+  // the preceding kernel (this chunk's forward/backward), which does not
+  // write them
+  int ws_armed[2] = {0, 0}, x_armed[2] = {0, 0}, a_armed = 0;
+  if (warp == 0 && lane == 0) {
+    if (a.inject && !injected_wait(&never, a.status, a.wait_ns)) *abort = 1;
+    for (int jj = 0; jj < nt && jj < 2 && !*abort; ++jj) {
+      const int col = 64 * (j0 + jj);
+      mbar_arrive_expect_tx(&ws_full[jj], ws_bytes);
+      for (int bx = 0; bx < 2; ++bx) {
+        tma_load_3d(w_slot(jj) + bx * UP_BOX, &m.w[l], &ws_full[jj], col + 32 * bx, 128 * mt, s);
+        tma_load_3d(s_slot(jj) + bx * UP_BOX, &m.s[l], &ws_full[jj], col + 32 * bx, 128 * mt, s);
+      }
+      ++ws_armed[jj];
+    }
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && !*abort) {
+      const long long brow = (long long)s * ly.b_rows_per_stream + ly.b_row_off;
+      mbar_arrive_expect_tx(&a_full, 2u * AB);
+      for (int f = 0; f < 2; ++f)
+        for (int kp = 0; kp < C / 64; ++kp) {
+          tma_load_2d(a_cg + f * C * 128 + kp * 64 * 128, &m.a[l], &a_full, 128 * mt + 64 * f, s * C + 64 * kp);
+          tma_load_2d(a_eg + f * C * 128 + kp * 64 * 128, &m.a2[l], &a_full, 128 * mt + 64 * f, s * C + 64 * kp);
+        }
+      a_armed = 1;
+      for (int jj = 0; jj < nt; ++jj) {
+        const int b = jj & 1, col = 64 * (j0 + jj);
+        if (jj >= 2) {
+          if (!up2_wait(&stage_free[b], (uint32_t)(((jj - 2) >> 1) & 1), a, abort)) break;
+          mbar_arrive_expect_tx(&ws_full[b], ws_bytes);
+          for (int bx = 0; bx < 2; ++bx) {
+            tma_load_3d(w_slot(b) + bx * UP_BOX, &m.w[l], &ws_full[b], col + 32 * bx, 128 * mt, s);
+            tma_load_3d(s_slot(b) + bx * UP_BOX, &m.s[l], &ws_full[b], col + 32 * bx, 128 * mt, s);
+          }
+          ++ws_armed[b];
+        }
+        mbar_arrive_expect_tx(&x_full[b], x_bytes);
+        for (int kp = 0; kp < C / 64; ++kp)
+          tma_load_2d(x_slot(b) + kp * 64 * 128, &m.b[l], &x_full[b], col, (int)(brow + 64 * kp));
+        ++x_armed[b];
+      }
+    }
+    if (lane == 0 && *abort) {
+      // copies still in flight into this CTA's shared memory finish first
+      if (a_armed) mbar_wait(&a_full, 0, a.wait_ns);
+      for (int b = 0; b < 2; ++b) {
+        if (ws_armed[b]) mbar_wait(&ws_full[b], (uint32_t)((ws_armed[b] - 1) & 1), a.wait_ns);
+        if (x_armed[b]) mbar_wait(&x_full[b], (uint32_t)((x_armed[b] - 1) & 1), a.wait_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, 64, true, true);
+      const uint32_t acg = smem_u32(a_cg), aeg = smem_u32(a_eg);
+      bool ok = up2_wait(&a_full, 0, a, abort);
+      for (int jj = 0; jj < nt && ok; ++jj) {
+        const int b = jj & 1;
+        if (!up2_wait(&x_full[b], (uint32_t)((jj >> 1) & 1), a, abort)) break;
+        if (jj >= 2 && !up2_wait(&acc_free[b], (uint32_t)(((jj - 2) >> 1) & 1), a, abort)) break;
+        tc_fence_after();
+        const uint32_t xb = smem_u32(x_slot(b));
+        const uint32_t acc = tm + 128u * (uint32_t)b;
+        for (int ks = 0; ks < C / 16; ++ks) {
+          const uint64_t bd = desc_mnmajor(xb, C, ks);
+          umma_bf16(acc, desc_mnmajor(acg, C, ks), bd, idesc, ks != 0);
+          umma_bf16(acc + 64, desc_mnmajor(aeg, C, ks), bd, idesc, ks != 0);
+        }
+        umma_commit(&mma_done[b]);
+      }
+      // every MMA this CTA issued has completed before TMEM is freed
+      umma_commit(&fin);
+      mbar_wait(&fin, 0, a.wait_ns);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ stores
+    if (lane == 0) {
+      for (int jj = 0; jj < nt; ++jj) {
+        const int b = jj & 1, col = 64 * (j0 + jj);
+        if (!up2_wait(&epi_done[b], (uint32_t)((jj >> 1) & 1), a, abort)) break;
+        for (int bx = 0; bx < 2; ++bx) {
+          tma_store_3d(&m.w[l], w_slot(b) + bx * UP_BOX, col + 32 * bx, 128 * mt, s);
+          tma_store_3d(&m.s[l], s_slot(b) + bx * UP_BOX, col + 32 * bx, 128 * mt, s);
+        }
+        tma_store_3d(&m.wb[l], x_slot(b), col, 128 * mt, s);
+        tma_store_commit_wait_read();
+        mbar_arrive(&stage_free[b]);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= UP2_EPI0) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3, h = (warp - UP2_EPI0) >> 2;
+    const int r = 32 * q + lane;               // TMEM lane = row of the block
+    const uint32_t lb = (uint32_t)(32 * q) << 16;
+    const float4 sc = *reinterpret_cast<const float4 *>(a.scal + 4 * ((long long)s * a.nchunks + a.chunk));
+    for (int jj = 0; jj < nt; ++jj) {
+      const int b = jj & 1;
+      const uint32_t ph = (uint32_t)((jj >> 1) & 1);
+      if (!up2_wait(&mma_done[b], ph, a, abort)) break;
+      if (!up2_wait(&ws_full[b], ph, a, abort)) break;
+      tc_fence_after();
+      float u0[16], u1[16], v0[16], v1[16];
+      const uint32_t acc = tm + lb + 128u * (uint32_t)b + 32u * (uint32_t)h;
+      tmem_ld16(acc, u0);
+      tmem_ld16(acc + 16, u1);
+      tmem_ld16(acc + 64, v0);
+      tmem_ld16(acc + 80, v1);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_free[b]);  // the MMA of tile jj + 2 may overwrite the pair
+      if (r < rows) {
+        unsigned char *wr = w_slot(b) + h * UP_BOX + r * 128;
+        unsigned char *sr = s_slot(b) + h * UP_BOX + r * 128;
+        unsigned char *br = x_slot(b) + r * 128;
+#pragma unroll
+        for (int jc = 0; jc < 8; ++jc) {
+          const uint32_t o = (uint32_t)((jc ^ (r & 7)) << 4);
+          const float *uw = jc < 4 ? u0 + 4 * jc : u1 + 4 * (jc - 4);
+          const float *us = jc < 4 ? v0 + 4 * jc : v1 + 4 * (jc - 4);
+          const float4 w = *reinterpret_cast<const float4 *>(wr + o);
+          const float4 x = *reinterpret_cast<const float4 *>(sr + o);
+          const float4 wn = make_float4(sc.x * w.x + sc.z * x.x + uw[0], sc.x * w.y + sc.z * x.y + uw[1],
+                                        sc.x * w.z + sc.z * x.z + uw[2], sc.x * w.w + sc.z * x.w + uw[3]);
+          const float4 sn = make_float4(sc.y * x.x + us[0], sc.y * x.y + us[1], sc.y * x.z + us[2],
+                                        sc.y * x.w + us[3]);
+          *reinterpret_cast<float4 *>(wr + o) = wn;
+          *reinterpret_cast<float4 *>(sr + o) = sn;
+          // bf16 row: columns 32 h + 4 jc .. + 3 in 16-byte chunk 4 h + jc / 2
+          const uint32_t ob = (uint32_t)((((4 * h + (jc >> 1)) ^ (r & 7)) << 4) + (jc & 1) * 8);
+          *reinterpret_cast<uint2 *>(br + ob) = make_uint2(pack_bf16(wn.x, wn.y), pack_bf16(wn.z, wn.w));
+        }
+      }
+      fence_proxy_async_smem();                // the TMA stores read these rows
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&epi_done[b]);
+    }
+  }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tm, 256);
+}
+
+// ------------------------------------------------------------------------
 // Fused forward + backward of one chunk, for memories whose every layer is at
 // most 256 wide. One CTA per (128-row tile of the chunk's [keys; queries],
 // stream) runs the whole chain that the per-phase kernels run as 2L - 1
@@ -517,6 +801,7 @@ struct FbArgs {
   const float *coef;                 // [streams, T, 2]
   int *status;
   unsigned long long wait_ns;
+  int inject;                        // test hook, as in GemmArgs
 };
 
 struct FbMaps {
@@ -571,7 +856,7 @@ __global__ void __launch_bounds__(FB_NT, 1)
   unsigned char *abuf =
       reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char *ring = abuf + FB_ABUF;
-  __shared__ uint64_t full[FB_STAGES], empty[FB_STAGES], xbar, done, ready;
+  __shared__ uint64_t full[FB_STAGES], empty[FB_STAGES], xbar, done, ready, never;
   __shared__ uint32_t tslot;
   __shared__ int abort_flag;
   __shared__ float2 cef[128];
@@ -592,6 +877,7 @@ __global__ void __launch_bounds__(FB_NT, 1)
     mbar_init(&xbar, 1);
     mbar_init(&done, 1);
     mbar_init(&ready, 1);
+    mbar_init(&never, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -604,7 +890,10 @@ __global__ void __launch_bounds__(FB_NT, 1)
 
   if (warp == FB_EPI / 32) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
+    if (lane == 0 && a.inject && !injected_wait(&never, a.status, a.wait_ns)) {
+      abort_flag = 1;                            // nothing issued yet; release the epilogue
+      mbar_arrive(&done);
+    } else if (lane == 0) {
       int total = 0;
       for (int p = 0; p < nphase; ++p) total += fb_phase(a, p).ns;
       int issued = 0, consumed = 0;
@@ -998,6 +1287,20 @@ cudaError_t launch_gemm(const GemmArgs &a, const CUtensorMap &mA, const CUtensor
   return cudaErrorInvalidValue;
 }
 
+cudaError_t launch_up2(const Up2Args &a, const UpMaps &m, int units, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)units);
+  cfg.blockDim = dim3(UP2_NT);
+  cfg.dynamicSmemBytes = up2_smem(a.C);
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tcl_update2_kernel, a, m);
+}
+
 cudaError_t launch_up(const UpArgs &a, const UpMaps &m, int tiles, size_t smem, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)tiles);
@@ -1025,8 +1328,29 @@ bool tcl_supported(const Problem &p) {
 
 
 static unsigned long long g_tcl_wait_ns = 2000000000ull;
+static int g_tcl_inject = 0;
 
 namespace {
+
+// Column tiles per unit of the pipelined update: 4 (longer pipelines) unless
+// that leaves fewer than 32 CTAs per launch; TM_TCL_TPU (1..16), read once
+// per process, overrides.
+int up2_tiles_per_unit(const Problem &p) {
+  static int forced = -1;
+  if (forced < 0) {
+    const char *e = std::getenv("TM_TCL_TPU");
+    forced = e ? std::atoi(e) : 0;
+    if (forced < 0 || forced > 16) forced = 0;
+  }
+  if (forced) return forced;
+  for (int tpu = 4; tpu > 1; tpu /= 2) {
+    long long units = 0;
+    for (int l = 1; l <= p.L; ++l)
+      units += (long long)p.streams * ((p.dims[l] + 127) / 128) * ((p.dims[l - 1] / 64 + tpu - 1) / tpu);
+    if (units >= 32) return tpu;
+  }
+  return 1;
+}
 
 // One group of streams: its slice of every tensor, its own workspace carve
 // and CUDA stream, and everything its launches need.
@@ -1045,6 +1369,9 @@ struct TclGroup {
   UpMaps um;
   int up_tiles;
   size_t up_smem_bytes;
+  bool up2;                      // pipelined update kernel (C <= 128)
+  Up2Args ua2;
+  int up2_units;
   bool fused;
   FbArgs fa;
   FbMaps fm;
@@ -1107,6 +1434,7 @@ cudaError_t TclGroup::setup() {
   base.coef = coef;
   base.status = p.status;
   base.wait_ns = g_tcl_wait_ns;
+  base.inject = g_tcl_inject;
   base.y = p.y;
   base.v = reinterpret_cast<const __nv_bfloat16 *>(p.v);
 
@@ -1119,6 +1447,7 @@ cudaError_t TclGroup::setup() {
   ua.scal = scal;
   ua.status = p.status;
   ua.wait_ns = g_tcl_wait_ns;
+  ua.inject = g_tcl_inject;
   up_tiles = 0;
   up_smem_bytes = 0;
   for (int l = 1; l <= L; ++l) {
@@ -1146,6 +1475,32 @@ cudaError_t TclGroup::setup() {
     if (sm > up_smem_bytes) up_smem_bytes = sm;
   }
 
+  // the pipelined update: units of (layer, stream, 128-row block, range of
+  // up to tpu 64-column tiles)
+  up2 = C <= 128;
+  if (up2) {
+    std::memset(&ua2, 0, sizeof ua2);
+    ua2.L = L;
+    ua2.C = C;
+    ua2.nchunks = nchunks;
+    ua2.scal = scal;
+    ua2.status = p.status;
+    ua2.wait_ns = g_tcl_wait_ns;
+    ua2.inject = g_tcl_inject;
+    ua2.tpu = up2_tiles_per_unit(p);
+    up2_units = 0;
+    for (int l = 1; l <= L; ++l) {
+      Up2Layer &u = ua2.l[l - 1];
+      u.M = p.dims[l];
+      u.mtiles = (p.dims[l] + 127) / 128;
+      u.ntiles = p.dims[l - 1] / 64;
+      u.nranges = (u.ntiles + ua2.tpu - 1) / ua2.tpu;
+      u.first = up2_units;
+      u.b_rows_per_stream = l == 1 ? T : 2 * C;
+      up2_units += S * u.mtiles * u.nranges;
+    }
+  }
+
   fused = p.fuse_fb && fb_ok(p);
   if (fused) {
     std::memset(&fa, 0, sizeof fa);
@@ -1167,6 +1522,7 @@ cudaError_t TclGroup::setup() {
     fa.coef = coef;
     fa.status = p.status;
     fa.wait_ns = g_tcl_wait_ns;
+    fa.inject = g_tcl_inject;
   }
   return cudaSuccess;
 }
@@ -1215,6 +1571,11 @@ cudaError_t TclGroup::chunk(int ch) {
     if (err != cudaSuccess) return err;
   }
   // weight-update contractions of every layer, with the fused state update
+  if (up2) {
+    ua2.chunk = ch;
+    ua2.l[0].b_row_off = (long long)ch * C;
+    return launch_up2(ua2, um, up2_units, stream);
+  }
   ua.chunk = ch;
   ua.l[0].b_row_off = (long long)ch * C;
   return launch_up(ua, um, up_tiles, up_smem_bytes, stream);
@@ -1301,6 +1662,8 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
     e = cudaFuncSetAttribute(tcl_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)up_smem(128, 2));
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tcl_update2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)up2_smem(128));
+    if (e != cudaSuccess) return e;
     attr_done = true;
   }
   const int G = tcl_groups(p);
@@ -1339,7 +1702,11 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
   return err;
 }
 
-void tcl_set_wait(unsigned long long wait_ns) { g_tcl_wait_ns = wait_ns ? wait_ns : 2000000000ull; }
+void tcl_set_debug(int inject_timeout, unsigned long long wait_ns) {
+  g_tcl_inject = inject_timeout ? 1 : 0;
+  g_tcl_wait_ns = wait_ns ? wait_ns : 2000000000ull;
+}
 unsigned long long tcl_wait_ns() { return g_tcl_wait_ns; }
+int tcl_inject() { return g_tcl_inject; }
 
 }  // namespace tmem

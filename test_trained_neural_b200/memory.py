@@ -111,6 +111,47 @@ class NeuralMemory:
             self.sync(workspace, stream)
         return y, W_end, S_end
 
+    def host_workspace_size(self, B, H, T, C, dtype=torch.bfloat16, segment_tokens=0) -> int:
+        out = ctypes.c_size_t()
+        code = N.TM_BF16 if dtype == torch.bfloat16 else N.TM_F32
+        N.check(self._lib.tm_host_workspace_size(self._h, B, H, T, C, code, int(segment_tokens),
+                                                 ctypes.byref(out)), "tm_host_workspace_size")
+        return int(out.value)
+
+    def run_host(self, k, v, q, theta, eta, alpha, W0, S0, C, y=None, W_end=None, S_end=None,
+                 workspace=None, segment_tokens=0, stream=None, sync=True):
+        """run() with every input and output in host memory (CPU tensors,
+        pinned for the copies to overlap the kernels): the library copies the
+        segments in and out itself, overlapped with the kernels. Returns
+        (y, W_end, S_end) as CPU tensors; with sync=False they are complete
+        once `stream` reaches this point."""
+        B, H, T, d = k.shape
+        dt = self._dtype_code(k)
+        for t in (k, v, q, theta, eta, alpha, W0, S0):
+            if t.is_cuda or not t.is_contiguous():
+                raise ValueError("run_host takes contiguous CPU tensors")
+        pin = k.is_pinned()
+        if y is None:
+            y = torch.empty((B, H, T, d), dtype=torch.float32, pin_memory=pin)
+        if W_end is None:
+            W_end = torch.empty_like(W0, pin_memory=pin)
+        if S_end is None:
+            S_end = torch.empty_like(S0, pin_memory=pin)
+        dev = torch.device("cuda", torch.cuda.current_device())
+        if workspace is None:
+            n = self.host_workspace_size(B, H, T, C, k.dtype, segment_tokens)
+            workspace = torch.empty(n, dtype=torch.uint8, device=dev)
+        if stream is None:
+            stream = torch.cuda.current_stream(dev)
+        code = self._lib.tm_run_host(self._h, B, H, T, C, dt, _ptr(k), _ptr(v), _ptr(q), _ptr(theta),
+                                     _ptr(eta), _ptr(alpha), _ptr(W0), _ptr(S0), _ptr(y), _ptr(W_end),
+                                     _ptr(S_end), int(segment_tokens), _ptr(workspace), workspace.numel(),
+                                     ctypes.c_void_p(stream.cuda_stream))
+        N.check(code, "tm_run_host")
+        if sync:
+            self.sync(workspace, stream)
+        return y, W_end, S_end
+
     def decode_step(self, k, v, q, theta, eta, alpha, W, S, y=None, stream=None):
         """One token per stream (k, v, q [B, H, d_h]; gates [B, H]): returns
         y = M_W(q) and updates W, S ([B, H, P] float32) in place."""

@@ -406,3 +406,47 @@ def test_tcl_matches_cluster_kernel():
     assert max(errs.values()) < TOL_BF16_TC, errs
 
 
+
+
+@pytest.mark.parametrize("path", ["tcl", "tcl-phased"])
+def test_tcl_timeout_is_reported_and_context_survives(path):
+    """The layered kernels' failure handling: with the test hook on, every CTA
+    of the forward/backward (fused or per phase) and update kernels first
+    waits on a barrier that nothing completes; the wait runs out after 1 ms,
+    the kernel records TM_ERR_TIMEOUT, issues nothing further and returns.
+    The next call on the same context (hook off) matches the oracle."""
+    from test_trained_neural_b200 import _native as N
+    from test_trained_neural_b200._native import TitansMemError
+    lib = N.load()
+    w = W.make(4, 64, 2, 1, 2, 256, 128, index=650) if path == "tcl" else W.make(2, 128, 3, 1, 1, 128, 64, index=651)
+    inp, dev = _dev_inputs(w)
+    mem = NeuralMemory(w.L, w.d, w.expansion, path=path)
+    assert lib.tm_set_debug(1, 1_000_000) == N.TM_OK
+    try:
+        for _ in range(2):          # a repeated call goes through graph capture and replay
+            with pytest.raises(TitansMemError) as ei:
+                run_lib(mem, dev, w.C)
+            assert ei.value.code == N.TM_ERR_TIMEOUT
+    finally:
+        lib.tm_set_debug(0, 0)
+    y, We, Se = run_lib(mem, dev, w.C)
+    ref = oracle.run_workload(w, inp)
+    errs = parity_errors(w.dims, inp["W0"], gpu_to_np(y, We, Se), ref)
+    assert max(errs.values()) < TOL_BF16_TC, errs
+
+
+@pytest.mark.parametrize("idx,T", [(1, 128), (2, 128), (3, 128), (4, 256)])
+def test_literal_gates_on_the_benchmark_path(idx, T):
+    """Each MLP workload with its gates drawn exactly as specified (no
+    damping), on the path the benchmark times, over a stream short enough
+    that the memory is still finite: every stream against the oracle."""
+    w = W.get_literal(idx)
+    inp = W.generate(w, T=T)
+    dev = to_dev(inp, w.B, w.H, w.dtype)
+    mem = NeuralMemory(w.L, w.d, w.expansion, path="auto")
+    assert mem.query_path(w.B, w.H, T, w.C) in ("tc", "tcl", "tcl-phased")
+    y, We, Se = run_lib(mem, dev, w.C)
+    ref = oracle.run_workload(w, inp)
+    assert np.isfinite(ref["W_end"]).all() and np.isfinite(ref["y"]).all()
+    errs = parity_errors(w.dims, inp["W0"], gpu_to_np(y, We, Se), ref)
+    assert max(errs.values()) < TOL_BF16_TC, (w.name, errs)
