@@ -102,15 +102,20 @@ bool tensor_path(tm_path path) {
          path == TM_PATH_TC_PHASED;
 }
 
-// Workspace after the status word. A tensor-core path with a shorter last
-// chunk runs it afterwards on the CUDA-core kernel, in the same space.
+// Bytes at the start of the workspace (after the status word) that hold the
+// fp16 copies of keys and queries on the tensor-core paths.
+size_t f16_bytes(tm_path path, const tmem::Problem &p) { return tensor_path(path) ? tmem::tokens_f16_bytes(p) : 0; }
+
+// Workspace after the status word: the fp16 token copies (tensor-core paths),
+// then the kernels' scratch. A tensor-core path with a shorter last chunk runs
+// it afterwards on the CUDA-core kernel, in the same scratch space.
 size_t scratch_bytes(tm_path path, const tmem::Problem &p) {
   size_t b = tmem::simt_scratch_bytes(p);
   if (!tensor_path(path)) return b;
-  const size_t m = (path == TM_PATH_TC || path == TM_PATH_TC_GLOBAL) ? tmem::tc_scratch_bytes(p)
-                                                                    : tmem::tcl_scratch_bytes(p);
-  if (p.T_run == p.T) return m;
-  return m > b ? m : b;
+  size_t m = (path == TM_PATH_TC || path == TM_PATH_TC_GLOBAL) ? tmem::tc_scratch_bytes(p)
+                                                              : tmem::tcl_scratch_bytes(p);
+  if (p.T_run < p.T && b > m) m = b;
+  return f16_bytes(path, p) + m;
 }
 
 }  // namespace
@@ -361,8 +366,8 @@ tm_status tm_launch_count(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtyp
   long long n = 1;
   if (tensor_path(path)) {
     n = p.T_run == 0 ? 0
-        : (path == TM_PATH_TC_LAYERED || path == TM_PATH_TC_PHASED) ? tmem::tcl_launch_count(p)
-                                                                    : tmem::tc_launch_count(p);
+        : 1 + ((path == TM_PATH_TC_LAYERED || path == TM_PATH_TC_PHASED) ? tmem::tcl_launch_count(p)
+                                                                         : tmem::tc_launch_count(p));
     if (p.T_run < p.T) n += 1;                 // the shorter last chunk
   }
   *out = n;
@@ -421,11 +426,19 @@ tm_status run_device(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype,
   p.W_end = W_end;
   p.S_end = S_end;
   p.status = reinterpret_cast<int *>(workspace);
-  p.scratch = static_cast<char *>(workspace) + tmem::kStatusBytes;
-  p.scratch_bytes = workspace_bytes - tmem::kStatusBytes;
+  const size_t f16b = f16_bytes(path, p);
+  char *after_status = static_cast<char *>(workspace) + tmem::kStatusBytes;
+  if (f16b) {
+    p.k16 = after_status;
+    p.q16 = after_status + f16b / 2;
+  }
+  p.scratch = after_status + f16b;
+  p.scratch_bytes = workspace_bytes - tmem::kStatusBytes - f16b;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (clear_status && cudaMemsetAsync(p.status, 0, sizeof(int), s) != cudaSuccess) return TM_ERR_CUDA;
+  // the tensor-core kernels read fp16 copies of the keys and queries
+  if (f16b && p.T_run > 0 && tmem::tokens_f16_launch(p, s) != cudaSuccess) return TM_ERR_CUDA;
   p.fuse_fb = path == TM_PATH_TC_LAYERED;
   if (path == TM_PATH_TC_LAYERED || path == TM_PATH_TC_PHASED) {
     const int groups = tmem::tcl_group_count(p);
@@ -456,7 +469,13 @@ tm_status run_device(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype,
       err = tmem::simt_launch(q, s);
     }
   }
-  return err == cudaSuccess ? TM_OK : TM_ERR_CUDA;
+  if (err != cudaSuccess) {
+    // a failed launch leaves its error pending in the runtime: consume it
+    // here (it is reported as TM_ERR_CUDA) so that later calls do not see it
+    cudaGetLastError();
+    return TM_ERR_CUDA;
+  }
+  return TM_OK;
 }
 
 size_t up256(size_t x) { return (x + 255) / 256 * 256; }

@@ -32,6 +32,7 @@ struct Problem {
   int streams;
   tm_dtype in_dtype;
   const void *k, *v, *q;
+  const void *k16, *q16;  // tensor-core paths: fp16 copies of k and q (workspace)
   const float *theta, *eta, *alpha;
   const float *W0, *S0;
   float *y, *W_end, *S_end;
@@ -55,6 +56,12 @@ bool problem_from_ctx(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype dt
 bool run_aliasing_ok(const Problem &p, const void *k, const void *v, const void *q, const float *theta,
                      const float *eta, const float *alpha, const float *W0, const float *S0, const float *y,
                      const float *W_end, const float *S_end);
+
+// fp16 copies of the keys and queries for the tensor-core paths: workspace
+// bytes (both copies, 256-byte aligned) and the conversion launch (p.k, p.q
+// bf16 -> p.k16, p.q16).
+size_t tokens_f16_bytes(const Problem &p);
+cudaError_t tokens_f16_launch(const Problem &p, cudaStream_t stream);
 
 // SIMT (CUDA-core, fp32) path.
 size_t simt_scratch_bytes(const Problem &p);

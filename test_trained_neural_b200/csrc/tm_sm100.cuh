@@ -159,17 +159,16 @@ __device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int rows, int ks)
 __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int rows, int ks) {
   return make_desc(base + (uint32_t)ks * 2048u, (uint32_t)rows * 128u, 1024u);
 }
-// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
+// Instruction descriptor, kind::f16: fp16 A and B (format code 0 in bits
+// 7-9 and 10-12), fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn) {
   return (1u << 4)                       // D format f32
-         | (1u << 7)                     // A bf16
-         | (1u << 10)                    // B bf16
          | ((a_mn ? 1u : 0u) << 15)      // A major
          | ((b_mn ? 1u : 0u) << 16)      // B major
          | ((uint32_t)(N >> 3) << 17)    // N / 8
          | ((uint32_t)(M >> 4) << 24);   // M / 16
 }
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                           uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -225,6 +224,14 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void 
 // memory sources have been read (the global writes complete with the grid).
 __device__ __forceinline__ void tma_store_commit_wait_read() {
   asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Close the bulk group of this thread's stores (no wait).
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's most recent bulk groups still read
+// their shared-memory sources.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

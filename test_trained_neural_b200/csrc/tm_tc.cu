@@ -4,19 +4,21 @@
 // CTA j of the cluster owns hidden units [64 j, 64 j + 64): rows of W1 and
 // columns of W2, so hidden = 64 G. Per chunk of C = 64 tokens:
 //
-//   A1  TMA loads keys and queries of the chunk as one 128-row bf16 tile
+//   A1  TMA loads keys and queries of the chunk as one 128-row fp16 tile
 //       (keys rows 0-63, queries rows 64-127), 128-byte swizzle.
 //   A5  the control warp turns the chunk's gates into per-token coefficients
 //       with warp shuffles (division-free reverse scan).
 //   A2  Z1 = [K;Q] W1_j^T        M=128 N=64  K=d   (keys and queries share W)
-//       X1 = silu(Z1)            epilogue, bf16 to shared memory
+//       X1 = silu(Z1)            epilogue, fp16 to shared memory
 //       Z2_j = X1 W2_j^T         M=128 N=d   K=64  (this CTA's partial sum)
-//       all-reduce of Z2 over the cluster with bulk copies between the CTAs'
-//       shared memories (the copy engine, mbarrier transaction counts, no
-//       thread-level cluster fences): each CTA stages its partial as bf16 rows
-//       and pushes rows [128/G p, 128/G (p+1)) to CTA p (reduce-scatter); CTA p
-//       sums them in fp32, writes y for query rows and G2 = 2 (Z2 - V) for key
-//       rows, and pushes its G2 rows to every CTA (all-gather) (A3).
+//       all-reduce of Z2 over the cluster through the CTAs' shared memories
+//       with asynchronous remote stores (st.async: each 16-byte piece counts
+//       its bytes on the receiver's mbarrier, no cluster fences): each thread
+//       sends its fp16 partial of rows [128/G p, 128/G (p+1)) straight into
+//       CTA p's receive buffer (reduce-scatter); CTA p sums them in fp32,
+//       writes y for query rows and G2 = 2 (Z2 - V) for key rows, and each of
+//       its threads sends its G2 piece into every CTA's G2 tile (all-gather)
+//       (A3).
 //   A4  G1 = (G2 W2_j) . silu'(Z1_K)        M=128(64 used) N=64 K=d
 //   A6+A7 the fp32 state of this CTA's slice, [W | S], lives in TMEM for the
 //       whole stream. Before the weight-update contractions of a chunk the
@@ -26,7 +28,7 @@
 //       [W1' | S1']^T = [W1 | S1]^T + K^T  [-c G1   | -e G1]     M=d N=128 K=64
 //       (c_i, e_i fold the momentum and forget gates of the chunk into the
 //        operands), so the tensor core itself emits the updated state; the
-//       epilogue only writes the bf16 copy of W' the next chunk multiplies with.
+//       epilogue only writes the fp16 copy of W' the next chunk multiplies with.
 //   A8  the loop over chunks; TMA for chunk c+1 overlaps the write-back.
 //       W_end / S_end are written once, after the last chunk.
 //
@@ -34,12 +36,24 @@
 //  gradients at the chunk-start weights written as matrix products, decay
 //  products folded per token.)
 //
-// Warp roles: warps 0-7 epilogue (warp w reads TMEM lanes 32 (w % 4) .. +31,
-// columns half w / 4), warp 8 control (TMA, MMA issue by lane 0, scan).
+// Operand format: every contraction takes fp16 operands (10 mantissa bits)
+// with fp32 accumulation. Keys and queries arrive as bf16 and are converted to
+// fp16 once per call before this kernel; weights, activations, gradients and
+// the exchanged partial sums are rounded to fp16. (With bf16's 7 mantissa bits
+// the rounding of these operands, although unbiased, drifts the state along a
+// near-symmetry of the depth-2 memory - W1 -> A W1, W2 -> W2 A^-1 for the
+// nearly linear SiLU at small pre-activations - by several percent over
+// thousands of chunks; fp16 cuts that drift eightfold at the same cost.)
+//
+// Warp roles: warps 0-15 epilogue (warp w reads TMEM lanes 32 (w % 4) .. +31
+// and a quarter w / 4 of the slice's 64 hidden columns; warps 0-7 also stage
+// and reduce the layer-2 exchange by column halves), warp 16 control (TMA,
+// MMA issue by lane 0, scan).
 // Every wait is bounded; on expiry the kernel records TM_ERR_TIMEOUT in the
 // status word, drains its copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <cstring>
 
@@ -53,9 +67,11 @@ using namespace sm100;
 
 constexpr int C = 64;           // chunk size of this kernel
 constexpr int HS = 64;          // hidden units per CTA
-constexpr int EPI_WARPS = 8;
+constexpr int EPI_WARPS = 16;   // warp w: TMEM lanes 32 (w % 4) .., hidden columns quarter w / 4
+constexpr int XCH_WARPS = 8;    // the first 8 stage and reduce the layer-2 exchange (column halves)
 constexpr int NTHREADS = (EPI_WARPS + 1) * 32;
-constexpr int EPI_THREADS = EPI_WARPS * 32;
+constexpr int XCH_THREADS = XCH_WARPS * 32;
+constexpr int CPT = HS / (EPI_WARPS / 4);   // hidden columns of a slice per epilogue thread (16)
 constexpr uint32_t TMEM_COLS = 512;
 
 struct TcArgs {
@@ -71,8 +87,8 @@ struct TcArgs {
   // Exchange through global memory (streams whose cluster does not fit
   // beside the others): per stream, receive buffers and G2 rows, double
   // buffered by chunk parity, and monotonic arrival counters.
-  unsigned char *xrecv;          // [stream][dest][parity][G x 2 x RP x d] bf16
-  unsigned char *xg2;            // [stream][parity][64 x d] bf16, row-block layout
+  unsigned char *xrecv;          // [stream][dest][parity][G x 2 x RP x d] fp16
+  unsigned char *xg2;            // [stream][parity][64 x d] fp16, row-block layout
   unsigned *xflag;               // [stream][G + 1] counters, 128 bytes apart
 };
 
@@ -82,11 +98,28 @@ __host__ __device__ constexpr size_t xrecv_bytes(int D, int G) { return (size_t)
 __host__ __device__ constexpr size_t xg2_bytes(int D) { return (size_t)2 * 64 * D * 2; }
 __host__ __device__ constexpr size_t xflag_bytes(int G) { return (size_t)(G + 1) * XFLAG_STRIDE * 4; }
 
+// Per-chunk coefficients. sig is a power of two that the S part of the
+// TMEM state carries for this chunk (S_tmem = sig S) and that the -e X1 and
+// -e G1 operands are multiplied by: e_i = theta_i prod_{j>i} eta_j reaches
+// 1e-6 for the first tokens of a chunk, and e_i x_i would otherwise fall among
+// fp16's subnormals, whose coarse spacing biases the momentum update; sig puts
+// theta_max sig in [8, 16).
 struct Coefs {
   float c[C];
   float e[C];
-  float Bw, As, cS, pad;
+  float Bw, As, cS, sig;
 };
+
+// The power of two 2^k with tmax 2^k in [8, 16), k clamped to [0, 40]; 1 when
+// tmax is not positive.
+__device__ __forceinline__ float chunk_scale(float tmax) {
+  if (!(tmax > 0.f)) return 1.f;
+  int ex;
+  frexpf(tmax, &ex);                 // tmax = m 2^ex, m in [0.5, 1)
+  int k = 4 - ex;
+  k = k < 0 ? 0 : (k > 40 ? 40 : k);
+  return ldexpf(1.f, k);
+}
 
 // Shared-memory map (bytes from a 1024-aligned base). Feature dims of the
 // d-wide buffers are allocated as 128 even for d = 64 so that the padded
@@ -101,8 +134,8 @@ struct Layout {
   static constexpr uint32_t X1S = X1 + 128 * 64 * 2;         // [64 tok x 128]  R=64
   static constexpr uint32_t G2 = X1S + 64 * 128 * 2;         // [64 tok x FD]   R=64
   static constexpr uint32_t G1S = G2 + 64 * FD * 2;          // [64 tok x 128]  R=64
-  static constexpr uint32_t SEND = G1S + 64 * 128 * 2;       // [128 x D] bf16 partial Z2
-  static constexpr uint32_t RECV = SEND + 128 * D * 2;       // G x [128/G x D] bf16
+  static constexpr uint32_t SEND = G1S + 64 * 128 * 2;       // [128 x D] fp16 partial Z2
+  static constexpr uint32_t RECV = SEND + 128 * D * 2;       // G x [128/G x D] fp16
   static constexpr uint32_t G2OWN = RECV + 128 * D * 2;      // owned rows of G2, RB atoms
   static constexpr uint32_t COEF = G2OWN + 64 * D * 2;       // 2 x Coefs
   static constexpr uint32_t BARS = COEF + 2 * sizeof(Coefs);
@@ -117,7 +150,7 @@ enum Bar {
 };
 
 // sigmoid(z) = 1/2 + tanh(z/2)/2, with the hardware tanh approximation (one
-// MUFU operation; its error is far below the bf16 rounding of the results).
+// MUFU operation; its error is far below the fp16 rounding of the results).
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -125,13 +158,15 @@ __device__ __forceinline__ float tanh_approx(float x) {
 }
 __device__ __forceinline__ float sigm(float z) { return fmaf(0.5f, tanh_approx(0.5f * z), 0.5f); }
 
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+// Two fp32 values as one fp16 pair (round to nearest even): the operand
+// format of every tensor-core contraction here.
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t *>(&h);
 }
 __device__ __forceinline__ uint4 pack8(const float *v) {
-  return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
-                    pack_bf16(v[6], v[7]));
+  return make_uint4(pack_h2(v[0], v[1]), pack_h2(v[2], v[3]), pack_h2(v[4], v[5]),
+                    pack_h2(v[6], v[7]));
 }
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
@@ -154,14 +189,14 @@ __device__ __forceinline__ bool try_wait_acquire_cluster(uint32_t bar, uint32_t 
       : "memory");
   return ok != 0;
 }
-// Copy `bytes` from this CTA's shared memory into CTA-of-cluster shared memory
-// (dst, bar are shared::cluster addresses); completion counts on the remote bar.
-__device__ __forceinline__ void bulk_push(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          dst),
-      "r"(src), "r"(bytes), "r"(bar)
-      : "memory");
+// 16 bytes into CTA-of-cluster shared memory (dst, bar are shared::cluster
+// addresses), counted as 16 transaction bytes on the remote mbarrier, whose
+// completion releases the write at cluster scope.
+__device__ __forceinline__ void st_async_v4(uint32_t dst, uint4 v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   dst),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar)
+               : "memory");
 }
 // Global-memory exchange: bulk copy shared -> global, completion, proxy fence,
 // release counter, acquire poll, bulk copy global -> shared.
@@ -284,10 +319,14 @@ __device__ void coef_scan_warp(Coefs &cf, const float *th, const float *et, cons
   cf.c[i1] = t1 * r1;
   cf.e[i0] = t0 * pe0;
   cf.e[i1] = t1 * pe1;
+  float tmax = fmaxf(t0, t1);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
   if (lane == 0) {
     cf.Bw = pa0 * f0;
     cf.As = pe0 * e0;
     cf.cS = e0 * r0;
+    cf.sig = chunk_scale(tmax);
   }
 }
 
@@ -296,6 +335,8 @@ __device__ void coef_scan_warp(Coefs &cf, const float *th, const float *et, cons
 // the exchange going through global memory (used for streams whose cluster
 // does not fit beside the others; all G CTAs of a stream must be resident).
 template <int D, int G, bool XG>
+// 17 warps: registers are allocated for whole groups of four warps (20
+// warps), so 96 registers a thread fill the SM's 64 K (one CTA per SM)
 __global__ void __launch_bounds__(NTHREADS, 1)
     tc_chunk_kernel(const TcArgs a, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_q) {
@@ -305,9 +346,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   constexpr int RP = 128 / G;                      // rows owned per CTA
   constexpr int RPK = RP < 64 ? RP : 64;           // key rows owned by a key owner
   constexpr int NQO = G >= 2 ? G / 2 : 0;          // owners of query rows only
-  constexpr int NPT = RP * D / 8 / EPI_THREADS;    // 16-byte chunks reduced per thread
+  constexpr int NPT = RP * D / 8 / XCH_THREADS;    // 16-byte chunks reduced per exchange thread
   constexpr int SWZ = (D / 16 < 8 ? D / 16 : 8) - 1; // chunk swizzle mask of a half row
-  static_assert(NPT >= 1 && RP * D / 8 % EPI_THREADS == 0, "reduce split");
+  static_assert(NPT >= 1 && RP * D / 8 % XCH_THREADS == 0, "reduce split");
+  static_assert(CPT == 16, "epilogue column split");
   constexpr int NSIG = 2 * G * (RP >= 32 ? RP / 32 : 1);   // row pushes a CTA receives per chunk
   constexpr int NKO = RP >= C ? 1 : C / RP;                 // CTAs owning key rows
   constexpr uint32_t XDEST = 2 * 128 * D;                   // bytes of one receive buffer
@@ -387,42 +429,39 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int row = 32 * q + lane;                     // TMEM lane of this thread
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     // TMEM-resident state: lane d, columns [W | S] of the slice; this thread
-    // holds hidden units 32 h .. 32 h + 31 of row d.
+    // holds hidden units CPT h .. CPT h + CPT - 1 of row d.
     //   t_s2: W2[d][64 j + n] (n < 64), S2 at n + 64
     //   t_s1: W1[64 j + n][d] (n < 64), S1 at n + 64
     if (row < D) {
-      float w[32], sv[32];
-      const long long g2 = (long long)Hd * D + (long long)row * Hd + HS * j + 32 * h;
+      float w[CPT], sv[CPT];
+      const long long g2 = (long long)Hd * D + (long long)row * Hd + HS * j + CPT * h;
 #pragma unroll
-      for (int i4 = 0; i4 < 8; ++i4) {
+      for (int i4 = 0; i4 < CPT / 4; ++i4) {
         const float4 a4 = *reinterpret_cast<const float4 *>(W0g + g2 + 4 * i4);
         const float4 b4 = *reinterpret_cast<const float4 *>(S0g + g2 + 4 * i4);
         w[4 * i4] = a4.x; w[4 * i4 + 1] = a4.y; w[4 * i4 + 2] = a4.z; w[4 * i4 + 3] = a4.w;
         sv[4 * i4] = b4.x; sv[4 * i4 + 1] = b4.y; sv[4 * i4 + 2] = b4.z; sv[4 * i4 + 3] = b4.w;
       }
-      tmem_st16(t_s2 + lane_base + 32 * h, *reinterpret_cast<float(*)[16]>(&w[0]));
-      tmem_st16(t_s2 + lane_base + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&w[16]));
-      tmem_st16(t_s2 + lane_base + 64 + 32 * h, *reinterpret_cast<float(*)[16]>(&sv[0]));
-      tmem_st16(t_s2 + lane_base + 64 + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&sv[16]));
+      tmem_st16(t_s2 + lane_base + CPT * h, w);
+      tmem_st16(t_s2 + lane_base + 64 + CPT * h, sv);
 #pragma unroll
-      for (int k8 = 0; k8 < 4; ++k8)
-        st_shared_v4(sbase + Lay::W2 + rb_chunk(D, row, 4 * h + k8), pack8(&w[8 * k8]));
+      for (int k8 = 0; k8 < CPT / 8; ++k8)
+        st_shared_v4(sbase + Lay::W2 + rb_chunk(D, row, (CPT / 8) * h + k8), pack8(&w[8 * k8]));
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const long long g1 = (long long)(HS * j + 32 * h + i) * D + row;
+      for (int i = 0; i < CPT; ++i) {
+        const long long g1 = (long long)(HS * j + CPT * h + i) * D + row;
         w[i] = W0g[g1];
         sv[i] = S0g[g1];
       }
-      tmem_st16(t_s1 + lane_base + 32 * h, *reinterpret_cast<float(*)[16]>(&w[0]));
-      tmem_st16(t_s1 + lane_base + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&w[16]));
-      tmem_st16(t_s1 + lane_base + 64 + 32 * h, *reinterpret_cast<float(*)[16]>(&sv[0]));
-      tmem_st16(t_s1 + lane_base + 64 + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&sv[16]));
+      tmem_st16(t_s1 + lane_base + CPT * h, w);
+      tmem_st16(t_s1 + lane_base + 64 + CPT * h, sv);
 #pragma unroll
-      for (int k8 = 0; k8 < 4; ++k8)
-        st_shared_v4(sbase + Lay::W1 + rb_chunk(D, row, 4 * h + k8), pack8(&w[8 * k8]));
+      for (int k8 = 0; k8 < CPT / 8; ++k8)
+        st_shared_v4(sbase + Lay::W1 + rb_chunk(D, row, (CPT / 8) * h + k8), pack8(&w[8 * k8]));
       tmem_wait_st();
     }
     warp_arrive_local(&bars[B_UPD], lane);
+    float sig_prev = 1.f;                              // S_tmem = sig_prev S (S0 loaded as is)
 
     for (int cch = 0; cch < nchunks; ++cch) {
       const uint32_t par = cch & 1;
@@ -432,32 +471,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       uint4 vv[NPT];
 #pragma unroll
       for (int i = 0; i < NPT; ++i) {
-        const int k = tid + i * EPI_THREADS, gr = (int)j * RP + k / (D / 8), c = k % (D / 8);
-        if (gr < C) vv[i] = *reinterpret_cast<const uint4 *>(a.v + (tb + gr) * D + 8 * c);
+        const int k = tid + i * XCH_THREADS, gr = (int)j * RP + k / (D / 8), c = k % (D / 8);
+        if (tid < XCH_THREADS && gr < C) vv[i] = *reinterpret_cast<const uint4 *>(a.v + (tb + gr) * D + 8 * c);
       }
       if (!wait_bar(&bars[B_COEF], par, a, abort_flag)) break;
       const Coefs &cf = coefs[par];
       // -------- A7, first half: W <- B W + c_S S, S <- A S in TMEM. Runs while
-      // F1 executes; the accumulating contractions later add the writes.
+      // F1 executes; the accumulating contractions later add the writes. S
+      // moves from the previous chunk's scale to this chunk's (exact: powers of
+      // two).
+      const float sig = cf.sig, inv_prev = 1.f / sig_prev;
+      const float cS_t = cf.cS * inv_prev, As_t = cf.As * (sig * inv_prev);
+      sig_prev = sig;
       if (row < D) {
 #pragma unroll
         for (int layer = 0; layer < 2; ++layer) {
-          const uint32_t ts = (layer ? t_s1 : t_s2) + lane_base + 32 * h;
-          float w[32], sv[32];
-          tmem_ld16(ts, *reinterpret_cast<float(*)[16]>(&w[0]));
-          tmem_ld16(ts + 16, *reinterpret_cast<float(*)[16]>(&w[16]));
-          tmem_ld16(ts + 64, *reinterpret_cast<float(*)[16]>(&sv[0]));
-          tmem_ld16(ts + 80, *reinterpret_cast<float(*)[16]>(&sv[16]));
+          const uint32_t ts = (layer ? t_s1 : t_s2) + lane_base + CPT * h;
+          float w[CPT], sv[CPT];
+          tmem_ld16(ts, w);
+          tmem_ld16(ts + 64, sv);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            w[i] = cf.Bw * w[i] + cf.cS * sv[i];
-            sv[i] = cf.As * sv[i];
+          for (int i = 0; i < CPT; ++i) {
+            w[i] = cf.Bw * w[i] + cS_t * sv[i];
+            sv[i] = As_t * sv[i];
           }
-          tmem_st16(ts, *reinterpret_cast<float(*)[16]>(&w[0]));
-          tmem_st16(ts + 16, *reinterpret_cast<float(*)[16]>(&w[16]));
-          tmem_st16(ts + 64, *reinterpret_cast<float(*)[16]>(&sv[0]));
-          tmem_st16(ts + 80, *reinterpret_cast<float(*)[16]>(&sv[16]));
+          tmem_st16(ts, w);
+          tmem_st16(ts + 64, sv);
         }
         tmem_wait_st();
       }
@@ -465,35 +505,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (!wait_bar(&bars[B_F1], par, a, abort_flag)) break;
       tc_fence_after();
       {
-        float z[32];
-        tmem_ld16(t_z1 + lane_base + 32 * h, *reinterpret_cast<float(*)[16]>(&z[0]));
-        tmem_ld16(t_z1 + lane_base + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&z[16]));
+        float z[CPT];
+        tmem_ld16(t_z1 + lane_base + CPT * h, z);
         tmem_wait_ld();
-        float x[32];
+        float x[CPT];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] = z[i] * sigm(z[i]);
+        for (int i = 0; i < CPT; ++i) x[i] = z[i] * sigm(z[i]);
 #pragma unroll
-        for (int k8 = 0; k8 < 4; ++k8)
-          st_shared_v4(sbase + Lay::X1 + rb_chunk(128, row, 4 * h + k8), pack8(&x[8 * k8]));
+        for (int k8 = 0; k8 < CPT / 8; ++k8)
+          st_shared_v4(sbase + Lay::X1 + rb_chunk(128, row, (CPT / 8) * h + k8), pack8(&x[8 * k8]));
         // X1 feeds the next MMA: publish it first
         warp_arrive_local(&bars[B_X1], lane);
         // the scaled copies are only needed by the W2 update, much later (they
         // reach the tensor cores through the fence of the B_G2OWN arrival)
         if (row < C) {
-          const float ci = -cf.c[row], ei = -cf.e[row];
+          const float ci = -cf.c[row], ei = -cf.e[row] * sig;
           float s8[8];
 #pragma unroll
-          for (int k8 = 0; k8 < 4; ++k8) {
+          for (int k8 = 0; k8 < CPT / 8; ++k8) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) s8[i] = ci * x[8 * k8 + i];
-            st_shared_v4(sbase + Lay::X1S + rb_chunk(64, row, 4 * h + k8), pack8(s8));
+            st_shared_v4(sbase + Lay::X1S + rb_chunk(64, row, (CPT / 8) * h + k8), pack8(s8));
 #pragma unroll
             for (int i = 0; i < 8; ++i) s8[i] = ei * x[8 * k8 + i];
-            st_shared_v4(sbase + Lay::X1S + rb_chunk(64, row, 8 + 4 * h + k8), pack8(s8));
+            st_shared_v4(sbase + Lay::X1S + rb_chunk(64, row, 8 + (CPT / 8) * h + k8), pack8(s8));
           }
         }
       }
-      // -------- E2: stage this CTA's partial Z2 as bf16, [half][row][d/2]
+      // -------- E2: stage this CTA's partial Z2 as fp16, [half][row][d/2]
       // (16-byte chunk index XOR row), and let each warp bulk-copy the rows it
       // staged into their owners' receive buffers (reduce-scatter by rows:
       // CTA p owns rows [RP p, RP p + RP)).
@@ -506,56 +545,71 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // (The global exchange double-buffers by chunk parity instead: a peer
       // writes chunk c+2 only after this CTA's push of chunk c+1, which
       // follows its reads of chunk c.)
-      if (!XG && NQO > 0 && q >= 2 && cch > 0 &&
+      // Only the first XCH_WARPS warps (column halves h = 0, 1) stage and push.
+      if (!XG && NQO > 0 && warp < XCH_WARPS && q >= 2 && cch > 0 &&
           !wait_bar(&bars[B_QFREE], (uint32_t)((cch - 1) & 1), a, abort_flag, true))
         break;
-      {
+      if (warp < XCH_WARPS) {
         constexpr int HALF = D / 2;                    // columns of Z2 per thread
-        float z[HALF];
+        if constexpr (!XG) {
+          // each 16-byte piece goes straight into the owner's receive buffer
+          // (row rin of this CTA's block, half h), counted on its B_RECV
+          const int p = row / RP, rin = row - p * RP;
+          const uint32_t rrow = mapa(sbase + Lay::RECV + (uint32_t)(j * 2 * RP * D + h * RP * D + rin * D), (uint32_t)p);
+          const uint32_t rbar = mapa(smem_u32(&bars[B_RECV]), (uint32_t)p);
 #pragma unroll
-        for (int c16 = 0; c16 < HALF / 16; ++c16)
-          tmem_ld16(t_z2 + lane_base + HALF * h + 16 * c16, *reinterpret_cast<float(*)[16]>(&z[16 * c16]));
-        tmem_wait_ld();
-        const uint32_t srow = sbase + Lay::SEND + (uint32_t)(h * 128 * D + row * D);
+          for (int c16 = 0; c16 < HALF / 16; ++c16) {
+            float z[16];
+            tmem_ld16(t_z2 + lane_base + HALF * h + 16 * c16, z);
+            tmem_wait_ld();
 #pragma unroll
-        for (int k8 = 0; k8 < HALF / 8; ++k8)
-          st_shared_v4(srow + (uint32_t)((k8 ^ (row & SWZ)) << 4), pack8(&z[8 * k8]));
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          constexpr int RPP = RP < 32 ? RP : 32;       // rows per push
-#pragma unroll
-          for (int i = 0; i < 32 / RPP; ++i) {
-            const int r0 = 32 * q + i * RPP, p = r0 / RP, rin = r0 - p * RP;
-            const uint32_t off = (uint32_t)(j * 2 * RP * D + h * RP * D + rin * D);
-            const uint32_t src = sbase + Lay::SEND + (uint32_t)(h * 128 * D + r0 * D);
-            if constexpr (XG)
-              bulk_store_global(xrv + (size_t)(p * 2 + (int)par) * XDEST + off, src, (uint32_t)(RPP * D));
-            else
-              bulk_push(mapa(sbase + Lay::RECV + off, (uint32_t)p), src, (uint32_t)(RPP * D),
-                        mapa(smem_u32(&bars[B_RECV]), (uint32_t)p));
+            for (int k8 = 0; k8 < 2; ++k8)
+              st_async_v4(rrow + (uint32_t)(((2 * c16 + k8) ^ (row & SWZ)) << 4), pack8(&z[8 * k8]), rbar);
           }
-          if constexpr (XG) {
+          tc_fence_before();
+        } else {
+          const uint32_t srow = sbase + Lay::SEND + (uint32_t)(h * 128 * D + row * D);
+#pragma unroll
+          for (int c16 = 0; c16 < HALF / 16; ++c16) {
+            float z[16];
+            tmem_ld16(t_z2 + lane_base + HALF * h + 16 * c16, z);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k8 = 0; k8 < 2; ++k8)
+              st_shared_v4(srow + (uint32_t)(((2 * c16 + k8) ^ (row & SWZ)) << 4), pack8(&z[8 * k8]));
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            constexpr int RPP = RP < 32 ? RP : 32;       // rows per push
+#pragma unroll
+            for (int i = 0; i < 32 / RPP; ++i) {
+              const int r0 = 32 * q + i * RPP, p = r0 / RP, rin = r0 - p * RP;
+              const uint32_t off = (uint32_t)(j * 2 * RP * D + h * RP * D + rin * D);
+              const uint32_t src = sbase + Lay::SEND + (uint32_t)(h * 128 * D + r0 * D);
+              bulk_store_global(xrv + (size_t)(p * 2 + (int)par) * XDEST + off, src, (uint32_t)(RPP * D));
+            }
             // the rows are in global memory before the owners are told
             bulk_commit_and_wait();
             fence_proxy_async_global();
 #pragma unroll
             for (int i = 0; i < 32 / RPP; ++i) red_release_add(xfl + ((32 * q + i * RPP) / RP) * XFLAG_STRIDE, 1u);
           }
+          __syncwarp();
         }
-        __syncwarp();
       }
       // -------- reduce my rows over the G partials (fp32 sums, fixed order):
       // y for query rows, G2 = 2 (Z2 - V) for key rows (A3)
       if (XG ? !wait_flag(xfl + j * XFLAG_STRIDE, (unsigned)(NSIG * (cch + 1)), a, abort_flag)
-             : !wait_bar(&bars[B_RECV], par, a, abort_flag))
+             : !wait_bar(&bars[B_RECV], par, a, abort_flag, true))
         break;
       {
         float acc[NPT][8];
 #pragma unroll
         for (int i = 0; i < NPT; ++i) {
-          const int k = tid + i * EPI_THREADS, r = k / (D / 8), c = k % (D / 8);
+          if (tid >= XCH_THREADS) break;
+          const int k = tid + i * XCH_THREADS, r = k / (D / 8), c = k % (D / 8);
           uint4 pv[G];
 #pragma unroll
           for (int s2 = 0; s2 < G; ++s2) {
@@ -570,9 +624,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
 #pragma unroll
           for (int s2 = 0; s2 < G; ++s2) {
-            const __nv_bfloat16 *pb = reinterpret_cast<const __nv_bfloat16 *>(&pv[s2]);
+            const __half *pb = reinterpret_cast<const __half *>(&pv[s2]);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[i][e] += __bfloat162float(pb[e]);
+            for (int e = 0; e < 8; ++e) acc[i][e] += __half2float(pb[e]);
           }
           const int gr = (int)j * RP + r;
           if (gr < C) {
@@ -580,14 +634,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             float g[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) g[e] = 2.f * (acc[i][e] - __bfloat162float(vb[e]));
-            st_shared_v4(sbase + Lay::G2OWN + rb_chunk(RPK, r, c), pack8(g));
+            if constexpr (XG) {
+              st_shared_v4(sbase + Lay::G2OWN + rb_chunk(RPK, r, c), pack8(g));
+            } else {
+              // all-gather: the chunk goes to the G2 tile of every CTA of
+              // the cluster (this one included), counted on its B_G2
+              const uint4 gv = pack8(g);
+              const uint32_t loc = sbase + Lay::G2 + rb_chunk(64, gr, c);
+#pragma unroll
+              for (int i2 = 0; i2 < G; ++i2) {
+                const uint32_t pc = (j + (uint32_t)i2) % G;
+                st_async_v4(mapa(loc, pc), gv, mapa(smem_u32(&bars[B_G2]), pc));
+              }
+            }
           }
         }
         warp_arrive_local(&bars[B_G2OWN], lane);
         // reads y of my query rows
 #pragma unroll
         for (int i = 0; i < NPT; ++i) {
-          const int k = tid + i * EPI_THREADS, r = k / (D / 8), c = k % (D / 8);
+          if (tid >= XCH_THREADS) break;
+          const int k = tid + i * XCH_THREADS, r = k / (D / 8), c = k % (D / 8);
           const int gr = (int)j * RP + r;
           if (gr >= C) {
             float *yp = a.y + (tb + (gr - C)) * D + 8 * c;
@@ -600,84 +667,80 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (!wait_bar(&bars[B_B1], par, a, abort_flag)) break;
       tc_fence_after();
       if (row < C) {
-        float gp[32], z[32];
-        tmem_ld16(t_g1 + lane_base + 32 * h, *reinterpret_cast<float(*)[16]>(&gp[0]));
-        tmem_ld16(t_g1 + lane_base + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&gp[16]));
-        tmem_ld16(t_z1 + lane_base + 32 * h, *reinterpret_cast<float(*)[16]>(&z[0]));
-        tmem_ld16(t_z1 + lane_base + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&z[16]));
+        float gp[CPT], z[CPT];
+        tmem_ld16(t_g1 + lane_base + CPT * h, gp);
+        tmem_ld16(t_z1 + lane_base + CPT * h, z);
         tmem_wait_ld();
-        const float ci = -cf.c[row], ei = -cf.e[row];
-        float g1[32];
+        const float ci = -cf.c[row], ei = -cf.e[row] * sig;
+        float g1[CPT];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
+        for (int i = 0; i < CPT; ++i) {
           const float s = sigm(z[i]);
           g1[i] = gp[i] * (s * (1.f + z[i] * (1.f - s)));
         }
         float s8[8];
 #pragma unroll
-        for (int k8 = 0; k8 < 4; ++k8) {
+        for (int k8 = 0; k8 < CPT / 8; ++k8) {
 #pragma unroll
           for (int i = 0; i < 8; ++i) s8[i] = ci * g1[8 * k8 + i];
-          st_shared_v4(sbase + Lay::G1S + rb_chunk(64, row, 4 * h + k8), pack8(s8));
+          st_shared_v4(sbase + Lay::G1S + rb_chunk(64, row, (CPT / 8) * h + k8), pack8(s8));
 #pragma unroll
           for (int i = 0; i < 8; ++i) s8[i] = ei * g1[8 * k8 + i];
-          st_shared_v4(sbase + Lay::G1S + rb_chunk(64, row, 8 + 4 * h + k8), pack8(s8));
+          st_shared_v4(sbase + Lay::G1S + rb_chunk(64, row, 8 + (CPT / 8) * h + k8), pack8(s8));
         }
       }
       warp_arrive_local(&bars[B_G1], lane);
-      // -------- A7, second half: the bf16 copies of W2' and W1' for the next chunk
+      // -------- A7, second half: the fp16 copies of W2' and W1' for the next chunk
       if (!wait_bar(&bars[B_U2], par, a, abort_flag)) break;
       tc_fence_after();
       if (row < D) {
-        float w[32];
-        tmem_ld16(t_s2 + lane_base + 32 * h, *reinterpret_cast<float(*)[16]>(&w[0]));
-        tmem_ld16(t_s2 + lane_base + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&w[16]));
+        float w[CPT];
+        tmem_ld16(t_s2 + lane_base + CPT * h, w);
         tmem_wait_ld();
 #pragma unroll
-        for (int k8 = 0; k8 < 4; ++k8)
-          st_shared_v4(sbase + Lay::W2 + rb_chunk(D, row, 4 * h + k8), pack8(&w[8 * k8]));
+        for (int k8 = 0; k8 < CPT / 8; ++k8)
+          st_shared_v4(sbase + Lay::W2 + rb_chunk(D, row, (CPT / 8) * h + k8), pack8(&w[8 * k8]));
       }
       if (!wait_bar(&bars[B_U1], par, a, abort_flag)) break;
       tc_fence_after();
       if (row < D) {
-        float w[32];
-        tmem_ld16(t_s1 + lane_base + 32 * h, *reinterpret_cast<float(*)[16]>(&w[0]));
-        tmem_ld16(t_s1 + lane_base + 32 * h + 16, *reinterpret_cast<float(*)[16]>(&w[16]));
+        float w[CPT];
+        tmem_ld16(t_s1 + lane_base + CPT * h, w);
         tmem_wait_ld();
 #pragma unroll
-        for (int k8 = 0; k8 < 4; ++k8)
-          st_shared_v4(sbase + Lay::W1 + rb_chunk(D, row, 4 * h + k8), pack8(&w[8 * k8]));
+        for (int k8 = 0; k8 < CPT / 8; ++k8)
+          st_shared_v4(sbase + Lay::W1 + rb_chunk(D, row, (CPT / 8) * h + k8), pack8(&w[8 * k8]));
       }
       warp_arrive_local(&bars[B_UPD], lane);
     }
     // -------- W_end, S_end: write the TMEM-resident state back once
     if (!*abort_flag && row < D) {
       tc_fence_after();
-      float w[32], sv[32];
+      float w[CPT], sv[CPT];
+      const float inv_sig = 1.f / sig_prev;            // S_tmem = sig S of the last chunk
       {
-        const uint32_t ts = t_s2 + lane_base + 32 * h;
-        tmem_ld16(ts, *reinterpret_cast<float(*)[16]>(&w[0]));
-        tmem_ld16(ts + 16, *reinterpret_cast<float(*)[16]>(&w[16]));
-        tmem_ld16(ts + 64, *reinterpret_cast<float(*)[16]>(&sv[0]));
-        tmem_ld16(ts + 80, *reinterpret_cast<float(*)[16]>(&sv[16]));
+        const uint32_t ts = t_s2 + lane_base + CPT * h;
+        tmem_ld16(ts, w);
+        tmem_ld16(ts + 64, sv);
         tmem_wait_ld();
-        const long long g2 = (long long)Hd * D + (long long)row * Hd + HS * j + 32 * h;
 #pragma unroll
-        for (int i4 = 0; i4 < 8; ++i4) {
+        for (int i = 0; i < CPT; ++i) sv[i] *= inv_sig;
+        const long long g2 = (long long)Hd * D + (long long)row * Hd + HS * j + CPT * h;
+#pragma unroll
+        for (int i4 = 0; i4 < CPT / 4; ++i4) {
           *reinterpret_cast<float4 *>(Wg + g2 + 4 * i4) = make_float4(w[4 * i4], w[4 * i4 + 1], w[4 * i4 + 2], w[4 * i4 + 3]);
           *reinterpret_cast<float4 *>(Sg + g2 + 4 * i4) = make_float4(sv[4 * i4], sv[4 * i4 + 1], sv[4 * i4 + 2], sv[4 * i4 + 3]);
         }
       }
       {
-        const uint32_t ts = t_s1 + lane_base + 32 * h;
-        tmem_ld16(ts, *reinterpret_cast<float(*)[16]>(&w[0]));
-        tmem_ld16(ts + 16, *reinterpret_cast<float(*)[16]>(&w[16]));
-        tmem_ld16(ts + 64, *reinterpret_cast<float(*)[16]>(&sv[0]));
-        tmem_ld16(ts + 80, *reinterpret_cast<float(*)[16]>(&sv[16]));
+        const uint32_t ts = t_s1 + lane_base + CPT * h;
+        tmem_ld16(ts, w);
+        tmem_ld16(ts + 64, sv);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const long long g1 = (long long)(HS * j + 32 * h + i) * D + row;
+        for (int i = 0; i < CPT; ++i) {
+          sv[i] *= inv_sig;
+          const long long g1 = (long long)(HS * j + CPT * h + i) * D + row;
           Wg[g1] = w[i];
           Sg[g1] = sv[i];
         }
@@ -685,10 +748,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   } else {
     // ---------------------------------------------------------------- control warp
-    const uint32_t i_f1 = idesc_bf16(128, 64, false, true);
-    const uint32_t i_f2 = idesc_bf16(128, D, false, false);
-    const uint32_t i_b1 = idesc_bf16(128, 64, false, true);
-    const uint32_t i_dw = idesc_bf16(128, 128, true, true);
+    const uint32_t i_f1 = idesc_f16(128, 64, false, true);
+    const uint32_t i_f2 = idesc_f16(128, D, false, false);
+    const uint32_t i_b1 = idesc_f16(128, 64, false, true);
+    const uint32_t i_dw = idesc_f16(128, 128, true, true);
     const uint32_t xkq = sbase + Lay::XKQ, x1 = sbase + Lay::X1, x1s = sbase + Lay::X1S;
     const uint32_t g2 = sbase + Lay::G2, g1s = sbase + Lay::G1S;
     const uint32_t w1 = sbase + Lay::W1, w2 = sbase + Lay::W2;
@@ -737,7 +800,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (lane == 0) {
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
-          umma_bf16(t_z1, desc_kmajor(xkq, 128, ks), desc_mnmajor(w1, D, ks), i_f1, ks > 0);
+          umma_f16(t_z1, desc_kmajor(xkq, 128, ks), desc_mnmajor(w1, D, ks), i_f1, ks > 0);
         umma_commit(&bars[B_F1]);
       }
       __syncwarp();
@@ -746,7 +809,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (lane == 0) {
 #pragma unroll
         for (int ks = 0; ks < HS / 16; ++ks)
-          umma_bf16(t_z2, desc_kmajor(x1, 128, ks), desc_kmajor(w2, D, ks), i_f2, ks > 0);
+          umma_f16(t_z2, desc_kmajor(x1, 128, ks), desc_kmajor(w2, D, ks), i_f2, ks > 0);
         umma_commit(&bars[B_F2]);
       }
       __syncwarp();
@@ -754,9 +817,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // after B_X1: the epilogue has then consumed this chunk's B_COEF phase,
       // so B_COEF can never run two phases ahead of its waiters.
       if (cch + 1 < nchunks) scan(cch + 1);
-      // all-gather of G2: key owners push their rows (whole 1 KB swizzle
-      // atoms) to every CTA; query owners report that they are done reading
-      // their receive buffer (B_QFREE, off the critical path).
+      // all-gather of G2: in the cluster form the reduce threads have sent
+      // their G2 pieces to every CTA themselves; query owners report here
+      // that they are done reading their receive buffer (B_QFREE, off the
+      // critical path). The global form writes its G2 rows out here.
       if (!wait_bar(&bars[B_G2OWN], par, a, abort_flag)) break;
       if (lane == 0) {
         if ((int)j * RP < C && XG) {
@@ -768,17 +832,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           bulk_commit_and_wait();
           fence_proxy_async_global();
           red_release_add(xfl + G * XFLAG_STRIDE, 1u);
-        } else if ((int)j * RP < C) {
-#pragma unroll
-          for (int i = 0; i < G; ++i) {
-            const uint32_t p = (j + (uint32_t)i) % G;
-#pragma unroll
-            for (int fb = 0; fb < D / 64; ++fb)
-              bulk_push(mapa(sbase + Lay::G2 + (uint32_t)(fb * 64 * 128) + j * (uint32_t)(RP * 128), p),
-                        sbase + Lay::G2OWN + (uint32_t)(fb * RPK * 128), (uint32_t)(RPK * 128),
-                        mapa(smem_u32(&bars[B_G2]), p));
-          }
-        } else if (!XG) {
+        } else if (!XG && (int)j * RP >= C) {
           // done reading this chunk's receive buffer: query rows of the next
           // chunk may be pushed here
 #pragma unroll
@@ -806,12 +860,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // A4: G1 pre-activation gradient = G2 W2_j
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
-          umma_bf16(t_g1, desc_kmajor(g2, 64, ks), desc_mnmajor(w2, D, ks), i_b1, ks > 0);
+          umma_f16(t_g1, desc_kmajor(g2, 64, ks), desc_mnmajor(w2, D, ks), i_b1, ks > 0);
         umma_commit(&bars[B_B1]);
         // A6+A7 for W2: [W2 | S2] += G2^T [-c X1_K | -e X1_K] onto the pre-scaled state
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks)
-          umma_bf16(t_s2, desc_mnmajor(g2, 64, ks), desc_mnmajor(x1s, 64, ks), i_dw, 1);
+          umma_f16(t_s2, desc_mnmajor(g2, 64, ks), desc_mnmajor(x1s, 64, ks), i_dw, 1);
         umma_commit(&bars[B_U2]);
       }
       __syncwarp();
@@ -821,7 +875,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // A6+A7 for W1: [W1 | S1]^T += K^T [-c G1 | -e G1] onto the pre-scaled state
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks)
-          umma_bf16(t_s1, desc_mnmajor(xkq, 128, ks), desc_mnmajor(g1s, 64, ks), i_dw, 1);
+          umma_f16(t_s1, desc_mnmajor(xkq, 128, ks), desc_mnmajor(g1s, 64, ks), i_dw, 1);
         umma_commit(&bars[B_U1]);
       }
       __syncwarp();
@@ -871,7 +925,8 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D map over [rows x d] bf16 tokens, box = 64 features x 64 tokens, 128B swizzle.
+// 2-D map over [rows x d] fp16 tokens (the converted keys or queries), box =
+// 64 features x 64 tokens, 128B swizzle.
 bool make_token_map(CUtensorMap *map, const void *base, long long rows, int d) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
@@ -880,7 +935,7 @@ bool make_token_map(CUtensorMap *map, const void *base, long long rows, int d) {
   cuuint64_t strides[1] = {(cuuint64_t)d * 2};
   cuuint32_t box[2] = {64, (cuuint32_t)C};
   cuuint32_t es[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1044,8 +1099,8 @@ cudaError_t launch_both(const Problem &p, cudaStream_t stream, int nc, int nx, u
   // streams [s0, s0 + n) of the problem
   auto run = [&](int s0, int n, bool xg, bool after) -> cudaError_t {
     CUtensorMap mk, mq;
-    const __nv_bfloat16 *k = static_cast<const __nv_bfloat16 *>(p.k) + (size_t)s0 * td;
-    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(p.q) + (size_t)s0 * td;
+    const __half *k = static_cast<const __half *>(p.k16) + (size_t)s0 * td;
+    const __half *q = static_cast<const __half *>(p.q16) + (size_t)s0 * td;
     if (!make_token_map(&mk, k, (long long)n * p.T, D) || !make_token_map(&mq, q, (long long)n * p.T, D))
       return cudaErrorInvalidValue;
     TcArgs a = base;

@@ -9,7 +9,7 @@
 //   backward   l = L..2  G_{l-1} = (G_l W_l) . silu'(Z_{l-1})
 //   update     l = 1..L  [U_W | U_S] = [-c G_l | -e G_l]^T X_{l-1}, epilogue
 //              W' = B W + c_S S + U_W, S' = A S + U_S (fp32 state in the
-//              caller's W_end / S_end) and the bf16 copy of W' for the next chunk
+//              caller's W_end / S_end) and the fp16 copy of W' for the next chunk
 // ("Titans, explained" steps 2-6; "Attack of the Titans", "Parallel
 //  training"). Launch order on one stream orders the phases. For widths up to
 // 256 one fused kernel runs a tile's whole forward and backward; wider layers
@@ -19,6 +19,7 @@
 // tiles are independent (batched over streams).
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <cstdlib>
 #include <cstring>
@@ -32,9 +33,15 @@ namespace {
 
 using namespace sm100;
 
+// Operand format of every contraction: fp16 (10 mantissa bits), fp32
+// accumulation. The keys and queries arrive as bf16 and are converted to fp16
+// once per call; the weight copies, activations, silu' and gradients the
+// kernels exchange are fp16. Values stay bf16 (read by the epilogues only).
+using op_t = __half;
+
 constexpr int NT = 256;          // 8 warps: warp w reads TMEM lanes 32 (w % 4) .. +31,
                                  // columns half w / 4 of the tile
-constexpr int KB = 64;           // K block (one 128-byte swizzle atom of bf16)
+constexpr int KB = 64;           // K block (one 128-byte swizzle atom of 2-byte elements)
 
 enum Kind { K_FWD = 0, K_FWD_LAST = 1, K_BWD = 2 };
 
@@ -47,10 +54,10 @@ struct GemmArgs {
   int b_rows_per_stream;
   int a_split_kq;                // layer-1 forward: rows < C from k, else from q
   // epilogue operands
-  __nv_bfloat16 *x_out;          // [streams, 2C, n] activations (forward)
-  __nv_bfloat16 *sp_out;         // [streams, C, n] silu'(Z) of key rows (forward)
-  const __nv_bfloat16 *sp_in;    // [streams, C, n] silu' of the layer below (backward)
-  __nv_bfloat16 *g_out, *gc_out, *ge_out;  // [streams, C, n] G, -c G, -e G
+  op_t *x_out;                   // [streams, 2C, n] activations (forward)
+  op_t *sp_out;                  // [streams, C, n] silu'(Z) of key rows (forward)
+  const op_t *sp_in;             // [streams, C, n] silu' of the layer below (backward)
+  op_t *g_out, *gc_out, *ge_out; // [streams, C, n] G, -c G, -e G
   float *y;                      // [streams, T, d] reads (last forward)
   const __nv_bfloat16 *v;        // [streams, T, d] values (last forward)
   const float *coef;             // [streams, T, 2] (c, e) per token
@@ -66,13 +73,14 @@ __device__ __forceinline__ float tanh_approx(float x) {
 }
 __device__ __forceinline__ float sigm(float z) { return fmaf(0.5f, tanh_approx(0.5f * z), 0.5f); }
 
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+// Two fp32 values as one fp16 pair (round to nearest even).
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t *>(&h);
 }
 __device__ __forceinline__ uint4 pack8(const float *v) {
-  return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
-                    pack_bf16(v[6], v[7]));
+  return make_uint4(pack_h2(v[0], v[1]), pack_h2(v[2], v[3]), pack_h2(v[4], v[5]),
+                    pack_h2(v[6], v[7]));
 }
 
 __device__ bool wait_b(uint64_t *bar, uint32_t par, const GemmArgs &a) {
@@ -165,8 +173,8 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
     if (a.inject) ok = injected_wait(&never, a.status, a.wait_ns);
     const uint32_t tx = (uint32_t)(A_BYTES + (uint32_t)a.N * KB * 2);
     uint32_t idesc;
-    if (kind == K_BWD) idesc = idesc_bf16(128, a.N, false, true);
-    else idesc = idesc_bf16(128, a.N, false, false);
+    if (kind == K_BWD) idesc = idesc_f16(128, a.N, false, true);
+    else idesc = idesc_f16(128, a.N, false, false);
     for (int kb = 0; kb < nk && kb < STAGES && ok; ++kb) {
       mbar_arrive_expect_tx(&full[kb], tx);
       load_stage(a, &mA, &mA2, &mB, sm + kb * STAGE_BYTES, &full[kb], s, mt, nt, kb);
@@ -179,10 +187,10 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
       const uint32_t base = smem_u32(sm + st * STAGE_BYTES);
       for (int ks = 0; ks < KB / 16; ++ks) {
         if (kind == K_BWD) {
-          umma_bf16(tm, desc_kmajor(base, 128, ks), desc_mnmajor(base + A_BYTES, 64, ks), idesc,
+          umma_f16(tm, desc_kmajor(base, 128, ks), desc_mnmajor(base + A_BYTES, 64, ks), idesc,
                     (kb | ks) != 0);
         } else {
-          umma_bf16(tm, desc_kmajor(base, 128, ks), desc_kmajor(base + A_BYTES, a.N, ks), idesc,
+          umma_f16(tm, desc_kmajor(base, 128, ks), desc_kmajor(base + A_BYTES, a.N, ks), idesc,
                     (kb | ks) != 0);
         }
       }
@@ -226,11 +234,11 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
             x[i] = z[i] * sg;
             sp[i] = sg * (1.f + z[i] * (1.f - sg));
           }
-          __nv_bfloat16 *xo = a.x_out + ((long long)s * 2 * a.C + r) * a.n_out + col;
+          op_t *xo = a.x_out + ((long long)s * 2 * a.C + r) * a.n_out + col;
           *reinterpret_cast<uint4 *>(xo) = pack8(x);
           *reinterpret_cast<uint4 *>(xo + 8) = pack8(x + 8);
           if (key) {
-            __nv_bfloat16 *so = a.sp_out + ((long long)s * a.C + r) * a.n_out + col;
+            op_t *so = a.sp_out + ((long long)s * a.C + r) * a.n_out + col;
             *reinterpret_cast<uint4 *>(so) = pack8(sp);
             *reinterpret_cast<uint4 *>(so + 8) = pack8(sp + 8);
           }
@@ -255,15 +263,15 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
               g[8 + i] = 2.f * (z[8 + i] - __bfloat162float(vb1[i]));
             }
           } else {
-            const __nv_bfloat16 *spi = a.sp_in + ((long long)s * a.C + r) * a.n_out + col;
+            const op_t *spi = a.sp_in + ((long long)s * a.C + r) * a.n_out + col;
             const uint4 s0 = *reinterpret_cast<const uint4 *>(spi);
             const uint4 s1 = *reinterpret_cast<const uint4 *>(spi + 8);
-            const __nv_bfloat16 *sb0 = reinterpret_cast<const __nv_bfloat16 *>(&s0);
-            const __nv_bfloat16 *sb1 = reinterpret_cast<const __nv_bfloat16 *>(&s1);
+            const op_t *sb0 = reinterpret_cast<const op_t *>(&s0);
+            const op_t *sb1 = reinterpret_cast<const op_t *>(&s1);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              g[i] = z[i] * __bfloat162float(sb0[i]);
-              g[8 + i] = z[8 + i] * __bfloat162float(sb1[i]);
+              g[i] = z[i] * __half2float(sb0[i]);
+              g[8 + i] = z[8 + i] * __half2float(sb1[i]);
             }
           }
           const float2 ce = *reinterpret_cast<const float2 *>(a.coef + 2 * tok);
@@ -303,7 +311,7 @@ __global__ void __launch_bounds__(NT, 1)
 // on tcgen05 (A = the MN-major -c G and -e G of the tile's rows, B = the
 // layer's inputs X; accumulators in TMEM columns 0.. and 128..), then
 //   W' = B W + c_S S + U_W,  S' = A S + U_S
-// and the bf16 copy of W' that the next chunk's forward reads.
+// and the fp16 copy of W' that the next chunk's forward reads.
 // The fp32 state tile travels by TMA both ways. Its loads (32-column boxes,
 // 128-byte swizzle) are issued when the CTA starts, beside the contraction's
 // operands: the previous chunk's update of these rows completed before the
@@ -329,9 +337,9 @@ struct UpArgs {
   int inject;                                  // test hook, as in GemmArgs
 };
 struct UpMaps {
-  CUtensorMap a[kMaxL], a2[kMaxL], b[kMaxL];   // -c G_l, -e G_l [S*C, d_l]; X_{l-1} (bf16, 64 x 64 boxes)
+  CUtensorMap a[kMaxL], a2[kMaxL], b[kMaxL];   // -c G_l, -e G_l [S*C, d_l]; X_{l-1} (fp16, 64 x 64 boxes)
   CUtensorMap w[kMaxL], s[kMaxL];              // fp32 W_l, S_l as {cols, rows, stream}, 32-column boxes
-  CUtensorMap wb[kMaxL];                       // bf16 W_l as {cols, rows, stream}, 64-column boxes
+  CUtensorMap wb[kMaxL];                       // fp16 W_l as {cols, rows, stream}, 64-column boxes
 };
 __host__ __device__ constexpr uint32_t up_stage_bytes(int N) { return 2 * A_BYTES + (uint32_t)N * KB * 2; }
 __host__ __device__ constexpr int up_stages(int nk) { return nk <= 2 ? 2 : 3; }
@@ -366,7 +374,7 @@ __global__ void __launch_bounds__(UP_NT, 1)
   const uint32_t SB = up_stage_bytes(N);
   unsigned char *wt = sm + STAGES * SB;        // W tile: N / 32 boxes
   unsigned char *st = wt + (N / 32) * UP_BOX;  // S tile
-  unsigned char *wbt = sm;                     // bf16 W' tile (N / 64 boxes), in the ring once the MMAs are done
+  unsigned char *wbt = sm;                     // fp16 W' tile (N / 64 boxes), in the ring once the MMAs are done
   const int R = ly.M < 128 ? ly.M : 128;       // rows of a box
   const int rows = ly.M - 128 * mt < 128 ? ly.M - 128 * mt : 128;   // rows of this tile
 
@@ -399,7 +407,7 @@ __global__ void __launch_bounds__(UP_NT, 1)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   int issued = 0, consumed = 0;                // operand stages requested / seen complete (thread 0)
   if (tid == 0) {
-    const uint32_t idesc = idesc_bf16(128, N, true, true);
+    const uint32_t idesc = idesc_f16(128, N, true, true);
     auto load = [&](int stg, int kb) {
       unsigned char *d = sm + stg * SB;
       const int row0 = s * a.C + kb * KB;
@@ -425,8 +433,8 @@ __global__ void __launch_bounds__(UP_NT, 1)
       const uint32_t base = smem_u32(sm + stg * SB);
       for (int ks = 0; ks < KB / 16; ++ks) {
         const uint64_t bd = desc_mnmajor(base + 2 * A_BYTES, 64, ks);
-        umma_bf16(tm, desc_mnmajor(base, 64, ks), bd, idesc, (kb | ks) != 0);
-        umma_bf16(tm + 128, desc_mnmajor(base + A_BYTES, 64, ks), bd, idesc, (kb | ks) != 0);
+        umma_f16(tm, desc_mnmajor(base, 64, ks), bd, idesc, (kb | ks) != 0);
+        umma_f16(tm + 128, desc_mnmajor(base + A_BYTES, 64, ks), bd, idesc, (kb | ks) != 0);
       }
       umma_commit(&empty[stg]);
       if (kb + STAGES < nk) {
@@ -461,7 +469,7 @@ __global__ void __launch_bounds__(UP_NT, 1)
       unsigned char *wr = wt + (cg / 32) * UP_BOX + r * 128;
       unsigned char *sr = st + (cg / 32) * UP_BOX + r * 128;
       unsigned char *br = wbt + (cg / 64) * UP_BOX + r * 128;
-      const int c16 = (cg % 64) / 8;           // 16-byte chunk of the bf16 row that column cg starts
+      const int c16 = (cg % 64) / 8;           // 16-byte chunk of the fp16 row that column cg starts
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const uint32_t o = (uint32_t)((j ^ (r & 7)) << 4);
@@ -476,7 +484,7 @@ __global__ void __launch_bounds__(UP_NT, 1)
         *reinterpret_cast<float4 *>(wr + o) = wn;
         *reinterpret_cast<float4 *>(sr + o) = sn;
         const uint32_t ob = (uint32_t)((((c16 + (j >> 1)) ^ (r & 7)) << 4) + (j & 1) * 8);
-        *reinterpret_cast<uint2 *>(br + ob) = make_uint2(pack_bf16(wn.x, wn.y), pack_bf16(wn.z, wn.w));
+        *reinterpret_cast<uint2 *>(br + ob) = make_uint2(pack_h2(wn.x, wn.y), pack_h2(wn.z, wn.w));
       }
     }
   }
@@ -506,23 +514,25 @@ __global__ void __launch_bounds__(UP_NT, 1)
 // The state update of every layer of a chunk, pipelined (chunks of at most 128
 // tokens). One CTA per unit = (layer l, stream, block of 128 rows of W_l, a
 // range of up to `tpu` 64-column tiles). The contraction's A operands, -c G
-// and -e G of the block's rows over the whole chunk (K = C), are loaded once;
-// the column tiles then stream through two shared-memory stages (X columns
-// and the fp32 W and S tiles) and two TMEM accumulator pairs (U_W | U_S), so
-// that tile j + 1's loads and MMAs overlap tile j's update and stores:
-//   warp 0      TMA loads (state tiles first: they do not depend on the
+// and -e G of the block's rows over the whole chunk (K = C), are loaded once.
+// The MMAs run per 64-column tile (X columns in one of two slots, the U_W | U_S
+// accumulators in one of two TMEM pairs); the fp32 W and S stream through four
+// slots of 32-column half tiles, so that up to four half tiles of state are in
+// flight while one is updated and stored:
+//   warp 0      TMA loads (state half tiles first: they do not depend on the
 //               previous kernel; the operands after griddepcontrol.wait)
 //   warp 1      TMEM allocation; MMA issue (M = 128 rows, N = 64, K = C)
-//   warp 2      TMA stores of W', S' and the bf16 W' of a tile, then frees
-//               the stage once the stores have read it
-//   warps 4-11  epilogue: the thread owning TMEM lane r (row r) and one half
-//               of the tile's columns computes W' = B W + c_S S + U_W,
-//               S' = A S + U_S in place and the bf16 W' into the X slot
+//   warp 2      TMA stores of W' and S' per half tile, of the fp16 W' per
+//               tile, each slot freed once its stores have read it
+//   warps 4-11  epilogue: the thread owning TMEM lane r (row r) and 16 of a
+//               half tile's 32 columns computes W' = B W + c_S S + U_W,
+//               S' = A S + U_S in place and the fp16 W' into the X slot
 // Every wait is bounded and also gives up once another role has flagged an
 // abort; after an abort the producer waits (bounded) for its copies in
 // flight and the MMA warp for its MMAs before TMEM is freed.
 constexpr int UP2_NT = 384;
 constexpr int UP2_EPI0 = 4;                    // first epilogue warp
+constexpr int UP2_WS = 4;                      // state half-tile slots
 struct Up2Layer {
   int M, mtiles, ntiles, nranges, first;       // rows of W_l, 128-row blocks, 64-column tiles, ranges, first unit
   int b_rows_per_stream;                       // rows of the X source per stream
@@ -536,12 +546,12 @@ struct Up2Args {
   unsigned long long wait_ns;
   int inject;                                  // test hook, as in GemmArgs
 };
-// shared memory: A operands, then two stages of {X (or bf16 W'), W, S}
+// shared memory: A operands, two X (or fp16 W') slots, four state slots
 __host__ __device__ constexpr uint32_t up2_a_bytes(int C) { return 2u * (uint32_t)C * 128u; }
 __host__ __device__ constexpr uint32_t up2_x_bytes(int C) { return (uint32_t)(C > 128 ? C : 128) * 128u; }
-__host__ __device__ constexpr uint32_t up2_stage_bytes(int C) { return up2_x_bytes(C) + 4u * UP_BOX; }
+__host__ __device__ constexpr uint32_t up2_ws_bytes() { return 2u * UP_BOX; }   // W and S, 32 columns each
 __host__ __device__ constexpr size_t up2_smem(int C) {
-  return 2 * (size_t)up2_a_bytes(C) + 2 * (size_t)up2_stage_bytes(C) + 1024;
+  return 2 * (size_t)up2_a_bytes(C) + 2 * (size_t)up2_x_bytes(C) + UP2_WS * (size_t)up2_ws_bytes() + 1024;
 }
 
 // Bounded wait that also returns (false) once *abort is set; on expiry it
@@ -567,8 +577,8 @@ __global__ void __launch_bounds__(UP2_NT, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *sm =
       reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t a_full, ws_full[2], x_full[2], mma_done[2], acc_free[2], epi_done[2], stage_free[2], fin,
-      never;
+  __shared__ uint64_t a_full, x_full[2], mma_done[2], acc_free[2], x_free[2];
+  __shared__ uint64_t ws_full[UP2_WS], epi_done[UP2_WS], ws_free[UP2_WS], fin, never;
   __shared__ uint32_t tslot;
   __shared__ int abort_flag;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -580,27 +590,31 @@ __global__ void __launch_bounds__(UP2_NT, 1)
   const int per = ly.mtiles * ly.nranges, i = u - ly.first;
   const int s = i / per, mt = (i % per) / ly.nranges, rg = i % ly.nranges;
   const int j0 = rg * a.tpu, j1 = (j0 + a.tpu < ly.ntiles) ? j0 + a.tpu : ly.ntiles;
-  const int nt = j1 - j0;                      // column tiles of this unit
+  const int nt = j1 - j0;                      // 64-column tiles of this unit
+  const int nh = 2 * nt;                       // 32-column half tiles
   const int C = a.C;
   const int R = ly.M < 128 ? ly.M : 128;       // rows of a state box
   const int rows = ly.M - 128 * mt < 128 ? ly.M - 128 * mt : 128;
-  const uint32_t AB = up2_a_bytes(C), XB = up2_x_bytes(C), SB = up2_stage_bytes(C);
+  const uint32_t AB = up2_a_bytes(C), XB = up2_x_bytes(C);
   unsigned char *a_cg = sm, *a_eg = sm + AB;
-  auto x_slot = [&](int b) { return sm + 2 * AB + b * SB; };
-  auto w_slot = [&](int b) { return sm + 2 * AB + b * SB + XB; };
-  auto s_slot = [&](int b) { return sm + 2 * AB + b * SB + XB + 2 * UP_BOX; };
-  const uint32_t ws_bytes = 4u * (uint32_t)R * 128u;
+  auto x_slot = [&](int b) { return sm + 2 * AB + b * XB; };
+  auto w_slot = [&](int b) { return sm + 2 * AB + 2 * XB + b * up2_ws_bytes(); };
+  auto s_slot = [&](int b) { return w_slot(b) + UP_BOX; };
+  const uint32_t ws_bytes = 2u * (uint32_t)R * 128u;
   const uint32_t x_bytes = (uint32_t)C * 128u;
 
   if (tid == 0) {
     mbar_init(&a_full, 1);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&ws_full[b], 1);
       mbar_init(&x_full[b], 1);
       mbar_init(&mma_done[b], 1);
       mbar_init(&acc_free[b], 8);
+      mbar_init(&x_free[b], 1);
+    }
+    for (int b = 0; b < UP2_WS; ++b) {
+      mbar_init(&ws_full[b], 1);
       mbar_init(&epi_done[b], 8);
-      mbar_init(&stage_free[b], 1);
+      mbar_init(&ws_free[b], 1);
     }
     mbar_init(&fin, 1);
     mbar_init(&never, 1);
@@ -614,21 +628,20 @@ __global__ void __launch_bounds__(UP2_NT, 1)
   const uint32_t tm = tslot;
   volatile int *abort = &abort_flag;
 
-  // state tiles of the first two column tiles: issued before the wait for
-  // the preceding kernel (this chunk's forward/backward), which does not
+  // state half tiles of the first UP2_WS half tiles: issued before the wait
+  // for the preceding kernel (this chunk's forward/backward), which does not
   // write them
-  int ws_armed[2] = {0, 0}, x_armed[2] = {0, 0}, a_armed = 0;
+  int ws_armed[UP2_WS] = {0, 0, 0, 0}, x_armed[2] = {0, 0}, a_armed = 0;
+  auto load_ws = [&](int h2) {                 // half tile h2 into slot h2 % UP2_WS
+    const int b = h2 % UP2_WS, col = 64 * j0 + 32 * h2;
+    mbar_arrive_expect_tx(&ws_full[b], ws_bytes);
+    tma_load_3d(w_slot(b), &m.w[l], &ws_full[b], col, 128 * mt, s);
+    tma_load_3d(s_slot(b), &m.s[l], &ws_full[b], col, 128 * mt, s);
+    ++ws_armed[b];
+  };
   if (warp == 0 && lane == 0) {
     if (a.inject && !injected_wait(&never, a.status, a.wait_ns)) *abort = 1;
-    for (int jj = 0; jj < nt && jj < 2 && !*abort; ++jj) {
-      const int col = 64 * (j0 + jj);
-      mbar_arrive_expect_tx(&ws_full[jj], ws_bytes);
-      for (int bx = 0; bx < 2; ++bx) {
-        tma_load_3d(w_slot(jj) + bx * UP_BOX, &m.w[l], &ws_full[jj], col + 32 * bx, 128 * mt, s);
-        tma_load_3d(s_slot(jj) + bx * UP_BOX, &m.s[l], &ws_full[jj], col + 32 * bx, 128 * mt, s);
-      }
-      ++ws_armed[jj];
-    }
+    for (int h2 = 0; h2 < nh && h2 < UP2_WS && !*abort; ++h2) load_ws(h2);
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
@@ -644,35 +657,34 @@ __global__ void __launch_bounds__(UP2_NT, 1)
         }
       a_armed = 1;
       for (int jj = 0; jj < nt; ++jj) {
-        const int b = jj & 1, col = 64 * (j0 + jj);
-        if (jj >= 2) {
-          if (!up2_wait(&stage_free[b], (uint32_t)(((jj - 2) >> 1) & 1), a, abort)) break;
-          mbar_arrive_expect_tx(&ws_full[b], ws_bytes);
-          for (int bx = 0; bx < 2; ++bx) {
-            tma_load_3d(w_slot(b) + bx * UP_BOX, &m.w[l], &ws_full[b], col + 32 * bx, 128 * mt, s);
-            tma_load_3d(s_slot(b) + bx * UP_BOX, &m.s[l], &ws_full[b], col + 32 * bx, 128 * mt, s);
-          }
-          ++ws_armed[b];
-        }
+        const int b = jj & 1;
+        if (jj >= 2 && !up2_wait(&x_free[b], (uint32_t)(((jj - 2) >> 1) & 1), a, abort)) break;
         mbar_arrive_expect_tx(&x_full[b], x_bytes);
         for (int kp = 0; kp < C / 64; ++kp)
-          tma_load_2d(x_slot(b) + kp * 64 * 128, &m.b[l], &x_full[b], col, (int)(brow + 64 * kp));
+          tma_load_2d(x_slot(b) + kp * 64 * 128, &m.b[l], &x_full[b], 64 * (j0 + jj), (int)(brow + 64 * kp));
         ++x_armed[b];
+        bool ok = true;
+        for (int h2 = 2 * jj; h2 < 2 * jj + 2; ++h2) {
+          if (h2 < UP2_WS) continue;           // issued before the wait
+          if (!up2_wait(&ws_free[h2 % UP2_WS], (uint32_t)(((h2 - UP2_WS) / UP2_WS) & 1), a, abort)) { ok = false; break; }
+          load_ws(h2);
+        }
+        if (!ok) break;
       }
     }
     if (lane == 0 && *abort) {
       // copies still in flight into this CTA's shared memory finish first
       if (a_armed) mbar_wait(&a_full, 0, a.wait_ns);
-      for (int b = 0; b < 2; ++b) {
-        if (ws_armed[b]) mbar_wait(&ws_full[b], (uint32_t)((ws_armed[b] - 1) & 1), a.wait_ns);
+      for (int b = 0; b < 2; ++b)
         if (x_armed[b]) mbar_wait(&x_full[b], (uint32_t)((x_armed[b] - 1) & 1), a.wait_ns);
-      }
+      for (int b = 0; b < UP2_WS; ++b)
+        if (ws_armed[b]) mbar_wait(&ws_full[b], (uint32_t)((ws_armed[b] - 1) & 1), a.wait_ns);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(128, 64, true, true);
+      const uint32_t idesc = idesc_f16(128, 64, true, true);
       const uint32_t acg = smem_u32(a_cg), aeg = smem_u32(a_eg);
       bool ok = up2_wait(&a_full, 0, a, abort);
       for (int jj = 0; jj < nt && ok; ++jj) {
@@ -684,8 +696,8 @@ __global__ void __launch_bounds__(UP2_NT, 1)
         const uint32_t acc = tm + 128u * (uint32_t)b;
         for (int ks = 0; ks < C / 16; ++ks) {
           const uint64_t bd = desc_mnmajor(xb, C, ks);
-          umma_bf16(acc, desc_mnmajor(acg, C, ks), bd, idesc, ks != 0);
-          umma_bf16(acc + 64, desc_mnmajor(aeg, C, ks), bd, idesc, ks != 0);
+          umma_f16(acc, desc_mnmajor(acg, C, ks), bd, idesc, ks != 0);
+          umma_f16(acc + 64, desc_mnmajor(aeg, C, ks), bd, idesc, ks != 0);
         }
         umma_commit(&mma_done[b]);
       }
@@ -696,18 +708,33 @@ __global__ void __launch_bounds__(UP2_NT, 1)
     __syncwarp();
   } else if (warp == 2) {
     // ------------------------------------------------------------ stores
+    // One bulk group per half tile (its W' and S', and on odd half tiles the
+    // tile's fp16 W'); a group's slots are released once the next group has
+    // been issued and the earlier ones have read their sources, so one group
+    // stays in flight while the next half tile is stored.
     if (lane == 0) {
-      for (int jj = 0; jj < nt; ++jj) {
-        const int b = jj & 1, col = 64 * (j0 + jj);
-        if (!up2_wait(&epi_done[b], (uint32_t)((jj >> 1) & 1), a, abort)) break;
-        for (int bx = 0; bx < 2; ++bx) {
-          tma_store_3d(&m.w[l], w_slot(b) + bx * UP_BOX, col + 32 * bx, 128 * mt, s);
-          tma_store_3d(&m.s[l], s_slot(b) + bx * UP_BOX, col + 32 * bx, 128 * mt, s);
+      int pend_ws = -1, pend_x = -1;           // slots of the newest group, released one group later
+      for (int h2 = 0; h2 < nh; ++h2) {
+        const int b = h2 % UP2_WS, col = 64 * j0 + 32 * h2;
+        if (!up2_wait(&epi_done[b], (uint32_t)((h2 / UP2_WS) & 1), a, abort)) break;
+        tma_store_3d(&m.w[l], w_slot(b), col, 128 * mt, s);
+        tma_store_3d(&m.s[l], s_slot(b), col, 128 * mt, s);
+        int xb = -1;
+        if (h2 & 1) {                          // the tile's fp16 W' is complete (both halves)
+          const int jj = h2 >> 1;
+          xb = jj & 1;
+          tma_store_3d(&m.wb[l], x_slot(xb), 64 * (j0 + jj), 128 * mt, s);
         }
-        tma_store_3d(&m.wb[l], x_slot(b), col, 128 * mt, s);
-        tma_store_commit_wait_read();
-        mbar_arrive(&stage_free[b]);
+        bulk_commit_group();
+        bulk_wait_group_read<1>();             // every group but this one has read its slots
+        if (pend_ws >= 0) mbar_arrive(&ws_free[pend_ws]);
+        if (pend_x >= 0) mbar_arrive(&x_free[pend_x]);
+        pend_ws = b;
+        pend_x = xb;
       }
+      bulk_wait_group_read<0>();
+      if (pend_ws >= 0) mbar_arrive(&ws_free[pend_ws]);
+      if (pend_x >= 0) mbar_arrive(&x_free[pend_x]);
     }
     __syncwarp();
   } else if (warp >= UP2_EPI0) {
@@ -716,47 +743,50 @@ __global__ void __launch_bounds__(UP2_NT, 1)
     const int r = 32 * q + lane;               // TMEM lane = row of the block
     const uint32_t lb = (uint32_t)(32 * q) << 16;
     const float4 sc = *reinterpret_cast<const float4 *>(a.scal + 4 * ((long long)s * a.nchunks + a.chunk));
-    for (int jj = 0; jj < nt; ++jj) {
-      const int b = jj & 1;
-      const uint32_t ph = (uint32_t)((jj >> 1) & 1);
-      if (!up2_wait(&mma_done[b], ph, a, abort)) break;
-      if (!up2_wait(&ws_full[b], ph, a, abort)) break;
-      tc_fence_after();
-      float u0[16], u1[16], v0[16], v1[16];
-      const uint32_t acc = tm + lb + 128u * (uint32_t)b + 32u * (uint32_t)h;
-      tmem_ld16(acc, u0);
-      tmem_ld16(acc + 16, u1);
-      tmem_ld16(acc + 64, v0);
-      tmem_ld16(acc + 80, v1);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_free[b]);  // the MMA of tile jj + 2 may overwrite the pair
-      if (r < rows) {
-        unsigned char *wr = w_slot(b) + h * UP_BOX + r * 128;
-        unsigned char *sr = s_slot(b) + h * UP_BOX + r * 128;
-        unsigned char *br = x_slot(b) + r * 128;
-#pragma unroll
-        for (int jc = 0; jc < 8; ++jc) {
-          const uint32_t o = (uint32_t)((jc ^ (r & 7)) << 4);
-          const float *uw = jc < 4 ? u0 + 4 * jc : u1 + 4 * (jc - 4);
-          const float *us = jc < 4 ? v0 + 4 * jc : v1 + 4 * (jc - 4);
-          const float4 w = *reinterpret_cast<const float4 *>(wr + o);
-          const float4 x = *reinterpret_cast<const float4 *>(sr + o);
-          const float4 wn = make_float4(sc.x * w.x + sc.z * x.x + uw[0], sc.x * w.y + sc.z * x.y + uw[1],
-                                        sc.x * w.z + sc.z * x.z + uw[2], sc.x * w.w + sc.z * x.w + uw[3]);
-          const float4 sn = make_float4(sc.y * x.x + us[0], sc.y * x.y + us[1], sc.y * x.z + us[2],
-                                        sc.y * x.w + us[3]);
-          *reinterpret_cast<float4 *>(wr + o) = wn;
-          *reinterpret_cast<float4 *>(sr + o) = sn;
-          // bf16 row: columns 32 h + 4 jc .. + 3 in 16-byte chunk 4 h + jc / 2
-          const uint32_t ob = (uint32_t)((((4 * h + (jc >> 1)) ^ (r & 7)) << 4) + (jc & 1) * 8);
-          *reinterpret_cast<uint2 *>(br + ob) = make_uint2(pack_bf16(wn.x, wn.y), pack_bf16(wn.z, wn.w));
+    bool ok = true;
+    for (int jj = 0; jj < nt && ok; ++jj) {
+      const int xb = jj & 1;
+      if (!up2_wait(&mma_done[xb], (uint32_t)((jj >> 1) & 1), a, abort)) break;
+      for (int hs = 0; hs < 2; ++hs) {
+        const int h2 = 2 * jj + hs, b = h2 % UP2_WS;
+        if (!up2_wait(&ws_full[b], (uint32_t)((h2 / UP2_WS) & 1), a, abort)) { ok = false; break; }
+        tc_fence_after();
+        // this thread's 16 columns of the half tile: U_W and U_S
+        float uw[16], us[16];
+        const uint32_t acc = tm + lb + 128u * (uint32_t)xb + 32u * (uint32_t)hs + 16u * (uint32_t)h;
+        tmem_ld16(acc, uw);
+        tmem_ld16(acc + 64, us);
+        tmem_wait_ld();
+        if (hs == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_free[xb]);   // the MMAs of tile jj + 2 may overwrite the pair
         }
+        if (r < rows) {
+          unsigned char *wr = w_slot(b) + r * 128;
+          unsigned char *sr = s_slot(b) + r * 128;
+          unsigned char *br = x_slot(xb) + r * 128;
+#pragma unroll
+          for (int jc = 0; jc < 4; ++jc) {
+            const uint32_t o = (uint32_t)(((4 * h + jc) ^ (r & 7)) << 4);
+            const float4 w = *reinterpret_cast<const float4 *>(wr + o);
+            const float4 x = *reinterpret_cast<const float4 *>(sr + o);
+            const float4 wn = make_float4(sc.x * w.x + sc.z * x.x + uw[4 * jc], sc.x * w.y + sc.z * x.y + uw[4 * jc + 1],
+                                          sc.x * w.z + sc.z * x.z + uw[4 * jc + 2], sc.x * w.w + sc.z * x.w + uw[4 * jc + 3]);
+            const float4 sn = make_float4(sc.y * x.x + us[4 * jc], sc.y * x.y + us[4 * jc + 1],
+                                          sc.y * x.z + us[4 * jc + 2], sc.y * x.w + us[4 * jc + 3]);
+            *reinterpret_cast<float4 *>(wr + o) = wn;
+            *reinterpret_cast<float4 *>(sr + o) = sn;
+            // fp16 row of the tile: columns 32 hs + 16 h + 4 jc .. + 3, in
+            // 16-byte chunk 4 hs + 2 h + jc / 2
+            const uint32_t ob = (uint32_t)((((4 * hs + 2 * h + (jc >> 1)) ^ (r & 7)) << 4) + (jc & 1) * 8);
+            *reinterpret_cast<uint2 *>(br + ob) = make_uint2(pack_h2(wn.x, wn.y), pack_h2(wn.z, wn.w));
+          }
+        }
+        fence_proxy_async_smem();              // the TMA stores read these rows
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&epi_done[b]);
       }
-      fence_proxy_async_smem();                // the TMA stores read these rows
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&epi_done[b]);
     }
   }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -769,9 +799,9 @@ __global__ void __launch_bounds__(UP2_NT, 1)
 // Fused forward + backward of one chunk, for memories whose every layer is at
 // most 256 wide. One CTA per (128-row tile of the chunk's [keys; queries],
 // stream) runs the whole chain that the per-phase kernels run as 2L - 1
-// launches: the tile's rows stay in shared memory (bf16, row-block layout,
+// launches: the tile's rows stay in shared memory (fp16, row-block layout,
 // overwritten in place by each epilogue) and the accumulator in TMEM, while
-// the bf16 weights stream through a ring of TMA stages whose prefetch runs
+// the fp16 weights stream through a ring of TMA stages whose prefetch runs
 // ahead across layer boundaries (the next layer's slices land during the
 // current epilogue). Rows of a tile are independent through every layer, so
 // no other CTA is involved.
@@ -780,7 +810,7 @@ __global__ void __launch_bounds__(UP2_NT, 1)
 //            of 64 rows); tiles without key rows stop after the forward.
 // Outputs are those the update GEMMs read: X_l and silu'(Z_l) of key rows,
 // -c G_l and -e G_l; and y for query rows.
-constexpr int FB_STAGES = 4;
+constexpr int FB_STAGES = 5;    // 64 KB tile + 5 x 32 KB ring: one slice of the next phase lands early
 constexpr uint32_t FB_STAGE = 256 * KB * 2;          // 32 KB: one 64-wide slice of W_l
 constexpr uint32_t FB_ABUF = 128 * 256 * 2;          // 64 KB: the tile's rows
 constexpr size_t FB_SMEM = FB_ABUF + FB_STAGES * FB_STAGE + 1024;
@@ -792,10 +822,10 @@ constexpr int FB_NT = FB_EPI + 32;   // and one producer warp (TMA loads, MMA is
 struct FbArgs {
   int L, C, T, chunk;
   int dims[kMaxL + 1];
-  __nv_bfloat16 *x_out[kMaxL + 1];   // [streams, 2C, d_l], key rows written (l = 1..L-1)
-  __nv_bfloat16 *sp_out[kMaxL + 1];  // [streams, C, d_l] silu'(Z_l) of key rows
-  __nv_bfloat16 *gc_out[kMaxL + 1];  // [streams, C, d_l] -c G_l
-  __nv_bfloat16 *ge_out[kMaxL + 1];  // [streams, C, d_l] -e G_l
+  op_t *x_out[kMaxL + 1];            // [streams, 2C, d_l], key rows written (l = 1..L-1)
+  op_t *sp_out[kMaxL + 1];           // [streams, C, d_l] silu'(Z_l) of key rows
+  op_t *gc_out[kMaxL + 1];           // [streams, C, d_l] -c G_l
+  op_t *ge_out[kMaxL + 1];           // [streams, C, d_l] -e G_l
   float *y;                          // [streams, T, d]
   const __nv_bfloat16 *v;            // [streams, T, d]
   const float *coef;                 // [streams, T, 2]
@@ -806,7 +836,7 @@ struct FbArgs {
 
 struct FbMaps {
   CUtensorMap k, q;
-  CUtensorMap w[kMaxL + 1];          // w[l]: bf16 W_l of every stream, [streams * d_l, d_{l-1}]
+  CUtensorMap w[kMaxL + 1];          // w[l]: fp16 W_l of every stream, [streams * d_l, d_{l-1}]
 };
 
 struct FbPhase {
@@ -868,7 +898,7 @@ __global__ void __launch_bounds__(FB_NT, 1)
   // key rows of this tile (keys precede queries)
   const int nkey = C - 128 * mt >= 128 ? 128 : (C - 128 * mt > 0 ? C - 128 * mt : 0);
   // silu'(Z_l) of key rows for the backward: the last two hidden layers keep
-  // it in TMEM (bf16 pairs in columns 256-383 and 384-511, beside the
+  // it in TMEM (fp16 pairs in columns 256-383 and 384-511, beside the
   // accumulator in 0-255); earlier layers go through global memory
   auto sp_slot = [&](int l) -> int { return L - 1 - l < 2 ? 256 + 128 * ((L - 1 - l) & 1) : -1; };
 
@@ -916,7 +946,7 @@ __global__ void __launch_bounds__(FB_NT, 1)
         // previous epilogue's output
         ok = p == 0 ? mbar_wait(&xbar, 0, a.wait_ns) : mbar_wait(&ready, (uint32_t)((p - 1) & 1), a.wait_ns);
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16(128, f.N, false, f.bwd != 0);
+        const uint32_t idesc = idesc_f16(128, f.N, false, f.bwd != 0);
         const uint32_t abase = smem_u32(abuf);
         // A phase has at most FB_STAGES slices and all of them were requested
         // before it began (the refills below run a phase ahead), so the MMAs
@@ -930,13 +960,17 @@ __global__ void __launch_bounds__(FB_NT, 1)
           for (int ks = 0; ks < KB / 16; ++ks) {
             const uint64_t ad = desc_kmajor(abase + kb * 128 * 128, 128, ks);
             const uint64_t bd = f.bwd ? desc_mnmajor(bb, 64, ks) : desc_kmajor(bb, f.N, ks);
-            umma_bf16(tm, ad, bd, idesc, (kb | ks) != 0);
+            umma_f16(tm, ad, bd, idesc, (kb | ks) != 0);
           }
           umma_commit(&empty[st]);
           ++consumed;
         }
         if (!ok) { atomicCAS(a.status, 0, kDevTimeout); abort_flag = 1; }
         umma_commit(&done);
+        // the last phase is under way: let the update launch behind this
+        // kernel start (its state loads do not depend on this kernel; it waits
+        // for this grid's completion before it reads the outputs)
+        if (p == nphase - 1) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
         // refill the consumed stages with the next phase's slices as the MMAs
         // finish; they land while the epilogue runs
         while (ok && issued < total && issued - FB_STAGES <= consumed - 1) {
@@ -982,12 +1016,12 @@ __global__ void __launch_bounds__(FB_NT, 1)
         if (pend_kind == 1) {
           *reinterpret_cast<uint4 *>(a.x_out[pend_l] + ((long long)s * 2 * C + 128 * mt + rr) * N + 8 * ch) = u;
         } else {
-          const __nv_bfloat16 *hb = reinterpret_cast<const __nv_bfloat16 *>(&u);
+          const op_t *hb = reinterpret_cast<const op_t *>(&u);
           const float2 k2 = cef[rr];
           float vc[8], ve[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const float g = __bfloat162float(hb[j]);
+            const float g = __half2float(hb[j]);
             vc[j] = -k2.x * g;
             ve[j] = -k2.y * g;
           }
@@ -1009,11 +1043,12 @@ __global__ void __launch_bounds__(FB_NT, 1)
       uint4 aux[8];
       const int spt = f.bwd ? sp_slot(f.l - 1) : -1;      // silu' of the layer below in TMEM?
       if (grad && key && spt < 0) {
-        const __nv_bfloat16 *src = f.bwd ? a.sp_out[f.l - 1] + ((long long)s * C + r) * N
-                                         : a.v + tok * N;
+        // fp16 silu' (backward) or bf16 values (last forward), 8 per 16 bytes
+        const uint4 *src = f.bwd ? reinterpret_cast<const uint4 *>(a.sp_out[f.l - 1] + ((long long)s * C + r) * N + cbeg)
+                                 : reinterpret_cast<const uint4 *>(a.v + tok * N + cbeg);
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          if (8 * i < N / 4) aux[i] = *reinterpret_cast<const uint4 *>(src + cbeg + 8 * i);
+          if (8 * i < N / 4) aux[i] = src[i];
       }
       flush();                                   // the previous phase's outputs
       if (tid == 0 && !mbar_wait(&done, (uint32_t)(p & 1), a.wait_ns)) {
@@ -1047,10 +1082,10 @@ __global__ void __launch_bounds__(FB_NT, 1)
             if (slot >= 0) {
               uint32_t pk[8];
 #pragma unroll
-              for (int i = 0; i < 8; ++i) pk[i] = pack_bf16(sp[2 * i], sp[2 * i + 1]);
+              for (int i = 0; i < 8; ++i) pk[i] = pack_h2(sp[2 * i], sp[2 * i + 1]);
               tmem_st8(tm + lb + (uint32_t)(slot + c0 / 2), pk);
             } else {
-              __nv_bfloat16 *so = a.sp_out[f.l] + ((long long)s * C + r) * N + c0;
+              op_t *so = a.sp_out[f.l] + ((long long)s * C + r) * N + c0;
               *reinterpret_cast<uint4 *>(so) = pack8(sp);
               *reinterpret_cast<uint4 *>(so + 8) = pack8(sp + 8);
             }
@@ -1074,11 +1109,12 @@ __global__ void __launch_bounds__(FB_NT, 1)
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             const uint4 u = aux[2 * step + i];
+            const op_t *hh = reinterpret_cast<const op_t *>(&u);
             const __nv_bfloat16 *hb = reinterpret_cast<const __nv_bfloat16 *>(&u);
             float g[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              const float h = __bfloat162float(hb[j]);
+              const float h = f.bwd ? __half2float(hh[j]) : __bfloat162float(hb[j]);
               g[j] = f.bwd ? z[8 * i + j] * h : 2.f * (z[8 * i + j] - h);
             }
             st_shared_v4(abuf + rb_chunk(128, row, c0 / 8 + i), pack8(g));
@@ -1104,46 +1140,90 @@ __global__ void __launch_bounds__(FB_NT, 1)
   if (warp == 0) tmem_dealloc(tm, 512);
 }
 
-// A5 for every chunk of every stream at once: one thread per (stream, chunk)
-// runs the reverse recurrence over its C tokens (0-based i within the chunk):
+// A5 for every chunk of every stream at once: one warp per (stream, chunk),
+// lane l holding tokens m l .. m l + m - 1 of the chunk (m = C / 32, 0-based i
+// within the chunk):
 //   pa_i = prod_{j>i}(1 - alpha_j), pe_i = prod_{j>i} eta_j,
 //   r_{C-1} = 1, r_i = pa_i + eta_{i+1} r_{i+1};  c_i = theta_i r_i, e_i = theta_i pe_i;
 //   B = prod(1 - alpha), A = prod eta, c_S = eta_0 r_0.
+// The suffix products are a suffix scan over lanes of each lane's products;
+// r is a chain of affine maps x -> pa_i + eta_{i+1} x, composed within each
+// lane, suffix-scanned over lanes, then unrolled within the lane. No division.
+constexpr int COEF_MAXM = kMaxC / 32;
 __global__ void tcl_coef_kernel(const float *theta, const float *eta, const float *alpha, int streams,
                                 int T, int C, int nchunks, float *coef, float *scal) {
-  const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (id >= (long long)streams * nchunks) return;
-  const long long s = id / nchunks, ch = id % nchunks;
+  const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= (long long)streams * nchunks) return;   // the whole warp leaves together
+  const long long s = wid / nchunks, ch = wid % nchunks;
   const long long t0 = s * T + ch * C;
-  float pa = 1.f, pe = 1.f, r = 1.f;
-  for (int i = C - 1; i >= 0; --i) {
-    if (i < C - 1) {
-      pa *= 1.f - alpha[t0 + i + 1];
-      pe *= eta[t0 + i + 1];
-      r = pa + eta[t0 + i + 1] * r;
+  const int m = C / 32;
+  float th[COEF_MAXM], et[COEF_MAXM], om[COEF_MAXM];
+  float Pa = 1.f, Pe = 1.f;
+#pragma unroll
+  for (int k = 0; k < COEF_MAXM; ++k)
+    if (k < m) {
+      const long long t = t0 + (long long)lane * m + k;
+      th[k] = theta[t];
+      et[k] = eta[t];
+      om[k] = 1.f - alpha[t];
+      Pa *= om[k];
+      Pe *= et[k];
     }
-    coef[2 * (t0 + i)] = theta[t0 + i] * r;
-    coef[2 * (t0 + i) + 1] = theta[t0 + i] * pe;
+  // products over the lanes after this one
+  float xa = Pa, xe = Pe;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float ya = __shfl_down_sync(0xffffffffu, xa, o), ye = __shfl_down_sync(0xffffffffu, xe, o);
+    if (lane + o < 32) { xa *= ya; xe *= ye; }
   }
-  float *o = scal + 4 * id;
-  o[0] = pa * (1.f - alpha[t0]);
-  o[1] = pe * eta[t0];
-  o[2] = eta[t0] * r;
-  o[3] = 0.f;
+  float na = __shfl_down_sync(0xffffffffu, xa, 1), ne = __shfl_down_sync(0xffffffffu, xe, 1);
+  if (lane == 31) { na = 1.f; ne = 1.f; }
+  float pa[COEF_MAXM], pe[COEF_MAXM], bn[COEF_MAXM];
+  const float eta_after = __shfl_down_sync(0xffffffffu, et[0], 1);   // eta of the next lane's first token
+  float A = 0.f, Bm = 1.f;                       // this lane's maps composed: x -> A + Bm x
+#pragma unroll
+  for (int k = COEF_MAXM - 1; k >= 0; --k)
+    if (k < m) {
+      pa[k] = na;
+      pe[k] = ne;
+      na *= om[k];
+      ne *= et[k];
+      bn[k] = k + 1 < m ? et[k + 1] : (lane == 31 ? 0.f : eta_after);   // eta_{i+1}; 0 past the chunk
+      A = pa[k] + bn[k] * A;
+      Bm = bn[k] * Bm;
+    }
+  // suffix scan of the lanes' maps: FA = r at this lane's first token
+  float FA = A, FB = Bm;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float ya = __shfl_down_sync(0xffffffffu, FA, o), yb = __shfl_down_sync(0xffffffffu, FB, o);
+    if (lane + o < 32) { FA = FA + FB * ya; FB = FB * yb; }
+  }
+  float r = __shfl_down_sync(0xffffffffu, FA, 1);   // r just after this lane's tokens (unused by lane 31)
+#pragma unroll
+  for (int k = COEF_MAXM - 1; k >= 0; --k)
+    if (k < m) {
+      r = pa[k] + bn[k] * r;
+      const long long t = t0 + (long long)lane * m + k;
+      *reinterpret_cast<float2 *>(coef + 2 * t) = make_float2(th[k] * r, th[k] * pe[k]);
+      if (lane == 0 && k == 0)
+        *reinterpret_cast<float4 *>(scal + 4 * wid) = make_float4(pa[0] * om[0], pe[0] * et[0], et[0] * r, 0.f);
+    }
 }
 
-// Copy W0/S0 into W_end/S_end (unless in place) and build the bf16 operand
+// Copy W0/S0 into W_end/S_end (unless in place) and build the fp16 operand
 // copies, stored layer-major ([streams, n_l, n_{l-1}] per layer) so that one
 // 2-D tensor map covers a layer of every stream.
 struct InitArgs {
   const float *W0, *S0;
   float *W, *S;
-  __nv_bfloat16 *Wbf;
+  op_t *Wbf;
   long long P;
   long long streams;
   int L;
   long long off[kMaxL + 1];      // layer offsets inside a parameter vector
-  long long boff[kMaxL + 1];     // layer offsets inside the bf16 copy
+  long long boff[kMaxL + 1];     // layer offsets inside the fp16 copy
 };
 
 __global__ void tcl_init_kernel(const InitArgs a) {
@@ -1158,7 +1238,7 @@ __global__ void tcl_init_kernel(const InitArgs a) {
     while (l + 1 < a.L && j >= a.off[l + 1]) ++l;
     const long long within = j - a.off[l];
     const long long per = a.off[l + 1] - a.off[l];
-    a.Wbf[a.boff[l] + s * per + within] = __float2bfloat16_rn(w);
+    a.Wbf[a.boff[l] + s * per + within] = __float2half_rn(w);
   }
 }
 
@@ -1179,7 +1259,7 @@ EncodeTiledFn encode_fn_l() {
   return fn;
 }
 
-// 2-D bf16 map over [rows x cols], box = 64 columns x box_rows rows, 128B swizzle.
+// 2-D fp16 map over [rows x cols], box = 64 columns x box_rows rows, 128B swizzle.
 bool map2d(CUtensorMap *m, const void *base, long long rows, int cols, int box_rows) {
   EncodeTiledFn fn = encode_fn_l();
   if (!fn) return false;
@@ -1188,7 +1268,7 @@ bool map2d(CUtensorMap *m, const void *base, long long rows, int cols, int box_r
   cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
   cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1360,7 +1440,7 @@ struct TclGroup {
   Carve cv;
   unsigned char *ws;
   float *coef, *scal;
-  __nv_bfloat16 *wbf;
+  op_t *wbf;
   int L, C, T, S, nchunks;
   InitArgs ia;
   CUtensorMap mk, mq, mwb[kMaxL + 1], mx[kMaxL + 1], mg[kMaxL + 1], mgc[kMaxL + 1], mge[kMaxL + 1];
@@ -1376,7 +1456,7 @@ struct TclGroup {
   FbArgs fa;
   FbMaps fm;
 
-  __nv_bfloat16 *bf(size_t off) const { return reinterpret_cast<__nv_bfloat16 *>(ws + off); }
+  op_t *bf(size_t off) const { return reinterpret_cast<op_t *>(ws + off); }
   // Widest tile that divides n and still gives about one CTA per SM.
   int tile_for(int n, int mtiles) const {
     for (int t = 256; t >= 64; t /= 2) {
@@ -1394,7 +1474,7 @@ cudaError_t TclGroup::setup() {
   ws = static_cast<unsigned char *>(p.scratch);
   coef = reinterpret_cast<float *>(ws + cv.coef);
   scal = reinterpret_cast<float *>(ws + cv.scal);
-  wbf = reinterpret_cast<__nv_bfloat16 *>(ws + cv.wbf);
+  wbf = reinterpret_cast<op_t *>(ws + cv.wbf);
   L = p.L; C = p.C; T = p.T; S = p.streams; nchunks = p.T_run / C;
   const int d = p.dims[0];
   cudaStream_t stream = st;
@@ -1410,13 +1490,13 @@ cudaError_t TclGroup::setup() {
   ia.boff[L] = bo;
   tcl_init_kernel<<<592, 256, 0, stream>>>(ia);
   const long long nct = (long long)S * nchunks;
-  tcl_coef_kernel<<<(unsigned)((nct + 127) / 128), 128, 0, stream>>>(p.theta, p.eta, p.alpha, S, T, C,
-                                                                     nchunks, coef, scal);
+  tcl_coef_kernel<<<(unsigned)((nct * 32 + 127) / 128), 128, 0, stream>>>(p.theta, p.eta, p.alpha, S, T, C,
+                                                                          nchunks, coef, scal);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
 
   // tensor maps, built once per call
-  if (!map2d(&mk, p.k, (long long)S * T, d, 64) || !map2d(&mq, p.q, (long long)S * T, d, 64))
+  if (!map2d(&mk, p.k16, (long long)S * T, d, 64) || !map2d(&mq, p.q16, (long long)S * T, d, 64))
     return cudaErrorInvalidValue;
   for (int l = 1; l <= L; ++l) {
     const int nl = p.dims[l], np = p.dims[l - 1];
@@ -1468,7 +1548,7 @@ cudaError_t TclGroup::setup() {
                (long long)p.P, 32, br) ||
         !map3d(&um.s[l - 1], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.S_end + p.layer_off[l - 1], np, nl, S,
                (long long)p.P, 32, br) ||
-        !map3d(&um.wb[l - 1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wbf + ia.boff[l - 1], np, nl, S,
+        !map3d(&um.wb[l - 1], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, wbf + ia.boff[l - 1], np, nl, S,
                (long long)nl * np, 64, br))
       return cudaErrorInvalidValue;
     const size_t sm = up_smem(u.N, C / KB);
@@ -1610,6 +1690,8 @@ Problem group_slice(const Problem &p, int g, int groups) {
   q.k = static_cast<const char *>(p.k) + s0 * td * el;
   q.v = static_cast<const char *>(p.v) + s0 * td * el;
   q.q = static_cast<const char *>(p.q) + s0 * td * el;
+  q.k16 = static_cast<const char *>(p.k16) + s0 * td * 2;   // fp16 copies
+  q.q16 = static_cast<const char *>(p.q16) + s0 * td * 2;
   q.theta = p.theta + (size_t)s0 * p.T;
   q.eta = p.eta + (size_t)s0 * p.T;
   q.alpha = p.alpha + (size_t)s0 * p.T;

@@ -9,11 +9,12 @@ result against tm_run on the same inputs (fp32 tolerance of the other tests)
 and against the float64 oracle. A larger problem runs first, then a smaller
 one with a different chunk size, so the second call finds the first call's
 leftovers in the shared array. Around a warmed-up call, the device's free
-memory and torch's allocation count do not move. It also checks that a
+memory does not move and torch's allocation count does not grow. It also checks that a
 problem too large for the array, and a call whose y overlaps an input, are
 refused before any launch. This file is collected last on purpose.
 """
 import ctypes
+import gc
 
 import numpy as np
 import pytest
@@ -94,12 +95,13 @@ def test_noalloc_allocates_nothing():
     We, Se = torch.empty_like(dev["W0"]), torch.empty_like(dev["S0"])
     assert call_noalloc(mem, dev, w.C, y, We, Se) == N.TM_OK    # set-up on this device
     torch.cuda.synchronize()
+    gc.collect()                 # tensors of earlier tests are released now, not during the calls
     free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
     for _ in range(3):
         assert call_noalloc(mem, dev, w.C, y, We, Se) == N.TM_OK
     torch.cuda.synchronize()
-    assert torch.cuda.mem_get_info()[0] == free0
-    assert torch.cuda.memory_allocated() == alloc0
+    assert torch.cuda.mem_get_info()[0] == free0          # the device's free memory did not move
+    assert torch.cuda.memory_allocated() <= alloc0
 
 
 def test_noalloc_refuses_problems_larger_than_its_array():
