@@ -11,14 +11,14 @@
 //   A2  Z1 = [K;Q] W1_j^T        M=128 N=64  K=d   (keys and queries share W)
 //       X1 = silu(Z1)            epilogue, fp16 to shared memory
 //       Z2_j = X1 W2_j^T         M=128 N=d   K=64  (this CTA's partial sum)
-//       all-reduce of Z2 over the cluster through the CTAs' shared memories
-//       with asynchronous remote stores (st.async: each 16-byte piece counts
-//       its bytes on the receiver's mbarrier, no cluster fences): each thread
-//       sends its fp16 partial of rows [128/G p, 128/G (p+1)) straight into
-//       CTA p's receive buffer (reduce-scatter); CTA p sums them in fp32,
-//       writes y for query rows and G2 = 2 (Z2 - V) for key rows, and each of
-//       its threads sends its G2 piece into every CTA's G2 tile (all-gather)
-//       (A3).
+//       all-reduce of Z2 over the cluster with bulk copies between the CTAs'
+//       shared memories (the copy engine, mbarrier transaction counts, no
+//       thread-level cluster fences): each CTA stages its partial as fp16 rows
+//       and pushes rows [128/G p, 128/G (p+1)) to CTA p (reduce-scatter); CTA p
+//       sums them in fp32, writes y for query rows and G2 = 2 (Z2 - V) for key
+//       rows, and pushes its G2 rows to every CTA (all-gather) (A3). (Per-thread
+//       asynchronous remote stores, st.async, measured slower here: 8.3 against
+//       7.3 us per chunk.)
 //   A4  G1 = (G2 W2_j) . silu'(Z1_K)        M=128(64 used) N=64 K=d
 //   A6+A7 the fp32 state of this CTA's slice, [W | S], lives in TMEM for the
 //       whole stream. Before the weight-update contractions of a chunk the
@@ -173,6 +173,17 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
                "r"(v.z), "r"(v.w)
                : "memory");
 }
+// N (a multiple of 16) consecutive TMEM columns of this thread's lane.
+template <int N>
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, float (&v)[N]) {
+#pragma unroll
+  for (int i = 0; i < N / 16; ++i) tmem_ld16(taddr + 16 * i, *reinterpret_cast<float(*)[16]>(&v[16 * i]));
+}
+template <int N>
+__device__ __forceinline__ void tmem_stn(uint32_t taddr, const float (&v)[N]) {
+#pragma unroll
+  for (int i = 0; i < N / 16; ++i) tmem_st16(taddr + 16 * i, *reinterpret_cast<const float(*)[16]>(&v[16 * i]));
+}
 __device__ __forceinline__ void arrive_remote_release(uint32_t bar_cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
                    bar_cluster_addr)
@@ -189,14 +200,14 @@ __device__ __forceinline__ bool try_wait_acquire_cluster(uint32_t bar, uint32_t 
       : "memory");
   return ok != 0;
 }
-// 16 bytes into CTA-of-cluster shared memory (dst, bar are shared::cluster
-// addresses), counted as 16 transaction bytes on the remote mbarrier, whose
-// completion releases the write at cluster scope.
-__device__ __forceinline__ void st_async_v4(uint32_t dst, uint4 v, uint32_t bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                   dst),
-               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar)
-               : "memory");
+// Copy `bytes` from this CTA's shared memory into CTA-of-cluster shared memory
+// (dst, bar are shared::cluster addresses); completion counts on the remote bar.
+__device__ __forceinline__ void bulk_push(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "r"(src), "r"(bytes), "r"(bar)
+      : "memory");
 }
 // Global-memory exchange: bulk copy shared -> global, completion, proxy fence,
 // release counter, acquire poll, bulk copy global -> shared.
@@ -349,7 +360,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   constexpr int NPT = RP * D / 8 / XCH_THREADS;    // 16-byte chunks reduced per exchange thread
   constexpr int SWZ = (D / 16 < 8 ? D / 16 : 8) - 1; // chunk swizzle mask of a half row
   static_assert(NPT >= 1 && RP * D / 8 % XCH_THREADS == 0, "reduce split");
-  static_assert(CPT == 16, "epilogue column split");
+  static_assert(CPT % 16 == 0, "epilogue column split");
   constexpr int NSIG = 2 * G * (RP >= 32 ? RP / 32 : 1);   // row pushes a CTA receives per chunk
   constexpr int NKO = RP >= C ? 1 : C / RP;                 // CTAs owning key rows
   constexpr uint32_t XDEST = 2 * 128 * D;                   // bytes of one receive buffer
@@ -442,8 +453,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         w[4 * i4] = a4.x; w[4 * i4 + 1] = a4.y; w[4 * i4 + 2] = a4.z; w[4 * i4 + 3] = a4.w;
         sv[4 * i4] = b4.x; sv[4 * i4 + 1] = b4.y; sv[4 * i4 + 2] = b4.z; sv[4 * i4 + 3] = b4.w;
       }
-      tmem_st16(t_s2 + lane_base + CPT * h, w);
-      tmem_st16(t_s2 + lane_base + 64 + CPT * h, sv);
+      tmem_stn(t_s2 + lane_base + CPT * h, w);
+      tmem_stn(t_s2 + lane_base + 64 + CPT * h, sv);
 #pragma unroll
       for (int k8 = 0; k8 < CPT / 8; ++k8)
         st_shared_v4(sbase + Lay::W2 + rb_chunk(D, row, (CPT / 8) * h + k8), pack8(&w[8 * k8]));
@@ -453,8 +464,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         w[i] = W0g[g1];
         sv[i] = S0g[g1];
       }
-      tmem_st16(t_s1 + lane_base + CPT * h, w);
-      tmem_st16(t_s1 + lane_base + 64 + CPT * h, sv);
+      tmem_stn(t_s1 + lane_base + CPT * h, w);
+      tmem_stn(t_s1 + lane_base + 64 + CPT * h, sv);
 #pragma unroll
       for (int k8 = 0; k8 < CPT / 8; ++k8)
         st_shared_v4(sbase + Lay::W1 + rb_chunk(D, row, (CPT / 8) * h + k8), pack8(&w[8 * k8]));
@@ -488,16 +499,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int layer = 0; layer < 2; ++layer) {
           const uint32_t ts = (layer ? t_s1 : t_s2) + lane_base + CPT * h;
           float w[CPT], sv[CPT];
-          tmem_ld16(ts, w);
-          tmem_ld16(ts + 64, sv);
+          tmem_ldn(ts, w);
+          tmem_ldn(ts + 64, sv);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < CPT; ++i) {
             w[i] = cf.Bw * w[i] + cS_t * sv[i];
             sv[i] = As_t * sv[i];
           }
-          tmem_st16(ts, w);
-          tmem_st16(ts + 64, sv);
+          tmem_stn(ts, w);
+          tmem_stn(ts + 64, sv);
         }
         tmem_wait_st();
       }
@@ -506,7 +517,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tc_fence_after();
       {
         float z[CPT];
-        tmem_ld16(t_z1 + lane_base + CPT * h, z);
+        tmem_ldn(t_z1 + lane_base + CPT * h, z);
         tmem_wait_ld();
         float x[CPT];
 #pragma unroll
@@ -551,58 +562,46 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       if (warp < XCH_WARPS) {
         constexpr int HALF = D / 2;                    // columns of Z2 per thread
-        if constexpr (!XG) {
-          // each 16-byte piece goes straight into the owner's receive buffer
-          // (row rin of this CTA's block, half h), counted on its B_RECV
-          const int p = row / RP, rin = row - p * RP;
-          const uint32_t rrow = mapa(sbase + Lay::RECV + (uint32_t)(j * 2 * RP * D + h * RP * D + rin * D), (uint32_t)p);
-          const uint32_t rbar = mapa(smem_u32(&bars[B_RECV]), (uint32_t)p);
+        const uint32_t srow = sbase + Lay::SEND + (uint32_t)(h * 128 * D + row * D);
 #pragma unroll
-          for (int c16 = 0; c16 < HALF / 16; ++c16) {
-            float z[16];
-            tmem_ld16(t_z2 + lane_base + HALF * h + 16 * c16, z);
-            tmem_wait_ld();
+        for (int c16 = 0; c16 < HALF / 16; ++c16) {
+          float z[16];
+          tmem_ld16(t_z2 + lane_base + HALF * h + 16 * c16, z);
+          tmem_wait_ld();
 #pragma unroll
-            for (int k8 = 0; k8 < 2; ++k8)
-              st_async_v4(rrow + (uint32_t)(((2 * c16 + k8) ^ (row & SWZ)) << 4), pack8(&z[8 * k8]), rbar);
-          }
-          tc_fence_before();
-        } else {
-          const uint32_t srow = sbase + Lay::SEND + (uint32_t)(h * 128 * D + row * D);
+          for (int k8 = 0; k8 < 2; ++k8)
+            st_shared_v4(srow + (uint32_t)(((2 * c16 + k8) ^ (row & SWZ)) << 4), pack8(&z[8 * k8]));
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          constexpr int RPP = RP < 32 ? RP : 32;       // rows per push
 #pragma unroll
-          for (int c16 = 0; c16 < HALF / 16; ++c16) {
-            float z[16];
-            tmem_ld16(t_z2 + lane_base + HALF * h + 16 * c16, z);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k8 = 0; k8 < 2; ++k8)
-              st_shared_v4(srow + (uint32_t)(((2 * c16 + k8) ^ (row & SWZ)) << 4), pack8(&z[8 * k8]));
-          }
-          fence_proxy_async_smem();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            constexpr int RPP = RP < 32 ? RP : 32;       // rows per push
-#pragma unroll
-            for (int i = 0; i < 32 / RPP; ++i) {
-              const int r0 = 32 * q + i * RPP, p = r0 / RP, rin = r0 - p * RP;
-              const uint32_t off = (uint32_t)(j * 2 * RP * D + h * RP * D + rin * D);
-              const uint32_t src = sbase + Lay::SEND + (uint32_t)(h * 128 * D + r0 * D);
+          for (int i = 0; i < 32 / RPP; ++i) {
+            const int r0 = 32 * q + i * RPP, p = r0 / RP, rin = r0 - p * RP;
+            const uint32_t off = (uint32_t)(j * 2 * RP * D + h * RP * D + rin * D);
+            const uint32_t src = sbase + Lay::SEND + (uint32_t)(h * 128 * D + r0 * D);
+            if constexpr (XG)
               bulk_store_global(xrv + (size_t)(p * 2 + (int)par) * XDEST + off, src, (uint32_t)(RPP * D));
-            }
+            else
+              bulk_push(mapa(sbase + Lay::RECV + off, (uint32_t)p), src, (uint32_t)(RPP * D),
+                        mapa(smem_u32(&bars[B_RECV]), (uint32_t)p));
+          }
+          if constexpr (XG) {
             // the rows are in global memory before the owners are told
             bulk_commit_and_wait();
             fence_proxy_async_global();
 #pragma unroll
             for (int i = 0; i < 32 / RPP; ++i) red_release_add(xfl + ((32 * q + i * RPP) / RP) * XFLAG_STRIDE, 1u);
           }
-          __syncwarp();
         }
+        __syncwarp();
       }
       // -------- reduce my rows over the G partials (fp32 sums, fixed order):
       // y for query rows, G2 = 2 (Z2 - V) for key rows (A3)
       if (XG ? !wait_flag(xfl + j * XFLAG_STRIDE, (unsigned)(NSIG * (cch + 1)), a, abort_flag)
-             : !wait_bar(&bars[B_RECV], par, a, abort_flag, true))
+             : !wait_bar(&bars[B_RECV], par, a, abort_flag))
         break;
       {
         float acc[NPT][8];
@@ -634,19 +633,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             float g[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) g[e] = 2.f * (acc[i][e] - __bfloat162float(vb[e]));
-            if constexpr (XG) {
-              st_shared_v4(sbase + Lay::G2OWN + rb_chunk(RPK, r, c), pack8(g));
-            } else {
-              // all-gather: the chunk goes to the G2 tile of every CTA of
-              // the cluster (this one included), counted on its B_G2
-              const uint4 gv = pack8(g);
-              const uint32_t loc = sbase + Lay::G2 + rb_chunk(64, gr, c);
-#pragma unroll
-              for (int i2 = 0; i2 < G; ++i2) {
-                const uint32_t pc = (j + (uint32_t)i2) % G;
-                st_async_v4(mapa(loc, pc), gv, mapa(smem_u32(&bars[B_G2]), pc));
-              }
-            }
+            st_shared_v4(sbase + Lay::G2OWN + rb_chunk(RPK, r, c), pack8(g));
           }
         }
         warp_arrive_local(&bars[B_G2OWN], lane);
@@ -668,8 +655,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tc_fence_after();
       if (row < C) {
         float gp[CPT], z[CPT];
-        tmem_ld16(t_g1 + lane_base + CPT * h, gp);
-        tmem_ld16(t_z1 + lane_base + CPT * h, z);
+        tmem_ldn(t_g1 + lane_base + CPT * h, gp);
+        tmem_ldn(t_z1 + lane_base + CPT * h, z);
         tmem_wait_ld();
         const float ci = -cf.c[row], ei = -cf.e[row] * sig;
         float g1[CPT];
@@ -695,7 +682,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tc_fence_after();
       if (row < D) {
         float w[CPT];
-        tmem_ld16(t_s2 + lane_base + CPT * h, w);
+        tmem_ldn(t_s2 + lane_base + CPT * h, w);
         tmem_wait_ld();
 #pragma unroll
         for (int k8 = 0; k8 < CPT / 8; ++k8)
@@ -705,7 +692,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tc_fence_after();
       if (row < D) {
         float w[CPT];
-        tmem_ld16(t_s1 + lane_base + CPT * h, w);
+        tmem_ldn(t_s1 + lane_base + CPT * h, w);
         tmem_wait_ld();
 #pragma unroll
         for (int k8 = 0; k8 < CPT / 8; ++k8)
@@ -720,8 +707,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float inv_sig = 1.f / sig_prev;            // S_tmem = sig S of the last chunk
       {
         const uint32_t ts = t_s2 + lane_base + CPT * h;
-        tmem_ld16(ts, w);
-        tmem_ld16(ts + 64, sv);
+        tmem_ldn(ts, w);
+        tmem_ldn(ts + 64, sv);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < CPT; ++i) sv[i] *= inv_sig;
@@ -734,8 +721,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       {
         const uint32_t ts = t_s1 + lane_base + CPT * h;
-        tmem_ld16(ts, w);
-        tmem_ld16(ts + 64, sv);
+        tmem_ldn(ts, w);
+        tmem_ldn(ts + 64, sv);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < CPT; ++i) {
@@ -817,10 +804,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // after B_X1: the epilogue has then consumed this chunk's B_COEF phase,
       // so B_COEF can never run two phases ahead of its waiters.
       if (cch + 1 < nchunks) scan(cch + 1);
-      // all-gather of G2: in the cluster form the reduce threads have sent
-      // their G2 pieces to every CTA themselves; query owners report here
-      // that they are done reading their receive buffer (B_QFREE, off the
-      // critical path). The global form writes its G2 rows out here.
+      // all-gather of G2: key owners push their rows (whole 1 KB swizzle
+      // atoms) to every CTA; query owners report that they are done reading
+      // their receive buffer (B_QFREE, off the critical path).
       if (!wait_bar(&bars[B_G2OWN], par, a, abort_flag)) break;
       if (lane == 0) {
         if ((int)j * RP < C && XG) {
@@ -832,7 +818,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           bulk_commit_and_wait();
           fence_proxy_async_global();
           red_release_add(xfl + G * XFLAG_STRIDE, 1u);
-        } else if (!XG && (int)j * RP >= C) {
+        } else if ((int)j * RP < C) {
+#pragma unroll
+          for (int i = 0; i < G; ++i) {
+            const uint32_t p = (j + (uint32_t)i) % G;
+#pragma unroll
+            for (int fb = 0; fb < D / 64; ++fb)
+              bulk_push(mapa(sbase + Lay::G2 + (uint32_t)(fb * 64 * 128) + j * (uint32_t)(RP * 128), p),
+                        sbase + Lay::G2OWN + (uint32_t)(fb * RPK * 128), (uint32_t)(RPK * 128),
+                        mapa(smem_u32(&bars[B_G2]), p));
+          }
+        } else if (!XG) {
           // done reading this chunk's receive buffer: query rows of the next
           // chunk may be pushed here
 #pragma unroll

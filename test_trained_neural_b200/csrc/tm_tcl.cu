@@ -515,18 +515,20 @@ __global__ void __launch_bounds__(UP_NT, 1)
 // tokens). One CTA per unit = (layer l, stream, block of 128 rows of W_l, a
 // range of up to `tpu` 64-column tiles). The contraction's A operands, -c G
 // and -e G of the block's rows over the whole chunk (K = C), are loaded once.
-// The MMAs run per 64-column tile (X columns in one of two slots, the U_W | U_S
-// accumulators in one of two TMEM pairs); the fp32 W and S stream through four
-// slots of 32-column half tiles, so that up to four half tiles of state are in
-// flight while one is updated and stored:
+// The MMAs run per 64-column tile (X columns in one of two slots, reused as
+// soon as the tile's MMAs are done; the U_W | U_S accumulators in one of two
+// TMEM pairs); the fp32 W and S stream through four slots of 32-column half
+// tiles, so that up to four half tiles of state are in flight while one is
+// updated and stored:
 //   warp 0      TMA loads (state half tiles first: they do not depend on the
 //               previous kernel; the operands after griddepcontrol.wait)
 //   warp 1      TMEM allocation; MMA issue (M = 128 rows, N = 64, K = C)
-//   warp 2      TMA stores of W' and S' per half tile, of the fp16 W' per
-//               tile, each slot freed once its stores have read it
+//   warp 2      TMA stores of W' and S' per half tile, each slot freed once
+//               its stores have read it
 //   warps 4-11  epilogue: the thread owning TMEM lane r (row r) and 16 of a
 //               half tile's 32 columns computes W' = B W + c_S S + U_W,
-//               S' = A S + U_S in place and the fp16 W' into the X slot
+//               S' = A S + U_S in place, and writes the fp16 W' of its 16
+//               columns (32 contiguous bytes) straight to global memory
 // Every wait is bounded and also gives up once another role has flagged an
 // abort; after an abort the producer waits (bounded) for its copies in
 // flight and the MMA warp for its MMAs before TMEM is freed.
@@ -537,6 +539,7 @@ struct Up2Layer {
   int M, mtiles, ntiles, nranges, first;       // rows of W_l, 128-row blocks, 64-column tiles, ranges, first unit
   int b_rows_per_stream;                       // rows of the X source per stream
   long long b_row_off;                         // first X row of the chunk (layer 1 reads the keys)
+  op_t *wb;                                    // fp16 copy of W_l, [streams, M, 64 ntiles] row-major
 };
 struct Up2Args {
   Up2Layer l[kMaxL];
@@ -546,7 +549,7 @@ struct Up2Args {
   unsigned long long wait_ns;
   int inject;                                  // test hook, as in GemmArgs
 };
-// shared memory: A operands, two X (or fp16 W') slots, four state slots
+// shared memory: A operands, two X slots, four state slots
 __host__ __device__ constexpr uint32_t up2_a_bytes(int C) { return 2u * (uint32_t)C * 128u; }
 __host__ __device__ constexpr uint32_t up2_x_bytes(int C) { return (uint32_t)(C > 128 ? C : 128) * 128u; }
 __host__ __device__ constexpr uint32_t up2_ws_bytes() { return 2u * UP_BOX; }   // W and S, 32 columns each
@@ -577,7 +580,7 @@ __global__ void __launch_bounds__(UP2_NT, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *sm =
       reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t a_full, x_full[2], mma_done[2], acc_free[2], x_free[2];
+  __shared__ uint64_t a_full, x_full[2], mma_done[2], acc_free[2];
   __shared__ uint64_t ws_full[UP2_WS], epi_done[UP2_WS], ws_free[UP2_WS], fin, never;
   __shared__ uint32_t tslot;
   __shared__ int abort_flag;
@@ -609,7 +612,6 @@ __global__ void __launch_bounds__(UP2_NT, 1)
       mbar_init(&x_full[b], 1);
       mbar_init(&mma_done[b], 1);
       mbar_init(&acc_free[b], 8);
-      mbar_init(&x_free[b], 1);
     }
     for (int b = 0; b < UP2_WS; ++b) {
       mbar_init(&ws_full[b], 1);
@@ -658,7 +660,8 @@ __global__ void __launch_bounds__(UP2_NT, 1)
       a_armed = 1;
       for (int jj = 0; jj < nt; ++jj) {
         const int b = jj & 1;
-        if (jj >= 2 && !up2_wait(&x_free[b], (uint32_t)(((jj - 2) >> 1) & 1), a, abort)) break;
+        // the slot's previous X (tile jj - 2) has been read by its MMAs
+        if (jj >= 2 && !up2_wait(&mma_done[b], (uint32_t)(((jj - 2) >> 1) & 1), a, abort)) break;
         mbar_arrive_expect_tx(&x_full[b], x_bytes);
         for (int kp = 0; kp < C / 64; ++kp)
           tma_load_2d(x_slot(b) + kp * 64 * 128, &m.b[l], &x_full[b], 64 * (j0 + jj), (int)(brow + 64 * kp));
@@ -708,33 +711,23 @@ __global__ void __launch_bounds__(UP2_NT, 1)
     __syncwarp();
   } else if (warp == 2) {
     // ------------------------------------------------------------ stores
-    // One bulk group per half tile (its W' and S', and on odd half tiles the
-    // tile's fp16 W'); a group's slots are released once the next group has
-    // been issued and the earlier ones have read their sources, so one group
-    // stays in flight while the next half tile is stored.
+    // One bulk group per half tile (its W' and S'); a group's slot is released
+    // once the next group has been issued and the earlier ones have read
+    // their sources, so one group stays in flight while the next is stored.
     if (lane == 0) {
-      int pend_ws = -1, pend_x = -1;           // slots of the newest group, released one group later
+      int pend = -1;                           // slot of the newest group, released one group later
       for (int h2 = 0; h2 < nh; ++h2) {
         const int b = h2 % UP2_WS, col = 64 * j0 + 32 * h2;
         if (!up2_wait(&epi_done[b], (uint32_t)((h2 / UP2_WS) & 1), a, abort)) break;
         tma_store_3d(&m.w[l], w_slot(b), col, 128 * mt, s);
         tma_store_3d(&m.s[l], s_slot(b), col, 128 * mt, s);
-        int xb = -1;
-        if (h2 & 1) {                          // the tile's fp16 W' is complete (both halves)
-          const int jj = h2 >> 1;
-          xb = jj & 1;
-          tma_store_3d(&m.wb[l], x_slot(xb), 64 * (j0 + jj), 128 * mt, s);
-        }
         bulk_commit_group();
-        bulk_wait_group_read<1>();             // every group but this one has read its slots
-        if (pend_ws >= 0) mbar_arrive(&ws_free[pend_ws]);
-        if (pend_x >= 0) mbar_arrive(&x_free[pend_x]);
-        pend_ws = b;
-        pend_x = xb;
+        bulk_wait_group_read<1>();             // every group but this one has read its slot
+        if (pend >= 0) mbar_arrive(&ws_free[pend]);
+        pend = b;
       }
       bulk_wait_group_read<0>();
-      if (pend_ws >= 0) mbar_arrive(&ws_free[pend_ws]);
-      if (pend_x >= 0) mbar_arrive(&x_free[pend_x]);
+      if (pend >= 0) mbar_arrive(&ws_free[pend]);
     }
     __syncwarp();
   } else if (warp >= UP2_EPI0) {
@@ -765,7 +758,7 @@ __global__ void __launch_bounds__(UP2_NT, 1)
         if (r < rows) {
           unsigned char *wr = w_slot(b) + r * 128;
           unsigned char *sr = s_slot(b) + r * 128;
-          unsigned char *br = x_slot(xb) + r * 128;
+          uint32_t hw[8];                      // fp16 W' of this thread's 16 columns
 #pragma unroll
           for (int jc = 0; jc < 4; ++jc) {
             const uint32_t o = (uint32_t)(((4 * h + jc) ^ (r & 7)) << 4);
@@ -777,11 +770,13 @@ __global__ void __launch_bounds__(UP2_NT, 1)
                                           sc.y * x.z + us[4 * jc + 2], sc.y * x.w + us[4 * jc + 3]);
             *reinterpret_cast<float4 *>(wr + o) = wn;
             *reinterpret_cast<float4 *>(sr + o) = sn;
-            // fp16 row of the tile: columns 32 hs + 16 h + 4 jc .. + 3, in
-            // 16-byte chunk 4 hs + 2 h + jc / 2
-            const uint32_t ob = (uint32_t)((((4 * hs + 2 * h + (jc >> 1)) ^ (r & 7)) << 4) + (jc & 1) * 8);
-            *reinterpret_cast<uint2 *>(br + ob) = make_uint2(pack_h2(wn.x, wn.y), pack_h2(wn.z, wn.w));
+            hw[2 * jc] = pack_h2(wn.x, wn.y);
+            hw[2 * jc + 1] = pack_h2(wn.z, wn.w);
           }
+          op_t *dst = ly.wb + (long long)s * ly.M * (64 * ly.ntiles) + (long long)(128 * mt + r) * (64 * ly.ntiles) +
+                      64 * (j0 + jj) + 32 * hs + 16 * h;
+          *reinterpret_cast<uint4 *>(dst) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4 *>(dst + 8) = make_uint4(hw[4], hw[5], hw[6], hw[7]);
         }
         fence_proxy_async_smem();              // the TMA stores read these rows
         __syncwarp();
@@ -886,7 +881,7 @@ __global__ void __launch_bounds__(FB_NT, 1)
   unsigned char *abuf =
       reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char *ring = abuf + FB_ABUF;
-  __shared__ uint64_t full[FB_STAGES], empty[FB_STAGES], xbar, done, ready, never;
+  __shared__ uint64_t full[FB_STAGES], empty[FB_STAGES], xbar, done, ready, flushed, never;
   __shared__ uint32_t tslot;
   __shared__ int abort_flag;
   __shared__ float2 cef[128];
@@ -906,7 +901,8 @@ __global__ void __launch_bounds__(FB_NT, 1)
     for (int i = 0; i < FB_STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     mbar_init(&xbar, 1);
     mbar_init(&done, 1);
-    mbar_init(&ready, 1);
+    mbar_init(&ready, FB_EPI / 32);
+    mbar_init(&flushed, FB_EPI / 32);
     mbar_init(&never, 1);
     abort_flag = 0;
     fence_barrier_init();
@@ -1001,17 +997,23 @@ __global__ void __launch_bounds__(FB_NT, 1)
       cef[tid] = *reinterpret_cast<const float2 *>(a.coef + 2 * ((long long)s * a.T + (long long)a.chunk * C + 128 * mt + tid));
     epi_sync();
     // Global traffic of the tile's outputs that the update reads (X, -c G,
-    // -e G) leaves from the tile in shared memory, row-contiguous, after the
-    // next phase's MMAs have been released (they only read the tile too).
+    // -e G) leaves from the tile in shared memory after the next phase's MMAs
+    // have been released (they only read the tile too). Each warp stores the
+    // part of the tile it wrote itself (its 32 rows, its quarter of the
+    // columns), whole row pieces per instruction, so that no warp waits for
+    // another before it overwrites the tile in the next epilogue, unless the
+    // next phase's width differs: then its column quarters overlap other
+    // warps' old ones, and every warp waits (bounded) until all have flushed
+    // (mbarrier `flushed`, one arrival per warp and phase).
     int pend_kind = 0, pend_l = 0, pend_N = 0;   // 1: X_l, 2: -c G_l and -e G_l
     auto flush = [&]() {
       if (!pend_kind || nkey == 0) return;
-      const int N = pend_N, nch = N / 8;
-      const int lnch = N == 64 ? 3 : (N == 128 ? 4 : (N == 256 ? 5 : 0));
-      for (int i = tid; i < nkey * nch; i += FB_EPI) {
-        int rr, ch;
-        if (lnch) { rr = i >> lnch; ch = i & (nch - 1); }
-        else { rr = i / nch; ch = i - rr * nch; }
+      const int N = pend_N, nchw = N / 4 / 8;    // 16-byte chunks of this warp's quarter of a row
+      const int ch0 = quarter * nchw;
+      for (int i = lane; i < 32 * nchw; i += 32) {
+        const int rr = 32 * (warp & 3) + i / nchw;   // tile row
+        const int ch = ch0 + i % nchw;
+        if (rr >= nkey) continue;
         const uint4 u = *reinterpret_cast<const uint4 *>(abuf + rb_chunk(128, rr, ch));
         if (pend_kind == 1) {
           *reinterpret_cast<uint4 *>(a.x_out[pend_l] + ((long long)s * 2 * C + 128 * mt + rr) * N + 8 * ch) = u;
@@ -1035,6 +1037,7 @@ __global__ void __launch_bounds__(FB_NT, 1)
     for (int p = 0; p < nphase; ++p) {
       const FbPhase f = fb_phase(a, p);
       const int N = f.N, cbeg = quarter * (N / 4), cend = cbeg + N / 4;
+      // (every warp handles TMEM lanes 32 (warp % 4).. and columns [cbeg, cend))
       const bool last_fwd = !f.bwd && f.l == L;
       const bool grad = f.bwd || last_fwd;
       // this thread's other operand of a gradient phase (V, or silu' of the
@@ -1050,12 +1053,18 @@ __global__ void __launch_bounds__(FB_NT, 1)
         for (int i = 0; i < 8; ++i)
           if (8 * i < N / 4) aux[i] = src[i];
       }
+      const bool width_change = pend_kind != 0 && nkey > 0 && pend_N != N;
       flush();                                   // the previous phase's outputs
-      if (tid == 0 && !mbar_wait(&done, (uint32_t)(p & 1), a.wait_ns)) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&flushed);
+      // one lane per warp waits for this phase's MMAs and, when the width
+      // changes, for every warp's flush of the old outputs
+      if (lane == 0 && (!mbar_wait(&done, (uint32_t)(p & 1), a.wait_ns) ||
+                        (width_change && !mbar_wait(&flushed, (uint32_t)(p & 1), a.wait_ns)))) {
         atomicCAS(a.status, 0, kDevTimeout);
         abort_flag = 1;
       }
-      epi_sync();
+      __syncwarp();
       if (*(volatile int *)&abort_flag) break;
       tc_fence_after();
 #pragma unroll
@@ -1122,11 +1131,12 @@ __global__ void __launch_bounds__(FB_NT, 1)
         }
       }
       if (!grad) tmem_wait_st();                 // silu' stored into TMEM above
-      // the tile (generic-proxy writes) is read by the next phase's MMAs
+      // the tile (generic-proxy writes) is read by the next phase's MMAs:
+      // every warp reports its part
       fence_proxy_async_smem();
       tc_fence_before();
-      epi_sync();
-      if (tid == 0) mbar_arrive(&ready);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ready);
       pend_kind = grad ? 2 : (nkey > 0 ? 1 : 0);
       pend_l = f.bwd ? f.l - 1 : f.l;
       pend_N = N;
@@ -1577,6 +1587,7 @@ cudaError_t TclGroup::setup() {
       u.nranges = (u.ntiles + ua2.tpu - 1) / ua2.tpu;
       u.first = up2_units;
       u.b_rows_per_stream = l == 1 ? T : 2 * C;
+      u.wb = wbf + ia.boff[l - 1];
       up2_units += S * u.mtiles * u.nranges;
     }
   }
