@@ -259,14 +259,28 @@ def sweep_chunk(args, w: W.Workload, sizes):
                           "workspace_bytes": ws.numel()}), flush=True)
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one run of the
-# chunk walker (the cluster kernel for 15 streams and the global-exchange
-# kernel for the 16th), from one ncu --set full capture of a shortened case
-# of the long d=128 workload (16 streams x 4096 tokens: 64.16 + 9.94 MB and
-# 4.32 + 0 MB; the summary is kept under profiles/). The traffic grows with
-# the tokens processed (inputs and reads stream through once, the state stays
-# on chip), so a full run is that figure scaled by tokens.
-CAPTURED_TRAFFIC = {("tc", "mlp2-d128-long"): (64.163584e6 + 9.935360e6 + 4.315904e6, 16 * 4096)}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) measured by ncu
+# inside the dominant kernels' launches on shortened cases (summaries under
+# profiles/), with the number of tokens each capture covered; a full run is
+# that figure scaled by tokens.
+# - long d=128 workload: the chunk walker (cluster kernel for 15 streams,
+#   global-exchange kernel for the 16th) on 16 streams x 65536 tokens, whose
+#   537 MB of reads y are several times L2 so their write-back is counted:
+#   784.7 + 483.3 MB and 52.5 + 4.6 MB. The state stays on chip, so the
+#   traffic is the token inputs and outputs and grows with the tokens.
+# - deep workload: one fused forward/backward launch and one update launch of
+#   a group of 8 streams for one chunk of 128 tokens: 4.01 + 0 MB and
+#   18.13 + 0 MB (the update's writes stay in L2 and are written back after
+#   its launch, outside the window).
+# - README-shape workload (d=384, 2 streams x 1024 tokens): every launch of
+#   one tm_run (token conversion, initial copy, coefficients, 16 chunks of
+#   three per-phase GEMM launches and one update): 487.9 MB read, 0 written
+#   inside the launches (ncu flushes the caches before each launch, so these
+#   reads are cold-cache).
+CAPTURED_TRAFFIC = {("tc", "mlp2-d128-long"): (784.695040e6 + 483.341568e6 + 52.528896e6 + 4.637184e6, 16 * 65536),
+                    ("tcl", "mlp4-d128-deep"): (4.007936e6 + 18.134528e6, 8 * 128),
+                    ("tcl", "mlp2-d384-readme"): (3.153e6 + 18.885e6 + 0.034e6
+                                                  + 16 * (2.579e6 + 3.269e6 + 2.875e6 + 20.394e6), 2 * 1024)}
 
 
 def traffic_per_launch(path: str, w: W.Workload):
@@ -574,9 +588,14 @@ def main():
                 "sm_mhz_seen": sm_mhz}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = traffic_per_launch(path_used, w)
+    fused = all(n <= 256 for n in w.dims)
+    upd = "tcl_update2_kernel" if w.C <= 128 else "tcl_update_kernel"
     roof["kernel"] = {"tc": "tc_chunk_kernel (cluster and global-exchange forms)",
-                      "tcl": "tcl_fb_kernel + tcl_update_kernel",
-                      "tcl-phased": "tcl_gemm_kernel"}.get(path_used, "simt_chunk_kernel")
+                      "tcl": ("tcl_fb_kernel + " if fused else "tcl_gemm_kernel + ") + upd,
+                      "tcl-phased": "tcl_gemm_kernel + " + upd}.get(path_used, "simt_chunk_kernel")
+    if roof["traffic"] is not None:
+        roof["traffic_scope"] = ("DRAM bytes inside the kernels' launches per tm_run, from an ncu capture "
+                                 "of a shortened case scaled by tokens (profiles/)")
 
     e2e = None
     if not args.no_e2e:

@@ -15,20 +15,33 @@
 namespace tmem {
 namespace {
 
-// 8 elements per thread and iteration (16-byte loads and stores), grid-stride.
-__global__ void tokens_f16_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__ q, uint4 *__restrict__ k16,
-                                  uint4 *__restrict__ q16, long long n8) {
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < 2 * n8;
-       i += (long long)gridDim.x * blockDim.x) {
-    const bool isk = i < n8;
-    const long long j = isk ? i : i - n8;
-    const uint4 u = isk ? k[j] : q[j];
-    const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&u);
-    uint4 o;
-    __half2 *h = reinterpret_cast<__half2 *>(&o);
+__device__ __forceinline__ uint4 to_f16x8(uint4 u) {
+  const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&u);
+  uint4 o;
+  __half2 *h = reinterpret_cast<__half2 *>(&o);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) h[e] = __float22half2_rn(__bfloat1622float2(b[e]));
-    (isk ? k16 : q16)[j] = o;
+  for (int e = 0; e < 4; ++e) h[e] = __float22half2_rn(__bfloat1622float2(b[e]));
+  return o;
+}
+
+// Grid-stride over 16-byte pieces (8 elements) of k then q; each thread keeps
+// four independent loads in flight before it converts and stores them.
+constexpr int CV_UNROLL = 4;
+__global__ void __launch_bounds__(256) tokens_f16_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__ q,
+                                                         uint4 *__restrict__ k16, uint4 *__restrict__ q16, long long n8) {
+  const long long total = 2 * n8, stride = (long long)gridDim.x * blockDim.x;
+  for (long long base = (long long)blockIdx.x * blockDim.x + threadIdx.x; base < total; base += stride * CV_UNROLL) {
+    uint4 u[CV_UNROLL];
+#pragma unroll
+    for (int r = 0; r < CV_UNROLL; ++r) {
+      const long long i = base + r * stride;
+      if (i < total) u[r] = i < n8 ? __ldcs(k + i) : __ldcs(q + (i - n8));
+    }
+#pragma unroll
+    for (int r = 0; r < CV_UNROLL; ++r) {
+      const long long i = base + r * stride;
+      if (i < total) (i < n8 ? k16[i] : q16[i - n8]) = to_f16x8(u[r]);
+    }
   }
 }
 
@@ -44,7 +57,7 @@ cudaError_t tokens_f16_launch(const Problem &p, cudaStream_t stream) {
   if (n % 8 != 0 || !p.k16 || !p.q16) return cudaErrorInvalidValue;
   const long long n8 = (long long)(n / 8);
   long long blocks = (2 * n8 + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks > 148 * 8) blocks = 148 * 8;     // 8 CTAs of 256 threads per SM
   tokens_f16_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
       static_cast<const uint4 *>(p.k), static_cast<const uint4 *>(p.q), static_cast<uint4 *>(const_cast<void *>(p.k16)),
       static_cast<uint4 *>(const_cast<void *>(p.q16)), n8);
