@@ -644,6 +644,12 @@ __global__ void __launch_bounds__(UP2_NT, 1)
   if (warp == 0 && lane == 0) {
     if (a.inject && !injected_wait(&never, a.status, a.wait_ns)) *abort = 1;
     for (int h2 = 0; h2 < nh && h2 < UP2_WS && !*abort; ++h2) load_ws(h2);
+    // the unit's later half tiles wait for a free slot; bring them into L2 now
+    // so that their loads, when the slots free up, do not wait on DRAM
+    for (int h2 = UP2_WS; h2 < nh && !*abort; ++h2) {
+      tma_prefetch_l2_3d(&m.w[l], 64 * j0 + 32 * h2, 128 * mt, s);
+      tma_prefetch_l2_3d(&m.s[l], 64 * j0 + 32 * h2, 128 * mt, s);
+    }
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
@@ -791,6 +797,241 @@ __global__ void __launch_bounds__(UP2_NT, 1)
 }
 
 // ------------------------------------------------------------------------
+// The state update with the contraction transposed (chunks of at most 128
+// tokens, every layer input width a multiple of 128). One CTA per unit =
+// (layer l, stream, block of 128 columns of W_l, block of up to 256 rows):
+//   U_W^T = X^T (-c G),  U_S^T = X^T (-e G)   (M = 128 columns, N = rows, K = C)
+// so that TMEM lane i holds column i of the block and TMEM column j row j.
+// A warp then owns 32 consecutive columns: it reads a row's W and S from a
+// staged slot as one 128-byte piece and writes W', S' (fp32) and the fp16 copy
+// of W' straight to global memory, each a whole row piece per instruction.
+// The state streams through 16-row slots (16 KB: W and S of 16 rows x 128
+// columns); once the MMAs have read the operands, their shared memory becomes
+// more slots, so most of a unit's state is in flight at once, and a slot is
+// refilled as soon as its four readers are done with it.
+//   warps 0-15  epilogue: warp w owns TMEM lanes (columns) 32 (w % 4) .. +31
+//               and the 16-row chunks i = w / 4, w / 4 + 4, ...
+//   warp 16     TMA loads (the first slots' state before waiting for the
+//               preceding kernel, which does not write it; the operands after)
+//   warp 17     TMEM allocation; MMA issue, rows 0-127 and 128-255 committed
+//               separately so that the epilogue starts on the first half
+// Every wait is bounded and gives up once another role has flagged an abort.
+constexpr int UP3_EPI = 16;                    // epilogue warps
+constexpr int UP3_NT = (UP3_EPI + 2) * 32;
+constexpr int UP3_SLOT = 16384;                // W and S of 16 rows x 128 fp32 columns
+constexpr int UP3_NSLOT_MEM = 14;              // slots' worth of dynamic shared memory
+constexpr int UP3_NS = 12;                     // slots in the ring (a multiple of 4)
+constexpr size_t UP3_SMEM = (size_t)UP3_NSLOT_MEM * UP3_SLOT + 1024;
+struct Up3Layer {
+  int M, cols, rblocks, cblocks, first;        // rows and columns of W_l, 256-row and 128-column blocks, first unit
+  int b_rows_per_stream;                       // rows of the X source per stream
+  long long b_row_off;                         // first X row of the chunk (layer 1 reads the keys)
+  float *w, *s;                                // fp32 W_l, S_l of stream 0 (stream stride P)
+  op_t *wb;                                    // fp16 copy of W_l, [streams, M, cols]
+};
+struct Up3Args {
+  Up3Layer l[kMaxL];
+  int L, C, chunk, nchunks;
+  long long P;
+  const float *scal;                           // [streams, nchunks, 4] (B, A, c_S, -)
+  int *status;
+  unsigned long long wait_ns;
+  int inject;                                  // test hook, as in GemmArgs
+};
+struct Up3Maps {
+  CUtensorMap a[kMaxL], a2[kMaxL], b[kMaxL];   // -c G_l, -e G_l [S*C, d_l]; X_{l-1} (fp16, 64 x 64 boxes)
+  CUtensorMap w[kMaxL], s[kMaxL];              // fp32 W_l, S_l as {cols, rows, stream}, 128 x 16 boxes
+};
+// operand bytes: X^T (128 columns x C) and -c G, -e G (256 rows x C each), fp16
+__host__ __device__ constexpr uint32_t up3_op_bytes(int C) { return 1280u * (uint32_t)C; }
+// slots before the operand region (the rest of the ring overlays the operands)
+__host__ __device__ constexpr int up3_dedicated(int C) {
+  return UP3_NSLOT_MEM - (int)((up3_op_bytes(C) + UP3_SLOT - 1) / UP3_SLOT);
+}
+
+__device__ bool up3_wait(uint64_t *bar, uint32_t par, const Up3Args &a, volatile int *abort) {
+  if (mbar_try_wait(bar, par)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i)
+      if (mbar_try_wait(bar, par)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > a.wait_ns) {
+      atomicCAS(a.status, 0, kDevTimeout);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(UP3_NT, 1)
+    tcl_update3_kernel(const __grid_constant__ Up3Args a, const __grid_constant__ Up3Maps m) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char *sm =
+      reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t full[UP3_NS], freed[UP3_NS], op_full, mma_done[2], fin, never;
+  __shared__ uint32_t tslot;
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  // this CTA's unit
+  const int u = blockIdx.x;
+  int l = 0;
+  while (l + 1 < a.L && u >= a.l[l + 1].first) ++l;
+  const Up3Layer &ly = a.l[l];
+  const int per = ly.rblocks * ly.cblocks, i0 = u - ly.first;
+  const int s = i0 / per, rb = (i0 % per) / ly.cblocks, cb = i0 % ly.cblocks;
+  const int N = ly.M - 256 * rb < 256 ? ly.M - 256 * rb : 256;   // rows of this unit (a multiple of 64)
+  const int nch = N / 16;                      // 16-row chunks
+  const int nhalf = N > 128 ? 2 : 1;
+  const int C = a.C;
+  const int NSD = up3_dedicated(C);
+  unsigned char *opa = sm + NSD * UP3_SLOT;    // X^T: 2 feature blocks of 64 columns x C
+  unsigned char *opc = opa + 256 * C;          // -c G: up to 4 feature blocks of 64 rows x C
+  unsigned char *ope = opc + 512 * C;          // -e G
+  auto slot_w = [&](int b) { return sm + b * UP3_SLOT; };
+
+  if (tid == 0) {
+    for (int b = 0; b < UP3_NS; ++b) {
+      mbar_init(&full[b], 1);
+      mbar_init(&freed[b], 4);                 // the four warps reading the slot's columns
+    }
+    mbar_init(&op_full, 1);
+    mbar_init(&mma_done[0], 1);
+    mbar_init(&mma_done[1], 1);
+    mbar_init(&fin, 1);
+    mbar_init(&never, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == UP3_EPI + 1) { tmem_alloc(&tslot, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = tslot;
+  volatile int *abort = &abort_flag;
+
+  int armed = 0, op_armed = 0;                 // chunks whose loads were issued; operands issued
+  auto load_chunk = [&](int i) {               // rows 16 i .. 16 i + 15 of the unit into slot i % NS
+    const int b = i % UP3_NS;
+    unsigned char *dst = slot_w(b);
+    mbar_arrive_expect_tx(&full[b], (uint32_t)UP3_SLOT);
+    tma_load_3d(dst, &m.w[l], &full[b], 128 * cb, 256 * rb + 16 * i, s);
+    tma_load_3d(dst + UP3_SLOT / 2, &m.s[l], &full[b], 128 * cb, 256 * rb + 16 * i, s);
+    armed = i + 1;
+  };
+  if (warp == UP3_EPI && lane == 0) {
+    if (a.inject && !injected_wait(&never, a.status, a.wait_ns)) *abort = 1;
+    for (int i = 0; i < nch && i < NSD && !*abort; ++i) load_chunk(i);
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  if (warp == UP3_EPI) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && !*abort) {
+      const long long brow = (long long)s * ly.b_rows_per_stream + ly.b_row_off;
+      mbar_arrive_expect_tx(&op_full, (uint32_t)(256 * C + 2 * 2 * N * C));
+      for (int kp = 0; kp < C / 64; ++kp) {
+        for (int f = 0; f < 2; ++f)
+          tma_load_2d(opa + f * C * 128 + kp * 64 * 128, &m.b[l], &op_full, 128 * cb + 64 * f, (int)(brow + 64 * kp));
+        for (int f = 0; f < N / 64; ++f) {
+          tma_load_2d(opc + f * C * 128 + kp * 64 * 128, &m.a[l], &op_full, 256 * rb + 64 * f, s * C + 64 * kp);
+          tma_load_2d(ope + f * C * 128 + kp * 64 * 128, &m.a2[l], &op_full, 256 * rb + 64 * f, s * C + 64 * kp);
+        }
+      }
+      op_armed = 1;
+      bool ops_free = false;                   // the MMAs have read the operand region
+      for (int i = armed; i < nch; ++i) {
+        const int b = i % UP3_NS, use = i / UP3_NS;
+        bool ok;
+        if (use == 0) {                        // first use of a slot over the operands
+          ok = ops_free || up3_wait(&mma_done[nhalf - 1], 0, a, abort);
+          ops_free = ok;
+        } else {
+          ok = up3_wait(&freed[b], (uint32_t)((use - 1) & 1), a, abort);
+        }
+        if (!ok) break;
+        load_chunk(i);
+      }
+    }
+    if (lane == 0 && *abort) {
+      // copies still in flight into this CTA's shared memory finish first
+      if (op_armed) mbar_wait(&op_full, 0, a.wait_ns);
+      for (int i = 0; i < armed; ++i)
+        if (i + UP3_NS >= armed) mbar_wait(&full[i % UP3_NS], (uint32_t)((i / UP3_NS) & 1), a.wait_ns);
+    }
+    __syncwarp();
+  } else if (warp == UP3_EPI + 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      if (up3_wait(&op_full, 0, a, abort)) {
+        tc_fence_after();
+        const uint32_t xa = smem_u32(opa), gc = smem_u32(opc), ge = smem_u32(ope);
+        for (int h = 0; h < nhalf; ++h) {
+          const int nh = N - 128 * h < 128 ? N - 128 * h : 128;
+          const uint32_t idesc = idesc_f16(128, nh, true, true);
+          const uint32_t boff = (uint32_t)(2 * h) * (uint32_t)C * 128u;   // feature blocks 2h, 2h + 1
+          for (int ks = 0; ks < C / 16; ++ks) {
+            const uint64_t ad = desc_mnmajor(xa, C, ks);
+            umma_f16(tm + 128u * (uint32_t)h, ad, desc_mnmajor(gc + boff, C, ks), idesc, ks != 0);
+            umma_f16(tm + 256u + 128u * (uint32_t)h, ad, desc_mnmajor(ge + boff, C, ks), idesc, ks != 0);
+          }
+          umma_commit(&mma_done[h]);
+        }
+      }
+      // every MMA this CTA issued has completed before TMEM is freed
+      umma_commit(&fin);
+      mbar_wait(&fin, 0, a.wait_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int lq = warp & 3, rq = warp >> 2;
+    const int col = 32 * lq + lane;            // column of the block = TMEM lane
+    const uint32_t lb = (uint32_t)(32 * lq) << 16;
+    const float4 sc = *reinterpret_cast<const float4 *>(a.scal + 4 * ((long long)s * a.nchunks + a.chunk));
+    const long long gcol = 128LL * cb + col;
+    float *wout = ly.w + (long long)s * a.P + gcol;
+    float *sout = ly.s + (long long)s * a.P + gcol;
+    op_t *bout = ly.wb + (long long)s * ly.M * ly.cols + gcol;
+    int seen = 0;                              // halves of the accumulator known complete
+    for (int i = rq; i < nch; i += 4) {
+      const int h = 16 * i >= 128 ? 1 : 0;
+      if (seen <= h) {
+        if (!up3_wait(&mma_done[h], 0, a, abort)) break;
+        seen = h + 1;
+      }
+      const int b = i % UP3_NS;
+      if (!up3_wait(&full[b], (uint32_t)((i / UP3_NS) & 1), a, abort)) break;
+      tc_fence_after();
+      float uw[16], us[16];
+      tmem_ld16(tm + lb + 16u * (uint32_t)i, uw);
+      tmem_ld16(tm + lb + 256u + 16u * (uint32_t)i, us);
+      tmem_wait_ld();
+      const float *ws_ = reinterpret_cast<const float *>(slot_w(b)) + col;
+      const float *ss_ = ws_ + UP3_SLOT / 8;   // S follows W in the slot (8 KB = 2048 floats)
+      const long long row0 = 256LL * rb + 16 * i;
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        const float w = ws_[128 * r], x = ss_[128 * r];
+        const float wn = sc.x * w + sc.z * x + uw[r];
+        const float sn = sc.y * x + us[r];
+        const long long o = (row0 + r) * ly.cols;
+        wout[o] = wn;
+        sout[o] = sn;
+        bout[o] = __float2half_rn(wn);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&freed[b]);   // the slot may be refilled
+    }
+  }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  if (warp == UP3_EPI + 1) tmem_dealloc(tm, 512);
+}
+
+// ------------------------------------------------------------------------
 // Fused forward + backward of one chunk, for memories whose every layer is at
 // most 256 wide. One CTA per (128-row tile of the chunk's [keys; queries],
 // stream) runs the whole chain that the per-phase kernels run as 2L - 1
@@ -818,7 +1059,9 @@ struct FbArgs {
   int L, C, T, chunk;
   int dims[kMaxL + 1];
   op_t *x_out[kMaxL + 1];            // [streams, 2C, d_l], key rows written (l = 1..L-1)
-  op_t *sp_out[kMaxL + 1];           // [streams, C, d_l] silu'(Z_l) of key rows
+  op_t *sp_out[kMaxL + 1];           // silu'(Z_l) of key rows, [streams, d_l / 8, C, 8]: 16-byte
+                                     // pieces of a row, consecutive rows adjacent (written and read
+                                     // back by the same thread; a warp's 32 rows are 512 contiguous bytes)
   op_t *gc_out[kMaxL + 1];           // [streams, C, d_l] -c G_l
   op_t *ge_out[kMaxL + 1];           // [streams, C, d_l] -e G_l
   float *y;                          // [streams, T, d]
@@ -912,6 +1155,22 @@ __global__ void __launch_bounds__(FB_NT, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = tslot;
+  // The tile's input rows (fp16 keys or queries) were converted before the
+  // chunk walk began, and every kernel of the walk waits for its predecessor
+  // before it signals its dependents, so they can be requested before waiting
+  // for the preceding kernel (the weights cannot).
+  auto load_x = [&]() {
+    const int d0 = a.dims[0];
+    mbar_arrive_expect_tx(&xbar, (uint32_t)(128 * d0 * 2));
+    for (int piece = 0; piece < 2; ++piece) {
+      const int r = 128 * mt + 64 * piece;
+      const CUtensorMap *src = r < C ? &m.k : &m.q;
+      const int row = s * a.T + a.chunk * C + (r < C ? r : r - C);
+      for (int f = 0; f < d0 / 64; ++f)
+        tma_load_2d(abuf + f * 128 * 128 + piece * 64 * 128, src, &xbar, 64 * f, row);
+    }
+  };
+  if (warp == FB_EPI / 32 && lane == 0 && !a.inject) load_x();
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == FB_EPI / 32) {
@@ -923,17 +1182,7 @@ __global__ void __launch_bounds__(FB_NT, 1)
       int total = 0;
       for (int p = 0; p < nphase; ++p) total += fb_phase(a, p).ns;
       int issued = 0, consumed = 0;
-      prefetch_tmap(&m.k);
-      prefetch_tmap(&m.q);
-      const int d0 = a.dims[0];
-      mbar_arrive_expect_tx(&xbar, (uint32_t)(128 * d0 * 2));
-      for (int piece = 0; piece < 2; ++piece) {
-        const int r = 128 * mt + 64 * piece;
-        const CUtensorMap *src = r < C ? &m.k : &m.q;
-        const int row = s * a.T + a.chunk * C + (r < C ? r : r - C);
-        for (int f = 0; f < d0 / 64; ++f)
-          tma_load_2d(abuf + f * 128 * 128 + piece * 64 * 128, src, &xbar, 64 * f, row);
-      }
+      if (a.inject) load_x();
       for (; issued < total && issued < FB_STAGES; ++issued) fb_load_slice(a, m, ring, full, s, issued);
       bool ok = true;
       for (int p = 0; p < nphase && ok; ++p) {
@@ -1047,11 +1296,17 @@ __global__ void __launch_bounds__(FB_NT, 1)
       const int spt = f.bwd ? sp_slot(f.l - 1) : -1;      // silu' of the layer below in TMEM?
       if (grad && key && spt < 0) {
         // fp16 silu' (backward) or bf16 values (last forward), 8 per 16 bytes
-        const uint4 *src = f.bwd ? reinterpret_cast<const uint4 *>(a.sp_out[f.l - 1] + ((long long)s * C + r) * N + cbeg)
-                                 : reinterpret_cast<const uint4 *>(a.v + tok * N + cbeg);
+        if (f.bwd) {
+          const uint4 *src = reinterpret_cast<const uint4 *>(a.sp_out[f.l - 1] + (long long)s * C * N) + (cbeg / 8) * C + r;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (8 * i < N / 4) aux[i] = src[i];
+          for (int i = 0; i < 8; ++i)
+            if (8 * i < N / 4) aux[i] = src[(long long)i * C];
+        } else {
+          const uint4 *src = reinterpret_cast<const uint4 *>(a.v + tok * N + cbeg);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (8 * i < N / 4) aux[i] = src[i];
+        }
       }
       const bool width_change = pend_kind != 0 && nkey > 0 && pend_N != N;
       flush();                                   // the previous phase's outputs
@@ -1094,9 +1349,9 @@ __global__ void __launch_bounds__(FB_NT, 1)
               for (int i = 0; i < 8; ++i) pk[i] = pack_h2(sp[2 * i], sp[2 * i + 1]);
               tmem_st8(tm + lb + (uint32_t)(slot + c0 / 2), pk);
             } else {
-              op_t *so = a.sp_out[f.l] + ((long long)s * C + r) * N + c0;
-              *reinterpret_cast<uint4 *>(so) = pack8(sp);
-              *reinterpret_cast<uint4 *>(so + 8) = pack8(sp + 8);
+              uint4 *so = reinterpret_cast<uint4 *>(a.sp_out[f.l] + (long long)s * C * N) + (c0 / 8) * C + r;
+              so[0] = pack8(sp);
+              so[C] = pack8(sp + 8);
             }
           }
         } else if (!key) {
@@ -1300,6 +1555,23 @@ bool map3d(CUtensorMap *m, CUtensorMapDataType dt, int el, const void *base, int
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over `streams` fp32 matrices [rows x cols] (matrix s at base + s *
+// stream_stride elements), box = box_cols x box_rows x 1, no swizzle: rows of
+// the box land in shared memory one after another (box_cols * 4 bytes each).
+bool map3d_f32_plain(CUtensorMap *m, const float *base, int cols, int rows, int streams, long long stream_stride,
+                     int box_cols, int box_rows) {
+  EncodeTiledFn fn = encode_fn_l();
+  if (!fn || (box_cols * 4) % 16 != 0 || box_cols > 256 || box_rows > 256) return false;
+  std::memset(m, 0, sizeof *m);
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)streams};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 4, (cuuint64_t)stream_stride * 4};
+  cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Workspace carve-up (bytes, 256-aligned pieces), per problem.
 struct Carve {
   size_t coef, scal, wbf, x[kMaxL + 1], sp[kMaxL + 1], g[kMaxL + 1], gc[kMaxL + 1], ge[kMaxL + 1];
@@ -1391,6 +1663,20 @@ cudaError_t launch_up2(const Up2Args &a, const UpMaps &m, int units, cudaStream_
   return cudaLaunchKernelEx(&cfg, tcl_update2_kernel, a, m);
 }
 
+cudaError_t launch_up3(const Up3Args &a, const Up3Maps &m, int units, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)units);
+  cfg.blockDim = dim3(UP3_NT);
+  cfg.dynamicSmemBytes = UP3_SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tcl_update3_kernel, a, m);
+}
+
 cudaError_t launch_up(const UpArgs &a, const UpMaps &m, int tiles, size_t smem, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)tiles);
@@ -1460,6 +1746,10 @@ struct TclGroup {
   int up_tiles;
   size_t up_smem_bytes;
   bool up2;                      // pipelined update kernel (C <= 128)
+  bool up3;                      // transposed update kernel (C <= 128, input widths multiples of 128)
+  Up3Args ua3;
+  Up3Maps um3;
+  int up3_units;
   Up2Args ua2;
   int up2_units;
   bool fused;
@@ -1592,6 +1882,43 @@ cudaError_t TclGroup::setup() {
     }
   }
 
+  // the transposed update: units of (layer, stream, 256-row block, 128-column block)
+  up3 = up2;
+  for (int l = 1; l <= L; ++l)
+    if (p.dims[l - 1] % 128 != 0 || p.dims[l] % 64 != 0) up3 = false;
+  if (up3) {
+    std::memset(&ua3, 0, sizeof ua3);
+    std::memset(&um3, 0, sizeof um3);
+    ua3.L = L;
+    ua3.C = C;
+    ua3.nchunks = nchunks;
+    ua3.P = (long long)p.P;
+    ua3.scal = scal;
+    ua3.status = p.status;
+    ua3.wait_ns = g_tcl_wait_ns;
+    ua3.inject = g_tcl_inject;
+    up3_units = 0;
+    for (int l = 1; l <= L; ++l) {
+      Up3Layer &u = ua3.l[l - 1];
+      u.M = p.dims[l];
+      u.cols = p.dims[l - 1];
+      u.rblocks = (u.M + 255) / 256;
+      u.cblocks = u.cols / 128;
+      u.first = up3_units;
+      u.b_rows_per_stream = l == 1 ? T : 2 * C;
+      u.w = p.W_end + p.layer_off[l - 1];
+      u.s = p.S_end + p.layer_off[l - 1];
+      u.wb = wbf + ia.boff[l - 1];
+      up3_units += S * u.rblocks * u.cblocks;
+      um3.a[l - 1] = mgc[l];
+      um3.a2[l - 1] = mge[l];
+      um3.b[l - 1] = l == 1 ? mk : mx[l - 1];
+      if (!map3d_f32_plain(&um3.w[l - 1], u.w, u.cols, u.M, S, (long long)p.P, 128, 16) ||
+          !map3d_f32_plain(&um3.s[l - 1], u.s, u.cols, u.M, S, (long long)p.P, 128, 16))
+        return cudaErrorInvalidValue;
+    }
+  }
+
   fused = p.fuse_fb && fb_ok(p);
   if (fused) {
     std::memset(&fa, 0, sizeof fa);
@@ -1662,6 +1989,11 @@ cudaError_t TclGroup::chunk(int ch) {
     if (err != cudaSuccess) return err;
   }
   // weight-update contractions of every layer, with the fused state update
+  if (up3) {
+    ua3.chunk = ch;
+    ua3.l[0].b_row_off = (long long)ch * C;
+    return launch_up3(ua3, um3, up3_units, stream);
+  }
   if (up2) {
     ua2.chunk = ch;
     ua2.l[0].b_row_off = (long long)ch * C;
@@ -1756,6 +2088,8 @@ cudaError_t tcl_launch(const Problem &p, cudaStream_t stream) {
                              (int)up_smem(128, 2));
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(tcl_update2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)up2_smem(128));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tcl_update3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)UP3_SMEM);
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
