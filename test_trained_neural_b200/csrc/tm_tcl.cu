@@ -73,6 +73,25 @@ __device__ __forceinline__ float tanh_approx(float x) {
 }
 __device__ __forceinline__ float sigm(float z) { return fmaf(0.5f, tanh_approx(0.5f * z), 0.5f); }
 
+// SiLU and its derivative of a pair of pre-activations in half precision,
+// for outputs that are fp16 operands anyway: with s = sigmoid(z) =
+// 1/2 + tanh(z/2)/2, x = z s and s' = s (1 + z (1 - s)). Returns the pairs
+// of x and s' as fp16 bits.
+__device__ __forceinline__ void silu_pair_h2(float z0, float z1, uint32_t &x, uint32_t &sp) {
+  const __half2 z = __floats2half2_rn(z0, z1);
+  const __half2 half = __float2half2_rn(0.5f), one = __float2half2_rn(1.0f);
+  __half2 h = __hmul2(z, half), t;
+  const uint32_t hb = *reinterpret_cast<const uint32_t *>(&h);
+  uint32_t tb;
+  asm("tanh.approx.f16x2 %0, %1;" : "=r"(tb) : "r"(hb));
+  t = *reinterpret_cast<const __half2 *>(&tb);
+  const __half2 sg = __hfma2(t, half, half);
+  const __half2 xx = __hmul2(z, sg);
+  const __half2 dd = __hmul2(sg, __hfma2(z, __hsub2(one, sg), one));
+  x = *reinterpret_cast<const uint32_t *>(&xx);
+  sp = *reinterpret_cast<const uint32_t *>(&dd);
+}
+
 // Two fp32 values as one fp16 pair (round to nearest even).
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
@@ -940,6 +959,12 @@ __global__ void __launch_bounds__(UP3_NT, 1)
         }
       }
       op_armed = 1;
+      // the later chunks wait for slots (over the operands, or refills); bring
+      // them into L2 behind the operands so that those loads do not wait on DRAM
+      for (int i = armed; i < nch; ++i) {
+        tma_prefetch_l2_3d(&m.w[l], 128 * cb, 256 * rb + 16 * i, s);
+        tma_prefetch_l2_3d(&m.s[l], 128 * cb, 256 * rb + 16 * i, s);
+      }
       bool ops_free = false;                   // the MMAs have read the operand region
       for (int i = armed; i < nch; ++i) {
         const int b = i % UP3_NS, use = i / UP3_NS;
@@ -994,6 +1019,7 @@ __global__ void __launch_bounds__(UP3_NT, 1)
     float *wout = ly.w + (long long)s * a.P + gcol;
     float *sout = ly.s + (long long)s * a.P + gcol;
     op_t *bout = ly.wb + (long long)s * ly.M * ly.cols + gcol;
+    const int cols = ly.cols;
     int seen = 0;                              // halves of the accumulator known complete
     for (int i = rq; i < nch; i += 4) {
       const int h = 16 * i >= 128 ? 1 : 0;
@@ -1010,16 +1036,20 @@ __global__ void __launch_bounds__(UP3_NT, 1)
       tmem_wait_ld();
       const float *ws_ = reinterpret_cast<const float *>(slot_w(b)) + col;
       const float *ss_ = ws_ + UP3_SLOT / 8;   // S follows W in the slot (8 KB = 2048 floats)
-      const long long row0 = 256LL * rb + 16 * i;
+      const int o0 = (256 * rb + 16 * i) * cols;   // element offset of the chunk's first row
+      float *wo = wout + o0, *so = sout + o0;
+      op_t *bo = bout + o0;
 #pragma unroll
       for (int r = 0; r < 16; ++r) {
         const float w = ws_[128 * r], x = ss_[128 * r];
         const float wn = sc.x * w + sc.z * x + uw[r];
         const float sn = sc.y * x + us[r];
-        const long long o = (row0 + r) * ly.cols;
-        wout[o] = wn;
-        sout[o] = sn;
-        bout[o] = __float2half_rn(wn);
+        *wo = wn;
+        *so = sn;
+        *bo = __float2half_rn(wn);
+        wo += cols;
+        so += cols;
+        bo += cols;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&freed[b]);   // the slot may be refilled
@@ -1331,27 +1361,22 @@ __global__ void __launch_bounds__(FB_NT, 1)
         tmem_wait_ld();
         if (!grad) {
           // hidden layer: X = silu(Z) for every row (the next operand), and
-          // silu'(Z) of key rows straight out
-          float x[16], sp[16];
+          // silu'(Z) of key rows straight out; both are fp16 operands, so they
+          // are computed in half precision, two at a time
+          uint32_t xh[8], sh[8];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float sg = sigm(z[i]);
-            x[i] = z[i] * sg;
-            sp[i] = sg * (1.f + z[i] * (1.f - sg));
-          }
+          for (int i = 0; i < 8; ++i) silu_pair_h2(z[2 * i], z[2 * i + 1], xh[i], sh[i]);
 #pragma unroll
-          for (int i = 0; i < 2; ++i) st_shared_v4(abuf + rb_chunk(128, row, c0 / 8 + i), pack8(x + 8 * i));
+          for (int i = 0; i < 2; ++i)
+            st_shared_v4(abuf + rb_chunk(128, row, c0 / 8 + i), make_uint4(xh[4 * i], xh[4 * i + 1], xh[4 * i + 2], xh[4 * i + 3]));
           if (key) {
             const int slot = sp_slot(f.l);
             if (slot >= 0) {
-              uint32_t pk[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) pk[i] = pack_h2(sp[2 * i], sp[2 * i + 1]);
-              tmem_st8(tm + lb + (uint32_t)(slot + c0 / 2), pk);
+              tmem_st8(tm + lb + (uint32_t)(slot + c0 / 2), sh);
             } else {
               uint4 *so = reinterpret_cast<uint4 *>(a.sp_out[f.l] + (long long)s * C * N) + (c0 / 8) * C + r;
-              so[0] = pack8(sp);
-              so[C] = pack8(sp + 8);
+              so[0] = make_uint4(sh[0], sh[1], sh[2], sh[3]);
+              so[C] = make_uint4(sh[4], sh[5], sh[6], sh[7]);
             }
           }
         } else if (!key) {
