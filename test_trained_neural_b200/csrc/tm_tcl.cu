@@ -49,6 +49,9 @@ struct GemmArgs {
   int kind;
   int C, T, chunk;               // chunk size, tokens per stream, chunk index
   int M, N, K;                   // per-stream GEMM: rows, cols, reduction
+  int streams, ksplit;           // grid z = streams x ksplit: K is split over ksplit CTAs per tile
+  float *part;                   // [tiles, ksplit, 128, N] fp32 partial tiles (ksplit > 1)
+  unsigned *cnt;                 // [tiles] arrivals per tile; the last CTA resets it to 0
   int n_out;                     // row length of the epilogue's outputs
   int a_rows_per_stream;         // rows of the A source per stream
   int b_rows_per_stream;
@@ -167,7 +170,10 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
   __shared__ uint32_t tslot;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   constexpr int kind = KIND;
-  const int nk = a.K / KB;
+  // this CTA's share of the reduction: K blocks [kb0, kb0 + nk)
+  const int nkt = a.K / KB;
+  const int kz = blockIdx.z / a.streams;
+  const int kb0 = nkt * kz / a.ksplit, nk = nkt * (kz + 1) / a.ksplit - kb0;
   const uint32_t ncols = 256u;
   constexpr int STAGES = 4;
   constexpr uint32_t STAGE_BYTES = STAGE_BYTES_MM;
@@ -196,7 +202,7 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
     else idesc = idesc_f16(128, a.N, false, false);
     for (int kb = 0; kb < nk && kb < STAGES && ok; ++kb) {
       mbar_arrive_expect_tx(&full[kb], tx);
-      load_stage(a, &mA, &mA2, &mB, sm + kb * STAGE_BYTES, &full[kb], s, mt, nt, kb);
+      load_stage(a, &mA, &mA2, &mB, sm + kb * STAGE_BYTES, &full[kb], s, mt, nt, kb0 + kb);
     }
     for (int kb = 0; kb < nk && ok; ++kb) {
       const int st = kb % STAGES;
@@ -217,7 +223,7 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
       if (kb + STAGES < nk) {
         if (!wait_b(&empty[st], ph, a)) { ok = false; break; }
         mbar_arrive_expect_tx(&full[st], tx);
-        load_stage(a, &mA, &mA2, &mB, sm + st * STAGE_BYTES, &full[st], s, mt, nt, kb + STAGES);
+        load_stage(a, &mA, &mA2, &mB, sm + st * STAGE_BYTES, &full[st], s, mt, nt, kb0 + kb + STAGES);
       }
     }
     umma_commit(&done);
@@ -234,6 +240,52 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
   const uint32_t lb = (uint32_t)(32 * (warp & 3)) << 16;
   const int half = warp >> 2;                    // this warp's half of the tile's columns
   const int cbeg = half * (a.N / 2), cend = cbeg + a.N / 2;
+  // Split K: every CTA of the tile stores its partial sums; the last to
+  // arrive adds them up (in split order, so the result does not depend on
+  // the arrival order) and runs the epilogue.
+  const int tile = (s * gridDim.y + mt) * gridDim.x + nt;
+  const float *parts = nullptr;
+  if (ok && a.ksplit > 1) {
+    __shared__ int last;
+    float *mine = a.part + ((long long)tile * a.ksplit + kz) * 128 * a.N + (long long)row * a.N;
+    for (int c0 = cbeg; c0 < cend; c0 += 16) {
+      float z[16];
+      tmem_ld16(tm + lb + c0, z);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i4 = 0; i4 < 4; ++i4)
+        __stcg(reinterpret_cast<float4 *>(mine + c0 + 4 * i4), make_float4(z[4 * i4], z[4 * i4 + 1], z[4 * i4 + 2], z[4 * i4 + 3]));
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      const unsigned prev = atomicAdd(a.cnt + tile, 1u);
+      last = prev == (unsigned)a.ksplit - 1;
+      if (last) a.cnt[tile] = 0;                 // every CTA of the tile has arrived: ready for the next launch
+    }
+    __syncthreads();
+    if (!last) ok = false;                       // not an error: another CTA finishes the tile
+    __threadfence();
+    parts = a.part + (long long)tile * a.ksplit * 128 * a.N + (long long)row * a.N;
+  }
+  // the tile's 16 sums from column c0 on, for this thread's row
+  auto sums = [&](int c0, float (&z)[16]) {
+    if (parts == nullptr) {
+      tmem_ld16(tm + lb + c0, z);
+      tmem_wait_ld();
+      return;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) z[i] = 0.f;
+    for (int k = 0; k < a.ksplit; ++k) {
+      const float4 *src = reinterpret_cast<const float4 *>(parts + (long long)k * 128 * a.N + c0);
+#pragma unroll
+      for (int i4 = 0; i4 < 4; ++i4) {
+        const float4 v = __ldcg(src + i4);
+        z[4 * i4] += v.x; z[4 * i4 + 1] += v.y; z[4 * i4 + 2] += v.z; z[4 * i4 + 3] += v.w;
+      }
+    }
+  };
   if (ok) {
     if constexpr (kind == K_FWD || kind == K_FWD_LAST || kind == K_BWD) {
       const int r = 128 * mt + row;              // row of the per-stream matrix
@@ -241,8 +293,7 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
       const bool valid = (kind == K_BWD) ? key : (r < 2 * a.C);
       for (int c0 = cbeg; c0 < cend; c0 += 16) {
         float z[16];
-        tmem_ld16(tm + lb + c0, z);
-        tmem_wait_ld();
+        sums(c0, z);
         if (!valid) continue;
         const int col = a.N * nt + c0;           // column in the per-stream output
         if (kind == K_FWD) {
@@ -319,7 +370,7 @@ template <int KIND>
 __global__ void __launch_bounds__(NT, 1)
     tcl_gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap mA,
                     const __grid_constant__ CUtensorMap mA2, const __grid_constant__ CUtensorMap mB) {
-  gemm_tile<KIND>(a, mA, mA2, mB, blockIdx.z, blockIdx.y, blockIdx.x);
+  gemm_tile<KIND>(a, mA, mA2, mB, blockIdx.z % a.streams, blockIdx.y, blockIdx.x);
 }
 
 // ------------------------------------------------------------------------
@@ -889,7 +940,7 @@ __global__ void __launch_bounds__(UP3_NT, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *sm =
       reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t full[UP3_NS], freed[UP3_NS], op_full, mma_done[2], fin, never;
+  __shared__ uint64_t full[UP3_NS], freed[UP3_NS], op_full[2], mma_done[2], fin, never;
   __shared__ uint32_t tslot;
   __shared__ int abort_flag;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -915,7 +966,8 @@ __global__ void __launch_bounds__(UP3_NT, 1)
       mbar_init(&full[b], 1);
       mbar_init(&freed[b], 4);                 // the four warps reading the slot's columns
     }
-    mbar_init(&op_full, 1);
+    mbar_init(&op_full[0], 1);
+    mbar_init(&op_full[1], 1);
     mbar_init(&mma_done[0], 1);
     mbar_init(&mma_done[1], 1);
     mbar_init(&fin, 1);
@@ -930,7 +982,7 @@ __global__ void __launch_bounds__(UP3_NT, 1)
   const uint32_t tm = tslot;
   volatile int *abort = &abort_flag;
 
-  int armed = 0, op_armed = 0;                 // chunks whose loads were issued; operands issued
+  int armed = 0, op_armed = 0;                 // chunks whose loads were issued; operand halves issued
   auto load_chunk = [&](int i) {               // rows 16 i .. 16 i + 15 of the unit into slot i % NS
     const int b = i % UP3_NS;
     unsigned char *dst = slot_w(b);
@@ -949,16 +1001,23 @@ __global__ void __launch_bounds__(UP3_NT, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0 && !*abort) {
       const long long brow = (long long)s * ly.b_rows_per_stream + ly.b_row_off;
-      mbar_arrive_expect_tx(&op_full, (uint32_t)(256 * C + 2 * 2 * N * C));
-      for (int kp = 0; kp < C / 64; ++kp) {
-        for (int f = 0; f < 2; ++f)
-          tma_load_2d(opa + f * C * 128 + kp * 64 * 128, &m.b[l], &op_full, 128 * cb + 64 * f, (int)(brow + 64 * kp));
-        for (int f = 0; f < N / 64; ++f) {
-          tma_load_2d(opc + f * C * 128 + kp * 64 * 128, &m.a[l], &op_full, 256 * rb + 64 * f, s * C + 64 * kp);
-          tma_load_2d(ope + f * C * 128 + kp * 64 * 128, &m.a2[l], &op_full, 256 * rb + 64 * f, s * C + 64 * kp);
+      // operands in two halves, so that the MMAs of rows 0-127 start while
+      // those of rows 128-255 are still arriving: X^T and the first rows of
+      // -c G, -e G, then the remaining rows
+      for (int h = 0; h < nhalf; ++h) {
+        const int f0 = 2 * h, f1 = (N / 64 < f0 + 2) ? N / 64 : f0 + 2;
+        mbar_arrive_expect_tx(&op_full[h], (uint32_t)((h == 0 ? 256 * C : 0) + 2 * (f1 - f0) * 128 * C));
+        for (int kp = 0; kp < C / 64; ++kp) {
+          if (h == 0)
+            for (int f = 0; f < 2; ++f)
+              tma_load_2d(opa + f * C * 128 + kp * 64 * 128, &m.b[l], &op_full[0], 128 * cb + 64 * f, (int)(brow + 64 * kp));
+          for (int f = f0; f < f1; ++f) {
+            tma_load_2d(opc + f * C * 128 + kp * 64 * 128, &m.a[l], &op_full[h], 256 * rb + 64 * f, s * C + 64 * kp);
+            tma_load_2d(ope + f * C * 128 + kp * 64 * 128, &m.a2[l], &op_full[h], 256 * rb + 64 * f, s * C + 64 * kp);
+          }
         }
+        op_armed = h + 1;
       }
-      op_armed = 1;
       // the later chunks wait for slots (over the operands, or refills); bring
       // them into L2 behind the operands so that those loads do not wait on DRAM
       for (int i = armed; i < nch; ++i) {
@@ -981,7 +1040,7 @@ __global__ void __launch_bounds__(UP3_NT, 1)
     }
     if (lane == 0 && *abort) {
       // copies still in flight into this CTA's shared memory finish first
-      if (op_armed) mbar_wait(&op_full, 0, a.wait_ns);
+      for (int h = 0; h < op_armed; ++h) mbar_wait(&op_full[h], 0, a.wait_ns);
       for (int i = 0; i < armed; ++i)
         if (i + UP3_NS >= armed) mbar_wait(&full[i % UP3_NS], (uint32_t)((i / UP3_NS) & 1), a.wait_ns);
     }
@@ -989,20 +1048,19 @@ __global__ void __launch_bounds__(UP3_NT, 1)
   } else if (warp == UP3_EPI + 1) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      if (up3_wait(&op_full, 0, a, abort)) {
+      const uint32_t xa = smem_u32(opa), gc = smem_u32(opc), ge = smem_u32(ope);
+      for (int h = 0; h < nhalf; ++h) {
+        if (!up3_wait(&op_full[h], 0, a, abort)) break;
         tc_fence_after();
-        const uint32_t xa = smem_u32(opa), gc = smem_u32(opc), ge = smem_u32(ope);
-        for (int h = 0; h < nhalf; ++h) {
-          const int nh = N - 128 * h < 128 ? N - 128 * h : 128;
-          const uint32_t idesc = idesc_f16(128, nh, true, true);
-          const uint32_t boff = (uint32_t)(2 * h) * (uint32_t)C * 128u;   // feature blocks 2h, 2h + 1
-          for (int ks = 0; ks < C / 16; ++ks) {
-            const uint64_t ad = desc_mnmajor(xa, C, ks);
-            umma_f16(tm + 128u * (uint32_t)h, ad, desc_mnmajor(gc + boff, C, ks), idesc, ks != 0);
-            umma_f16(tm + 256u + 128u * (uint32_t)h, ad, desc_mnmajor(ge + boff, C, ks), idesc, ks != 0);
-          }
-          umma_commit(&mma_done[h]);
+        const int nh = N - 128 * h < 128 ? N - 128 * h : 128;
+        const uint32_t idesc = idesc_f16(128, nh, true, true);
+        const uint32_t boff = (uint32_t)(2 * h) * (uint32_t)C * 128u;   // feature blocks 2h, 2h + 1
+        for (int ks = 0; ks < C / 16; ++ks) {
+          const uint64_t ad = desc_mnmajor(xa, C, ks);
+          umma_f16(tm + 128u * (uint32_t)h, ad, desc_mnmajor(gc + boff, C, ks), idesc, ks != 0);
+          umma_f16(tm + 256u + 128u * (uint32_t)h, ad, desc_mnmajor(ge + boff, C, ks), idesc, ks != 0);
         }
+        umma_commit(&mma_done[h]);
       }
       // every MMA this CTA issued has completed before TMEM is freed
       umma_commit(&fin);
@@ -1600,10 +1658,52 @@ bool map3d_f32_plain(CUtensorMap *m, const float *base, int cols, int rows, int 
 // Workspace carve-up (bytes, 256-aligned pieces), per problem.
 struct Carve {
   size_t coef, scal, wbf, x[kMaxL + 1], sp[kMaxL + 1], g[kMaxL + 1], gc[kMaxL + 1], ge[kMaxL + 1];
+  size_t part, cnt, cnt_bytes;       // split-K partial sums and per-tile arrival counters
   size_t total;
 };
 
 size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+bool fb_ok(const Problem &p);
+
+// Widest output tile of a per-phase GEMM that divides n and still gives about
+// one CTA per SM (S streams, mtiles row tiles).
+int phase_tile(int n, int mtiles, int S) {
+  for (int t = 256; t >= 64; t /= 2) {
+    if (n % t) continue;
+    if ((long long)S * mtiles * (n / t) >= 128 || t == 64) return t;
+  }
+  return 64;
+}
+// Split of a per-phase GEMM's reduction over several CTAs per output tile,
+// for grids that leave most SMs idle and long reductions (K >= 1024): the
+// partial tiles cost a store, a fence and a re-read, which shorter
+// reductions do not earn back.
+int phase_ksplit(long long ctas, int nk) {
+  if (ctas >= 64 || nk < 16) return 1;
+  for (int ks = 4; ks >= 2; --ks)
+    if (ctas * ks <= 148) return ks;
+  return 1;
+}
+// Largest partial-sum buffer (bytes) and tile count of the split phases.
+void phase_split_sizes(const Problem &p, size_t *part_bytes, size_t *tiles) {
+  *part_bytes = 0;
+  *tiles = 0;
+  if (p.fuse_fb && fb_ok(p)) return;           // the fused kernel runs instead
+  const int C = p.C, S = p.streams;
+  auto one = [&](int n_out, int M, int K) {
+    const int mtiles = (M + 127) / 128, N = phase_tile(n_out, mtiles, S);
+    const long long ctas = (long long)S * mtiles * (n_out / N);
+    const int ks = phase_ksplit(ctas, K / KB);
+    if (ks > 1) {
+      const size_t b = (size_t)ctas * ks * 128 * N * sizeof(float);
+      if (b > *part_bytes) *part_bytes = b;
+      if ((size_t)ctas > *tiles) *tiles = (size_t)ctas;
+    }
+  };
+  for (int l = 1; l <= p.L; ++l) one(p.dims[l], 2 * C, p.dims[l - 1]);
+  for (int l = p.L; l >= 2; --l) one(p.dims[l - 1], C, p.dims[l]);
+}
 
 Carve carve(const Problem &p) {
   Carve c{};
@@ -1622,6 +1722,11 @@ Carve carve(const Problem &p) {
     c.gc[l] = take(S * p.C * p.dims[l] * 2);
     c.ge[l] = take(S * p.C * p.dims[l] * 2);
   }
+  size_t pb, nt;
+  phase_split_sizes(p, &pb, &nt);
+  c.part = pb ? take(pb) : 0;
+  c.cnt = nt ? take(nt * sizeof(unsigned)) : 0;
+  c.cnt_bytes = nt * sizeof(unsigned);
   c.total = off;
   return c;
 }
@@ -1657,7 +1762,7 @@ cudaError_t launch_fb(const FbArgs &a, const FbMaps &m, int streams, cudaStream_
 cudaError_t launch_gemm(const GemmArgs &a, const CUtensorMap &mA, const CUtensorMap &mA2,
                         const CUtensorMap &mB, int streams, int mtiles, int ntiles, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)ntiles, (unsigned)mtiles, (unsigned)streams);
+  cfg.gridDim = dim3((unsigned)ntiles, (unsigned)mtiles, (unsigned)(streams * a.ksplit));
   cfg.blockDim = dim3(NT);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = st;
@@ -1783,13 +1888,7 @@ struct TclGroup {
 
   op_t *bf(size_t off) const { return reinterpret_cast<op_t *>(ws + off); }
   // Widest tile that divides n and still gives about one CTA per SM.
-  int tile_for(int n, int mtiles) const {
-    for (int t = 256; t >= 64; t /= 2) {
-      if (n % t) continue;
-      if ((long long)S * mtiles * (n / t) >= 128 || t == 64) return t;
-    }
-    return 64;
-  }
+  int tile_for(int n, int mtiles) const { return phase_tile(n, mtiles, S); }
   cudaError_t setup();
   cudaError_t chunk(int ch);
 };
@@ -1836,6 +1935,14 @@ cudaError_t TclGroup::setup() {
   std::memset(&base, 0, sizeof base);
   base.C = C;
   base.T = T;
+  base.streams = S;
+  base.ksplit = 1;
+  if (cv.part) base.part = reinterpret_cast<float *>(ws + cv.part);
+  if (cv.cnt) {
+    base.cnt = reinterpret_cast<unsigned *>(ws + cv.cnt);
+    err = cudaMemsetAsync(base.cnt, 0, cv.cnt_bytes, stream);   // each split tile's last CTA resets its counter
+    if (err != cudaSuccess) return err;
+  }
   base.coef = coef;
   base.status = p.status;
   base.wait_ns = g_tcl_wait_ns;
@@ -1991,6 +2098,7 @@ cudaError_t TclGroup::chunk(int ch) {
     a.a_split_kq = l == 1;
     a.a_rows_per_stream = 2 * C;
     a.b_rows_per_stream = nl;
+    a.ksplit = base.cnt ? phase_ksplit((long long)S * (2 * C / 128) * (nl / a.N), np / KB) : 1;
     if (l < L) { a.x_out = bf(cv.x[l]); a.sp_out = bf(cv.sp[l]); }
     a.g_out = bf(cv.g[L]); a.gc_out = bf(cv.gc[L]); a.ge_out = bf(cv.ge[L]);
     err = launch_gemm(a, l == 1 ? mk : mx[l - 1], mq, mwb[l], S, 2 * C / 128, nl / a.N, stream);
@@ -2008,6 +2116,7 @@ cudaError_t TclGroup::chunk(int ch) {
     a.n_out = np;
     a.a_rows_per_stream = C;
     a.b_rows_per_stream = nl;
+    a.ksplit = base.cnt ? phase_ksplit((long long)S * ((C + 127) / 128) * (np / a.N), nl / KB) : 1;
     a.sp_in = bf(cv.sp[l - 1]);
     a.g_out = bf(cv.g[l - 1]); a.gc_out = bf(cv.gc[l - 1]); a.ge_out = bf(cv.ge[l - 1]);
     err = launch_gemm(a, mg[l], mg[l], mwb[l], S, (C + 127) / 128, np / a.N, stream);

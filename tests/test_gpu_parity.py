@@ -307,6 +307,7 @@ TCL_SHAPES = [  # L, d, expansion, B, H, T, C
     (2, 128, 2, 1, 1, 512, 256),    # C = 256: four key/query row tiles, pipelined K loop
     (2, 64, 2, 3, 3, 256, 64),      # 9 streams: two concurrent groups of 4 and 5
     (4, 64, 2, 2, 4, 256, 128),     # 8 streams in two groups, depth 4
+    (2, 128, 8, 1, 1, 128, 64),     # hidden 1024: the last forward's K = 1024 split over 4 CTAs per tile
 ]
 
 
