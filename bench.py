@@ -274,13 +274,13 @@ def sweep_chunk(args, w: W.Workload, sizes):
 #   its launch, outside the window).
 # - README-shape workload (d=384, 2 streams x 1024 tokens): every launch of
 #   one tm_run (token conversion, initial copy, coefficients, 16 chunks of
-#   three per-phase GEMM launches and one update): 487.9 MB read, 0 written
+#   three per-phase GEMM launches and one update): 488.2 MB read, 0 written
 #   inside the launches (ncu flushes the caches before each launch, so these
 #   reads are cold-cache).
 CAPTURED_TRAFFIC = {("tc", "mlp2-d128-long"): (784.695040e6 + 483.341568e6 + 52.528896e6 + 4.637184e6, 16 * 65536),
                     ("tcl", "mlp4-d128-deep"): (4.007936e6 + 18.134528e6, 8 * 128),
-                    ("tcl", "mlp2-d384-readme"): (3.153e6 + 18.885e6 + 0.034e6
-                                                  + 16 * (2.579e6 + 3.269e6 + 2.875e6 + 20.394e6), 2 * 1024)}
+                    ("tcl", "mlp2-d384-readme"): (3.152e6 + 18.885e6 + 0.034e6
+                                                  + 16 * (2.585e6 + 3.275e6 + 2.880e6 + 20.395e6), 2 * 1024)}
 
 
 def traffic_per_launch(path: str, w: W.Workload):
@@ -589,7 +589,8 @@ def main():
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = traffic_per_launch(path_used, w)
     fused = all(n <= 256 for n in w.dims)
-    upd = "tcl_update2_kernel" if w.C <= 128 else "tcl_update_kernel"
+    transposed = all(w.dims[l - 1] % 128 == 0 and w.dims[l] % 64 == 0 for l in range(1, len(w.dims)))
+    upd = ("tcl_update3_kernel" if transposed else "tcl_update2_kernel") if w.C <= 128 else "tcl_update_kernel"
     roof["kernel"] = {"tc": "tc_chunk_kernel (cluster and global-exchange forms)",
                       "tcl": ("tcl_fb_kernel + " if fused else "tcl_gemm_kernel + ") + upd,
                       "tcl-phased": "tcl_gemm_kernel + " + upd}.get(path_used, "simt_chunk_kernel")

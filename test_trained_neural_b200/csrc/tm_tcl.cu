@@ -42,6 +42,7 @@ using op_t = __half;
 constexpr int NT = 256;          // 8 warps: warp w reads TMEM lanes 32 (w % 4) .. +31,
                                  // columns half w / 4 of the tile
 constexpr int KB = 64;           // K block (one 128-byte swizzle atom of 2-byte elements)
+constexpr int kMaxSplit = 4;     // CTAs per output tile sharing a per-phase GEMM's reduction
 
 enum Kind { K_FWD = 0, K_FWD_LAST = 1, K_BWD = 2 };
 
@@ -275,16 +276,28 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs &a, const CUtensorMap &
       tmem_wait_ld();
       return;
     }
+    // every partial of the 16 columns requested at once (at most 4 splits),
+    // then added in split order
+    float4 v[kMaxSplit][4];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) z[i] = 0.f;
-    for (int k = 0; k < a.ksplit; ++k) {
-      const float4 *src = reinterpret_cast<const float4 *>(parts + (long long)k * 128 * a.N + c0);
+    for (int k = 0; k < kMaxSplit; ++k)
+      if (k < a.ksplit) {
+        const float4 *src = reinterpret_cast<const float4 *>(parts + (long long)k * 128 * a.N + c0);
 #pragma unroll
-      for (int i4 = 0; i4 < 4; ++i4) {
-        const float4 v = __ldcg(src + i4);
-        z[4 * i4] += v.x; z[4 * i4 + 1] += v.y; z[4 * i4 + 2] += v.z; z[4 * i4 + 3] += v.w;
+        for (int i4 = 0; i4 < 4; ++i4) v[k][i4] = __ldcg(src + i4);
       }
+#pragma unroll
+    for (int i4 = 0; i4 < 4; ++i4) {
+      z[4 * i4] = v[0][i4].x; z[4 * i4 + 1] = v[0][i4].y; z[4 * i4 + 2] = v[0][i4].z; z[4 * i4 + 3] = v[0][i4].w;
     }
+#pragma unroll
+    for (int k = 1; k < kMaxSplit; ++k)
+      if (k < a.ksplit) {
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4) {
+          z[4 * i4] += v[k][i4].x; z[4 * i4 + 1] += v[k][i4].y; z[4 * i4 + 2] += v[k][i4].z; z[4 * i4 + 3] += v[k][i4].w;
+        }
+      }
   };
   if (ok) {
     if constexpr (kind == K_FWD || kind == K_FWD_LAST || kind == K_BWD) {
@@ -1681,7 +1694,7 @@ int phase_tile(int n, int mtiles, int S) {
 // reductions do not earn back.
 int phase_ksplit(long long ctas, int nk) {
   if (ctas >= 64 || nk < 16) return 1;
-  for (int ks = 4; ks >= 2; --ks)
+  for (int ks = kMaxSplit; ks >= 2; --ks)
     if (ctas * ks <= 148) return ks;
   return 1;
 }
