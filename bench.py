@@ -277,7 +277,13 @@ def sweep_chunk(args, w: W.Workload, sizes):
 #   three per-phase GEMM launches and one update): 488.2 MB read, 0 written
 #   inside the launches (ncu flushes the caches before each launch, so these
 #   reads are cold-cache).
-CAPTURED_TRAFFIC = {("tc", "mlp2-d128-long"): (784.695040e6 + 483.341568e6 + 52.528896e6 + 4.637184e6, 16 * 65536),
+# - d=64 eight-head workload: the cluster walker on 32 streams x 32768 tokens
+#   (y 268 MB, twice L2): 424.2 MB read, 242.1 MB written.
+# - linear d=64 workload (fp32, CUDA-core kernel, 256 tokens): 0.319 MB read,
+#   nothing written back inside the launch.
+CAPTURED_TRAFFIC = {("tc", "mlp2-d64-h8"): (424.181e6 + 242.146e6, 32 * 32768),
+                    ("simt", "linear-d64"): (0.319e6, 256),
+                    ("tc", "mlp2-d128-long"): (784.695040e6 + 483.341568e6 + 52.528896e6 + 4.637184e6, 16 * 65536),
                     ("tcl", "mlp4-d128-deep"): (4.007936e6 + 18.134528e6, 8 * 128),
                     ("tcl", "mlp2-d384-readme"): (3.152e6 + 18.885e6 + 0.034e6
                                                   + 16 * (2.585e6 + 3.275e6 + 2.880e6 + 20.395e6), 2 * 1024)}
