@@ -642,7 +642,7 @@ def main():
         e_ms_max = max_over_ranks(statistics.mean(e_ms), world)
         e2e = {"value": aggregate_throughput(cnt["tokens"], world, e_ms_max * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e_ms_max,
-               "api": "tm_run_host", "segment_tokens": seg or "default (about T/8)",
+               "api": "tm_run_host", "segment_tokens": seg or "default (T/16 with a ramp of shorter segments at both ends)",
                "equal_to_device_run": same}
 
     cpu = None

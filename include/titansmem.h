@@ -205,9 +205,12 @@ TM_API tm_status tm_run_noalloc(tm_ctx *ctx, int B, int H, int T, int C, tm_dtyp
  * "titans-pytorch" review, "NeuralMemory as a standalone module"), with the
  * host <-> device copies inside the call and overlapped with the kernels.
  *
- * T is walked in segments of `segment_tokens` tokens per stream (0 = about
- * T / 8, rounded up to whole chunks; otherwise a multiple of C, or >= T);
- * the last segment takes the rest. While the kernels run segment i, the
+ * T is walked in segments of `segment_tokens` tokens per stream (a multiple
+ * of C, or >= T; the last segment takes the rest). With segment_tokens = 0
+ * the library chooses: middle segments of about T / 16 whole chunks, and the
+ * first and last three ramping up from and down to an eighth of that, so that
+ * the copies no kernel runs beside (the first segment's inputs, the last
+ * one's reads) are short. While the kernels run segment i, the
  * inputs of segment i + 1 are copied in on one side stream and the reads y
  * of segment i - 1 copied out on another (one cudaMemcpy2DAsync per tensor
  * and segment). W0/S0 go in before the first segment, W_end/S_end come out

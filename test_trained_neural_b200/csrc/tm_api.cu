@@ -4,6 +4,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <new>
+#include <vector>
 
 #include "tm_internal.h"
 
@@ -480,13 +481,53 @@ tm_status run_device(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype,
 
 size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Segment length of tm_run_host: the caller's, or about an eighth of T
-// rounded up to whole chunks.
-int host_segment(int T, int C, int segment_tokens) {
-  if (segment_tokens > 0) return segment_tokens < T ? segment_tokens : T;
-  const int n = (T + 7) / 8;
-  const int seg = (n + C - 1) / C * C;
-  return seg < T ? seg : T;
+// Segments of tm_run_host, as token counts in order. A caller's
+// segment_tokens > 0 gives equal segments (the last one shorter). Otherwise
+// the middle segments are about T / 16 (whole chunks) and the first and last
+// three ramp up from and down to an eighth of that: the copies of the first
+// segment's inputs and of the last one's reads are the only ones no kernel
+// runs beside, so keeping those segments short leaves the host link busy for
+// almost the whole call, while the middle ones stay long enough that each
+// tm_run's fixed cost is small. Every segment but the last is a multiple of C.
+std::vector<int> host_segments(int T, int C, int segment_tokens) {
+  std::vector<int> lens;
+  if (segment_tokens > 0) {
+    const int seg = segment_tokens < T ? segment_tokens : T;
+    for (int t = 0; t < T; t += seg) lens.push_back(T - t < seg ? T - t : seg);
+    return lens;
+  }
+  const int Tc = T - T % C;                    // tokens in whole chunks
+  const int base = ((T + 15) / 16 + C - 1) / C * C;
+  auto down = [&](int x) { x = x / C * C; return x < C ? C : x; };
+  const int ramp[3] = {down(base / 8), down(base / 4), down(base / 2)};
+  const int ends = 2 * (ramp[0] + ramp[1] + ramp[2]);
+  if (base >= Tc || Tc - ends < base) {
+    // too short for a ramp: equal segments of about T / 16
+    for (int t = 0; t < T; t += base) lens.push_back(T - t < base ? T - t : base);
+    return lens;
+  }
+  for (int r : ramp) lens.push_back(r);
+  int mid = Tc - ends;
+  while (mid > 0) {
+    const int n = mid < base ? mid : base;
+    lens.push_back(n);
+    mid -= n;
+  }
+  for (int i = 2; i >= 0; --i) lens.push_back(ramp[i]);
+  lens.back() += T - Tc;                       // a shorter final chunk goes with the last segment
+  return lens;
+}
+
+// Longest segment and whether every segment but the last is whole chunks.
+int host_segment_max(const std::vector<int> &lens) {
+  int m = 0;
+  for (int n : lens) m = n > m ? n : m;
+  return m;
+}
+bool host_segments_ok(const std::vector<int> &lens, int C) {
+  for (size_t i = 0; i + 1 < lens.size(); ++i)
+    if (lens[i] % C != 0) return false;
+  return true;
 }
 
 // Device workspace of tm_run_host: tm_run's workspace for one segment first
@@ -496,10 +537,10 @@ struct HostCarve {
   size_t run, run_bytes, W, S, buf[2], k, v, q, th, et, al, y, total;
 };
 
-tm_status host_carve(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype dt, int seg, HostCarve *c) {
-  const int last = T - (T - 1) / seg * seg;    // tokens of the last segment
+tm_status host_carve(const tm_ctx *ctx, int B, int H, int T, int C, tm_dtype dt, const std::vector<int> &lens,
+                     HostCarve *c) {
+  const int seg = host_segment_max(lens);
   size_t ws = 0;
-  const int lens[2] = {seg, last};
   for (int t : lens) {
     size_t b = 0;
     const tm_status st = tm_workspace_size(ctx, B, H, t, C, dt, &b);
@@ -548,10 +589,10 @@ tm_status tm_host_workspace_size(const tm_ctx *ctx, int B, int H, int T, int C, 
   if (!bytes || segment_tokens < 0) return TM_ERR_INVALID_ARG;
   tm_status st = check_shape(ctx, B, H, T, C, in_dtype);
   if (st != TM_OK) return st;
-  const int seg = host_segment(T, C, segment_tokens);
-  if (seg < T && seg % C != 0) return TM_ERR_INVALID_ARG;
+  const std::vector<int> lens = host_segments(T, C, segment_tokens);
+  if (!host_segments_ok(lens, C)) return TM_ERR_INVALID_ARG;
   HostCarve c;
-  st = host_carve(ctx, B, H, T, C, in_dtype, seg, &c);
+  st = host_carve(ctx, B, H, T, C, in_dtype, lens, &c);
   if (st != TM_OK) return st;
   *bytes = c.total;
   return TM_OK;
@@ -571,19 +612,18 @@ tm_status tm_run_host(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TM_ERR_INVALID_ARG;
   const tmem::Problem p = make_problem(ctx, B, H, T, C, in_dtype);
   if (!tmem::run_aliasing_ok(p, k, v, q, theta, eta, alpha, W0, S0, y, W_end, S_end)) return TM_ERR_INVALID_ARG;
-  const int seg = host_segment(T, C, segment_tokens);
-  if (seg < T && seg % C != 0) return TM_ERR_INVALID_ARG;
+  const std::vector<int> lens = host_segments(T, C, segment_tokens);
+  if (!host_segments_ok(lens, C)) return TM_ERR_INVALID_ARG;
   HostCarve c;
-  st = host_carve(ctx, B, H, T, C, in_dtype, seg, &c);
+  st = host_carve(ctx, B, H, T, C, in_dtype, lens, &c);
   if (st != TM_OK) return st;
   if (workspace_bytes < c.total) return TM_ERR_OOM;
   {
     // every segment's path must be one tm_run supports
     tm_path path;
-    const int last = T - (T - 1) / seg * seg;
-    if (tm_query_path(ctx, B, H, seg, C, in_dtype, &path) != TM_OK ||
-        tm_query_path(ctx, B, H, last, C, in_dtype, &path) != TM_OK)
-      return TM_ERR_UNSUPPORTED;
+    for (size_t i = 0; i < lens.size(); ++i)
+      if ((i == 0 || lens[i] != lens[i - 1]) && tm_query_path(ctx, B, H, lens[i], C, in_dtype, &path) != TM_OK)
+        return TM_ERR_UNSUPPORTED;
   }
   if (!ensure_host(ctx)) return TM_ERR_CUDA;
 
@@ -592,13 +632,15 @@ tm_status tm_run_host(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype
   const size_t S = (size_t)p.streams, d = (size_t)ctx->d, el = in_dtype == TM_BF16 ? 2 : 4;
   const size_t st_bytes = S * ctx->P * 4;
   float *dW = reinterpret_cast<float *>(ws + c.W), *dS = reinterpret_cast<float *>(ws + c.S);
-  const int nseg = (T + seg - 1) / seg;
-  auto seg_len = [&](int i) { return i + 1 < nseg ? seg : T - i * seg; };
+  const int nseg = (int)lens.size();
+  std::vector<size_t> start((size_t)nseg);
+  for (int i = 0, t = 0; i < nseg; t += lens[(size_t)i], ++i) start[(size_t)i] = (size_t)t;
+  auto seg_len = [&](int i) { return lens[(size_t)i]; };
   // One strided copy per tensor and segment: the segment's rows of every
   // stream, [S rows] x [n tokens x width] bytes.
   auto copy_in = [&](int i) -> cudaError_t {
     unsigned char *b = ws + c.buf[i & 1];
-    const size_t t0 = (size_t)i * seg, n = (size_t)seg_len(i);
+    const size_t t0 = start[(size_t)i], n = (size_t)seg_len(i);
     const void *src[6] = {k, v, q, theta, eta, alpha};
     const size_t off[6] = {c.k, c.v, c.q, c.th, c.et, c.al};
     const size_t w[6] = {d * el, d * el, d * el, 4, 4, 4};
@@ -639,7 +681,7 @@ tm_status tm_run_host(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype
     if (e == cudaSuccess) e = cudaEventRecord(ctx->y_ready[b], s);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ctx->d2h, ctx->y_ready[b], 0);
     if (e == cudaSuccess)
-      e = cudaMemcpy2DAsync(y + (size_t)i * seg * d, (size_t)T * d * 4, yb, (size_t)n * d * 4, (size_t)n * d * 4, S,
+      e = cudaMemcpy2DAsync(y + start[(size_t)i] * d, (size_t)T * d * 4, yb, (size_t)n * d * 4, (size_t)n * d * 4, S,
                             cudaMemcpyDeviceToHost, ctx->d2h);
     if (e == cudaSuccess) e = cudaEventRecord(ctx->y_free[b], ctx->d2h);
     if (e != cudaSuccess) st = TM_ERR_CUDA;
