@@ -412,13 +412,22 @@ def bench_backward(args, w: W.Workload):
     P1 = w.dims[0] * w.dims[1]
     flops = (22.0 * w.P if w.L == 1 else 32.0 * w.P - 6.0 * P1 if w.L == 2 else 34.0 * w.P - 8.0 * P1) * tokens
     peaks = measured_peaks()
-    alu_peak = SM_COUNT * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
     tf = flops / t / 1e12
+    if w.dtype == "bf16":
+        # bf16 inputs: the chunk's products run on tcgen05 with TF32 operands,
+        # whose dense rate is half the bf16 one
+        peak = 0.5 * peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                "peak_source": peaks["source"] + " bf16 burst (cuBLAS) x 1/2 (TF32 / BF16 nominal)",
+                "kernel": "backward%s_kernel<true> (tcgen05 kind::tf32 products)" % ("1" if w.L == 1 else "2" if w.L == 2 else "L")}
+    else:
+        peak = SM_COUNT * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
+        roof = {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 x max clock",
+                "kernel": "backward%s_kernel<false> (fp32 FFMA)" % ("1" if w.L == 1 else "2" if w.L == 2 else "L")}
     print(json.dumps({"metric": "backward tokens/sec", "value": tokens / t, "unit": "tokens/s", "ms": t * 1e3,
                       "workload": w.name, "finite": bool(all(torch.isfinite(v).all() for v in out.values())),
-                      "roofline": {"bound": "alu", "achieved": tf, "peak": alu_peak, "unit": "TFLOP/s",
-                                   "frac": tf / alu_peak,
-                                   "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 x max clock"}}), flush=True)
+                      "roofline": roof}), flush=True)
 
 
 def bench_prologue(args, w: W.Workload):

@@ -263,9 +263,14 @@ TM_API tm_status tm_sync(tm_ctx *ctx, void *workspace, void *stream);
  *   other arguments as for tm_run (chunk size C, a shorter last chunk allowed)
  *
  * Supported: every depth 1 to 4 (the surprise is itself a gradient, so the
- * backward takes second derivatives through the MLP), fp32 arithmetic, any
- * C the forward accepts; TM_ERR_UNSUPPORTED otherwise. The forward is recomputed inside
- * (chunk-start states kept in the workspace: tm_backward_workspace_size()).
+ * backward takes second derivatives through the MLP), any C the forward
+ * accepts; TM_ERR_UNSUPPORTED otherwise. Arithmetic: fp32 throughout for fp32
+ * inputs or TM_PATH_SIMT; for bf16 inputs on the other paths the chunk's
+ * matrix products run on the tensor cores with TF32 operands (rounded to
+ * nearest, fp32's exponent range) and fp32 accumulation, the rest in fp32.
+ * The forward is recomputed inside (chunk-start states kept in the workspace:
+ * tm_backward_workspace_size()); tm_sync(ctx, workspace, stream) reports a
+ * device-side error of the call (its waits are bounded).
  * Pointers 16-byte aligned; outputs must not overlap inputs or each other.
  * Errors as for tm_run. Asynchronous on `stream`; allocates nothing.
  */

@@ -763,6 +763,12 @@ tm_status tm_backward(tm_ctx *ctx, int B, int H, int T, int C, tm_dtype in_dtype
   p.S0 = S0;
   p.scratch = static_cast<char *>(workspace) + tmem::kStatusBytes;
   p.scratch_bytes = workspace_bytes - tmem::kStatusBytes;
+  // bf16 inputs on a tensor-core path: the reverse pass's products on tcgen05
+  // (TF32 operands); fp32 inputs or TM_PATH_SIMT: fp32 FFMA throughout
+  p.bw_tc = in_dtype == TM_BF16 && ctx->path != TM_PATH_SIMT;
+  p.status = static_cast<int *>(workspace);
+  if (cudaMemsetAsync(workspace, 0, sizeof(int), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return TM_ERR_CUDA;
   const cudaError_t e = tmem::backward_launch(p, dy, dW_end, dS_end, dk, dv, dq, dtheta, deta, dalpha, dW0, dS0,
                                               reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? TM_OK : TM_ERR_CUDA;

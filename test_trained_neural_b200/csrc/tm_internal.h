@@ -40,6 +40,7 @@ struct Problem {
   void *scratch;          // per-stream activations (SIMT path)
   int fuse_fb;            // layered path: fused forward + backward launch where supported
   int tc_global;          // cluster-kernel path: every stream exchanges through global memory
+  int bw_tc;              // backward: the chunk's products on tcgen05 (TF32) rather than fp32 FFMA
   // layered path: CUDA streams and events (owned by the context) for groups
   // 1.. of the streams; group 0 runs on the caller's stream
   void *side_streams[kMaxGroups - 1];

@@ -24,6 +24,7 @@
 #include <cuda_bf16.h>
 
 #include "tm_internal.h"
+#include "tm_tcgemm.cuh"
 
 namespace tmem {
 namespace {
@@ -347,6 +348,8 @@ __global__ void __launch_bounds__(NT) simt_chunk_kernel(KArgs a) {
 // and (dc, de, dB, dA, dcS) go back through the coefficient scan to the gates.
 struct BArgs {
   int d, T, C, bf16;
+  int *status;                   // device status word (bounded waits of the tensor-core products)
+  unsigned long long wait_ns;
   const void *k, *v, *q;
   const float *theta, *eta, *alpha, *W0, *S0, *dy, *dW_end, *dS_end;
   float *dk, *dv, *dq, *dtheta, *deta, *dalpha, *dW0, *dS0;
@@ -411,9 +414,36 @@ __device__ void gate_reverse(int Cc, const float *th, const float *et, const flo
   }
 }
 
-__global__ void __launch_bounds__(NT) simt_backward_kernel(BArgs a) {
+template <bool TC>
+__global__ void __launch_bounds__(NT) backward1_kernel(BArgs a) {
   __shared__ SmemT sm;
   __shared__ float red[NT / 32];
+  extern __shared__ __align__(1024) unsigned char tcg_dyn[];
+  __shared__ TcGemm tg;
+  if constexpr (TC) tcg_init(tg, tcg_dyn, a.status, a.wait_ns);
+  // the chunk's products: tcgen05 (TF32 operands, fp32 accumulation) or fp32 FFMA tiles
+  auto mm = [&](int M_, int N_, int K_, const float *A_, long long sam, long long sak, const float *B_,
+                long long sbn, long long sbk, auto epi) {
+    if constexpr (TC) tc_gemm(tg, M_, N_, K_, A_, sam, sak, B_, sbn, sbk, epi);
+    else gemm(sm, M_, N_, K_, A_, sam, sak, B_, sbn, sbk, epi);
+  };
+  // the forward pass's state update of one layer (A6 + A7): on the tensor
+  // cores as two products, U_W with the tokens' c and U_S with their e
+  auto upd = [&](int rows, int cols, int Cn, const float *G, const float *X, float *Wl, float *Sl) {
+    if constexpr (TC) {
+      const Coef &cf = sm.coef;
+      tc_gemm(tg, rows, cols, Cn, G, 1, rows, X, 1, cols, [&](int r, int c, float u) {
+        const long long idx = (long long)r * cols + c;
+        Wl[idx] = cf.Bw * Wl[idx] + cf.cS * Sl[idx] - u;
+      }, cf.c);
+      tc_gemm(tg, rows, cols, Cn, G, 1, rows, X, 1, cols, [&](int r, int c, float u) {
+        const long long idx = (long long)r * cols + c;
+        Sl[idx] = cf.As * Sl[idx] - u;
+      }, cf.e);
+    } else {
+      update_layer(sm, rows, cols, Cn, G, X, Wl, Sl);
+    }
+  };
   const int s = blockIdx.x, d = a.d, T = a.T, C = a.C, dd = d * d;
   const int nch = (T + C - 1) / C;
   float *p = a.scratch + (long long)s * a.scratch_per_stream;
@@ -471,9 +501,9 @@ __global__ void __launch_bounds__(NT) simt_backward_kernel(BArgs a) {
     chunk_coefficients(sm.coef, a.theta + tok0 + t0, a.eta + tok0 + t0, a.alpha + tok0 + t0, Cc);
     load_chunk(t0, Cc, false);
     // G = 2 (K W^T - V): the surprise factor of every token
-    gemm(sm, Cc, d, d, K, d, 1, Wc, d, 1, [&](int i, int r, float z) { R[i * d + r] = 2.f * (z - V[i * d + r]); });
+    mm(Cc, d, d, K, d, 1, Wc, d, 1, [&](int i, int r, float z) { R[i * d + r] = 2.f * (z - V[i * d + r]); });
     __syncthreads();
-    update_layer(sm, d, d, Cc, R, K, Wc, Sc);
+    upd(d, d, Cc, R, K, Wc, Sc);
     __syncthreads();
   }
   // ---- reverse
@@ -489,12 +519,12 @@ __global__ void __launch_bounds__(NT) simt_backward_kernel(BArgs a) {
     chunk_coefficients(sm.coef, th, et, al, Cc);
     load_chunk(t0, Cc, true);
     // residuals r_i and the products with gW, gS
-    gemm(sm, Cc, d, d, K, d, 1, W, d, 1, [&](int i, int r, float z) { R[i * d + r] = z - V[i * d + r]; });
-    gemm(sm, Cc, d, d, K, d, 1, gW, d, 1, [&](int i, int r, float z) { Am[i * d + r] = z; });
-    gemm(sm, Cc, d, d, K, d, 1, gS, d, 1, [&](int i, int r, float z) { Bm[i * d + r] = z; });
+    mm(Cc, d, d, K, d, 1, W, d, 1, [&](int i, int r, float z) { R[i * d + r] = z - V[i * d + r]; });
+    mm(Cc, d, d, K, d, 1, gW, d, 1, [&](int i, int r, float z) { Am[i * d + r] = z; });
+    mm(Cc, d, d, K, d, 1, gS, d, 1, [&](int i, int r, float z) { Bm[i * d + r] = z; });
     __syncthreads();
-    gemm(sm, Cc, d, d, R, d, 1, gW, 1, d, [&](int i, int j, float z) { Pm[i * d + j] = z; });
-    gemm(sm, Cc, d, d, R, d, 1, gS, 1, d, [&](int i, int j, float z) { Qm[i * d + j] = z; });
+    mm(Cc, d, d, R, d, 1, gW, 1, d, [&](int i, int j, float z) { Pm[i * d + j] = z; });
+    mm(Cc, d, d, R, d, 1, gS, 1, d, [&](int i, int j, float z) { Qm[i * d + j] = z; });
     for (int e = threadIdx.x; e < Cc * d; e += NT) {
       const int i = e / d;
       Mm[e] = -(sm.coef.c[i] * Am[e] + sm.coef.e[i] * Bm[e]);
@@ -523,11 +553,11 @@ __global__ void __launch_bounds__(NT) simt_backward_kernel(BArgs a) {
     const float dB = block_sum(pw, red), dcS = block_sum(pws, red), dA = block_sum(pss, red);
     // token gradients
     const long long gt = (tok0 + t0) * d;
-    gemm(sm, Cc, d, d, Mm, d, 1, W, 1, d, [&](int i, int j, float z) {
+    mm(Cc, d, d, Mm, d, 1, W, 1, d, [&](int i, int j, float z) {
       const int e = i * d + j;
       a.dk[gt + e] = 2.f * z - 2.f * sm.coef.c[i] * Pm[e] - 2.f * sm.coef.e[i] * Qm[e];
     });
-    gemm(sm, Cc, d, d, DY, d, 1, W, 1, d, [&](int i, int j, float z) { a.dq[gt + i * d + j] = z; });
+    mm(Cc, d, d, DY, d, 1, W, 1, d, [&](int i, int j, float z) { a.dq[gt + i * d + j] = z; });
     for (int e = threadIdx.x; e < Cc * d; e += NT) a.dv[gt + e] = -2.f * Mm[e];
     // gates: back through the coefficient scan (one thread, in order)
     if (threadIdx.x == 0)
@@ -535,9 +565,9 @@ __global__ void __launch_bounds__(NT) simt_backward_kernel(BArgs a) {
                    a.dalpha + tok0 + t0, pa, pe, rho, dpa, dpe, drho);
     // the state gradients at the chunk start
     const float Bw = sm.coef.Bw, As = sm.coef.As, cS = sm.coef.cS;
-    gemm(sm, d, d, Cc, Mm, 1, d, K, 1, d, [&](int r, int j, float z) { gWn[r * d + j] = Bw * gW[r * d + j] + 2.f * z; });
+    mm(d, d, Cc, Mm, 1, d, K, 1, d, [&](int r, int j, float z) { gWn[r * d + j] = Bw * gW[r * d + j] + 2.f * z; });
     __syncthreads();
-    gemm(sm, d, d, Cc, DY, 1, d, Q, 1, d, [&](int r, int j, float z) { gWn[r * d + j] += z; });
+    mm(d, d, Cc, DY, 1, d, Q, 1, d, [&](int r, int j, float z) { gWn[r * d + j] += z; });
     __syncthreads();
     for (int e = threadIdx.x; e < dd; e += NT) {
       gS[e] = cS * gW[e] + As * gS[e];
@@ -549,6 +579,7 @@ __global__ void __launch_bounds__(NT) simt_backward_kernel(BArgs a) {
     a.dW0[sw + e] = gW[e];
     a.dS0[sw + e] = gS[e];
   }
+  if constexpr (TC) tcg_release(tg);
 }
 
 
@@ -573,6 +604,8 @@ __device__ __forceinline__ float silu_second(float z) {
 
 struct BArgs2 {
   int d, n, o, T, C, bf16;
+  int *status;                   // device status word (bounded waits of the tensor-core products)
+  unsigned long long wait_ns;
   long long P;
   const void *k, *v, *q;
   const float *theta, *eta, *alpha, *W0, *S0, *dy, *dW_end, *dS_end;
@@ -587,9 +620,36 @@ __host__ __device__ inline long long backward2_floats(int d, int n, int o, int T
   return 2 * nch * P + 5 * P + 20LL * C * m + 8LL * C;
 }
 
-__global__ void __launch_bounds__(NT) simt_backward2_kernel(BArgs2 a) {
+template <bool TC>
+__global__ void __launch_bounds__(NT) backward2_kernel(BArgs2 a) {
   __shared__ SmemT sm;
   __shared__ float red[NT / 32];
+  extern __shared__ __align__(1024) unsigned char tcg_dyn[];
+  __shared__ TcGemm tg;
+  if constexpr (TC) tcg_init(tg, tcg_dyn, a.status, a.wait_ns);
+  // the chunk's products: tcgen05 (TF32 operands, fp32 accumulation) or fp32 FFMA tiles
+  auto mm = [&](int M_, int N_, int K_, const float *A_, long long sam, long long sak, const float *B_,
+                long long sbn, long long sbk, auto epi) {
+    if constexpr (TC) tc_gemm(tg, M_, N_, K_, A_, sam, sak, B_, sbn, sbk, epi);
+    else gemm(sm, M_, N_, K_, A_, sam, sak, B_, sbn, sbk, epi);
+  };
+  // the forward pass's state update of one layer (A6 + A7): on the tensor
+  // cores as two products, U_W with the tokens' c and U_S with their e
+  auto upd = [&](int rows, int cols, int Cn, const float *G, const float *X, float *Wl, float *Sl) {
+    if constexpr (TC) {
+      const Coef &cf = sm.coef;
+      tc_gemm(tg, rows, cols, Cn, G, 1, rows, X, 1, cols, [&](int r, int c, float u) {
+        const long long idx = (long long)r * cols + c;
+        Wl[idx] = cf.Bw * Wl[idx] + cf.cS * Sl[idx] - u;
+      }, cf.c);
+      tc_gemm(tg, rows, cols, Cn, G, 1, rows, X, 1, cols, [&](int r, int c, float u) {
+        const long long idx = (long long)r * cols + c;
+        Sl[idx] = cf.As * Sl[idx] - u;
+      }, cf.e);
+    } else {
+      update_layer(sm, rows, cols, Cn, G, X, Wl, Sl);
+    }
+  };
   const int s = blockIdx.x, d = a.d, n = a.n, o = a.o, T = a.T, C = a.C;
   const long long P = a.P, nd = (long long)n * d;
   const int nch = (T + C - 1) / C;
@@ -633,14 +693,14 @@ __global__ void __launch_bounds__(NT) simt_backward2_kernel(BArgs2 a) {
   };
   // forward of the keys at (W1, W2): Z1, X1, G2, H = G2 W2, G1
   auto keys_forward = [&](int Cc, const float *W1, const float *W2) {
-    gemm(sm, Cc, n, d, K, d, 1, W1, d, 1, [&](int i, int j, float z) {
+    mm(Cc, n, d, K, d, 1, W1, d, 1, [&](int i, int j, float z) {
       Z1[i * n + j] = z;
       X1[i * n + j] = silu(z);
     });
     __syncthreads();
-    gemm(sm, Cc, o, n, X1, n, 1, W2, n, 1, [&](int i, int r, float z) { G2[i * o + r] = 2.f * (z - V[i * o + r]); });
+    mm(Cc, o, n, X1, n, 1, W2, n, 1, [&](int i, int r, float z) { G2[i * o + r] = 2.f * (z - V[i * o + r]); });
     __syncthreads();
-    gemm(sm, Cc, n, o, G2, o, 1, W2, 1, n, [&](int i, int j, float z) {
+    mm(Cc, n, o, G2, o, 1, W2, 1, n, [&](int i, int j, float z) {
       H[i * n + j] = z;
       G1[i * n + j] = z * silu_prime(Z1[i * n + j]);
     });
@@ -661,8 +721,8 @@ __global__ void __launch_bounds__(NT) simt_backward2_kernel(BArgs2 a) {
     chunk_coefficients(sm.coef, a.theta + tok0 + t0, a.eta + tok0 + t0, a.alpha + tok0 + t0, Cc);
     load_chunk(t0, Cc, false);
     keys_forward(Cc, Wc, Wc + nd);
-    update_layer(sm, o, n, Cc, G2, X1, Wc + nd, Sc + nd);
-    update_layer(sm, n, d, Cc, G1, K, Wc, Sc);
+    upd(o, n, Cc, G2, X1, Wc + nd, Sc + nd);
+    upd(n, d, Cc, G1, K, Wc, Sc);
     __syncthreads();
   }
   // ---- reverse
@@ -680,14 +740,14 @@ __global__ void __launch_bounds__(NT) simt_backward2_kernel(BArgs2 a) {
     chunk_coefficients(sm.coef, th, et, al, Cc);
     load_chunk(t0, Cc, true);
     keys_forward(Cc, W1, W2);
-    gemm(sm, Cc, n, d, Q, d, 1, W1, d, 1, [&](int i, int j, float z) {
+    mm(Cc, n, d, Q, d, 1, W1, d, 1, [&](int i, int j, float z) {
       ZQ[i * n + j] = z;
       XQ[i * n + j] = silu(z);
     });
-    gemm(sm, Cc, n, d, K, d, 1, gW1, d, 1, [&](int i, int j, float z) { KW1[i * n + j] = z; });
-    gemm(sm, Cc, n, d, K, d, 1, gS1, d, 1, [&](int i, int j, float z) { KS1[i * n + j] = z; });
-    gemm(sm, Cc, o, n, X1, n, 1, gW2, n, 1, [&](int i, int r, float z) { XW2[i * o + r] = z; });
-    gemm(sm, Cc, o, n, X1, n, 1, gS2, n, 1, [&](int i, int r, float z) { XS2[i * o + r] = z; });
+    mm(Cc, n, d, K, d, 1, gW1, d, 1, [&](int i, int j, float z) { KW1[i * n + j] = z; });
+    mm(Cc, n, d, K, d, 1, gS1, d, 1, [&](int i, int j, float z) { KS1[i * n + j] = z; });
+    mm(Cc, o, n, X1, n, 1, gW2, n, 1, [&](int i, int r, float z) { XW2[i * o + r] = z; });
+    mm(Cc, o, n, X1, n, 1, gS2, n, 1, [&](int i, int r, float z) { XS2[i * o + r] = z; });
     __syncthreads();
     // coefficient gradients: dc_i = -<gW, u_i>, de_i = -<gS, u_i>
     for (int i = threadIdx.x / 32; i < Cc; i += NT / 32) {
@@ -722,45 +782,45 @@ __global__ void __launch_bounds__(NT) simt_backward2_kernel(BArgs2 a) {
     }
     __syncthreads();
     // dG2 = b + dH W2^T (TO)
-    gemm(sm, Cc, o, n, T1, n, 1, W2, n, 1, [&](int i, int r, float z) { TO[i * o + r] = z + XW2[i * o + r]; });
+    mm(Cc, o, n, T1, n, 1, W2, n, 1, [&](int i, int r, float z) { TO[i * o + r] = z + XW2[i * o + r]; });
     __syncthreads();
     // state gradient of W2: B gW2 + G2^T dH + 2 dG2^T X1 + DY^T XQ
     const float Bw = sm.coef.Bw, As = sm.coef.As, cS = sm.coef.cS;
     float *gWn1 = gWn, *gWn2 = gWn + nd;
-    gemm(sm, o, n, Cc, G2, 1, o, T1, 1, n, [&](int r, int j, float z) { gWn2[r * n + j] = Bw * gW2[r * n + j] + z; });
+    mm(o, n, Cc, G2, 1, o, T1, 1, n, [&](int r, int j, float z) { gWn2[r * n + j] = Bw * gW2[r * n + j] + z; });
     __syncthreads();
-    gemm(sm, o, n, Cc, TO, 1, o, X1, 1, n, [&](int r, int j, float z) { gWn2[r * n + j] += 2.f * z; });
+    mm(o, n, Cc, TO, 1, o, X1, 1, n, [&](int r, int j, float z) { gWn2[r * n + j] += 2.f * z; });
     __syncthreads();
-    gemm(sm, o, n, Cc, DY, 1, o, XQ, 1, n, [&](int r, int j, float z) { gWn2[r * n + j] += z; });
+    mm(o, n, Cc, DY, 1, o, XQ, 1, n, [&](int r, int j, float z) { gWn2[r * n + j] += z; });
     __syncthreads();
     const long long gt_in = (tok0 + t0) * d, gt_out = (tok0 + t0) * o;
     for (int e = threadIdx.x; e < Cc * o; e += NT) a.dv[gt_out + e] = -2.f * TO[e];
     // dX1 = 2 dG2 W2 - c (G2 gW2) - e (G2 gS2)  (into T1, dH no longer needed)
-    gemm(sm, Cc, n, o, TO, o, 1, W2, 1, n, [&](int i, int j, float z) { T1[i * n + j] = 2.f * z; });
+    mm(Cc, n, o, TO, o, 1, W2, 1, n, [&](int i, int j, float z) { T1[i * n + j] = 2.f * z; });
     __syncthreads();
-    gemm(sm, Cc, n, o, G2, o, 1, gW2, 1, n, [&](int i, int j, float z) { T1[i * n + j] -= sm.coef.c[i] * z; });
+    mm(Cc, n, o, G2, o, 1, gW2, 1, n, [&](int i, int j, float z) { T1[i * n + j] -= sm.coef.c[i] * z; });
     __syncthreads();
-    gemm(sm, Cc, n, o, G2, o, 1, gS2, 1, n, [&](int i, int j, float z) { T1[i * n + j] -= sm.coef.e[i] * z; });
+    mm(Cc, n, o, G2, o, 1, gS2, 1, n, [&](int i, int j, float z) { T1[i * n + j] -= sm.coef.e[i] * z; });
     __syncthreads();
     // dZ1 = dX1 . silu'(z1) + dSP . silu''(z1)  (T1)
     for (int e = threadIdx.x; e < Cc * n; e += NT) T1[e] = T1[e] * silu_prime(Z1[e]) + T2[e] * silu_second(Z1[e]);
     __syncthreads();
     // reads: dZQ = (DY W2) . silu'(zq)  (T2)
-    gemm(sm, Cc, n, o, DY, o, 1, W2, 1, n, [&](int i, int j, float z) { T2[i * n + j] = z * silu_prime(ZQ[i * n + j]); });
+    mm(Cc, n, o, DY, o, 1, W2, 1, n, [&](int i, int j, float z) { T2[i * n + j] = z * silu_prime(ZQ[i * n + j]); });
     __syncthreads();
     // state gradient of W1: B gW1 + dZ1^T K + dZQ^T Q
-    gemm(sm, n, d, Cc, T1, 1, n, K, 1, d, [&](int j, int mm, float z) { gWn1[j * d + mm] = Bw * gW1[j * d + mm] + z; });
+    mm(n, d, Cc, T1, 1, n, K, 1, d, [&](int j, int mm, float z) { gWn1[j * d + mm] = Bw * gW1[j * d + mm] + z; });
     __syncthreads();
-    gemm(sm, n, d, Cc, T2, 1, n, Q, 1, d, [&](int j, int mm, float z) { gWn1[j * d + mm] += z; });
+    mm(n, d, Cc, T2, 1, n, Q, 1, d, [&](int j, int mm, float z) { gWn1[j * d + mm] += z; });
     __syncthreads();
     // dk = dZ1 W1 - c (G1 gW1) - e (G1 gS1);  dq = dZQ W1
-    gemm(sm, Cc, d, n, T1, n, 1, W1, 1, d, [&](int i, int mm, float z) { a.dk[gt_in + i * d + mm] = z; });
+    mm(Cc, d, n, T1, n, 1, W1, 1, d, [&](int i, int mm, float z) { a.dk[gt_in + i * d + mm] = z; });
     __syncthreads();
-    gemm(sm, Cc, d, n, G1, n, 1, gW1, 1, d, [&](int i, int mm, float z) { a.dk[gt_in + i * d + mm] -= sm.coef.c[i] * z; });
+    mm(Cc, d, n, G1, n, 1, gW1, 1, d, [&](int i, int mm, float z) { a.dk[gt_in + i * d + mm] -= sm.coef.c[i] * z; });
     __syncthreads();
-    gemm(sm, Cc, d, n, G1, n, 1, gS1, 1, d, [&](int i, int mm, float z) { a.dk[gt_in + i * d + mm] -= sm.coef.e[i] * z; });
+    mm(Cc, d, n, G1, n, 1, gS1, 1, d, [&](int i, int mm, float z) { a.dk[gt_in + i * d + mm] -= sm.coef.e[i] * z; });
     __syncthreads();
-    gemm(sm, Cc, d, n, T2, n, 1, W1, 1, d, [&](int i, int mm, float z) { a.dq[gt_in + i * d + mm] = z; });
+    mm(Cc, d, n, T2, n, 1, W1, 1, d, [&](int i, int mm, float z) { a.dq[gt_in + i * d + mm] = z; });
     // chunk scalars
     float pw = 0.f, pws = 0.f, pss = 0.f;
     for (long long e = threadIdx.x; e < P; e += NT) {
@@ -782,6 +842,7 @@ __global__ void __launch_bounds__(NT) simt_backward2_kernel(BArgs2 a) {
     a.dW0[sw + e] = gW[e];
     a.dS0[sw + e] = gS[e];
   }
+  if constexpr (TC) tcg_release(tg);
 }
 
 
@@ -801,6 +862,8 @@ constexpr int BWL_ARRAYS = 2 + 9 * (kMaxL + 1) + 3;   // V, DY; 9 per level; P1,
 
 struct BArgsL {
   int L, T, C, bf16, maxw;
+  int *status;                   // device status word (bounded waits of the tensor-core products)
+  unsigned long long wait_ns;
   int dims[kMaxL + 1];
   long long off[kMaxL + 1];
   long long P;
@@ -816,9 +879,36 @@ __host__ __device__ inline long long backwardL_floats(long long P, int maxw, int
   return 2 * nch * P + 5 * P + (long long)BWL_ARRAYS * C * maxw + 8LL * C;
 }
 
-__global__ void __launch_bounds__(NT) simt_backwardL_kernel(BArgsL a) {
+template <bool TC>
+__global__ void __launch_bounds__(NT) backwardL_kernel(BArgsL a) {
   __shared__ SmemT sm;
   __shared__ float red[NT / 32];
+  extern __shared__ __align__(1024) unsigned char tcg_dyn[];
+  __shared__ TcGemm tg;
+  if constexpr (TC) tcg_init(tg, tcg_dyn, a.status, a.wait_ns);
+  // the chunk's products: tcgen05 (TF32 operands, fp32 accumulation) or fp32 FFMA tiles
+  auto mm = [&](int M_, int N_, int K_, const float *A_, long long sam, long long sak, const float *B_,
+                long long sbn, long long sbk, auto epi) {
+    if constexpr (TC) tc_gemm(tg, M_, N_, K_, A_, sam, sak, B_, sbn, sbk, epi);
+    else gemm(sm, M_, N_, K_, A_, sam, sak, B_, sbn, sbk, epi);
+  };
+  // the forward pass's state update of one layer (A6 + A7): on the tensor
+  // cores as two products, U_W with the tokens' c and U_S with their e
+  auto upd = [&](int rows, int cols, int Cn, const float *G, const float *X, float *Wl, float *Sl) {
+    if constexpr (TC) {
+      const Coef &cf = sm.coef;
+      tc_gemm(tg, rows, cols, Cn, G, 1, rows, X, 1, cols, [&](int r, int c, float u) {
+        const long long idx = (long long)r * cols + c;
+        Wl[idx] = cf.Bw * Wl[idx] + cf.cS * Sl[idx] - u;
+      }, cf.c);
+      tc_gemm(tg, rows, cols, Cn, G, 1, rows, X, 1, cols, [&](int r, int c, float u) {
+        const long long idx = (long long)r * cols + c;
+        Sl[idx] = cf.As * Sl[idx] - u;
+      }, cf.e);
+    } else {
+      update_layer(sm, rows, cols, Cn, G, X, Wl, Sl);
+    }
+  };
   const int s = blockIdx.x, L = a.L, T = a.T, C = a.C, mw = a.maxw;
   const int *nn = a.dims;
   const long long P = a.P;
@@ -871,7 +961,7 @@ __global__ void __launch_bounds__(NT) simt_backwardL_kernel(BArgsL a) {
       const int r = nn[l], cl = nn[l - 1];
       float *Zl = Z[l], *Xl = X[l];
       const bool last = l == L;
-      gemm(sm, Cc, r, cl, X[l - 1], cl, 1, W + a.off[l - 1], cl, 1, [&](int i, int j, float z) {
+      mm(Cc, r, cl, X[l - 1], cl, 1, W + a.off[l - 1], cl, 1, [&](int i, int j, float z) {
         Zl[i * r + j] = z;
         Xl[i * r + j] = last ? z : silu(z);
       });
@@ -885,7 +975,7 @@ __global__ void __launch_bounds__(NT) simt_backwardL_kernel(BArgsL a) {
     for (int l = L; l >= 2; --l) {
       const int r = nn[l], cl = nn[l - 1];
       float *Hl = Hk[l - 1], *Gl = Gk[l - 1], *Zl = Zk[l - 1];
-      gemm(sm, Cc, cl, r, Gk[l], r, 1, W + a.off[l - 1], 1, cl, [&](int i, int j, float z) {
+      mm(Cc, cl, r, Gk[l], r, 1, W + a.off[l - 1], 1, cl, [&](int i, int j, float z) {
         Hl[i * cl + j] = z;
         Gl[i * cl + j] = z * silu_prime(Zl[i * cl + j]);
       });
@@ -908,7 +998,7 @@ __global__ void __launch_bounds__(NT) simt_backwardL_kernel(BArgsL a) {
     load_chunk(t0, Cc, false);
     forward(Cc, Wc, Xk, Zk);
     keys_backward(Cc, Wc);
-    for (int l = 1; l <= L; ++l) update_layer(sm, nn[l], nn[l - 1], Cc, Gk[l], Xk[l - 1], Wc + a.off[l - 1], Sc + a.off[l - 1]);
+    for (int l = 1; l <= L; ++l) upd(nn[l], nn[l - 1], Cc, Gk[l], Xk[l - 1], Wc + a.off[l - 1], Sc + a.off[l - 1]);
     __syncthreads();
   }
   // ---- reverse
@@ -934,8 +1024,8 @@ __global__ void __launch_bounds__(NT) simt_backwardL_kernel(BArgsL a) {
     for (int l = 1; l <= L; ++l) {
       const int r = nn[l], cl = nn[l - 1];
       const float *gWl = gW + a.off[l - 1], *gSl = gS + a.off[l - 1];
-      gemm(sm, Cc, r, cl, Xk[l - 1], cl, 1, gWl, cl, 1, [&](int i, int j, float z) { P1[i * r + j] = z; });
-      gemm(sm, Cc, r, cl, Xk[l - 1], cl, 1, gSl, cl, 1, [&](int i, int j, float z) { P2[i * r + j] = z; });
+      mm(Cc, r, cl, Xk[l - 1], cl, 1, gWl, cl, 1, [&](int i, int j, float z) { P1[i * r + j] = z; });
+      mm(Cc, r, cl, Xk[l - 1], cl, 1, gSl, cl, 1, [&](int i, int j, float z) { P2[i * r + j] = z; });
       __syncthreads();
       for (int i = threadIdx.x / 32; i < Cc; i += NT / 32) {
         float x = 0.f, y = 0.f;
@@ -953,9 +1043,9 @@ __global__ void __launch_bounds__(NT) simt_backwardL_kernel(BArgsL a) {
       }
       __syncthreads();
       float *dXl = dX[l - 1];
-      gemm(sm, Cc, cl, r, Gk[l], r, 1, gWl, 1, cl, [&](int i, int j, float z) { dXl[i * cl + j] = -sm.coef.c[i] * z; });
+      mm(Cc, cl, r, Gk[l], r, 1, gWl, 1, cl, [&](int i, int j, float z) { dXl[i * cl + j] = -sm.coef.c[i] * z; });
       __syncthreads();
-      gemm(sm, Cc, cl, r, Gk[l], r, 1, gSl, 1, cl, [&](int i, int j, float z) { dXl[i * cl + j] -= sm.coef.e[i] * z; });
+      mm(Cc, cl, r, Gk[l], r, 1, gSl, 1, cl, [&](int i, int j, float z) { dXl[i * cl + j] -= sm.coef.e[i] * z; });
       __syncthreads();
     }
     // back through the keys' backward recursion
@@ -967,9 +1057,9 @@ __global__ void __launch_bounds__(NT) simt_backwardL_kernel(BArgsL a) {
       }
       __syncthreads();
       float *gWnl = gWn + a.off[l - 1], *dGl = dG[l];
-      gemm(sm, r, cl, Cc, Gk[l], 1, r, dH, 1, cl, [&](int rr, int j, float z) { gWnl[rr * cl + j] += z; });
+      mm(r, cl, Cc, Gk[l], 1, r, dH, 1, cl, [&](int rr, int j, float z) { gWnl[rr * cl + j] += z; });
       __syncthreads();
-      gemm(sm, Cc, r, cl, dH, cl, 1, W + a.off[l - 1], cl, 1, [&](int i, int rr, float z) { dGl[i * r + rr] += z; });
+      mm(Cc, r, cl, dH, cl, 1, W + a.off[l - 1], cl, 1, [&](int i, int rr, float z) { dGl[i * r + rr] += z; });
       __syncthreads();
     }
     const long long gout = (tok0 + t0) * dL, gin = (tok0 + t0) * d0;
@@ -990,9 +1080,9 @@ __global__ void __launch_bounds__(NT) simt_backwardL_kernel(BArgsL a) {
       }
       __syncthreads();
       float *gWnl = gWn + a.off[l - 1], *dXl = dX[l - 1];
-      gemm(sm, r, cl, Cc, dZ, 1, r, Xk[l - 1], 1, cl, [&](int rr, int j, float z) { gWnl[rr * cl + j] += z; });
+      mm(r, cl, Cc, dZ, 1, r, Xk[l - 1], 1, cl, [&](int rr, int j, float z) { gWnl[rr * cl + j] += z; });
       __syncthreads();
-      gemm(sm, Cc, cl, r, dZ, r, 1, W + a.off[l - 1], 1, cl, [&](int i, int j, float z) { dXl[i * cl + j] += z; });
+      mm(Cc, cl, r, dZ, r, 1, W + a.off[l - 1], 1, cl, [&](int i, int j, float z) { dXl[i * cl + j] += z; });
       __syncthreads();
     }
     for (int e = threadIdx.x; e < Cc * d0; e += NT) a.dk[gin + e] = dX[0][e];
@@ -1006,9 +1096,9 @@ __global__ void __launch_bounds__(NT) simt_backwardL_kernel(BArgsL a) {
       for (int e = threadIdx.x; e < Cc * r; e += NT) dZ[e] = l == L ? dXq[L][e] : dXq[l][e] * silu_prime(Zq[l][e]);
       __syncthreads();
       float *gWnl = gWn + a.off[l - 1], *dXl = dXq[l - 1];
-      gemm(sm, r, cl, Cc, dZ, 1, r, Xq[l - 1], 1, cl, [&](int rr, int j, float z) { gWnl[rr * cl + j] += z; });
+      mm(r, cl, Cc, dZ, 1, r, Xq[l - 1], 1, cl, [&](int rr, int j, float z) { gWnl[rr * cl + j] += z; });
       __syncthreads();
-      gemm(sm, Cc, cl, r, dZ, r, 1, W + a.off[l - 1], 1, cl, [&](int i, int j, float z) { dXl[i * cl + j] = z; });
+      mm(Cc, cl, r, dZ, r, 1, W + a.off[l - 1], 1, cl, [&](int i, int j, float z) { dXl[i * cl + j] = z; });
       __syncthreads();
     }
     for (int e = threadIdx.x; e < Cc * d0; e += NT) a.dq[gin + e] = dXq[0][e];
@@ -1033,6 +1123,7 @@ __global__ void __launch_bounds__(NT) simt_backwardL_kernel(BArgsL a) {
     a.dW0[sw + e] = gW[e];
     a.dS0[sw + e] = gS[e];
   }
+  if constexpr (TC) tcg_release(tg);
 }
 
 }  // namespace
@@ -1089,6 +1180,18 @@ cudaError_t backward_launch(const Problem &p, const float *dy, const float *dW_e
                             float *dk, float *dv, float *dq, float *dtheta, float *deta, float *dalpha,
                             float *dW0, float *dS0, cudaStream_t stream) {
   if (!backward_supported(p)) return cudaErrorNotSupported;
+  if (p.bw_tc) {
+    static bool attr_done = false;
+    if (!attr_done) {
+      const void *kerns[3] = {(const void *)backward1_kernel<true>, (const void *)backward2_kernel<true>,
+                              (const void *)backwardL_kernel<true>};
+      for (const void *k : kerns) {
+        const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TCG_SMEM);
+        if (e != cudaSuccess) return e;
+      }
+      attr_done = true;
+    }
+  }
   if (p.L >= 3) {
     BArgsL b;
     b.L = p.L;
@@ -1110,7 +1213,10 @@ cudaError_t backward_launch(const Problem &p, const float *dy, const float *dW_e
     b.dW0 = dW0; b.dS0 = dS0;
     b.scratch = static_cast<float *>(p.scratch);
     b.scratch_per_stream = backwardL_floats(b.P, b.maxw, p.T, p.C);
-    simt_backwardL_kernel<<<p.streams, NT, 0, stream>>>(b);
+    b.status = p.status;
+    b.wait_ns = tcl_wait_ns();
+    if (p.bw_tc) backwardL_kernel<true><<<p.streams, NT, TCG_SMEM, stream>>>(b);
+    else backwardL_kernel<false><<<p.streams, NT, 0, stream>>>(b);
     return cudaGetLastError();
   }
   if (p.L == 2) {
@@ -1130,7 +1236,10 @@ cudaError_t backward_launch(const Problem &p, const float *dy, const float *dW_e
     b.dW0 = dW0; b.dS0 = dS0;
     b.scratch = static_cast<float *>(p.scratch);
     b.scratch_per_stream = backward2_floats(b.d, b.n, b.o, p.T, p.C);
-    simt_backward2_kernel<<<p.streams, NT, 0, stream>>>(b);
+    b.status = p.status;
+    b.wait_ns = tcl_wait_ns();
+    if (p.bw_tc) backward2_kernel<true><<<p.streams, NT, TCG_SMEM, stream>>>(b);
+    else backward2_kernel<false><<<p.streams, NT, 0, stream>>>(b);
     return cudaGetLastError();
   }
   BArgs a;
@@ -1147,7 +1256,10 @@ cudaError_t backward_launch(const Problem &p, const float *dy, const float *dW_e
   a.dW0 = dW0; a.dS0 = dS0;
   a.scratch = static_cast<float *>(p.scratch);
   a.scratch_per_stream = 2 * nch * d * d + 5 * d * d + 10 * C * d + 8 * C;
-  simt_backward_kernel<<<p.streams, NT, 0, stream>>>(a);
+  a.status = p.status;
+  a.wait_ns = tcl_wait_ns();
+  if (p.bw_tc) backward1_kernel<true><<<p.streams, NT, TCG_SMEM, stream>>>(a);
+  else backward1_kernel<false><<<p.streams, NT, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
