@@ -893,17 +893,19 @@ __global__ void __launch_bounds__(UP2_NT, 1)
 // more slots, so most of a unit's state is in flight at once, and a slot is
 // refilled as soon as its four readers are done with it.
 //   warps 0-15  epilogue: warp w owns TMEM lanes (columns) 32 (w % 4) .. +31
-//               and the 16-row chunks i = w / 4, w / 4 + 4, ...
+//               and the 16-row chunks i = w / 4, w / 4 + 4, ... (UP3_RQ = 4 row groups)
 //   warp 16     TMA loads (the first slots' state before waiting for the
 //               preceding kernel, which does not write it; the operands after)
 //   warp 17     TMEM allocation; MMA issue, rows 0-127 and 128-255 committed
 //               separately so that the epilogue starts on the first half
 // Every wait is bounded and gives up once another role has flagged an abort.
 constexpr int UP3_EPI = 16;                    // epilogue warps
+constexpr int UP3_RQ = UP3_EPI / 4;            // row groups (each reads every column of its chunks)
 constexpr int UP3_NT = (UP3_EPI + 2) * 32;
 constexpr int UP3_SLOT = 16384;                // W and S of 16 rows x 128 fp32 columns
 constexpr int UP3_NSLOT_MEM = 14;              // slots' worth of dynamic shared memory
-constexpr int UP3_NS = 12;                     // slots in the ring (a multiple of 4)
+constexpr int UP3_NS = 12;                     // slots in the ring (a multiple of the row groups)
+static_assert(UP3_NS % UP3_RQ == 0, "a slot is always read by the same row group");
 constexpr size_t UP3_SMEM = (size_t)UP3_NSLOT_MEM * UP3_SLOT + 1024;
 struct Up3Layer {
   int M, cols, rblocks, cblocks, first;        // rows and columns of W_l, 256-row and 128-column blocks, first unit
@@ -1092,7 +1094,7 @@ __global__ void __launch_bounds__(UP3_NT, 1)
     op_t *bout = ly.wb + (long long)s * ly.M * ly.cols + gcol;
     const int cols = ly.cols;
     int seen = 0;                              // halves of the accumulator known complete
-    for (int i = rq; i < nch; i += 4) {
+    for (int i = rq; i < nch; i += UP3_RQ) {
       const int h = 16 * i >= 128 ? 1 : 0;
       if (seen <= h) {
         if (!up3_wait(&mma_done[h], 0, a, abort)) break;
