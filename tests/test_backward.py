@@ -73,6 +73,27 @@ def test_backward_matches_gradient_oracle(cfg, path):
     assert max(worst.values()) < (TOL_TC if tc else TOL), worst
 
 
+@pytest.mark.gpu
+def test_tensor_core_backward_is_bit_identical_across_runs():
+    """The TF32 products sum over k in a fixed order: repeated calls agree bit for bit."""
+    L, d, e, B, H, T, C = 4, 128, 2, 1, 2, 96, 32
+    w = W.make(L, d, e, B, H, T, C, index=790)
+    dev = to_dev(W.generate(w), B, H, "bf16")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(7)
+    dy = torch.randn((B, H, T, d), generator=g, device="cuda")
+    dW = torch.randn(dev["W0"].shape, generator=g, device="cuda")
+    dS = torch.randn(dev["S0"].shape, generator=g, device="cuda")
+    mem = NeuralMemory(L, d, e)
+    run = lambda: mem.backward(dev["k"], dev["v"], dev["q"], dev["theta"], dev["eta"], dev["alpha"], dev["W0"],
+                               dev["S0"], dy, dW, dS, C)
+    a = run()
+    b = run()
+    torch.cuda.synchronize()
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
+
+
 def test_backward_refuses_before_any_launch():
     lib = N.load()
     h = ctypes.c_void_p()

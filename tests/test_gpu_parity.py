@@ -113,6 +113,32 @@ def test_state_carry_and_determinism(path):
     assert torch.equal(Wb, We) and torch.equal(Sb, Se)
 
 
+@pytest.mark.parametrize("shape", [(2, 128, 8, 2, 1, 256, 64), (4, 128, 2, 1, 2, 384, 128)],
+                         ids=["split-K-hidden1024", "transposed-update-deep"])
+def test_layered_runs_are_bit_identical(shape):
+    """The split reduction adds its partial tiles in split order and the
+    transposed update's chunks are fixed per warp: two runs (and a run split
+    in two with the state carried) give the same bits."""
+    L, d, e, B, H, T, C = shape
+    w = W.make(L, d, e, B, H, T, C, index=330 + d + e)
+    _, dev = _dev_inputs(w)
+    mem = NeuralMemory(w.L, w.d, w.expansion, path="tcl")
+    y, We, Se = run_lib(mem, dev, w.C)
+    for _ in range(2):
+        y_b, We_b, Se_b = run_lib(mem, dev, w.C)
+        assert torch.equal(y, y_b) and torch.equal(We, We_b) and torch.equal(Se, Se_b)
+    T1 = 2 * C
+    first = {k: (v[:, :, :T1].contiguous() if k in ("k", "v", "q", "theta", "eta", "alpha") else v)
+             for k, v in dev.items()}
+    ya, Wa, Sa = run_lib(mem, first, w.C)
+    second = {k: (v[:, :, T1:].contiguous() if k in ("k", "v", "q", "theta", "eta", "alpha") else v)
+              for k, v in dev.items()}
+    second["W0"], second["S0"] = Wa, Sa
+    yb, Wb, Sb = run_lib(mem, second, w.C)
+    assert torch.equal(torch.cat([ya, yb], dim=2), y)
+    assert torch.equal(Wb, We) and torch.equal(Sb, Se)
+
+
 @pytest.mark.parametrize("path", ["simt", "tc", "tcl"])
 def test_streams_independent_and_permutable(path):
     w = W.make(2, 64, 1, 1, 4, 128, 64, index=303)
