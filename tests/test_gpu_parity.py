@@ -435,7 +435,7 @@ def test_tcl_matches_cluster_kernel():
 
 
 
-@pytest.mark.parametrize("path", ["tcl", "tcl-phased"])
+@pytest.mark.parametrize("path", ["tcl", "tcl-phased", "tcl-phased-split"])
 def test_tcl_timeout_is_reported_and_context_survives(path):
     """The layered kernels' failure handling: with the test hook on, every CTA
     of the forward/backward (fused or per phase) and update kernels first
@@ -445,9 +445,14 @@ def test_tcl_timeout_is_reported_and_context_survives(path):
     from test_trained_neural_b200 import _native as N
     from test_trained_neural_b200._native import TitansMemError
     lib = N.load()
-    w = W.make(4, 64, 2, 1, 2, 256, 128, index=650) if path == "tcl" else W.make(2, 128, 3, 1, 1, 128, 64, index=651)
+    # "tcl": fused kernel and the update for 64-wide inputs; "tcl-phased": the
+    # per-phase GEMMs and the transposed update; "-split": hidden 1024, whose
+    # last forward splits K = 1024 over 4 CTAs per tile
+    w = {"tcl": W.make(4, 64, 2, 1, 2, 256, 128, index=650),
+         "tcl-phased": W.make(2, 128, 3, 1, 1, 128, 64, index=651),
+         "tcl-phased-split": W.make(2, 128, 8, 1, 1, 128, 64, index=652)}[path]
     inp, dev = _dev_inputs(w)
-    mem = NeuralMemory(w.L, w.d, w.expansion, path=path)
+    mem = NeuralMemory(w.L, w.d, w.expansion, path=path.replace("-split", ""))
     assert lib.tm_set_debug(1, 1_000_000) == N.TM_OK
     try:
         for _ in range(2):          # a repeated call goes through graph capture and replay
