@@ -350,6 +350,7 @@ struct BArgs {
   int d, T, C, bf16;
   int *status;                   // device status word (bounded waits of the tensor-core products)
   unsigned long long wait_ns;
+  int inject;                    // test hook (tm_set_debug), tensor-core products only
   const void *k, *v, *q;
   const float *theta, *eta, *alpha, *W0, *S0, *dy, *dW_end, *dS_end;
   float *dk, *dv, *dq, *dtheta, *deta, *dalpha, *dW0, *dS0;
@@ -420,7 +421,7 @@ __global__ void __launch_bounds__(NT) backward1_kernel(BArgs a) {
   __shared__ float red[NT / 32];
   extern __shared__ __align__(1024) unsigned char tcg_dyn[];
   __shared__ TcGemm tg;
-  if constexpr (TC) tcg_init(tg, tcg_dyn, a.status, a.wait_ns);
+  if constexpr (TC) tcg_init(tg, tcg_dyn, a.status, a.wait_ns, a.inject);
   // the chunk's products: tcgen05 (TF32 operands, fp32 accumulation) or fp32 FFMA tiles
   auto mm = [&](int M_, int N_, int K_, const float *A_, long long sam, long long sak, const float *B_,
                 long long sbn, long long sbk, auto epi) {
@@ -606,6 +607,7 @@ struct BArgs2 {
   int d, n, o, T, C, bf16;
   int *status;                   // device status word (bounded waits of the tensor-core products)
   unsigned long long wait_ns;
+  int inject;                    // test hook (tm_set_debug), tensor-core products only
   long long P;
   const void *k, *v, *q;
   const float *theta, *eta, *alpha, *W0, *S0, *dy, *dW_end, *dS_end;
@@ -626,7 +628,7 @@ __global__ void __launch_bounds__(NT) backward2_kernel(BArgs2 a) {
   __shared__ float red[NT / 32];
   extern __shared__ __align__(1024) unsigned char tcg_dyn[];
   __shared__ TcGemm tg;
-  if constexpr (TC) tcg_init(tg, tcg_dyn, a.status, a.wait_ns);
+  if constexpr (TC) tcg_init(tg, tcg_dyn, a.status, a.wait_ns, a.inject);
   // the chunk's products: tcgen05 (TF32 operands, fp32 accumulation) or fp32 FFMA tiles
   auto mm = [&](int M_, int N_, int K_, const float *A_, long long sam, long long sak, const float *B_,
                 long long sbn, long long sbk, auto epi) {
@@ -864,6 +866,7 @@ struct BArgsL {
   int L, T, C, bf16, maxw;
   int *status;                   // device status word (bounded waits of the tensor-core products)
   unsigned long long wait_ns;
+  int inject;                    // test hook (tm_set_debug), tensor-core products only
   int dims[kMaxL + 1];
   long long off[kMaxL + 1];
   long long P;
@@ -885,7 +888,7 @@ __global__ void __launch_bounds__(NT) backwardL_kernel(BArgsL a) {
   __shared__ float red[NT / 32];
   extern __shared__ __align__(1024) unsigned char tcg_dyn[];
   __shared__ TcGemm tg;
-  if constexpr (TC) tcg_init(tg, tcg_dyn, a.status, a.wait_ns);
+  if constexpr (TC) tcg_init(tg, tcg_dyn, a.status, a.wait_ns, a.inject);
   // the chunk's products: tcgen05 (TF32 operands, fp32 accumulation) or fp32 FFMA tiles
   auto mm = [&](int M_, int N_, int K_, const float *A_, long long sam, long long sak, const float *B_,
                 long long sbn, long long sbk, auto epi) {
@@ -1215,6 +1218,7 @@ cudaError_t backward_launch(const Problem &p, const float *dy, const float *dW_e
     b.scratch_per_stream = backwardL_floats(b.P, b.maxw, p.T, p.C);
     b.status = p.status;
     b.wait_ns = tcl_wait_ns();
+    b.inject = tcl_inject();
     if (p.bw_tc) backwardL_kernel<true><<<p.streams, NT, TCG_SMEM, stream>>>(b);
     else backwardL_kernel<false><<<p.streams, NT, 0, stream>>>(b);
     return cudaGetLastError();
@@ -1238,6 +1242,7 @@ cudaError_t backward_launch(const Problem &p, const float *dy, const float *dW_e
     b.scratch_per_stream = backward2_floats(b.d, b.n, b.o, p.T, p.C);
     b.status = p.status;
     b.wait_ns = tcl_wait_ns();
+    b.inject = tcl_inject();
     if (p.bw_tc) backward2_kernel<true><<<p.streams, NT, TCG_SMEM, stream>>>(b);
     else backward2_kernel<false><<<p.streams, NT, 0, stream>>>(b);
     return cudaGetLastError();
@@ -1258,6 +1263,7 @@ cudaError_t backward_launch(const Problem &p, const float *dy, const float *dW_e
   a.scratch_per_stream = 2 * nch * d * d + 5 * d * d + 10 * C * d + 8 * C;
   a.status = p.status;
   a.wait_ns = tcl_wait_ns();
+  a.inject = tcl_inject();
   if (p.bw_tc) backward1_kernel<true><<<p.streams, NT, TCG_SMEM, stream>>>(a);
   else backward1_kernel<false><<<p.streams, NT, 0, stream>>>(a);
   return cudaGetLastError();

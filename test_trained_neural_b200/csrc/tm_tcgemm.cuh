@@ -41,6 +41,8 @@ constexpr size_t TCG_SMEM = TCG_A_BYTES + TCG_B_BYTES + 1024;   // dynamic share
 
 struct TcGemm {
   uint64_t bar;          // MMA completion
+  uint64_t never;        // test hook: a barrier nothing completes
+  int inject;            // test hook on: the CTA's first product first waits on `never`
   uint32_t uses;         // completed phases of bar
   uint32_t tmem;         // TMEM base (256 columns)
   int *status;
@@ -78,11 +80,14 @@ __device__ __forceinline__ uint32_t tcg_off(int rows, int r, int k) {
 
 // Set up by the whole CTA at kernel start (dyn: the kernel's dynamic shared
 // memory, TCG_SMEM bytes).
-__device__ __forceinline__ void tcg_init(TcGemm &g, unsigned char *dyn, int *status, unsigned long long wait_ns) {
+__device__ __forceinline__ void tcg_init(TcGemm &g, unsigned char *dyn, int *status, unsigned long long wait_ns,
+                                         int inject) {
   using namespace sm100;
   unsigned char *al = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(dyn) + 1023) & ~uintptr_t(1023));
   if (threadIdx.x == 0) {
     mbar_init(&g.bar, 1);
+    mbar_init(&g.never, 1);
+    g.inject = inject;
     g.uses = 0;
     g.status = status;
     g.wait_ns = wait_ns;
@@ -160,6 +165,12 @@ __device__ __noinline__ bool tcg_block(TcGemm &g, int M, int N, int K, int m0, i
   const uint32_t idesc = idesc_tf32(128, np);
   uint32_t uses = g.uses;                       // read by every thread; updated identically
   bool ok = true;
+  if (g.inject && uses == 0 && !mbar_wait(&g.never, 0, g.wait_ns)) {
+    // test hook: the wait ran out as a lost MMA completion would; recorded,
+    // and the call goes on (its products are still issued and awaited)
+    if (tid == 0) atomicCAS(g.status, 0, kDevTimeout);
+    ok = false;
+  }
   for (int k0 = 0; k0 < K; k0 += TCG_KR) {
     // ---- stage the round's operands (zeros outside M, N, K)
     tcg_stage(g.a, 128, 7, 128 * TCG_KR, sak == 1, A, sam, sak, m0, M - m0, k0, K, kscale);

@@ -166,16 +166,18 @@ class NeuralMemory:
         N.check(code, "tm_decode_step")
         return y
 
-    def backward(self, k, v, q, theta, eta, alpha, W0, S0, dy, dW_end, dS_end, C, stream=None):
+    def backward(self, k, v, q, theta, eta, alpha, W0, S0, dy, dW_end, dS_end, C, stream=None, workspace=None):
         """Gradients of sum <dy, y> + <dW_end, W_end> + <dS_end, S_end> for the
         run with these inputs (any depth). Returns a dict of float32 tensors dk,
-        dv, dq, dtheta, deta, dalpha, dW0, dS0."""
+        dv, dq, dtheta, deta, dalpha, dW0, dS0. With a caller's workspace (uint8,
+        at least backward_workspace_size bytes), sync(workspace) then reports
+        the call's device-side status."""
         B, H, T, d = k.shape
         dt = self._dtype_code(k)
-        n = ctypes.c_size_t()
-        N.check(self._lib.tm_backward_workspace_size(self._h, B, H, T, C, dt, ctypes.byref(n)),
-                "tm_backward_workspace_size")
-        ws = torch.empty(int(n.value), dtype=torch.uint8, device=k.device)
+        if workspace is None:
+            workspace = torch.empty(self.backward_workspace_size(B, H, T, C, k.dtype), dtype=torch.uint8,
+                                    device=k.device)
+        ws = workspace
         f32 = dict(dtype=torch.float32, device=k.device)
         out = {"dk": torch.empty((B, H, T, d), **f32), "dv": torch.empty((B, H, T, d), **f32),
                "dq": torch.empty((B, H, T, d), **f32), "dtheta": torch.empty((B, H, T), **f32),
@@ -190,6 +192,13 @@ class NeuralMemory:
             _ptr(ws), ws.numel(), ctypes.c_void_p(stream.cuda_stream))
         N.check(code, "tm_backward")
         return out
+
+    def backward_workspace_size(self, B, H, T, C, dtype) -> int:
+        n = ctypes.c_size_t()
+        dt = N.TM_BF16 if dtype == torch.bfloat16 else N.TM_F32
+        N.check(self._lib.tm_backward_workspace_size(self._h, B, H, T, C, dt, ctypes.byref(n)),
+                "tm_backward_workspace_size")
+        return int(n.value)
 
     def sync(self, workspace, stream=None):
         if stream is None:

@@ -126,6 +126,42 @@ def test_tensor_core_backward_matches_fp32_at_full_length(idx):
     assert max(worst.values()) < TOL_TC, worst
 
 
+@pytest.mark.gpu
+def test_tensor_core_backward_timeout_is_reported_and_context_survives():
+    """With the test hook on (tm_set_debug), each CTA's first tensor-core
+    product first waits on a barrier that nothing completes: the wait runs out
+    after 1 ms, TM_ERR_TIMEOUT is recorded in the call's workspace and reported
+    by tm_sync, and nothing hangs. The next call on the same context (hook off)
+    matches the fp32 form."""
+    from test_trained_neural_b200._native import TitansMemError
+    lib = N.load()
+    L, d, e, B, H, T, C = 2, 64, 4, 1, 2, 128, 64
+    w = W.make(L, d, e, B, H, T, C, index=795)
+    dev = to_dev(W.generate(w), B, H, "bf16")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(3)
+    dy = torch.randn((B, H, T, d), generator=g, device="cuda")
+    dW = torch.randn(dev["W0"].shape, generator=g, device="cuda")
+    dS = torch.randn(dev["S0"].shape, generator=g, device="cuda")
+    mem = NeuralMemory(L, d, e)
+    args = (dev["k"], dev["v"], dev["q"], dev["theta"], dev["eta"], dev["alpha"], dev["W0"], dev["S0"], dy, dW, dS, C)
+    ws = torch.empty(mem.backward_workspace_size(B, H, T, C, torch.bfloat16), dtype=torch.uint8, device="cuda")
+    assert lib.tm_set_debug(1, 1_000_000) == N.TM_OK
+    try:
+        mem.backward(*args, workspace=ws)
+        with pytest.raises(TitansMemError) as ei:
+            mem.sync(ws)
+        assert ei.value.code == N.TM_ERR_TIMEOUT
+    finally:
+        lib.tm_set_debug(0, 0)
+    got = mem.backward(*args, workspace=ws)
+    mem.sync(ws)
+    ref = NeuralMemory(L, d, e, path="simt").backward(*args)
+    torch.cuda.synchronize()
+    for k in got:
+        assert rel(got[k].double().cpu().numpy(), ref[k].double().cpu().numpy()) < TOL_TC, k
+
+
 def test_backward_refuses_before_any_launch():
     lib = N.load()
     h = ctypes.c_void_p()
