@@ -95,6 +95,11 @@ __global__ void __launch_bounds__(DT, 1) decode2_kernel(const DecArgs a) {
   float *W1g = W + (long long)DHS * j * D, *S1g = S + (long long)DHS * j * D;   // rows of W1 [hid x D]
   float *W2g = W + (long long)hid * D, *S2g = S + (long long)hid * D;           // W2 [D x hid]
 
+  // Consecutive steps are launched with programmatic serialization: the next
+  // step may be launched now, and this one reads nothing (state or token)
+  // before the previous kernel of the stream has completed.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // stage the slices (asynchronous 16-byte copies, all in flight) and the token
   for (int i = tid; i < DHS * D / 4; i += DT) {
     cp_async16(W1s + 4 * i, W1g + 4 * i);
@@ -225,6 +230,9 @@ __global__ void __launch_bounds__(DT) decode1_kernel(const DecArgs a, int rows_p
   const int s = blockIdx.x / ctas;
   const int r = (blockIdx.x % ctas) * rows_per_cta + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
+  // launched with programmatic serialization, as the depth-2 step
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (r >= d) return;
   float *Wr = a.W + (long long)s * a.P + (long long)r * d;
   float *Sr = a.S + (long long)s * a.P + (long long)r * d;
@@ -261,13 +269,15 @@ cudaError_t launch2(const DecArgs &a, int streams, cudaStream_t st) {
   cfg.blockDim = dim3(DT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = (unsigned)a.G;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, decode2_kernel<D>, a);
 }
 
@@ -304,8 +314,16 @@ cudaError_t decode_launch(const Problem &p, const void *k, const void *v, const 
   if (p.L == 1) {
     const int rows = DT / 32;
     const int ctas = (a.d + rows - 1) / rows;
-    decode1_kernel<<<(unsigned)(p.streams * ctas), DT, 0, st>>>(a, rows);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.streams * ctas));
+    cfg.blockDim = dim3(DT);
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode1_kernel, a, rows);
   }
   return a.d == 64 ? launch2<64>(a, p.streams, st) : launch2<128>(a, p.streams, st);
 }
