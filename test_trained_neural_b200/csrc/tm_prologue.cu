@@ -89,18 +89,20 @@ __device__ __forceinline__ void store4(void *p, long long i, const float o[4]) {
 template <typename T>
 __device__ __forceinline__ T pick(int z, T a, T b, T c) { return z == 0 ? a : (z == 1 ? b : c); }
 
-// MAXW: taps held in registers (4 or 8; taps beyond the filter width are zero)
-template <bool BF16, bool WIDE, int MAXW>
+// MAXW: taps held in registers (4 or 8; taps beyond the filter width are zero);
+// RBT: output rows per row group (more rows amortise the w - 1 halo rows and
+// the CTA's start over more work, fewer rows give small problems more CTAs)
+template <bool BF16, bool WIDE, int MAXW, int RBT = RB>
 __global__ void __launch_bounds__(NT, (!WIDE && MAXW == 4) ? 3 : 2) prologue_kernel(const ProArgs a) {
   using El = typename std::conditional<BF16, __nv_bfloat16, float>::type;
-  __shared__ float part[NT / 32][RB];        // per-warp partial sums of squares (d > 128)
+  __shared__ float part[NT / 32][RBT];        // per-warp partial sums of squares (d > 128)
   const int s = blockIdx.y, z = blockIdx.z;
   const int d = a.d, w = a.w, T = a.T;
   const int d4 = d / 4;
   const int g = threadIdx.x % d4, rl = threadIdx.x / d4;
   const int RL = blockDim.x / d4;
   const int c = 4 * g;
-  const long long tb = (long long)(blockIdx.x * RL + rl) * RB;   // first output row
+  const long long tb = (long long)(blockIdx.x * RL + rl) * RBT;   // first output row
   const El *in = static_cast<const El *>(pick(z, a.in[0], a.in[1], a.in[2]));
   const El *hist = static_cast<const El *>(pick(z, a.hist[0], a.hist[1], a.hist[2]));
   const float *fp = pick(z, a.filt[0], a.filt[1], a.filt[2]) + ((long long)(s % a.H) * d + c) * w;
@@ -108,9 +110,9 @@ __global__ void __launch_bounds__(NT, (!WIDE && MAXW == 4) ? 3 : 2) prologue_ker
   const long long base = (long long)s * T * d;
 
   // raw[i] holds input row tb - (MAXW - 1) + i; only rows i >= MAXW - w feed a tap
-  Raw<BF16> raw[RB + MAXW - 1];
+  Raw<BF16> raw[RBT + MAXW - 1];
 #pragma unroll
-  for (int i = 0; i < RB + MAXW - 1; ++i) {
+  for (int i = 0; i < RBT + MAXW - 1; ++i) {
     const long long t = tb - (MAXW - 1) + i;
     const bool live = i + w >= MAXW && t < T && (t >= 0 || hist != nullptr);
     const El *p = t >= 0 ? in + base + t * d + c : hist + ((long long)s * (w - 1) + (w - 1 + t)) * d + c;
@@ -132,7 +134,7 @@ __global__ void __launch_bounds__(NT, (!WIDE && MAXW == 4) ? 3 : 2) prologue_ker
     // more CTAs and more loads in flight per SM)
     const int width = d4;
 #pragma unroll
-    for (int r = 0; r < RB; ++r) {
+    for (int r = 0; r < RBT; ++r) {
       float o[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < MAXW; ++j) {
@@ -155,59 +157,59 @@ __global__ void __launch_bounds__(NT, (!WIDE && MAXW == 4) ? 3 : 2) prologue_ker
     }
     return;
   } else {
-  float o[RB][4];
+  float o[RBT][4];
 #pragma unroll
-  for (int r = 0; r < RB; ++r)
+  for (int r = 0; r < RBT; ++r)
 #pragma unroll
     for (int e = 0; e < 4; ++e) o[r][e] = 0.f;
 #pragma unroll
-  for (int i = 0; i < RB + MAXW - 1; ++i) {
+  for (int i = 0; i < RBT + MAXW - 1; ++i) {
     float x[4];
     raw[i].to_f32(x);
 #pragma unroll
     for (int j = 0; j < MAXW; ++j) {
       const int r = i + j - (MAXW - 1);      // output row that input row i feeds through tap j
-      if (r < 0 || r >= RB) continue;
+      if (r < 0 || r >= RBT) continue;
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[r][e] = fmaf(f[j][e], x[e], o[r][e]);
     }
   }
 
   if (norm) {
-    float ss[RB];
+    float ss[RBT];
 #pragma unroll
-    for (int r = 0; r < RB; ++r) {
+    for (int r = 0; r < RBT; ++r) {
       ss[r] = 0.f;
 #pragma unroll
       for (int e = 0; e < 4; ++e) ss[r] = fmaf(o[r][e], o[r][e], ss[r]);
     }
     const int width = d4 < 32 ? d4 : 32;
 #pragma unroll
-    for (int r = 0; r < RB; ++r)
+    for (int r = 0; r < RBT; ++r)
       for (int off = width / 2; off > 0; off >>= 1) ss[r] += __shfl_xor_sync(0xffffffffu, ss[r], off);
     if (d4 > 32) {                           // row group spans d4/32 whole warps
       const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
       if (lane == 0)
 #pragma unroll
-        for (int r = 0; r < RB; ++r) part[warp][r] = ss[r];
+        for (int r = 0; r < RBT; ++r) part[warp][r] = ss[r];
       __syncthreads();
       const int w0 = rl * (d4 / 32);
 #pragma unroll
-      for (int r = 0; r < RB; ++r) {
+      for (int r = 0; r < RBT; ++r) {
         float t = 0.f;
         for (int k = 0; k < d4 / 32; ++k) t += part[w0 + k][r];
         ss[r] = t;
       }
     }
 #pragma unroll
-    for (int r = 0; r < RB; ++r) {
+    for (int r = 0; r < RBT; ++r) {
       const float scale = ss[r] > 0.f ? 1.f / sqrtf(ss[r]) : 0.f;
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[r][e] *= scale;
     }
   }
 #pragma unroll
-  for (int r = 0; r < RB; ++r) {
+  for (int r = 0; r < RBT; ++r) {
     const long long t = tb + r;
     if (t < T) store4<BF16>(out, base + t * d + c, o[r]);
   }
@@ -242,12 +244,18 @@ cudaError_t prologue_launch(int streams, int H, int T, int d, int w, bool bf16, 
     a.out[i] = out[i];
   }
   const int RL = rows_groups_per_cta(d);
-  const int rows = RL * RB;
+  const bool wide = d / 4 > 32, short_filter = w <= 4;
+  // bf16, d <= 128, short filter, at least 2^20 rows per tensor: 16 rows per
+  // row group (measured on 16 streams x 262144 tokens of d = 128: 3.06 ->
+  // 2.79 ms; on 32 x 8192 tokens of d = 64 the 8-row form stays faster)
+  const bool long_rows = bf16 && !wide && short_filter && (long long)streams * T >= (1LL << 20);
+  const int rows = RL * (long_rows ? 2 * RB : RB);
   dim3 grid((unsigned)((T + rows - 1) / rows), (unsigned)streams, 3);
   const dim3 block((unsigned)(RL * (d / 4)));
-  const bool wide = d / 4 > 32, short_filter = w <= 4;
   auto go = [&](auto kern) { kern<<<grid, block, 0, stream>>>(a); };
-  if (bf16) {
+  if (long_rows) {
+    go(prologue_kernel<true, false, 4, 2 * RB>);
+  } else if (bf16) {
     if (wide) short_filter ? go(prologue_kernel<true, true, 4>) : go(prologue_kernel<true, true, 8>);
     else short_filter ? go(prologue_kernel<true, false, 4>) : go(prologue_kernel<true, false, 8>);
   } else {

@@ -88,6 +88,8 @@ def _f64(a, dtype):
     (1, 1, 70, 768, 5, "bf16", True),       # widest row: six warps per row
     (3, 1, 9, 128, 2, "f32", True),         # sequence shorter than one tile
     (1, 2, 100, 128, 6, "bf16", True),      # filter wider than 4 taps, rows inside one warp
+    (2, 8, 65600, 128, 4, "bf16", True),    # >= 2^20 rows: 16 output rows per row group, ragged end
+    (1, 2, 524300, 32, 4, "bf16", False),   # the same form with 8-lane row groups
 ])
 def test_prologue_matches_oracle(B, H, T, d, width, dtype, hist):
     from test_trained_neural_b200 import prologue
